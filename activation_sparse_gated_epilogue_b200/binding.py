@@ -1,0 +1,196 @@
+"""ctypes binding of libsge.so: argument marshalling only.
+
+Each function has the name of the C entry point it calls and takes torch
+tensors on a CUDA device; outputs not given are allocated with torch (device
+memory is the only thing PyTorch provides here) and returned.  Launches go on
+the current torch stream of the tensors' device unless ``stream`` is given.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+SGE_F32, SGE_BF16 = 0, 1
+_DTYPES = {torch.float32: SGE_F32, torch.bfloat16: SGE_BF16}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libsge.so")
+_lib = None
+
+
+class LibraryError(RuntimeError):
+    """A C entry point returned an error code (message from sge_last_error)."""
+
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed (code {code}): {msg}")
+        self.code = code
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def library() -> ctypes.CDLL:
+    """Load libsge.so (built in-tree by ``python -m
+    activation_sparse_gated_epilogue_b200.build``); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m activation_sparse_gated_epilogue_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        sigs = {
+            "sge_version": (I, []),
+            "sge_last_error": (ctypes.c_char_p, []),
+            "twell_gate_pack": (I, [P, P, I64, I64, I64, I, I, I, P, P, P, P, P]),
+            "twell_fused_up_down": (I, [P, P, P, P, P, P, P, I64, I64, I64, I, I, I, P]),
+            "dense_ffn_fwd": (I, [P, P, P, P, P, P, I64, I64, I64, P, P]),
+        }
+        for name, (res, args) in sigs.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _call(name: str, *args) -> None:
+    lib = library()
+    rc = getattr(lib, name)(*args)
+    if rc != 0:
+        raise LibraryError(name, rc, lib.sge_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t: torch.Tensor, name: str, dtype=None, shape=None) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _stream(dev: torch.device, stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream(dev) if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {t.dtype}")
+    return _DTYPES[t.dtype]
+
+
+def new_diag(device) -> torch.Tensor:
+    """A zeroed int32[4] diagnostics word (see include/sge.h)."""
+    return torch.zeros(4, dtype=torch.int32, device=device)
+
+
+@dataclass
+class TwELL:
+    """Device TwELL buffers: count [N][F/T] u8, idx [N][F/T][C] u8,
+    val [N][F/T][C] in the activation dtype."""
+    count: torch.Tensor
+    idx: torch.Tensor
+    val: torch.Tensor
+    tile: int
+    cap: int
+
+    @property
+    def n_rows(self) -> int:
+        return self.count.shape[0]
+
+    @property
+    def n_cols(self) -> int:
+        return self.count.shape[1] * self.tile
+
+    @staticmethod
+    def empty(n: int, f: int, tile: int, cap: int, dtype, device) -> "TwELL":
+        nt = f // tile
+        return TwELL(torch.empty((n, nt), dtype=torch.uint8, device=device),
+                     torch.empty((n, nt, cap), dtype=torch.uint8, device=device),
+                     torch.empty((n, nt, cap), dtype=dtype, device=device), tile, cap)
+
+
+def twell_gate_pack(x: torch.Tensor, wg_t: torch.Tensor, tile: int, cap: int,
+                    out: Optional[TwELL] = None, diag: Optional[torch.Tensor] = None,
+                    stream=None) -> TwELL:
+    """TwELL of ReLU(x W_gate), produced in the gate GEMM's epilogue."""
+    _check(x, "x")
+    n, d = x.shape
+    f = wg_t.shape[0]
+    _check(wg_t, "wg_t", x.dtype, (f, d))
+    if out is None:
+        out = TwELL.empty(n, f, tile, cap, x.dtype, x.device)
+    else:
+        _check(out.count, "count", torch.uint8, (n, f // tile))
+        _check(out.idx, "idx", torch.uint8, (n, f // tile, cap))
+        _check(out.val, "val", x.dtype, (n, f // tile, cap))
+    if diag is not None:
+        _check(diag, "diag", torch.int32, (4,))
+    _call("twell_gate_pack", _ptr(x), _ptr(wg_t), n, d, f, _dtype_code(x), tile, cap,
+          _ptr(out.count), _ptr(out.idx), _ptr(out.val), _ptr(diag), _stream(x.device, stream))
+    return out
+
+
+def twell_fused_up_down(x: torch.Tensor, tw: TwELL, wu_t: torch.Tensor, wd: torch.Tensor,
+                        y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """y = sum over TwELL entries of a * (x . W_up[:, j]) * W_down[j] (h never stored)."""
+    _check(x, "x")
+    n, d = x.shape
+    f = wu_t.shape[0]
+    _check(wu_t, "wu_t", x.dtype, (f, d))
+    _check(wd, "wd", x.dtype, (f, d))
+    _check(tw.count, "count", torch.uint8, (n, f // tw.tile))
+    _check(tw.idx, "idx", torch.uint8, (n, f // tw.tile, tw.cap))
+    _check(tw.val, "val", x.dtype, (n, f // tw.tile, tw.cap))
+    if y is None:
+        y = torch.empty_like(x)
+    _check(y, "y", x.dtype, (n, d))
+    _call("twell_fused_up_down", _ptr(x), _ptr(tw.count), _ptr(tw.idx), _ptr(tw.val),
+          _ptr(wu_t), _ptr(wd), _ptr(y), n, d, f, _dtype_code(x), tw.tile, tw.cap,
+          _stream(x.device, stream))
+    return y
+
+
+def twell_ffn_forward(x, wg_t, wu_t, wd, tile: int, cap: int, tw: Optional[TwELL] = None,
+                      y: Optional[torch.Tensor] = None, diag: Optional[torch.Tensor] = None,
+                      stream=None):
+    """The sparse inference forward: gate GEMM + TwELL epilogue, then the
+    fused up/down kernel.  Returns (y, twell)."""
+    tw = twell_gate_pack(x, wg_t, tile, cap, out=tw, diag=diag, stream=stream)
+    y = twell_fused_up_down(x, tw, wu_t, wd, y=y, stream=stream)
+    return y, tw
+
+
+def dense_ffn_fwd(x: torch.Tensor, wg_t: torch.Tensor, wu_t: torch.Tensor, wd_t: torch.Tensor,
+                  h: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                  diag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Dense bf16 gated FFN (baseline).  ``wd_t`` is W_down transposed, [d][F]."""
+    _check(x, "x", torch.bfloat16)
+    n, d = x.shape
+    f = wg_t.shape[0]
+    _check(wg_t, "wg_t", torch.bfloat16, (f, d))
+    _check(wu_t, "wu_t", torch.bfloat16, (f, d))
+    _check(wd_t, "wd_t", torch.bfloat16, (d, f))
+    if h is None:
+        h = torch.empty((n, f), dtype=torch.bfloat16, device=x.device)
+    if y is None:
+        y = torch.empty_like(x)
+    _check(h, "h", torch.bfloat16, (n, f))
+    _check(y, "y", torch.bfloat16, (n, d))
+    _call("dense_ffn_fwd", _ptr(x), _ptr(wg_t), _ptr(wu_t), _ptr(wd_t), _ptr(h), _ptr(y),
+          n, d, f, _ptr(diag), _stream(x.device, stream))
+    return y

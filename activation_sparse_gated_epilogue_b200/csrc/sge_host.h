@@ -1,0 +1,36 @@
+// Host-side helpers shared by the library's .cu files: error reporting,
+// argument checks, device properties and TMA descriptor encoding.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/sge.h"
+
+namespace sge {
+
+// Records a message for sge_last_error() and returns `code`.
+int fail(int code, const char* fmt, ...);
+void clear_error();
+
+// SGE_OK, or SGE_ERR_CUDA with the message of the pending launch error.
+int check_launch(const char* what);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Multiprocessor count of the current device (cached per device).
+int sm_count();
+
+// Sets the dynamic shared memory limit of a kernel once per process.
+int set_smem_limit(const void* kernel, int bytes);
+
+// 2-D bf16 tensor map over a row-major [rows][cols] matrix with row pitch
+// `pitch_elems`, box [box_rows][64] (64 bf16 = one 128-byte swizzle row),
+// 128-byte swizzle, out-of-bounds elements read as zero.
+int make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                   uint64_t pitch_elems, uint32_t box_rows);
+
+}  // namespace sge

@@ -1,0 +1,222 @@
+// Persistent tcgen05 GEMM engine for sm_100a:  D[M][N] = A[M][K] . B[N][K]^T
+// (both operands K-major bf16, fp32 accumulation in tensor memory), with a
+// pluggable epilogue that reads the accumulator tile straight out of TMEM.
+//
+// One CTA per SM (192 threads, 6 warps), looping over output tiles:
+//   warp 0      TMA producer: A and B tiles (128-byte swizzle) into a ring of
+//               STAGES shared-memory stages, completion on `full` mbarriers.
+//   warp 1      TMEM allocator and MMA issuer: one elected thread issues
+//               tcgen05.mma (M = 128, N = BN, K = 16 per instruction) and
+//               releases each stage with tcgen05.commit -> `empty`.
+//   warps 2..5  epilogue: tcgen05.ld of the tile (thread i of warp w holds
+//               accumulator row 32*(w%4) + i), then the Epilogue functor.
+// The accumulator is double-buffered in TMEM so the epilogue of one tile
+// overlaps the main loop of the next.  With NB = 2 the engine multiplies A
+// by two B matrices at once into two accumulators (gate and up projections
+// of the dense gated FFN share the A tile).
+//
+// No cluster launch and no TMA multicast: every CTA loads its own tiles.
+// Every wait is bounded (sge::mbar_wait); a timeout sets SGE_FLAG_TIMEOUT in
+// diag, raises a CTA-wide abort flag, and the CTA drains its in-flight TMA
+// loads and MMAs (bounded) before freeing TMEM and returning.
+#pragma once
+
+#include "sge_common.cuh"
+
+namespace sge {
+
+constexpr int kBM = 128;  // UMMA M: rows of A per tile = TMEM lanes
+constexpr int kBK = 64;   // K per stage: one 128-byte swizzle row of bf16
+constexpr int kGemmThreads = 192;
+
+template <int BN_, int NB_>
+struct TcShape {
+  static constexpr int BN = BN_;
+  static constexpr int NB = NB_;
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + NB * B_BYTES;
+  static constexpr int STAGES = (196 * 1024) / STAGE_BYTES > 8 ? 8 : (196 * 1024) / STAGE_BYTES;
+  static constexpr int ACC_COLS = BN * NB;
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+  static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM columns");
+  static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1024-byte aligned sub-tiles");
+};
+
+struct TileCoord {
+  int m_blk, n_blk;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(int tile, int m_blocks) {
+  return TileCoord{tile % m_blocks, tile / m_blocks};
+}
+
+// Bounded wait that also gives up when another role of the CTA aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag, int32_t* diag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if ((i & 63) == 0 && globaltimer_ns() - t0 > kWaitNs) break;
+  }
+  if (diag) atomicOr(reinterpret_cast<int*>(diag + SGE_DIAG_FLAGS), SGE_FLAG_TIMEOUT);
+  *abort_flag = 1;
+  return false;
+}
+
+template <class Shape, class Epilogue>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
+                   const __grid_constant__ CUtensorMap map_b0,
+                   const __grid_constant__ CUtensorMap map_b1, int M, int N, int K,
+                   Epilogue epi, int32_t* diag) {
+  constexpr int BN = Shape::BN, NB = Shape::NB, STAGES = Shape::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Shape::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tmem_full = empty + STAGES;
+  uint64_t* tmem_empty = tmem_full + 2;
+  uint64_t* drain = tmem_empty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int m_blocks = (M + kBM - 1) / kBM;
+  const int n_blocks = (N + BN - 1) / BN;
+  const int num_tiles = m_blocks * n_blocks;
+  const int k_blocks = (K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tmem_full[a], 1);
+      mbar_init(&tmem_empty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&map_a);
+    tma_prefetch_desc(&map_b0);
+    if (NB == 2) tma_prefetch_desc(&map_b1);
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, Shape::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t armed = 0;  // bit s: stage s has a load whose completion is unobserved
+      uint32_t armed_par = 0;
+      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
+        const TileCoord tc = tile_coord(tile, m_blocks);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, diag)) break;
+          uint8_t* sa = smem + s * Shape::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], Shape::STAGE_BYTES);
+          tma_load_2d(sa, &map_a, &full[s], kb * kBK, tc.m_blk * kBM);
+          tma_load_2d(sa + Shape::A_BYTES, &map_b0, &full[s], kb * kBK, tc.n_blk * BN);
+          if (NB == 2)
+            tma_load_2d(sa + Shape::A_BYTES + Shape::B_BYTES, &map_b1, &full[s], kb * kBK,
+                        tc.n_blk * BN);
+          armed |= 1u << s;
+          armed_par = (armed_par & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      // Drain: every stage's most recent load has landed before we leave
+      // (immediate in the normal path, where the MMA already consumed it).
+      for (int t = 0; t < STAGES; ++t)
+        if (armed & (1u << t)) mbar_wait(&full[t], (armed_par >> t) & 1, diag);
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(kBM, BN);
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      bool issued = false;
+      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        if (!wait_or_abort(&tmem_empty[acc], ((it >> 1) & 1) ^ 1, abort_flag, diag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * Shape::ACC_COLS;
+        bool ok = true;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!wait_or_abort(&full[s], ph, abort_flag, diag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * Shape::STAGE_BYTES);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t adesc = umma_desc_sw128(sa + k * 32);
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+              const uint64_t bdesc = umma_desc_sw128(sa + Shape::A_BYTES + b * Shape::B_BYTES + k * 32);
+              umma_bf16(d_tmem + b * BN, adesc, bdesc, idesc, (kb | k) != 0);
+            }
+          }
+          issued = true;
+          umma_commit(&empty[s]);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tmem_full[acc]);
+      }
+      // Drain: all issued MMAs complete before TMEM is released.
+      if (issued) {
+        umma_commit(drain);
+        mbar_wait(drain, 0, diag);
+      }
+    }
+  } else {
+    // --------------------------------------------------------- epilogue
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const bool ok = wait_or_abort(&tmem_full[acc], (it >> 1) & 1, abort_flag, diag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const TileCoord tc = tile_coord(tile, m_blocks);
+      const uint32_t taddr = tmem_base + acc * Shape::ACC_COLS + (static_cast<uint32_t>(quarter * 32) << 16);
+      const int64_t row = static_cast<int64_t>(tc.m_blk) * kBM + quarter * 32 + lane;
+      epi.template run<BN>(taddr, row, tc.n_blk, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tmem_empty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Shape::TMEM_COLS);
+  }
+}
+
+}  // namespace sge

@@ -1,0 +1,388 @@
+"""Benchmark of the activation-sparse gated FFN forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of the whole sparse inference path over one batch:
+gate GEMM with the TwELL epilogue (twell_gate_pack) followed by the fused
+up/down kernel (twell_fused_up_down), on the 1B-shaped bf16 workload
+(N=8192 tokens, d=2048, F=8192, T=C=128, mean gate density 1%, per-token
+scale LogNormal(0, 0.7)) unless --workload names another.  Inputs are seeded
+synthetic data resident in HBM; L2 is flushed (a 256 MB write) between timed
+steps and the flush is outside the per-step CUDA events.
+
+Prints one JSON line (rank 0).  `value` is tokens/s over all ranks (weak
+scaling: every rank runs its own batch, no collective on the data path).
+Also reported: the library's dense bf16 FFN and a cuBLAS (torch.matmul)
+dense FFN on the same inputs, the roofline of each kernel, an end-to-end
+number through host buffers, and the fp64 CPU oracle on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse gated-FFN tokens/s at 1B shape bf16 (%HBM roofline; vs dense FFN)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "source": "fallback"}
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flop x 1.965 GHz
+FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+# DRAM bytes per launch from the committed ncu captures (profiles/), keyed by
+# the source hash of the kernel they were taken on; null once it changes.
+TRAFFIC = {}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=300)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--workload", default="ffn_1b_bf16")
+    p.add_argument("--impl", default="own", choices=["own", "reference"])
+    p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def src_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "activation_sparse_gated_epilogue_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sge_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            self.proc.wait(timeout=10)
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        loaded = [s for s, p in zip(sm, pw)] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "samples": len(rows), "reasons": reasons}
+
+
+# ------------------------------------------------------------- own arm
+
+def run_own(args, rank, world, local_rank):
+    import activation_sparse_gated_epilogue_b200 as sge
+    from activation_sparse_gated_epilogue_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = synth.CONFIGS[args.workload]
+    inp = synth.make_inputs(cfg)
+    n, d, f, tile, cap = cfg.n_tokens, cfg.d_model, cfg.d_ff, cfg.tile, cfg.cap
+    x, wg, wu, wd = (getattr(inp, k).to(dev) for k in ("x", "wg_t", "wu_t", "wd"))
+    wd_t = wd.t().contiguous()
+    tw = sge.TwELL.empty(n, f, tile, cap, x.dtype, dev)
+    y = torch.empty_like(x)
+    h = torch.empty((n, f), dtype=x.dtype, device=dev)
+    y_dense = torch.empty_like(x)
+    diag = sge.new_diag(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+
+    def timed(fns, steps, warm):
+        """Per-step CUDA events around each fn (same stream), L2 flush between."""
+        evs = []
+        for s in range(warm + steps):
+            flush.zero_()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+            e[0].record(stream)
+            for i, fn in enumerate(fns):
+                fn()
+                e[i + 1].record(stream)
+            if s >= warm:
+                evs.append(e)
+        return evs
+
+    def reduce_max(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    gate = lambda: sge.twell_gate_pack(x, wg, tile, cap, out=tw, diag=diag)
+    fused = lambda: sge.twell_fused_up_down(x, tw, wu, wd, y=y)
+    dense = lambda: sge.dense_ffn_fwd(x, wg, wu, wd_t, h=h, y=y_dense)
+
+    # ---- the sparse forward: timed region
+    timed([gate, fused], 0, args.warmup)
+    barrier()
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        evs = timed([gate, fused], args.steps, 0)
+        barrier()
+    clocks = clk.summary()
+    t_gate = [e[0].elapsed_time(e[1]) for e in evs]
+    t_fused = [e[1].elapsed_time(e[2]) for e in evs]
+    total_ms = reduce_max(sum(a + b for a, b in zip(t_gate, t_fused)))
+    ms_step = total_ms / args.steps
+    value = n * world * args.steps / (total_ms / 1e3)
+
+    nnz = int(tw.count.to(torch.int64).sum().item())
+    density = nnz / (n * f)
+
+    # ---- dense baselines on the same inputs (own tcgen05 and cuBLAS)
+    evd = timed([dense], min(args.steps, 100), 3)
+    ms_dense = statistics.mean(e[0].elapsed_time(e[1]) for e in evd)
+
+    def cublas():
+        hh = torch.relu(x @ wg.t()) * (x @ wu.t())
+        return hh @ wd
+    evc = timed([cublas], min(args.steps, 50), 3)
+    ms_cublas = statistics.mean(e[0].elapsed_time(e[1]) for e in evc)
+
+    # ---- end to end through host buffers (copies inside the timed region)
+    x_host = inp.x.pin_memory()
+    y_host = torch.empty(x_host.shape, dtype=x_host.dtype).pin_memory()
+    x_dev2 = torch.empty_like(x)
+
+    def e2e():
+        x_dev2.copy_(x_host, non_blocking=True)
+        sge.twell_gate_pack(x_dev2, wg, tile, cap, out=tw, diag=diag)
+        sge.twell_fused_up_down(x_dev2, tw, wu, wd, y=y)
+        y_host.copy_(y, non_blocking=True)
+    e2e_steps = min(args.steps, 50)
+    barrier()
+    eve = timed([e2e], e2e_steps, 3)
+    barrier()
+    e2e_ms = reduce_max(sum(e[0].elapsed_time(e[1]) for e in eve))
+    e2e_value = n * world * e2e_steps / (e2e_ms / 1e3)
+    diag_host = diag.tolist()
+
+    if rank != 0:
+        return None
+
+    pk = peaks()
+    mg = statistics.mean(t_gate)
+    mf = statistics.mean(t_fused)
+    flops_gate = 2.0 * n * d * f
+    bf16_peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    gate_tf = flops_gate / (mg / 1e3) / 1e12
+    flops_fused = 4.0 * nnz * d
+    fused_tf = flops_fused / (mf / 1e3) / 1e12
+    # unique HBM bytes of the fused kernel: x, the weight rows it touches
+    # (at most all of W_up and W_down), TwELL entries and counts, y
+    bytes_fused = (2 * n * d + 2 * 2 * f * d + 3 * nnz + n * (f // tile) + 2 * n * d)
+    gate_src = src_hash("gate_pack.cu", "tc_gemm.cuh", "sge_common.cuh")
+    fused_src = src_hash("fused_up_down.cu", "sge_common.cuh")
+    tr_gate = TRAFFIC.get(gate_src)
+    tr_fused = TRAFFIC.get(fused_src)
+    k_gate = {"kernel": "twell_gate_pack (tcgen05 GEMM + TwELL epilogue)", "bound": "tensor",
+              "achieved": round(gate_tf, 1), "peak": bf16_peak, "unit": "TFLOP/s",
+              "frac": round(gate_tf / bf16_peak, 4), "traffic": tr_gate,
+              "ms": round(mg, 4), "share": round(mg / (mg + mf), 3),
+              "algorithmic": f"2*N*d*F = {flops_gate:.3e} flop per launch",
+              "peak_note": "bf16_tflops_sustained of measured peaks (seconds-long loop)"}
+    k_fused = {"kernel": "twell_fused_up_down", "bound": "alu", "achieved": round(fused_tf, 2),
+               "peak": round(FP32_SIMT_TFLOPS, 1), "unit": "TFLOP/s",
+               "frac": round(fused_tf / FP32_SIMT_TFLOPS, 4), "traffic": tr_fused,
+               "ms": round(mf, 4), "share": round(mf / (mg + mf), 3),
+               "algorithmic": f"4*nnz*d = {flops_fused:.3e} flop per launch (nnz={nnz})",
+               "hbm_gbs_unique": round(bytes_fused / (mf / 1e3) / 1e9, 1),
+               "peak_note": "fp32 FMA peak of the CUDA cores, 148 SMs x 128 lanes x 2 x 1.965 GHz"}
+    dominant = k_gate if mg >= mf else k_fused
+    rest = k_fused if dominant is k_gate else k_gate
+    roofline_time_ms = flops_gate / (bf16_peak * 1e12) * 1e3 + flops_fused / (FP32_SIMT_TFLOPS * 1e12) * 1e3
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; tokens x d_model x d_ff shaped like a 1B FFN)",
+        "config": {"workload": f"{cfg.name}: N={n} d={d} F={f} T={tile} C={cap} "
+                               f"target density {cfg.rho} sigma={cfg.sigma}",
+                   "realised_density": round(density, 5), "nnz": nnz,
+                   "l2": "flushed between steps (256 MB write outside the step events)",
+                   "parallelism": f"replicas x{world} (token batches independent)"},
+        "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")},
+        "kernels": [dominant, rest],
+        "step_roofline_ms": round(roofline_time_ms, 4),
+        "step_roofline_frac": round(roofline_time_ms / ms_step, 4),
+        "dense": {"own_tcgen05_ms": round(ms_dense, 4), "cublas_ms": round(ms_cublas, 4),
+                  "speedup_vs_own_dense": round(ms_dense / ms_step, 3),
+                  "speedup_vs_cublas_dense": round(ms_cublas / ms_step, 3)},
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+                "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+        "diag": diag_host,
+        "gpu": torch.cuda.get_device_name(dev),
+        "peaks_source": pk["source"],
+    }
+    return out
+
+
+# ------------------------------------------------------ CPU oracle timing
+
+def oracle_sample(cfg, budget_s: float, max_tokens: int):
+    """Time the fp64 oracle's sparse forward on the first tokens of the
+    workload; the sample grows until it costs about `budget_s`."""
+    import oracle
+    from activation_sparse_gated_epilogue_b200 import synth
+    inp = synth.make_inputs(cfg)
+    xf, wgf, wuf, wdf = (inp.as_f64(k) for k in ("x", "wg_t", "wu_t", "wd"))
+    oracle.build()
+
+    def run(k):
+        t0 = time.perf_counter()
+        oracle.sparse_ffn(xf[:k], wgf, wuf, wdf, cfg.tile, cfg.cap, oracle.VAL_BF16)
+        return time.perf_counter() - t0
+
+    k = min(8, max_tokens)
+    t = run(k)
+    while t < budget_s / 4 and k < max_tokens:
+        k = min(max_tokens, int(k * max(2.0, min(8.0, budget_s / max(t, 1e-3) / 2))))
+        t = run(k)
+    return k, t
+
+
+def cpu_baseline(cfg, budget_s=12.0):
+    k, t = oracle_sample(cfg, budget_s, cfg.n_tokens)
+    return {"value": round(k / t, 2), "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+            "sample": f"first {k} of {cfg.n_tokens} tokens of {cfg.name}: fp64 gate GEMM, "
+                      f"TwELL pack, fused up/down ({t:.1f} s, OpenMP over tokens)"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step is a bounded token sample."""
+    import oracle
+    from activation_sparse_gated_epilogue_b200 import synth
+    cfg = synth.CONFIGS[args.workload]
+    inp = synth.make_inputs(cfg)
+    xf, wgf, wuf, wdf = (inp.as_f64(k) for k in ("x", "wg_t", "wu_t", "wd"))
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.sparse_ffn(xf[:4], wgf, wuf, wdf, cfg.tile, cfg.cap, oracle.VAL_BF16)
+    per_tok = (time.perf_counter() - t0) / 4
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    k = int(max(1, min(cfg.n_tokens, budget / max(per_tok, 1e-6))))
+    times = []
+    for s in range(args.warmup + args.steps):
+        off = (s * k) % max(1, cfg.n_tokens - k)
+        t0 = time.perf_counter()
+        oracle.sparse_ffn(xf[off:off + k], wgf, wuf, wdf, cfg.tile, cfg.cap, oracle.VAL_BF16)
+        if s >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = k * args.steps / total
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{cfg.name}: N={cfg.n_tokens} d={cfg.d_model} F={cfg.d_ff} "
+                                   f"T={cfg.tile} C={cfg.cap}",
+                       "sample_tokens_per_step": k},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": host_cores(),
+                             "kind": "oracle",
+                             "sample": f"{k} consecutive tokens of {cfg.name} per step"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    out = run_own(args, rank, world, local_rank)
+    if rank == 0:
+        from activation_sparse_gated_epilogue_b200 import synth
+        out["cpu_baseline"] = None if args.no_cpu else cpu_baseline(synth.CONFIGS[args.workload])
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,150 @@
+/*
+ * sge.h -- C ABI of the activation-sparse gated-epilogue FFN library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method: "Sparser, Faster, Lighter Transformer Language Models" (Cetin,
+ * Peluchetti, Castillo, Naruse, Murakami, Jones; ICML 2026).  The feed-forward
+ * block is the gated FFN
+ *
+ *     y = (ReLU(x W_gate) (.) (x W_up)) W_down
+ *
+ * (pwwt.cn summary, section 01 and figure "Gated FFN up, gate and down
+ * projection"; the printed formula is lost, this is its plain reading with
+ * no bias terms).  ReLU makes most hidden activations exact zeros; the gate
+ * activations are packed into TwELL (tile-wise ELLPACK) directly in the gate
+ * GEMM's epilogue (section 02, figures "TwELL cuts the column direction into
+ * tiles" and "gate projection with TwELL storage generation"), and one fused
+ * kernel does the up and down projections over the nonzeros only, without
+ * writing the hidden activation h to memory (section 02, last paragraph).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers, row-major and contiguous, owned
+ *    by the caller; the library never allocates or frees device memory and
+ *    keeps no pointer after the call returns.
+ *  - Every pointer must be 16-byte aligned; d_model must be a multiple of 8.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *    are asynchronous on that stream; outputs are overwritten (beta = 0).
+ *  - The return value is SGE_OK or an error code, decided on the host before
+ *    anything is launched (bad argument, unsupported shape, launch failure);
+ *    sge_last_error() then holds a message (thread-local).
+ *  - Data-dependent conditions found on the device are reported in the
+ *    caller's optional `diag` word (int32[4], device memory), which kernels
+ *    ADD to (atomically), so the caller zeroes it when it wants fresh counts:
+ *      diag[SGE_DIAG_OVERFLOW_TILES]  TwELL tiles whose count exceeded C
+ *      diag[SGE_DIAG_SPILL_ROWS]      hybrid rows with nnz > K
+ *      diag[SGE_DIAG_DROPPED_ROWS]    spill rows beyond S_max (not computed)
+ *      diag[SGE_DIAG_FLAGS]           OR of SGE_FLAG_* bits
+ *    SGE_FLAG_TIMEOUT means a bounded pipeline wait gave up (a bug or a
+ *    stuck device); the outputs of that call are then undefined.
+ *
+ * Weights are stored neuron-major (row j is the j-th hidden unit):
+ *    wg_t[F][d] = W_gate^T,  wu_t[F][d] = W_up^T,  wd[F][d] = W_down.
+ *
+ * TwELL layout (per row t, per column tile b of width T, capacity C slots):
+ *    count[N][F/T]     uint8   true number of active columns (may exceed C)
+ *    idx  [N][F/T][C]  uint8   local column (0..T-1) of the stored entries,
+ *                              ascending
+ *    val  [N][F/T][C]  dtype   ReLU(g) of the stored entries, rounded to
+ *                              nearest even
+ * A column is active iff its fp32 gate pre-activation g > 0.  Only the first
+ * min(count, C) slots of a tile are written and read.
+ */
+#ifndef SGE_H
+#define SGE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* return codes */
+#define SGE_OK 0
+#define SGE_ERR_ARG 1         /* null / misaligned pointer, bad size */
+#define SGE_ERR_UNSUPPORTED 2 /* valid but not implemented shape or dtype */
+#define SGE_ERR_CUDA 3        /* CUDA runtime / driver error at launch */
+
+/* element types */
+#define SGE_F32 0
+#define SGE_BF16 1
+
+/* diag word slots and flags */
+#define SGE_DIAG_OVERFLOW_TILES 0
+#define SGE_DIAG_SPILL_ROWS 1
+#define SGE_DIAG_DROPPED_ROWS 2
+#define SGE_DIAG_FLAGS 3
+#define SGE_FLAG_TIMEOUT 1
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int sge_version(void);
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char* sge_last_error(void);
+
+/*
+ * twell_gate_pack -- gate projection with TwELL produced in the epilogue.
+ * (pwwt.cn summary, section 02: TwELL generated directly in the epilogue of
+ * the gate projection, no separate conversion kernel, no dense gate
+ * activation in global memory.)
+ *
+ *   G = x W_gate  (fp32 accumulation), then per row t and tile b:
+ *   count[t][b] = #{j in tile b : G[t][j] > 0}; the first min(count, C) active
+ *   columns (ascending) are stored as idx = j - bT, val = ReLU(G[t][j]).
+ *
+ *   x      [N][d]   dtype     input activations
+ *   wg_t   [F][d]   dtype     W_gate transposed (neuron-major)
+ *   dtype  SGE_BF16: tcgen05 tensor-core GEMM (bf16 x bf16 -> fp32);
+ *          SGE_F32:  CUDA-core fp32 FMA GEMM (exact fp32 products).
+ *   tile   T: 16, 32, 64 or 128, dividing F
+ *   cap    C: 1 <= C <= T
+ *   count, idx, val: TwELL output as laid out above (val in `dtype`)
+ *   diag   nullable int32[4]; adds the number of tiles with count > C
+ * Errors: SGE_ERR_ARG for null/misaligned pointers, N, d or F < 1, d % 8 != 0,
+ * F % T != 0, C outside [1, T]; SGE_ERR_UNSUPPORTED for other T or dtype.
+ */
+int twell_gate_pack(const void* x, const void* wg_t, int64_t n_tokens, int64_t d_model,
+                    int64_t d_ff, int dtype, int tile, int cap, uint8_t* count, uint8_t* idx,
+                    void* val, int32_t* diag, void* stream);
+
+/*
+ * twell_fused_up_down -- up and down projections over the TwELL nonzeros in
+ * one pass.  (pwwt.cn summary, section 02, last paragraph: one custom kernel
+ * does the up and down projections in a single traversal, fusing the two
+ * products so that the intermediate h never goes to global memory.)
+ *
+ *   y[t] = sum over stored entries (j, a) of row t of
+ *          a * (x[t] . wu_t[j]) * wd[j]
+ *   with fp32 accumulation; y is written in `dtype`.
+ *
+ *   x [N][d], wu_t [F][d], wd [F][d], y [N][d] in dtype; count/idx/val the
+ *   TwELL produced by twell_gate_pack with the same T and C.
+ * Errors: as twell_gate_pack; SGE_ERR_UNSUPPORTED for d > 4096.
+ */
+int twell_fused_up_down(const void* x, const uint8_t* count, const uint8_t* idx, const void* val,
+                        const void* wu_t, const void* wd, void* y, int64_t n_tokens,
+                        int64_t d_model, int64_t d_ff, int dtype, int tile, int cap, void* stream);
+
+/*
+ * dense_ffn_fwd -- the dense gated FFN the method is compared against
+ * (pwwt.cn summary, lead and section 04: speed-ups are quoted against the
+ * dense model).  bf16 only, on tcgen05 tensor cores:
+ *   h = bf16(ReLU(x W_gate) (.) (x W_up))   (one GEMM, two accumulators)
+ *   y = bf16(h W_down)
+ *
+ *   x [N][d], wg_t [F][d], wu_t [F][d]   bf16
+ *   wd_t [d][F]  bf16  W_down TRANSPOSED (row i = column i of W_down), the
+ *                      K-major layout of the second GEMM's B operand
+ *   h  [N][F]  bf16  caller-provided workspace for the hidden activation
+ *   y  [N][d]  bf16
+ * Errors: SGE_ERR_ARG as above and for F % 8 != 0.
+ */
+int dense_ffn_fwd(const void* x, const void* wg_t, const void* wu_t, const void* wd_t, void* h,
+                  void* y, int64_t n_tokens, int64_t d_model, int64_t d_ff, int32_t* diag,
+                  void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SGE_H */

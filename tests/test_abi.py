@@ -1,0 +1,93 @@
+"""The C-ABI library loads without a GPU, exports every symbol include/sge.h
+declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import activation_sparse_gated_epilogue_b200 as sge
+from activation_sparse_gated_epilogue_b200 import build as sge_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sge.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("defined",)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sge_build.build()
+    return sge.library()
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for want in ("twell_gate_pack", "twell_fused_up_down", "dense_ffn_fwd", "sge_last_error"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", sge.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+
+
+def test_version_and_error_string(lib):
+    assert lib.sge_version() >= 100
+    assert isinstance(lib.sge_last_error(), bytes)
+
+
+def _gate(lib, **kw):
+    a = dict(x=None, w=None, n=8, d=64, f=256, dt=sge.SGE_BF16, tile=128, cap=128,
+             count=None, idx=None, val=None, diag=None, stream=None)
+    a.update(kw)
+    return lib.twell_gate_pack(a["x"], a["w"], a["n"], a["d"], a["f"], a["dt"], a["tile"], a["cap"],
+                               a["count"], a["idx"], a["val"], a["diag"], a["stream"])
+
+
+def test_bad_arguments_are_rejected_on_host(lib):
+    assert _gate(lib, d=60) == 1                  # d % 8
+    assert _gate(lib, tile=48) == 2               # unsupported tile
+    assert _gate(lib, f=200, tile=64) == 1        # T does not divide F
+    assert _gate(lib, cap=0) == 1
+    assert _gate(lib, cap=129) == 1
+    assert _gate(lib, n=-1) == 1
+    assert _gate(lib) == 1                        # null pointers
+    assert b"null" in lib.sge_last_error()
+    assert _gate(lib, dt=7, x=ctypes.c_void_p(16), w=ctypes.c_void_p(16), count=ctypes.c_void_p(16),
+                 idx=ctypes.c_void_p(16), val=ctypes.c_void_p(16)) == 2
+    assert _gate(lib, x=ctypes.c_void_p(17), w=ctypes.c_void_p(16), count=ctypes.c_void_p(16),
+                 idx=ctypes.c_void_p(16), val=ctypes.c_void_p(16)) == 1   # misaligned
+    assert b"aligned" in lib.sge_last_error()
+
+
+def test_empty_input_is_a_no_op(lib):
+    assert _gate(lib, n=0) == 0
+    assert lib.twell_fused_up_down(None, None, None, None, None, None, None, 0, 64, 256,
+                                   sge.SGE_BF16, 128, 128, None) == 0
+    assert lib.dense_ffn_fwd(None, None, None, None, None, None, 0, 64, 256, None, None) == 0
+
+
+def test_fused_rejects_bad_arguments(lib):
+    assert lib.twell_fused_up_down(None, None, None, None, None, None, None, 8, 12, 256,
+                                   sge.SGE_BF16, 128, 128, None) == 1
+    assert lib.twell_fused_up_down(None, None, None, None, None, None, None, 8, 64, 256,
+                                   sge.SGE_BF16, 128, 128, None) == 1
+    assert lib.dense_ffn_fwd(None, None, None, None, None, None, 8, 64, 100, None, None) == 1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        sge.twell_gate_pack(x, torch.zeros(128, 64, dtype=torch.bfloat16), 128, 128)

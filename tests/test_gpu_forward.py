@@ -1,0 +1,228 @@
+"""GPU parity of the inference path (gate GEMM + TwELL epilogue, fused
+up/down, dense baseline) against the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import activation_sparse_gated_epilogue_b200 as sge
+import oracle
+from activation_sparse_gated_epilogue_b200 import synth
+from tests._util import (BF16_TOL, F32_TOL, FLIP_EPS, assert_twell_equal,
+                         compare_twell_inexact, to_f64)
+
+pytestmark = pytest.mark.gpu
+
+KIND = {torch.bfloat16: oracle.VAL_BF16, torch.float32: oracle.VAL_F32}
+
+
+def _dev(inp, dev):
+    return [getattr(inp, k).to(dev) for k in ("x", "wg_t", "wu_t", "wd")]
+
+
+def _f64(inp):
+    return [inp.as_f64(k) for k in ("x", "wg_t", "wu_t", "wd")]
+
+
+def _upload_twell(tw: oracle.TwELL, dtype, dev):
+    return sge.TwELL(torch.from_numpy(tw.count).to(dev), torch.from_numpy(tw.idx).to(dev),
+                     torch.from_numpy(tw.val).to(dtype).to(dev), tw.tile, tw.cap)
+
+
+# ------------------------------------------------- gate GEMM + TwELL epilogue
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("n,d,f,tile,cap", [
+    (300, 200, 640, 128, 128),    # ragged M, K tail, ragged N block
+    (257, 136, 512, 64, 64),
+    (128, 64, 256, 32, 5),        # overflow
+    (520, 264, 768, 16, 16),
+    (64, 512, 1024, 128, 12),
+])
+def test_gate_pack_exact_on_grid_inputs(cuda_device, dtype, n, d, f, tile, cap):
+    """Grid inputs make G exact in fp32, so counts, indices and values are
+    bit-exact against the oracle, including overflow truncation."""
+    inp = synth.make_grid_inputs(n, d, f, dtype, rho=0.05, seed=n + d)
+    x, wg, _, _ = _dev(inp, cuda_device)
+    diag = sge.new_diag(cuda_device)
+    tw = sge.twell_gate_pack(x, wg, tile, cap, diag=diag)
+    ora = oracle.twell_pack(oracle.gate_preact(inp.as_f64("x"), inp.as_f64("wg_t")), tile, cap,
+                            KIND[dtype])
+    torch.cuda.synchronize()
+    assert_twell_equal(tw, ora)
+    assert int(diag[0]) == ora.overflow
+
+
+def test_gate_pack_identity_weights(cuda_device):
+    """x := G (bf16), W_gate := I: the GEMM reproduces G exactly, so the
+    epilogue's TwELL equals the oracle's pack of G bit for bit."""
+    rng = np.random.default_rng(3)
+    n, f = 384, 512
+    g = torch.from_numpy(rng.standard_normal((n, f)) - 1.0).to(torch.bfloat16)
+    eye = torch.eye(f, dtype=torch.bfloat16)
+    tw = sge.twell_gate_pack(g.to(cuda_device), eye.to(cuda_device), 128, 128)
+    ora = oracle.twell_pack(g.double().numpy(), 128, 128, oracle.VAL_BF16)
+    torch.cuda.synchronize()
+    assert_twell_equal(tw, ora)
+
+
+@pytest.mark.parametrize("name,cap", [("ffn_0p5b_bf16", 128), ("tiny_fp32", 64), ("tiny_fp32", 16)])
+def test_gate_pack_gaussian_sign_flips(cuda_device, name, cap):
+    """Realistic inputs: tiles disagree only where near-zero gates explain it
+    (|g| < 1e-3); values agree within one bf16 ulp / the fp32 tolerance."""
+    cfg = synth.CONFIGS[name]
+    inp = synth.make_inputs(cfg, n_tokens=512)
+    x, wg, _, _ = _dev(inp, cuda_device)
+    tw = sge.twell_gate_pack(x, wg, cfg.tile, cap)
+    g = oracle.gate_preact(inp.as_f64("x"), inp.as_f64("wg_t"))
+    kind = KIND[cfg.torch_dtype]
+    ora = oracle.twell_pack(g, cfg.tile, cap, kind)
+    torch.cuda.synchronize()
+    bad_rows, bad_tiles = compare_twell_inexact(tw, ora, g, kind)
+    assert bad_tiles <= max(2, 0.002 * ora.count.size)
+    print(f"{name} C={cap}: {bad_tiles} tiles differ by near-zero sign flips")
+
+
+# ------------------------------------------------------------ fused up/down
+
+@pytest.mark.parametrize("dtype,tol", [(torch.bfloat16, BF16_TOL), (torch.float32, F32_TOL)])
+@pytest.mark.parametrize("n,d,f,tile,cap", [
+    (300, 264, 640, 64, 64),      # d tail inside the last 16-byte chunk group
+    (129, 1024, 512, 128, 128),
+    (77, 520, 768, 32, 6),        # truncated tiles
+    (64, 2560, 1024, 128, 128),   # the 2B d_model
+])
+def test_fused_up_down_matches_oracle(cuda_device, dtype, tol, n, d, f, tile, cap):
+    """Both sides get the same TwELL (the oracle's pack of its fp64 G)."""
+    inp = synth.make_inputs(synth.CONFIGS["ffn_0p5b_bf16"].with_(
+        n_tokens=n, d_model=d, d_ff=f, dtype="bf16" if dtype == torch.bfloat16 else "f32",
+        rho=0.05))
+    xf, wgf, wuf, wdf = _f64(inp)
+    ora_tw = oracle.twell_pack(oracle.gate_preact(xf, wgf), tile, cap, KIND[dtype])
+    x, _, wu, wd = _dev(inp, cuda_device)
+    y = sge.twell_fused_up_down(x, _upload_twell(ora_tw, dtype, cuda_device), wu, wd)
+    want = oracle.fused_up_down(xf, ora_tw, wuf, wdf)
+    err = oracle.max_abs_rel(to_f64(y), want)
+    assert err <= tol, err
+
+
+def test_fused_up_down_zero_density(cuda_device):
+    n, d, f = 64, 256, 512
+    inp = synth.make_inputs(synth.CONFIGS["ffn_0p5b_bf16"].with_(n_tokens=n, d_model=d, d_ff=f),
+                            tau=1e4)
+    x, wg, wu, wd = _dev(inp, cuda_device)
+    y, tw = sge.twell_ffn_forward(x, wg, wu, wd, 128, 128)
+    torch.cuda.synchronize()
+    assert int(tw.count.sum()) == 0
+    assert torch.all(y == 0)
+
+
+def test_full_density_equals_dense(cuda_device):
+    """tau -> -inf: every gate is active, TwELL with C = T is dense and the
+    sparse forward equals the dense FFN (oracle)."""
+    n, d, f = 96, 256, 512
+    inp = synth.make_inputs(synth.CONFIGS["ffn_0p5b_bf16"].with_(n_tokens=n, d_model=d, d_ff=f),
+                            tau=-1e3)
+    x, wg, wu, wd = _dev(inp, cuda_device)
+    y, tw = sge.twell_ffn_forward(x, wg, wu, wd, 128, 128)
+    want = oracle.dense_ffn(*_f64(inp))
+    torch.cuda.synchronize()
+    assert int(tw.count.sum()) == n * f
+    assert oracle.max_abs_rel(to_f64(y), want) <= BF16_TOL
+
+
+# --------------------------------------------------------------- end to end
+
+def _e2e_check(inp, dev, tile, cap, tol, rows=None):
+    x, wg, wu, wd = _dev(inp, dev)
+    diag = sge.new_diag(dev)
+    y, tw = sge.twell_ffn_forward(x, wg, wu, wd, tile, cap, diag=diag)
+    torch.cuda.synchronize()
+    xf, wgf, wuf, wdf = _f64(inp)
+    if rows is not None:
+        xf = xf[rows]
+    kind = KIND[inp.x.dtype]
+    y_ora, tw_ora, g = oracle.sparse_ffn(xf, wgf, wuf, wdf, tile, cap, kind)
+    bad_rows, bad_tiles = compare_twell_inexact(tw, tw_ora, g, kind, rows=rows)
+    # rows whose stored entries differ (near-zero sign flips) are left out of
+    # the y bar and counted
+    assert bad_rows.sum() <= max(2, 0.02 * len(bad_rows))
+    yg = to_f64(y) if rows is None else to_f64(y)[rows]
+    ok = ~bad_rows
+    err = oracle.max_abs_rel(yg[ok], y_ora[ok])
+    assert err <= tol, err
+    return err, bad_tiles, int(diag[0])
+
+
+def test_e2e_tiny_fp32(cuda_device):
+    cfg = synth.CONFIGS["tiny_fp32"]
+    inp = synth.make_inputs(cfg)
+    err, flips, over = _e2e_check(inp, cuda_device, cfg.tile, cfg.cap, F32_TOL)
+    ora_over = oracle.twell_pack(oracle.gate_preact(inp.as_f64("x"), inp.as_f64("wg_t")),
+                                 cfg.tile, cfg.cap, oracle.VAL_F32).overflow
+    assert abs(over - ora_over) <= flips       # overflow count agrees up to flipped tiles
+    print(f"tiny fp32: max-abs-rel {err:.2e}, {flips} flips, {over} overflowing tiles")
+
+
+def test_e2e_0p5b_bf16(cuda_device):
+    cfg = synth.CONFIGS["ffn_0p5b_bf16"]
+    err, flips, _ = _e2e_check(synth.make_inputs(cfg), cuda_device, cfg.tile, cfg.cap, BF16_TOL,
+                               rows=np.arange(0, cfg.n_tokens, 8))
+    print(f"0.5B bf16: max-abs-rel {err:.2e}, {flips} flips")
+
+
+@pytest.mark.parametrize("name", ["ffn_1b_bf16", "ffn_2b_bf16"])
+def test_e2e_full_size_sampled_rows(cuda_device, name):
+    """Full-size workload in the bench's launch configuration; the oracle
+    checks a sample of rows (first, last, and a strided set)."""
+    cfg = synth.CONFIGS[name]
+    inp = synth.make_inputs(cfg)
+    n = cfg.n_tokens
+    rows = np.unique(np.concatenate([[0, 1, n - 1], np.arange(5, n, n // 24)]))
+    err, flips, _ = _e2e_check(inp, cuda_device, cfg.tile, cfg.cap, BF16_TOL, rows=rows)
+    print(f"{name}: max-abs-rel {err:.2e} on {len(rows)} rows, {flips} flips")
+
+
+# ------------------------------------------------------------ dense baseline
+
+@pytest.mark.parametrize("n,d,f", [(300, 264, 640), (256, 1024, 2048)])
+def test_dense_ffn_matches_oracle(cuda_device, n, d, f):
+    inp = synth.make_inputs(synth.CONFIGS["ffn_0p5b_bf16"].with_(n_tokens=n, d_model=d, d_ff=f,
+                                                                 rho=0.3))
+    x, wg, wu, wd = _dev(inp, cuda_device)
+    y = sge.dense_ffn_fwd(x, wg, wu, wd.t().contiguous())
+    want = oracle.dense_ffn(*_f64(inp))
+    err = oracle.max_abs_rel(to_f64(y), want)
+    assert err <= BF16_TOL, err
+
+
+def test_dense_ffn_full_size_sampled(cuda_device):
+    cfg = synth.CONFIGS["ffn_1b_bf16"]
+    inp = synth.make_inputs(cfg)
+    x, wg, wu, wd = _dev(inp, cuda_device)
+    y = sge.dense_ffn_fwd(x, wg, wu, wd.t().contiguous())
+    rows = np.arange(3, cfg.n_tokens, cfg.n_tokens // 16)
+    xf, wgf, wuf, wdf = _f64(inp)
+    want = oracle.dense_ffn(xf[rows], wgf, wuf, wdf)
+    err = oracle.max_abs_rel(to_f64(y)[rows], want)
+    assert err <= BF16_TOL, err
+
+
+def test_diag_counts_overflow_tiles(cuda_device):
+    cfg = synth.CONFIGS["tiny_fp32"]
+    inp = synth.make_grid_inputs(256, 256, 1024, torch.float32, rho=0.05)
+    x, wg, _, _ = _dev(inp, cuda_device)
+    diag = sge.new_diag(cuda_device)
+    sge.twell_gate_pack(x, wg, 64, 4, diag=diag)
+    sge.twell_gate_pack(x, wg, 64, 4, diag=diag)       # accumulates
+    ora = oracle.twell_pack(oracle.gate_preact(inp.as_f64("x"), inp.as_f64("wg_t")), 64, 4,
+                            oracle.VAL_F32)
+    torch.cuda.synchronize()
+    assert int(diag[0]) == 2 * ora.overflow
+    assert int(diag[3]) == 0
+
+
+def test_library_errors_raise(cuda_device):
+    x = torch.zeros(8, 64, dtype=torch.bfloat16, device=cuda_device)
+    w = torch.zeros(200, 64, dtype=torch.bfloat16, device=cuda_device)
+    with pytest.raises(sge.LibraryError):
+        sge.twell_gate_pack(x, w, 64, 64)          # 64 does not divide 200
