@@ -52,6 +52,8 @@ def parse():
     p.add_argument("--workload", default="ffn_1b_bf16")
     p.add_argument("--impl", default="own", choices=["own", "reference"])
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    p.add_argument("--profile", action="store_true",
+                   help="run only warmup + steps of the sparse step (for ncu captures); no JSON")
     return p.parse_args()
 
 
@@ -172,6 +174,7 @@ def run_own(args, rank, world, local_rank):
                 e[i + 1].record(stream)
             if s >= warm:
                 evs.append(e)
+        torch.cuda.synchronize(dev)
         return evs
 
     def reduce_max(v: float) -> float:
@@ -184,6 +187,10 @@ def run_own(args, rank, world, local_rank):
     gate = lambda: sge.twell_gate_pack(x, wg, tile, cap, out=tw, diag=diag)
     fused = lambda: sge.twell_fused_up_down(x, tw, wu, wd, y=y)
     dense = lambda: sge.dense_ffn_fwd(x, wg, wu, wd_t, h=h, y=y_dense)
+
+    if args.profile:
+        timed([gate, fused], args.steps, args.warmup)
+        return None
 
     # ---- the sparse forward: timed region
     timed([gate, fused], 0, args.warmup)
@@ -375,7 +382,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     out = run_own(args, rank, world, local_rank)
-    if rank == 0:
+    if rank == 0 and out is not None:
         from activation_sparse_gated_epilogue_b200 import synth
         out["cpu_baseline"] = None if args.no_cpu else cpu_baseline(synth.CONFIGS[args.workload])
         print(json.dumps(out), flush=True)

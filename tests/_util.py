@@ -44,14 +44,16 @@ def assert_twell_equal(tw_gpu, tw_ora: "oracle.TwELL"):
 
 
 def compare_twell_inexact(tw_gpu, tw_ora: "oracle.TwELL", g_ora: np.ndarray, val_kind: int,
-                          rows=None):
+                          abs_sum: np.ndarray, rows=None):
     """GPU TwELL (fp32 gate accumulation) vs the oracle's (fp64 gates).
 
     A tile may disagree (different count, or different stored indices, which
     a sign flip causes in a truncated tile by shifting its window) only if it
     holds oracle gates with |g| < FLIP_EPS, at least as many as the count
-    difference.  Values of agreeing tiles match within one ulp (bf16) or the
-    fp32 tolerance.  Returns (bad-row mask, number of disagreeing tiles)."""
+    difference.  Values of agreeing tiles match within one ulp of the value
+    dtype plus the fp32 accumulation allowance 2^-16 * sum_i |x_i w_i|
+    (``abs_sum``, [N][F]).  Returns (bad-row mask, number of disagreeing
+    tiles)."""
     c, i, v = twell_host(tw_gpu)
     if rows is not None:
         c, i, v = c[rows], i[rows], v[rows]
@@ -69,8 +71,9 @@ def compare_twell_inexact(tw_gpu, tw_ora: "oracle.TwELL", g_ora: np.ndarray, val
         "a tile disagrees without a near-zero gate to explain it"
     ok = (~tile_bad)[:, :, None] & keep_o
     vg, vo = v[ok], tw_ora.val[ok]
-    if val_kind == oracle.VAL_BF16:
-        assert np.all(np.abs(vg - vo) <= 2.0 ** -7 * np.abs(vo) * 1.0001)
-    else:
-        assert oracle.max_abs_rel(vg, vo) <= F32_TOL
+    t_i, b_i, s_i = np.nonzero(ok)
+    s_abs = abs_sum[t_i, b_i * tile + tw_ora.idx[t_i, b_i, s_i].astype(np.int64)]
+    ulp = 2.0 ** -7 if val_kind == oracle.VAL_BF16 else 2.0 ** -23
+    excess = np.abs(vg - vo) - ulp * np.abs(vo) * 1.0001
+    assert np.all(excess <= 2.0 ** -16 * s_abs), float(np.max(excess / s_abs))
     return tile_bad.any(1), int(tile_bad.sum())

@@ -77,7 +77,8 @@ def test_gate_pack_gaussian_sign_flips(cuda_device, name, cap):
     kind = KIND[cfg.torch_dtype]
     ora = oracle.twell_pack(g, cfg.tile, cap, kind)
     torch.cuda.synchronize()
-    bad_rows, bad_tiles = compare_twell_inexact(tw, ora, g, kind)
+    abs_sum = np.abs(inp.as_f64("x")) @ np.abs(inp.as_f64("wg_t")).T
+    bad_rows, bad_tiles = compare_twell_inexact(tw, ora, g, kind, abs_sum)
     assert bad_tiles <= max(2, 0.002 * ora.count.size)
     print(f"{name} C={cap}: {bad_tiles} tiles differ by near-zero sign flips")
 
@@ -93,6 +94,8 @@ def test_gate_pack_gaussian_sign_flips(cuda_device, name, cap):
 ])
 def test_fused_up_down_matches_oracle(cuda_device, dtype, tol, n, d, f, tile, cap):
     """Both sides get the same TwELL (the oracle's pack of its fp64 G)."""
+    if dtype == torch.float32 and d > 1280:
+        pytest.skip("fp32 fused up/down supports d_model <= 1280 (see test_fused_fp32_d_limit)")
     inp = synth.make_inputs(synth.CONFIGS["ffn_0p5b_bf16"].with_(
         n_tokens=n, d_model=d, d_ff=f, dtype="bf16" if dtype == torch.bfloat16 else "f32",
         rho=0.05))
@@ -103,6 +106,15 @@ def test_fused_up_down_matches_oracle(cuda_device, dtype, tol, n, d, f, tile, ca
     want = oracle.fused_up_down(xf, ora_tw, wuf, wdf)
     err = oracle.max_abs_rel(to_f64(y), want)
     assert err <= tol, err
+
+
+def test_fused_fp32_d_limit(cuda_device):
+    x = torch.zeros(4, 1288, dtype=torch.float32, device=cuda_device)
+    w = torch.zeros(128, 1288, dtype=torch.float32, device=cuda_device)
+    tw = sge.TwELL.empty(4, 128, 128, 128, torch.float32, cuda_device)
+    tw.count.zero_()
+    with pytest.raises(sge.LibraryError, match="too large"):
+        sge.twell_fused_up_down(x, tw, w, w)
 
 
 def test_fused_up_down_zero_density(cuda_device):
@@ -142,7 +154,8 @@ def _e2e_check(inp, dev, tile, cap, tol, rows=None):
         xf = xf[rows]
     kind = KIND[inp.x.dtype]
     y_ora, tw_ora, g = oracle.sparse_ffn(xf, wgf, wuf, wdf, tile, cap, kind)
-    bad_rows, bad_tiles = compare_twell_inexact(tw, tw_ora, g, kind, rows=rows)
+    abs_sum = np.abs(xf) @ np.abs(wgf).T
+    bad_rows, bad_tiles = compare_twell_inexact(tw, tw_ora, g, kind, abs_sum, rows=rows)
     # rows whose stored entries differ (near-zero sign flips) are left out of
     # the y bar and counted
     assert bad_rows.sum() <= max(2, 0.02 * len(bad_rows))
