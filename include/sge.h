@@ -95,7 +95,7 @@ const char* sge_last_error(void);
  *   x      [N][d]   dtype     input activations
  *   wg_t   [F][d]   dtype     W_gate transposed (neuron-major)
  *   dtype  SGE_BF16: tcgen05 tensor-core GEMM (bf16 x bf16 -> fp32);
- *          SGE_F32:  CUDA-core fp32 FMA GEMM (exact fp32 products).
+ *          SGE_F32:  CUDA-core fp32 FMA GEMM.
  *   tile   T: 16, 32, 64 or 128, dividing F
  *   cap    C: 1 <= C <= T
  *   count, idx, val: TwELL output as laid out above (val in `dtype`)
@@ -119,7 +119,8 @@ int twell_gate_pack(const void* x, const void* wg_t, int64_t n_tokens, int64_t d
  *
  *   x [N][d], wu_t [F][d], wd [F][d], y [N][d] in dtype; count/idx/val the
  *   TwELL produced by twell_gate_pack with the same T and C.
- * Errors: as twell_gate_pack; SGE_ERR_UNSUPPORTED for d > 4096.
+ * Errors: as twell_gate_pack; SGE_ERR_UNSUPPORTED for d > 8192 (bf16) or
+ * d > 4096 (fp32).
  */
 int twell_fused_up_down(const void* x, const uint8_t* count, const uint8_t* idx, const void* val,
                         const void* wu_t, const void* wd, void* y, int64_t n_tokens,
