@@ -5,8 +5,7 @@
 //   GEMM 1 (two accumulators, shared A tile):  G = x W_gate, U = x W_up,
 //          epilogue h = bf16(ReLU(G) * U) -> h [N][F]
 //   GEMM 2:  y = bf16(h W_down) with W_down given transposed (K-major).
-#include "sge_host.h"
-#include "tc_gemm.cuh"
+#include "tc_launch.cuh"
 
 namespace sge {
 
@@ -77,21 +76,6 @@ struct EpiStoreBf16 {
   }
 };
 
-template <class Shape, class Epi>
-int launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, int64_t m,
-                   int64_t n, int64_t k, const Epi& epi, int32_t* diag, cudaStream_t st,
-                   const char* what) {
-  auto kern = tc_gemm_kernel<Shape, Epi>;
-  int rc = set_smem_limit(reinterpret_cast<const void*>(kern), Shape::SMEM_BYTES);
-  if (rc) return rc;
-  const int64_t tiles = ((m + kBM - 1) / kBM) * ((n + Shape::BN - 1) / Shape::BN);
-  const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  kern<<<grid, kGemmThreads, Shape::SMEM_BYTES, st>>>(ma, mb0, mb1, static_cast<int>(m),
-                                                      static_cast<int>(n), static_cast<int>(k), epi,
-                                                      diag);
-  return check_launch(what);
-}
-
 }  // namespace sge
 
 using namespace sge;
@@ -110,18 +94,18 @@ extern "C" int dense_ffn_fwd(const void* x, const void* wg_t, const void* wu_t, 
       !aligned16(y))
     return fail(SGE_ERR_ARG, "dense_ffn_fwd: pointer not 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  using S1 = TcShape<128, 2>;
-  using S2 = TcShape<256, 1>;
+  using S1 = TcPairShape<128, 2>;
+  using S2 = TcPairShape<256, 1>;
   CUtensorMap mx, mg, mu, mh, md;
   int rc;
   if ((rc = make_tmap_bf16(&mx, x, n_tokens, d_model, d_model, kBM))) return rc;
-  if ((rc = make_tmap_bf16(&mg, wg_t, d_ff, d_model, d_model, S1::BN))) return rc;
-  if ((rc = make_tmap_bf16(&mu, wu_t, d_ff, d_model, d_model, S1::BN))) return rc;
+  if ((rc = make_tmap_bf16(&mg, wg_t, d_ff, d_model, d_model, S1::BN / 2))) return rc;
+  if ((rc = make_tmap_bf16(&mu, wu_t, d_ff, d_model, d_model, S1::BN / 2))) return rc;
   if ((rc = make_tmap_bf16(&mh, h, n_tokens, d_ff, d_ff, kBM))) return rc;
-  if ((rc = make_tmap_bf16(&md, wd_t, d_model, d_ff, d_ff, S2::BN))) return rc;
+  if ((rc = make_tmap_bf16(&md, wd_t, d_model, d_ff, d_ff, S2::BN / 2))) return rc;
   EpiGated e1{static_cast<uint16_t*>(h), n_tokens, static_cast<int>(d_ff)};
-  if ((rc = launch_tc_gemm<S1>(mx, mg, mu, n_tokens, d_ff, d_model, e1, diag, st, "dense_ffn_fwd gate/up")))
+  if ((rc = launch_tc_gemm_pair<S1>(mx, mg, mu, n_tokens, d_ff, d_model, e1, diag, st, "dense_ffn_fwd gate/up")))
     return rc;
   EpiStoreBf16 e2{static_cast<uint16_t*>(y), n_tokens, static_cast<int>(d_model)};
-  return launch_tc_gemm<S2>(mh, md, md, n_tokens, d_model, d_ff, e2, diag, st, "dense_ffn_fwd down");
+  return launch_tc_gemm_pair<S2>(mh, md, md, n_tokens, d_model, d_ff, e2, diag, st, "dense_ffn_fwd down");
 }

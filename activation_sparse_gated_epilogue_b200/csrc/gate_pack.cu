@@ -13,8 +13,7 @@
 // tile is a sequential in-thread scan over its columns in ascending order.
 // fp32: a CUDA-core FMA GEMM (64 x 128 tiles) with the same pack from a
 // shared-memory copy of the tile.
-#include "sge_host.h"
-#include "tc_gemm.cuh"
+#include "tc_launch.cuh"
 
 namespace sge {
 
@@ -155,26 +154,15 @@ __global__ void __launch_bounds__(256) gate_pack_f32_kernel(const float* __restr
 template <int T>
 static int launch_bf16(const void* x, const void* wg_t, int64_t n, int64_t d, int64_t f, int cap,
                        uint8_t* count, uint8_t* idx, void* val, int32_t* diag, cudaStream_t st) {
-  using Shape = TcShape<256, 1>;
+  using Shape = TcPairShape<256, 1>;
   CUtensorMap ma, mb;
   int rc = make_tmap_bf16(&ma, x, n, d, d, kBM);
   if (rc) return rc;
-  rc = make_tmap_bf16(&mb, wg_t, f, d, d, Shape::BN);
+  rc = make_tmap_bf16(&mb, wg_t, f, d, d, Shape::BN / 2);
   if (rc) return rc;
   EpiTwell<T> epi{count, idx, static_cast<uint16_t*>(val), n, static_cast<int>(f), cap, diag};
-  auto kern = tc_gemm_kernel<Shape, EpiTwell<T>>;
-  static int smem_set = 0;
-  if (!smem_set) {
-    rc = set_smem_limit(reinterpret_cast<const void*>(kern), Shape::SMEM_BYTES);
-    if (rc) return rc;
-    smem_set = 1;
-  }
-  const int64_t tiles = ((n + kBM - 1) / kBM) * ((f + Shape::BN - 1) / Shape::BN);
-  const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  kern<<<grid, kGemmThreads, Shape::SMEM_BYTES, st>>>(ma, mb, mb, static_cast<int>(n),
-                                                      static_cast<int>(f), static_cast<int>(d),
-                                                      epi, diag);
-  return check_launch("twell_gate_pack (bf16 tcgen05)");
+  return launch_tc_gemm_pair<Shape>(ma, mb, mb, n, f, d, epi, diag, st,
+                                    "twell_gate_pack (bf16 tcgen05 pair)");
 }
 
 template <int T>

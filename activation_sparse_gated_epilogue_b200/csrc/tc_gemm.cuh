@@ -219,4 +219,188 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// CTA-pair variant (cta_group::2): a cluster of two CTAs on two SMs computes a
+// 256 x BN tile.  CTA r loads rows [128 r, 128 r + 128) of the A tile and
+// half of each B tile (BN/2 rows) into its own shared memory; both CTAs'
+// TMA bytes complete on the leader's (rank 0) `full` barrier.  The leader's
+// MMA thread issues M = 256 tcgen05.mma instructions that read A and B from
+// both CTAs and write each CTA's 128 accumulator rows into that CTA's TMEM;
+// its commits arrive on both CTAs' barriers (multicast commit).  Each CTA's
+// epilogue drains its own TMEM and releases the accumulator on the leader's
+// `tmem_empty` barrier (count 8: four warps in each CTA).  Per SM this moves
+// half the B bytes of the single-CTA engine for the same work.
+template <int BN_, int NB_>
+struct TcPairShape {
+  static constexpr int BN = BN_;  // N of one MMA (both CTAs together)
+  static constexpr int NB = NB_;
+  static constexpr int BM = 2 * kBM;
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = (BN / 2) * kBK * 2;  // this CTA's half
+  static constexpr int STAGE_BYTES = A_BYTES + NB * B_BYTES;
+  static constexpr int STAGES = (196 * 1024) / STAGE_BYTES > 8 ? 8 : (196 * 1024) / STAGE_BYTES;
+  static constexpr int ACC_COLS = BN * NB;
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=256");
+  static_assert(TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0, "TMEM columns");
+  static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1024-byte aligned sub-tiles");
+};
+
+template <class Shape, class Epilogue>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
+                        const __grid_constant__ CUtensorMap map_b0,
+                        const __grid_constant__ CUtensorMap map_b1, int M, int N, int K,
+                        Epilogue epi, int32_t* diag) {
+  constexpr int BN = Shape::BN, NB = Shape::NB, STAGES = Shape::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Shape::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tmem_full = empty + STAGES;
+  uint64_t* tmem_empty = tmem_full + 2;
+  uint64_t* drain = tmem_empty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(cluster_id_x());
+  const int n_pairs = static_cast<int>(cluster_count_x());
+  const int m_blocks = (M + Shape::BM - 1) / Shape::BM;
+  const int n_blocks = (N + BN - 1) / BN;
+  const int num_tiles = m_blocks * n_blocks;
+  const int k_blocks = (K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tmem_full[a], 1);
+      mbar_init(&tmem_empty[a], 8);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&map_a);
+    tma_prefetch_desc(&map_b0);
+    if (NB == 2) tma_prefetch_desc(&map_b1);
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_holder, Shape::TMEM_COLS);
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive / TMA
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t armed = 0, armed_par = 0;
+      for (int tile = pair; tile < num_tiles && !*abort_flag; tile += n_pairs) {
+        const TileCoord tc = tile_coord(tile, m_blocks);
+        const int a_row = tc.m_blk * Shape::BM + static_cast<int>(rank) * kBM;
+        const int b_row = tc.n_blk * BN + static_cast<int>(rank) * (BN / 2);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, diag)) break;
+          uint8_t* sa = smem + s * Shape::STAGE_BYTES;
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * Shape::STAGE_BYTES);
+          tma_load_2d_pair(sa, &map_a, &full[s], kb * kBK, a_row);
+          tma_load_2d_pair(sa + Shape::A_BYTES, &map_b0, &full[s], kb * kBK, b_row);
+          if (NB == 2)
+            tma_load_2d_pair(sa + Shape::A_BYTES + Shape::B_BYTES, &map_b1, &full[s], kb * kBK, b_row);
+          armed |= 1u << s;
+          armed_par = (armed_par & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      // Drain: the leader's barrier counts both CTAs' bytes, so once the
+      // leader has seen every armed stage land, no load of either CTA is in
+      // flight (the closing cluster barrier holds the other CTA until then).
+      if (leader)
+        for (int t = 0; t < STAGES; ++t)
+          if (armed & (1u << t)) mbar_wait(&full[t], (armed_par >> t) & 1, diag);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(Shape::BM, BN);
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      for (int tile = pair; tile < num_tiles && !*abort_flag; tile += n_pairs, ++it) {
+        const int acc = it & 1;
+        if (!wait_or_abort(&tmem_empty[acc], ((it >> 1) & 1) ^ 1, abort_flag, diag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * Shape::ACC_COLS;
+        bool ok = true;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!wait_or_abort(&full[s], ph, abort_flag, diag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * Shape::STAGE_BYTES);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t adesc = umma_desc_sw128(sa + k * 32);
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+              const uint64_t bdesc = umma_desc_sw128(sa + Shape::A_BYTES + b * Shape::B_BYTES + k * 32);
+              umma2_bf16(d_tmem + b * BN, adesc, bdesc, idesc, (kb | k) != 0);
+            }
+          }
+          umma2_commit_mc(&empty[s], 0x3);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma2_commit_mc(&tmem_full[acc], 0x3);
+      }
+      // Drain: both CTAs learn that every issued MMA has completed.
+      umma2_commit_mc(drain, 0x3);
+    }
+    if (lane == 0) mbar_wait(drain, 0, diag);
+    __syncwarp();
+  } else {
+    // --------------------------------------------------------- epilogue
+    const int quarter = warp & 3;
+    const uint32_t leader_tmem_empty0 = mapa_shared(smem_u32(&tmem_empty[0]), 0);
+    int it = 0;
+    for (int tile = pair; tile < num_tiles; tile += n_pairs, ++it) {
+      const int acc = it & 1;
+      const bool ok = wait_or_abort(&tmem_full[acc], (it >> 1) & 1, abort_flag, diag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const TileCoord tc = tile_coord(tile, m_blocks);
+      const uint32_t taddr = tmem_base + acc * Shape::ACC_COLS + (static_cast<uint32_t>(quarter * 32) << 16);
+      const int64_t row = static_cast<int64_t>(tc.m_blk) * Shape::BM + rank * kBM + quarter * 32 + lane;
+      epi.template run<BN>(taddr, row, tc.n_blk, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_tmem_empty0 + acc * 8);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while its pair may still touch its barriers or TMEM
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, Shape::TMEM_COLS);
+  }
+}
+
 }  // namespace sge
