@@ -28,10 +28,10 @@
 
 namespace sge {
 
-constexpr int kUdThreads = 256;
+constexpr int kUdThreads = 128;
 constexpr int kUdWarps = kUdThreads / 32;
 constexpr int kMaxEntries = 512;  // entries per chunk held in shared memory
-constexpr int kUnroll = 8;        // entries in flight per thread
+constexpr int kUnroll = 8;        // entries per reduction group
 constexpr int kMaxTiles = 512;    // TwELL tiles per chunk
 
 template <bool BF16>
@@ -56,14 +56,20 @@ struct Elem<true> {
           : "r"(xs[i]), "r"(ws[i]));
     return acc;
   }
-  __device__ __forceinline__ static void axpy(float h, const uint4& w, float (&y)[8]) {
+  // y += h * w with h already rounded to bf16 (hb), exact products
+  __device__ __forceinline__ static void axpy(uint16_t hb, const uint4& w, float (&y)[8]) {
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      y[2 * i] = fmaf(h, __uint_as_float(ws[i] << 16), y[2 * i]);
-      y[2 * i + 1] = fmaf(h, __uint_as_float(ws[i] & 0xFFFF0000u), y[2 * i + 1]);
-    }
+    for (int i = 0; i < 4; ++i)
+      asm("{\n\t.reg .b16 wl, wh;\n\t"
+          "mov.b32 {wl, wh}, %2;\n\t"
+          "fma.rn.f32.bf16 %0, %3, wl, %0;\n\t"
+          "fma.rn.f32.bf16 %1, %3, wh, %1;\n\t}"
+          : "+f"(y[2 * i]), "+f"(y[2 * i + 1])
+          : "r"(ws[i]), "h"(hb));
   }
+  using HType = uint16_t;
+  __device__ __forceinline__ static HType h_of(float h) { return f32_to_bf16_bits(h); }
   __device__ __forceinline__ static float load_val(const void* p, int64_t i) {
     return __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(p)[i]) << 16);
   }
@@ -93,6 +99,8 @@ struct Elem<false> {
     y[2] = fmaf(h, __uint_as_float(w.z), y[2]);
     y[3] = fmaf(h, __uint_as_float(w.w), y[3]);
   }
+  using HType = float;
+  __device__ __forceinline__ static HType h_of(float h) { return h; }
   __device__ __forceinline__ static float load_val(const void* p, int64_t i) {
     return static_cast<const float*>(p)[i];
   }
@@ -138,7 +146,7 @@ __device__ __forceinline__ int reduce8_entry(int lane) {
 }
 
 template <int NV, bool BF16>
-__global__ void __launch_bounds__(kUdThreads, NV == 1 ? 4 : (NV == 2 ? 3 : 2))
+__global__ void __launch_bounds__(kUdThreads, NV == 1 ? 6 : (NV == 2 ? 5 : (NV == 3 ? 4 : 3)))
     fused_up_down_kernel(const void* __restrict__ x, const uint8_t* __restrict__ count,
                          const uint8_t* __restrict__ idx, const void* __restrict__ val,
                          const void* __restrict__ wu_t, const void* __restrict__ wd,
@@ -146,8 +154,7 @@ __global__ void __launch_bounds__(kUdThreads, NV == 1 ? 4 : (NV == 2 ? 3 : 2))
   using E = Elem<BF16>;
   constexpr int VEC = E::VEC;
   constexpr int ESZ = BF16 ? 2 : 4;
-  __shared__ int s_j[kMaxEntries];
-  __shared__ float s_a[kMaxEntries];
+  __shared__ int2 s_jh[kMaxEntries];  // (column j, a bits); after phase U: (j, h bits)
   __shared__ float s_upart[kUdWarps][kMaxEntries];
   __shared__ int s_tile_off[kMaxTiles + 1];
   __shared__ int s_chunk[2];  // [0] first tile after the chunk, [1] entries in the chunk
@@ -216,8 +223,7 @@ __global__ void __launch_bounds__(kUdThreads, NV == 1 ? 4 : (NV == 2 ? 3 : 2))
       const int b = b0 + lo;
       const int s = e - s_tile_off[lo];
       const int64_t seg = t * nt + b;
-      s_j[e] = b * tile + idx[seg * cap + s];
-      s_a[e] = E::load_val(val, seg * cap + s);
+      s_jh[e] = make_int2(b * tile + idx[seg * cap + s], __float_as_int(E::load_val(val, seg * cap + s)));
     }
     __syncthreads();
 
@@ -229,13 +235,12 @@ __global__ void __launch_bounds__(kUdThreads, NV == 1 ? 4 : (NV == 2 ? 3 : 2))
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int e = e0 + u;
-        const int j = e < n_e ? s_j[e] : -1;
+        const int j = e < n_e ? s_jh[e].x : -1;
+        const uint4* row = reinterpret_cast<const uint4*>(wub + static_cast<int64_t>(j) * row_bytes);
 #pragma unroll
         for (int k = 0; k < NV; ++k) {
           const int v = tid + k * kUdThreads;
-          w[u][k] = (j >= 0 && v < nvec)
-                        ? __ldg(reinterpret_cast<const uint4*>(wub + static_cast<int64_t>(j) * row_bytes) + v)
-                        : make_uint4(0, 0, 0, 0);
+          w[u][k] = (j >= 0 && v < nvec) ? __ldg(row + v) : make_uint4(0, 0, 0, 0);
         }
       }
 #pragma unroll
@@ -253,12 +258,15 @@ __global__ void __launch_bounds__(kUdThreads, NV == 1 ? 4 : (NV == 2 ? 3 : 2))
     }
     __syncthreads();
 
-    // ---- h = a * u (fixed-order sum over warps); reuse s_a for h
+    // ---- h = a * u (fixed-order sum over warps), rounded as phase D uses it
     for (int e = tid; e < n_e; e += kUdThreads) {
       float u = 0.0f;
 #pragma unroll
       for (int w8 = 0; w8 < kUdWarps; ++w8) u += s_upart[w8][e];
-      s_a[e] = s_a[e] * u;
+      const typename E::HType hq = E::h_of(__int_as_float(s_jh[e].y) * u);
+      int bits;
+      if constexpr (BF16) bits = static_cast<int>(hq); else bits = __float_as_int(hq);
+      s_jh[e].y = bits;
     }
     __syncthreads();
 
@@ -266,25 +274,23 @@ __global__ void __launch_bounds__(kUdThreads, NV == 1 ? 4 : (NV == 2 ? 3 : 2))
     const char* wdb = static_cast<const char*>(wd);
     for (int e0 = 0; e0 < n_e; e0 += kUnroll) {
       uint4 w[kUnroll][NV];
+      typename E::HType hv[kUnroll];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int e = e0 + u;
-        const int j = e < n_e ? s_j[e] : -1;
+        const int2 jh = e < n_e ? s_jh[e] : make_int2(-1, 0);
+        if constexpr (BF16) hv[u] = static_cast<uint16_t>(jh.y); else hv[u] = __int_as_float(jh.y);
+        const uint4* row = reinterpret_cast<const uint4*>(wdb + static_cast<int64_t>(jh.x) * row_bytes);
 #pragma unroll
         for (int k = 0; k < NV; ++k) {
           const int v = tid + k * kUdThreads;
-          w[u][k] = (j >= 0 && v < nvec)
-                        ? __ldg(reinterpret_cast<const uint4*>(wdb + static_cast<int64_t>(j) * row_bytes) + v)
-                        : make_uint4(0, 0, 0, 0);
+          w[u][k] = (jh.x >= 0 && v < nvec) ? __ldg(row + v) : make_uint4(0, 0, 0, 0);
         }
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int e = e0 + u;
-        const float h = e < n_e ? s_a[e] : 0.0f;
+      for (int u = 0; u < kUnroll; ++u)
 #pragma unroll
-        for (int k = 0; k < NV; ++k) E::axpy(h, w[u][k], acc[k]);
-      }
+        for (int k = 0; k < NV; ++k) E::axpy(hv[u], w[u][k], acc[k]);
     }
     b0 = b1;
     __syncthreads();  // the next chunk rewrites the shared lists
@@ -316,6 +322,7 @@ static int dispatch_ud(const void* x, const uint8_t* count, const uint8_t* idx, 
   const int64_t nv = (d + PER - 1) / PER;
   if (nv <= 1) return launch_ud<1, BF16>(x, count, idx, val, wu_t, wd, y, n, d, f, tile, cap, st);
   if (nv <= 2) return launch_ud<2, BF16>(x, count, idx, val, wu_t, wd, y, n, d, f, tile, cap, st);
+  if (nv <= 3) return launch_ud<3, BF16>(x, count, idx, val, wu_t, wd, y, n, d, f, tile, cap, st);
   if (nv <= 4) return launch_ud<4, BF16>(x, count, idx, val, wu_t, wd, y, n, d, f, tile, cap, st);
   return fail(SGE_ERR_UNSUPPORTED, "twell_fused_up_down: d_model %lld too large (max %d)",
               (long long)d, 4 * PER);

@@ -17,7 +17,11 @@
 
 namespace sge {
 
-// Epilogue: ReLU + TwELL pack of one 128 x BN accumulator tile.
+// Epilogue: ReLU + TwELL pack of one 128 x BN accumulator tile.  Each thread
+// owns one row.  Per 32-column chunk it builds the bit mask of active
+// columns (g > 0; NaN and -0 are inactive), then visits only the set bits in
+// ascending order, so the cost is ~2 instructions per column plus a few
+// dozen per stored entry.
 template <int T>
 struct EpiTwell {
   uint8_t* count;
@@ -28,39 +32,73 @@ struct EpiTwell {
   int cap;
   int32_t* diag;
 
+  // r[jj] for a run-time jj in [0, 32) without local memory: a 5-level
+  // select tree over the 32 registers.
+  __device__ __forceinline__ static uint32_t pick(const uint32_t (&r)[32], int jj) {
+    uint32_t a[16], b[8], c4[4], d2[2];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a[i] = (jj & 16) ? r[i + 16] : r[i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) b[i] = (jj & 8) ? a[i + 8] : a[i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c4[i] = (jj & 4) ? b[i + 4] : b[i];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) d2[i] = (jj & 2) ? c4[i + 2] : c4[i];
+    return (jj & 1) ? d2[1] : d2[0];
+  }
+
+  // Store the active columns of `m` (bits of r) as entries of tile `seg`,
+  // local index = bit + idx_off; c counts every active column.
+  __device__ __forceinline__ void emit(uint32_t m, const uint32_t (&r)[32], int& c, int64_t seg,
+                                       bool ok, int idx_off) const {
+    while (m) {
+      const int jj = __ffs(m) - 1;
+      m &= m - 1;
+      if (ok && c < cap) {
+        idx[seg * cap + c] = static_cast<uint8_t>(jj + idx_off);
+        val[seg * cap + c] = f32_to_bf16_bits(__uint_as_float(pick(r, jj)));
+      }
+      ++c;
+    }
+  }
+
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {
     static_assert(BN % T == 0 && BN % 32 == 0, "tile must divide the GEMM N block");
+    static_assert(T == 16 || T % 32 == 0, "tile width");
     const bool row_ok = row < n_rows;
     const int64_t nt = n_cols / T;
     int overflow = 0;
     int c = 0;
-    int64_t seg = 0;
-    bool tile_ok = false;
-#pragma unroll
+#pragma unroll 1
     for (int ch = 0; ch < BN / 32; ++ch) {
       uint32_t r[32];
       tmem_ld32(taddr + ch * 32, r);
       tmem_ld_wait();
+      uint32_t m = 0;
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
-        constexpr int kT = T;
-        const int col = ch * 32 + jj;  // column inside the N block (compile time)
-        if (col % kT == 0) {
-          const int gcol = n_blk * BN + col;
-          tile_ok = row_ok && gcol < n_cols;
-          seg = row * nt + gcol / kT;
+      for (int jj = 0; jj < 32; ++jj) m |= (__uint_as_float(r[jj]) > 0.0f ? 1u : 0u) << jj;
+      const int col0 = n_blk * BN + ch * 32;  // global column of bit 0
+      if constexpr (T == 16) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int gcol = col0 + 16 * half;
+          const bool ok = row_ok && gcol < n_cols;
+          const int64_t seg = row * nt + gcol / T;
           c = 0;
-        }
-        const float v = __uint_as_float(r[jj]);
-        if (v > 0.0f) {
-          if (tile_ok && c < cap) {
-            idx[seg * cap + c] = static_cast<uint8_t>(col % kT);
-            val[seg * cap + c] = f32_to_bf16_bits(v);
+          emit(half ? (m & 0xFFFF0000u) : (m & 0xFFFFu), r, c, seg, ok, -16 * half);
+          if (ok) {
+            count[seg] = static_cast<uint8_t>(c);
+            overflow += c > cap;
           }
-          ++c;
         }
-        if (col % kT == kT - 1 && tile_ok) {
+      } else {
+        const int off = (ch * 32) % T;  // offset of this chunk inside its tile
+        if (off == 0) c = 0;
+        const bool ok = row_ok && col0 < n_cols;
+        const int64_t seg = row * nt + col0 / T;
+        emit(m, r, c, seg, ok, off);
+        if (off + 32 == T && ok) {
           count[seg] = static_cast<uint8_t>(c);
           overflow += c > cap;
         }
