@@ -28,8 +28,6 @@
 
 namespace sge {
 
-constexpr int kUdThreads = 128;
-constexpr int kUdWarps = kUdThreads / 32;
 constexpr int kMaxEntries = 512;  // entries per chunk held in shared memory
 constexpr int kUnroll = 8;        // entries per reduction group
 constexpr int kMaxTiles = 512;    // TwELL tiles per chunk
@@ -145,8 +143,8 @@ __device__ __forceinline__ int reduce8_entry(int lane) {
   return ((lane & 16) ? 4 : 0) + ((lane & 8) ? 2 : 0) + ((lane & 4) ? 1 : 0);
 }
 
-template <int NV, bool BF16>
-__global__ void __launch_bounds__(kUdThreads, NV == 1 ? 6 : (NV == 2 ? 5 : (NV == 3 ? 4 : 3)))
+template <int THREADS, int NV, bool BF16>
+__global__ void __launch_bounds__(THREADS, THREADS == 256 ? 2 : (NV == 1 ? 6 : (NV == 2 ? 5 : (NV == 3 ? 4 : 3))))
     fused_up_down_kernel(const void* __restrict__ x, const uint8_t* __restrict__ count,
                          const uint8_t* __restrict__ idx, const void* __restrict__ val,
                          const void* __restrict__ wu_t, const void* __restrict__ wd,
@@ -154,6 +152,8 @@ __global__ void __launch_bounds__(kUdThreads, NV == 1 ? 6 : (NV == 2 ? 5 : (NV =
   using E = Elem<BF16>;
   constexpr int VEC = E::VEC;
   constexpr int ESZ = BF16 ? 2 : 4;
+  constexpr int kUdThreads = THREADS;
+  constexpr int kUdWarps = THREADS / 32;
   __shared__ int2 s_jh[kMaxEntries];  // (column j, a bits); after phase U: (j, h bits)
   __shared__ float s_upart[kUdWarps][kMaxEntries];
   __shared__ int s_tile_off[kMaxTiles + 1];
@@ -304,28 +304,34 @@ __global__ void __launch_bounds__(kUdThreads, NV == 1 ? 6 : (NV == 2 ? 5 : (NV =
   }
 }
 
-template <int NV, bool BF16>
+template <int THREADS, int NV, bool BF16>
 static int launch_ud(const void* x, const uint8_t* count, const uint8_t* idx, const void* val,
                      const void* wu_t, const void* wd, void* y, int64_t n, int64_t d, int64_t f,
                      int tile, int cap, cudaStream_t st) {
   if (n > 0x7fffffff) return fail(SGE_ERR_UNSUPPORTED, "twell_fused_up_down: too many rows");
-  fused_up_down_kernel<NV, BF16><<<static_cast<unsigned>(n), kUdThreads, 0, st>>>(
+  fused_up_down_kernel<THREADS, NV, BF16><<<static_cast<unsigned>(n), THREADS, 0, st>>>(
       x, count, idx, val, wu_t, wd, y, static_cast<int>(d), static_cast<int>(f), tile, cap);
   return check_launch("twell_fused_up_down");
 }
 
+// A row is covered by THREADS x NV 16-byte vectors: 128 threads with 1..4
+// vectors each, 256 threads with 4 for the widest rows.
 template <bool BF16>
 static int dispatch_ud(const void* x, const uint8_t* count, const uint8_t* idx, const void* val,
                        const void* wu_t, const void* wd, void* y, int64_t n, int64_t d, int64_t f,
                        int tile, int cap, cudaStream_t st) {
-  constexpr int PER = kUdThreads * Elem<BF16>::VEC;  // elements covered per vector round
-  const int64_t nv = (d + PER - 1) / PER;
-  if (nv <= 1) return launch_ud<1, BF16>(x, count, idx, val, wu_t, wd, y, n, d, f, tile, cap, st);
-  if (nv <= 2) return launch_ud<2, BF16>(x, count, idx, val, wu_t, wd, y, n, d, f, tile, cap, st);
-  if (nv <= 3) return launch_ud<3, BF16>(x, count, idx, val, wu_t, wd, y, n, d, f, tile, cap, st);
-  if (nv <= 4) return launch_ud<4, BF16>(x, count, idx, val, wu_t, wd, y, n, d, f, tile, cap, st);
+  constexpr int VEC = Elem<BF16>::VEC;
+  const int64_t nvec = d / VEC;
+#define SGE_UD(TH, NV) \
+  if (nvec <= (TH) * (NV)) return launch_ud<TH, NV, BF16>(x, count, idx, val, wu_t, wd, y, n, d, f, tile, cap, st);
+  SGE_UD(128, 1)
+  SGE_UD(128, 2)
+  SGE_UD(128, 3)
+  SGE_UD(128, 4)
+  SGE_UD(256, 4)
+#undef SGE_UD
   return fail(SGE_ERR_UNSUPPORTED, "twell_fused_up_down: d_model %lld too large (max %d)",
-              (long long)d, 4 * PER);
+              (long long)d, 256 * 4 * VEC);
 }
 
 }  // namespace sge
