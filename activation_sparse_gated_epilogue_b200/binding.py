@@ -48,7 +48,9 @@ def library() -> ctypes.CDLL:
             "sge_version": (I, []),
             "sge_last_error": (ctypes.c_char_p, []),
             "twell_gate_pack": (I, [P, P, I64, I64, I64, I, I, I, P, P, P, P, P]),
-            "twell_fused_up_down": (I, [P, P, P, P, P, P, P, I64, I64, I64, I, I, I, P]),
+            "twell_fused_up_down_workspace_bytes": (ctypes.c_size_t, [I64]),
+            "twell_fused_up_down": (I, [P, P, P, P, P, P, P, I64, I64, I64, I, I, I, P,
+                                        ctypes.c_size_t, P]),
             "dense_ffn_fwd": (I, [P, P, P, P, P, P, I64, I64, I64, P, P]),
         }
         for name, (res, args) in sigs.items():
@@ -145,8 +147,15 @@ def twell_gate_pack(x: torch.Tensor, wg_t: torch.Tensor, tile: int, cap: int,
     return out
 
 
+def fused_workspace(n_tokens: int, device) -> torch.Tensor:
+    """Scratch for twell_fused_up_down (heavy-token list and work cursors)."""
+    nbytes = library().twell_fused_up_down_workspace_bytes(n_tokens)
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
 def twell_fused_up_down(x: torch.Tensor, tw: TwELL, wu_t: torch.Tensor, wd: torch.Tensor,
-                        y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                        y: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
     """y = sum over TwELL entries of a * (x . W_up[:, j]) * W_down[j] (h never stored)."""
     _check(x, "x")
     n, d = x.shape
@@ -159,19 +168,22 @@ def twell_fused_up_down(x: torch.Tensor, tw: TwELL, wu_t: torch.Tensor, wd: torc
     if y is None:
         y = torch.empty_like(x)
     _check(y, "y", x.dtype, (n, d))
+    if workspace is None:
+        workspace = fused_workspace(n, x.device)
+    _check(workspace, "workspace", torch.uint8)
     _call("twell_fused_up_down", _ptr(x), _ptr(tw.count), _ptr(tw.idx), _ptr(tw.val),
           _ptr(wu_t), _ptr(wd), _ptr(y), n, d, f, _dtype_code(x), tw.tile, tw.cap,
-          _stream(x.device, stream))
+          _ptr(workspace), workspace.numel(), _stream(x.device, stream))
     return y
 
 
 def twell_ffn_forward(x, wg_t, wu_t, wd, tile: int, cap: int, tw: Optional[TwELL] = None,
                       y: Optional[torch.Tensor] = None, diag: Optional[torch.Tensor] = None,
-                      stream=None):
+                      workspace: Optional[torch.Tensor] = None, stream=None):
     """The sparse inference forward: gate GEMM + TwELL epilogue, then the
     fused up/down kernel.  Returns (y, twell)."""
     tw = twell_gate_pack(x, wg_t, tile, cap, out=tw, diag=diag, stream=stream)
-    y = twell_fused_up_down(x, tw, wu_t, wd, y=y, stream=stream)
+    y = twell_fused_up_down(x, tw, wu_t, wd, y=y, workspace=workspace, stream=stream)
     return y, tw
 
 

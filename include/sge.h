@@ -114,17 +114,27 @@ int twell_gate_pack(const void* x, const void* wg_t, int64_t n_tokens, int64_t d
  * products so that the intermediate h never goes to global memory.)
  *
  *   y[t] = sum over stored entries (j, a) of row t of
- *          a * (x[t] . wu_t[j]) * wd[j]
- *   with fp32 accumulation; y is written in `dtype`.
+ *          h * wd[j],  h = a * (x[t] . wu_t[j])
+ *   with fp32 accumulation of both products; for bf16, h is rounded to bf16
+ *   before the down projection (the precision the dense bf16 FFN gives h).
+ *   y is written in `dtype`.
  *
  *   x [N][d], wu_t [F][d], wd [F][d], y [N][d] in dtype; count/idx/val the
  *   TwELL produced by twell_gate_pack with the same T and C.
- * Errors: as twell_gate_pack; SGE_ERR_UNSUPPORTED for d > 8192 (bf16) or
- * d > 4096 (fp32).
+ *   workspace  device scratch of at least
+ *              twell_fused_up_down_workspace_bytes(N) bytes, 16-byte aligned,
+ *              owned by the caller; it holds the list of heavy tokens (those
+ *              processed by a whole SM) and work cursors, and must not be
+ *              shared by calls that may run concurrently.
+ * Errors: as twell_gate_pack; SGE_ERR_ARG for a missing or short workspace;
+ * SGE_ERR_UNSUPPORTED for d > 4096 (bf16) or d > 2048 (fp32).
  */
+size_t twell_fused_up_down_workspace_bytes(int64_t n_tokens);
+
 int twell_fused_up_down(const void* x, const uint8_t* count, const uint8_t* idx, const void* val,
                         const void* wu_t, const void* wd, void* y, int64_t n_tokens,
-                        int64_t d_model, int64_t d_ff, int dtype, int tile, int cap, void* stream);
+                        int64_t d_model, int64_t d_ff, int dtype, int tile, int cap,
+                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * dense_ffn_fwd -- the dense gated FFN the method is compared against
