@@ -39,9 +39,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flop x 1.965 GHz
 FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
-# DRAM bytes per launch from the committed ncu captures (profiles/), keyed by
-# the source hash of the kernel they were taken on; null once it changes.
-TRAFFIC = {}
+# DRAM bytes (read + write) per launch from the committed ncu captures
+# (profiles/*.md), keyed by the source hash of the kernel they were taken on;
+# a kernel whose source changed since gets null.
+TRAFFIC = {
+    "c5973eaffc07627f": 80.4e6,   # gate GEMM + TwELL, profiles/gate_gemm_twell_ffn_1b_bf16.md
+    "fe89ac0e242a0959": 364.4e6,  # fused up/down, profiles/fused_up_down_ffn_1b_bf16.md
+}
 
 
 def parse():
@@ -245,7 +249,7 @@ def run_own(args, rank, world, local_rank):
     mg = statistics.mean(t_gate)
     mf = statistics.mean(t_fused)
     flops_gate = 2.0 * n * d * f
-    bf16_peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    bf16_peak = pk["bf16_tflops"]
     gate_tf = flops_gate / (mg / 1e3) / 1e12
     flops_fused = 4.0 * nnz * d
     fused_tf = flops_fused / (mf / 1e3) / 1e12
@@ -256,12 +260,14 @@ def run_own(args, rank, world, local_rank):
     fused_src = src_hash("fused_up_down.cu", "sge_common.cuh")
     tr_gate = TRAFFIC.get(gate_src)
     tr_fused = TRAFFIC.get(fused_src)
+    tr_gate = None if tr_gate is None else int(tr_gate)
+    tr_fused = None if tr_fused is None else int(tr_fused)
     k_gate = {"kernel": "twell_gate_pack (tcgen05 GEMM + TwELL epilogue)", "bound": "tensor",
               "achieved": round(gate_tf, 1), "peak": bf16_peak, "unit": "TFLOP/s",
               "frac": round(gate_tf / bf16_peak, 4), "traffic": tr_gate,
               "ms": round(mg, 4), "share": round(mg / (mg + mf), 3),
               "algorithmic": f"2*N*d*F = {flops_gate:.3e} flop per launch",
-              "peak_note": "bf16_tflops_sustained of measured peaks (seconds-long loop)"}
+              "peak_note": "bf16_tflops (burst) of measured peaks: the step keeps SM clocks at max"}
     k_fused = {"kernel": "twell_fused_up_down (classify + persistent fused kernel)", "bound": "alu", "achieved": round(fused_tf, 2),
                "peak": round(FP32_SIMT_TFLOPS, 1), "unit": "TFLOP/s",
                "frac": round(fused_tf / FP32_SIMT_TFLOPS, 4), "traffic": tr_fused,
@@ -269,6 +275,7 @@ def run_own(args, rank, world, local_rank):
                "algorithmic": f"4*nnz*d = {flops_fused:.3e} flop per launch (nnz={nnz})",
                "hbm_gbs_unique": round(bytes_fused / (mf / 1e3) / 1e9, 1),
                "peak_note": "fp32 FMA peak of the CUDA cores, 148 SMs x 128 lanes x 2 x 1.965 GHz"}
+    k_gate["traffic_unit"] = k_fused["traffic_unit"] = "bytes per launch (ncu dram read + write)"
     dominant = k_gate if mg >= mf else k_fused
     rest = k_fused if dominant is k_gate else k_gate
     roofline_time_ms = flops_gate / (bf16_peak * 1e12) * 1e3 + flops_fused / (FP32_SIMT_TFLOPS * 1e12) * 1e3
