@@ -32,6 +32,8 @@
 //     accumulates h_e * W_down[j] into its y registers.
 // h lives only in shared memory.  Results do not depend on which CTA or
 // group processes a token: no atomics touch data.
+#include <mutex>
+
 #include "sge_host.h"
 #include "sge_common.cuh"
 
@@ -551,4 +553,106 @@ extern "C" int twell_fused_up_down(const void* x, const uint8_t* count, const ui
   if (dtype == SGE_BF16) return dispatch_ud<true>(prm, st);
   if (dtype == SGE_F32) return dispatch_ud<false>(prm, st);
   return fail(SGE_ERR_UNSUPPORTED, "twell_fused_up_down: dtype %d", dtype);
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant.
+//
+// Some callers cannot allocate device memory for a workspace: code that runs
+// where no allocator may be called (an embedding runtime that forbids
+// cudaMalloc after start-up, a memory-capped inference server that has
+// handed all device memory to its own pools, a plugin that receives only the
+// tensors it works on).  For them the workspace of twell_fused_up_down lives
+// in this file-scope device array instead, sized for at most
+// kNoAllocMaxTokens tokens; every GPU that loads the library holds it until
+// the process exits.  In host code `g_fused_scratch` names a host-side stand-in,
+// not a device address, so its device address is looked up per device with
+// cudaGetSymbolAddress, once, with that device current.
+
+constexpr int64_t kNoAllocMaxTokens = 262144;
+constexpr size_t kNoAllocScratchBytes =
+    (kWsHeader + 5 * static_cast<size_t>(kNoAllocMaxTokens) + 15) & ~static_cast<size_t>(15);
+
+static __device__ __align__(256) uint8_t g_fused_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_fused_scratch on the current device (looked up once).
+int scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "twell_fused_up_down_noalloc: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(SGE_ERR_UNSUPPORTED, "twell_fused_up_down_noalloc: device %d beyond %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_fused_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(SGE_ERR_CUDA, "twell_fused_up_down_noalloc: cudaGetSymbolAddress: %s",
+                  cudaGetErrorString(e));
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return SGE_OK;
+}
+
+}  // namespace
+
+extern "C" int64_t twell_fused_up_down_noalloc_max_tokens(void) { return kNoAllocMaxTokens; }
+
+extern "C" int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, const uint8_t* idx,
+                                           const void* val, const void* wu_t, const void* wd,
+                                           void* y, int64_t n_tokens, int64_t d_model,
+                                           int64_t d_ff, int dtype, int tile, int cap,
+                                           void* stream) {
+  clear_error();
+  if (n_tokens < 0 || d_model < 1 || d_ff < 1)
+    return fail(SGE_ERR_ARG, "twell_fused_up_down_noalloc: bad sizes");
+  if (n_tokens > kNoAllocMaxTokens)
+    return fail(SGE_ERR_UNSUPPORTED,
+                "twell_fused_up_down_noalloc: %lld tokens exceed the built-in scratch limit of %lld; "
+                "use twell_fused_up_down with a workspace",
+                (long long)n_tokens, (long long)kNoAllocMaxTokens);
+  if (d_model % 8) return fail(SGE_ERR_ARG, "twell_fused_up_down_noalloc: d_model %% 8 != 0");
+  if (tile < 1 || tile > 255 || d_ff % tile)
+    return fail(SGE_ERR_ARG, "twell_fused_up_down_noalloc: tile must divide d_ff and be <= 255");
+  if (cap < 1 || cap > tile)
+    return fail(SGE_ERR_ARG, "twell_fused_up_down_noalloc: cap outside [1, tile]");
+  if (d_ff >= (1LL << 31)) return fail(SGE_ERR_UNSUPPORTED, "twell_fused_up_down_noalloc: d_ff beyond 2^31");
+  if (n_tokens == 0) return SGE_OK;
+  if (!x || !count || !idx || !val || !wu_t || !wd || !y)
+    return fail(SGE_ERR_ARG, "twell_fused_up_down_noalloc: null pointer");
+  if (!aligned16(x) || !aligned16(wu_t) || !aligned16(wd) || !aligned16(y) || !aligned16(val))
+    return fail(SGE_ERR_ARG, "twell_fused_up_down_noalloc: pointer not 16-byte aligned");
+  void* scratch = nullptr;
+  int rc = scratch_address(&scratch);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  UdParams prm;
+  prm.x = x;
+  prm.count = count;
+  prm.idx = idx;
+  prm.val = val;
+  prm.wu_t = wu_t;
+  prm.wd = wd;
+  prm.y = y;
+  prm.ws = static_cast<int*>(scratch);
+  prm.heavy_flag = static_cast<const uint8_t*>(scratch) + kWsHeader + 4 * static_cast<size_t>(n_tokens);
+  prm.n_rows = n_tokens;
+  prm.d = static_cast<int>(d_model);
+  prm.n_cols = static_cast<int>(d_ff);
+  prm.tile = tile;
+  prm.cap = cap;
+  // the array keeps the previous call's contents: the cursors start at zero
+  cudaError_t e = cudaMemsetAsync(scratch, 0, kWsHeader, st);
+  if (e != cudaSuccess)
+    return fail(SGE_ERR_CUDA, "twell_fused_up_down_noalloc: %s", cudaGetErrorString(e));
+  if (dtype == SGE_BF16) return dispatch_ud<true>(prm, st);
+  if (dtype == SGE_F32) return dispatch_ud<false>(prm, st);
+  return fail(SGE_ERR_UNSUPPORTED, "twell_fused_up_down_noalloc: dtype %d", dtype);
 }

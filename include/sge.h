@@ -137,6 +137,35 @@ int twell_fused_up_down(const void* x, const uint8_t* count, const uint8_t* idx,
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * twell_fused_up_down_noalloc -- twell_fused_up_down for callers that cannot
+ * allocate device memory.  The paper has no counterpart: this is a
+ * deployment convenience of this library.
+ *
+ * Some callers have no way to obtain a workspace: runtimes that forbid
+ * cudaMalloc once they are serving, servers that have given all device memory
+ * to their own pools, plugins that only receive the tensors they operate on.
+ * This entry point takes the same arguments as twell_fused_up_down minus the
+ * workspace and allocates nothing (no cudaMalloc, no cudaFree, no allocating
+ * library routine).  Its scratch is a fixed device array built into the
+ * library, sized for at most twell_fused_up_down_noalloc_max_tokens()
+ * tokens (262144; about 1.3 MB, held on every GPU that loads the library
+ * until the process exits).  Larger N is rejected with SGE_ERR_UNSUPPORTED.
+ *
+ * The first call on a device looks up the array's device address on that
+ * device (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  Every call shares the one array, so calls that may overlap on
+ * the GPU (different streams, or different host threads on the same device)
+ * race and must be serialised by the caller.  Results equal those of
+ * twell_fused_up_down.
+ */
+int64_t twell_fused_up_down_noalloc_max_tokens(void);
+
+int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, const uint8_t* idx,
+                                const void* val, const void* wu_t, const void* wd, void* y,
+                                int64_t n_tokens, int64_t d_model, int64_t d_ff, int dtype,
+                                int tile, int cap, void* stream);
+
+/*
  * dense_ffn_fwd -- the dense gated FFN the method is compared against
  * (pwwt.cn summary, lead and section 04: speed-ups are quoted against the
  * dense model).  bf16 only, on tcgen05 tensor cores:

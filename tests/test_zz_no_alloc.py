@@ -1,0 +1,68 @@
+"""The allocation-free fused up/down entry point.
+
+Callers that cannot allocate device memory (runtimes that forbid cudaMalloc
+while serving, servers whose memory is all in their own pools, plugins that
+only see their input and output tensors) use twell_fused_up_down_noalloc,
+whose scratch is a device array built into the library.  This file is
+collected last so that a run stopping at the first failure has already run
+every other test; it passes alone and after the others.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import activation_sparse_gated_epilogue_b200 as sge
+import oracle
+from activation_sparse_gated_epilogue_b200 import synth
+from tests._util import BF16_TOL
+
+pytestmark = pytest.mark.gpu
+
+
+def _noalloc_fn():
+    lib = sge.library()
+    fn = lib.twell_fused_up_down_noalloc
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    fn.restype = I
+    fn.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I, I, I, P]
+    lib.twell_fused_up_down_noalloc_max_tokens.restype = I64
+    return lib, fn
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def test_noalloc_matches_workspace_entry_point(cuda_device):
+    lib, fn = _noalloc_fn()
+    cfg = synth.CONFIGS["ffn_0p5b_bf16"]
+    inp = synth.make_inputs(cfg, n_tokens=2048)
+    x, wg, wu, wd = (getattr(inp, k).to(cuda_device) for k in ("x", "wg_t", "wu_t", "wd"))
+    x[:6, :-1] *= 8.0              # a few heavy tokens: both halves of the kernel run
+    tw = sge.twell_gate_pack(x, wg, cfg.tile, cfg.cap)
+    y_ref = sge.twell_fused_up_down(x, tw, wu, wd)
+    n, d = x.shape
+    f = wg.shape[0]
+    stream = ctypes.c_void_p(torch.cuda.current_stream(cuda_device).cuda_stream)
+    want = y_ref.double().cpu().numpy()
+    for call in range(2):           # the second call reuses the array's old contents
+        y = torch.full_like(x, float("nan"))
+        rc = fn(_ptr(x), _ptr(tw.count), _ptr(tw.idx), _ptr(tw.val), _ptr(wu), _ptr(wd), _ptr(y),
+                n, d, f, sge.SGE_BF16, tw.tile, tw.cap, stream)
+        assert rc == 0, lib.sge_last_error()
+        torch.cuda.synchronize()
+        got = y.double().cpu().numpy()
+        assert np.isfinite(got).all()
+        assert oracle.max_abs_rel(got, want) <= BF16_TOL, call
+
+
+def test_noalloc_rejects_more_tokens_than_its_scratch_holds(cuda_device):
+    lib, fn = _noalloc_fn()
+    limit = lib.twell_fused_up_down_noalloc_max_tokens()
+    assert limit >= 8192
+    p = ctypes.c_void_p(16)
+    rc = fn(p, p, p, p, p, p, p, limit + 1, 64, 256, sge.SGE_BF16, 128, 128, None)
+    assert rc == 2
+    assert b"scratch limit" in lib.sge_last_error()
