@@ -9,11 +9,11 @@ or a tensor is not on a CUDA device, the call raises.
 from .binding import (  # noqa: F401
     SGE_BF16, SGE_F32, TwELL, LibraryError, library, library_path,
     twell_gate_pack, twell_fused_up_down, twell_ffn_forward, dense_ffn_fwd, new_diag,
-    fused_workspace,
+    fused_workspace, Hybrid, hybrid_pack, hybrid_ffn_fwd, hybrid_fwd_workspace,
 )
 
 __all__ = [
     "SGE_BF16", "SGE_F32", "TwELL", "LibraryError", "library", "library_path",
     "twell_gate_pack", "twell_fused_up_down", "twell_ffn_forward", "dense_ffn_fwd", "new_diag",
-    "fused_workspace",
+    "fused_workspace", "Hybrid", "hybrid_pack", "hybrid_ffn_fwd", "hybrid_fwd_workspace",
 ]

@@ -22,6 +22,18 @@ _LIB_PATH = os.path.join(_HERE, "libsge.so")
 _lib = None
 
 
+class _SgeHybrid(ctypes.Structure):
+    """Mirror of `sge_hybrid` in include/sge.h."""
+    _fields_ = [("n_tokens", ctypes.c_int64), ("d_ff", ctypes.c_int64),
+                ("ell_cap", ctypes.c_int32), ("s_max", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("row_nnz", ctypes.c_void_p), ("spill_slot", ctypes.c_void_p),
+                ("spill_rows", ctypes.c_void_p), ("n_spill", ctypes.c_void_p),
+                ("ell_idx", ctypes.c_void_p), ("ell_a", ctypes.c_void_p),
+                ("ell_u", ctypes.c_void_p), ("spill_a", ctypes.c_void_p),
+                ("spill_u", ctypes.c_void_p)]
+
+
 class LibraryError(RuntimeError):
     """A C entry point returned an error code (message from sge_last_error)."""
 
@@ -52,6 +64,10 @@ def library() -> ctypes.CDLL:
             "twell_fused_up_down": (I, [P, P, P, P, P, P, P, I64, I64, I64, I, I, I, P,
                                         ctypes.c_size_t, P]),
             "dense_ffn_fwd": (I, [P, P, P, P, P, P, I64, I64, I64, P, P]),
+            "hybrid_pack": (I, [P, P, P, I, I, ctypes.POINTER(_SgeHybrid), P, P]),
+            "hybrid_ffn_fwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I]),
+            "hybrid_ffn_fwd": (I, [P, ctypes.POINTER(_SgeHybrid), P, P, P, P, I64, P,
+                                   ctypes.c_size_t, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -205,4 +221,82 @@ def dense_ffn_fwd(x: torch.Tensor, wg_t: torch.Tensor, wu_t: torch.Tensor, wd_t:
     _check(y, "y", torch.bfloat16, (n, d))
     _call("dense_ffn_fwd", _ptr(x), _ptr(wg_t), _ptr(wu_t), _ptr(wd_t), _ptr(h), _ptr(y),
           n, d, f, _ptr(diag), _stream(x.device, stream))
+    return y
+
+
+@dataclass
+class Hybrid:
+    """Device buffers of the hybrid format (see `sge_hybrid` in include/sge.h)."""
+    n_tokens: int
+    d_ff: int
+    ell_cap: int
+    s_max: int
+    row_nnz: torch.Tensor
+    spill_slot: torch.Tensor
+    spill_rows: torch.Tensor
+    n_spill: torch.Tensor
+    ell_idx: torch.Tensor
+    ell_a: torch.Tensor
+    ell_u: torch.Tensor
+    spill_a: torch.Tensor
+    spill_u: torch.Tensor
+
+    @staticmethod
+    def empty(n: int, f: int, ell_cap: int, s_max: int, device) -> "Hybrid":
+        kk, ss = max(ell_cap, 1), max(s_max, 1)
+        z = lambda *shape, dt: torch.empty(shape, dtype=dt, device=device)
+        return Hybrid(n, f, ell_cap, s_max, z(n, dt=torch.int32), z(n, dt=torch.int32),
+                      z(ss, dt=torch.int32), z(1, dt=torch.int32), z(n, kk, dt=torch.uint16),
+                      z(n, kk, dt=torch.bfloat16), z(n, kk, dt=torch.bfloat16),
+                      z(ss, f, dt=torch.bfloat16), z(ss, f, dt=torch.bfloat16))
+
+    def c_struct(self) -> _SgeHybrid:
+        for name in ("row_nnz", "spill_slot", "spill_rows", "n_spill", "ell_idx", "ell_a", "ell_u",
+                     "spill_a", "spill_u"):
+            _check(getattr(self, name), name)
+        return _SgeHybrid(self.n_tokens, self.d_ff, self.ell_cap, self.s_max, SGE_BF16, 0,
+                          self.row_nnz.data_ptr(), self.spill_slot.data_ptr(),
+                          self.spill_rows.data_ptr(), self.n_spill.data_ptr(),
+                          self.ell_idx.data_ptr(), self.ell_a.data_ptr(), self.ell_u.data_ptr(),
+                          self.spill_a.data_ptr(), self.spill_u.data_ptr())
+
+
+def hybrid_pack(tw: TwELL, ell_cap: int, s_max: int, out: Optional[Hybrid] = None,
+                diag: Optional[torch.Tensor] = None, stream=None) -> Hybrid:
+    """Route each row of a bf16 TwELL to the ELL part (nnz <= K) or the dense spill."""
+    _check(tw.count, "count", torch.uint8)
+    _check(tw.val, "val", torch.bfloat16)
+    n, f = tw.n_rows, tw.n_cols
+    if out is None:
+        out = Hybrid.empty(n, f, ell_cap, s_max, tw.count.device)
+    cs = out.c_struct()
+    _call("hybrid_pack", _ptr(tw.count), _ptr(tw.idx), _ptr(tw.val), tw.tile, tw.cap,
+          ctypes.byref(cs), _ptr(diag), _stream(tw.count.device, stream))
+    return out
+
+
+def hybrid_fwd_workspace(d_model: int, d_ff: int, s_max: int, device) -> torch.Tensor:
+    nbytes = library().hybrid_ffn_fwd_workspace_bytes(d_model, d_ff, s_max)
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
+def hybrid_ffn_fwd(x: torch.Tensor, hy: Hybrid, wu_t: torch.Tensor, wd: torch.Tensor,
+                   wd_t: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """y from the hybrid form; fills hy.ell_u and hy.spill_u."""
+    _check(x, "x", torch.bfloat16)
+    n, d = x.shape
+    f = hy.d_ff
+    _check(wu_t, "wu_t", torch.bfloat16, (f, d))
+    _check(wd, "wd", torch.bfloat16, (f, d))
+    if wd_t is None:
+        wd_t = wd.t().contiguous()
+    _check(wd_t, "wd_t", torch.bfloat16, (d, f))
+    if y is None:
+        y = torch.empty_like(x)
+    if workspace is None:
+        workspace = hybrid_fwd_workspace(d, f, hy.s_max, x.device)
+    cs = hy.c_struct()
+    _call("hybrid_ffn_fwd", _ptr(x), ctypes.byref(cs), _ptr(wu_t), _ptr(wd), _ptr(wd_t), _ptr(y), d,
+          _ptr(workspace), workspace.numel(), _stream(x.device, stream))
     return y

@@ -1,0 +1,475 @@
+// Hybrid sparse format for training: compact ELL rows plus a dense spill.
+//
+// "Sparser, Faster, Lighter Transformer Language Models": the pwwt.cn summary,
+// section 03 and figure "基于混合格式的稀疏矩阵算子路由计算逻辑", routes tokens
+// with few active gates to a highly compressed ELL matrix and the occasional
+// highly active token to a dense backup path run on tensor cores; the
+// kongchang.com page ("定制CUDA内核：融合与压缩") adds that TwELL is compressed
+// into this hybrid form to minimise activation storage.
+//
+//   hybrid_pack     TwELL -> row nnz, routing (nnz <= K: ELL row, else spill
+//                   row, spill rows numbered in ascending token order), ELL
+//                   columns and values, dense spill rows of a.
+//   hybrid_ffn_fwd  ELL rows: the fused sparse up/down (u saved for the
+//                   backward pass); spill rows: gathered and run as tcgen05
+//                   GEMMs, U = X_s W_up (u saved, h = a (.) u), Y_s = H_s W_down,
+//                   the rows scattered back into y.
+#include "sparse_common.cuh"
+#include "tc_launch.cuh"
+
+namespace sge {
+
+constexpr uint16_t kEllPad = 0xFFFF;
+constexpr int kPackThreads = 1024;
+
+struct HybridView {
+  int64_t n;
+  int f, k, s_max;
+  int32_t* row_nnz;
+  int32_t* spill_slot;
+  int32_t* spill_rows;
+  int32_t* n_spill;
+  uint16_t* ell_idx;
+  uint16_t* ell_a;
+  uint16_t* ell_u;
+  uint16_t* spill_a;
+  uint16_t* spill_u;
+};
+
+// ---------------------------------------------------------------- pack
+
+// One CTA: per-row stored entry counts, routing, and the ascending ranks of
+// the spill rows (block-wide exclusive scan over contiguous row ranges).
+__global__ void __launch_bounds__(kPackThreads)
+    hybrid_route_kernel(const uint8_t* __restrict__ count, int nt, int cap, HybridView hv,
+                        int32_t* diag) {
+  __shared__ int s_scan[kPackThreads];
+  const int tid = threadIdx.x;
+  const int64_t per = (hv.n + kPackThreads - 1) / kPackThreads;
+  const int64_t r0 = tid * per, r1 = min(hv.n, r0 + per);
+  int local = 0;
+  for (int64_t t = r0; t < r1; ++t) {
+    const uint8_t* c = count + t * nt;
+    int nnz = 0;
+    for (int b = 0; b < nt; ++b) nnz += min(static_cast<int>(c[b]), cap);
+    hv.row_nnz[t] = nnz;
+    local += nnz > hv.k;
+  }
+  s_scan[tid] = local;
+  __syncthreads();
+  for (int o = 1; o < kPackThreads; o <<= 1) {  // inclusive Hillis-Steele scan
+    const int v = tid >= o ? s_scan[tid - o] : 0;
+    __syncthreads();
+    s_scan[tid] += v;
+    __syncthreads();
+  }
+  int rank = s_scan[tid] - local;
+  for (int64_t t = r0; t < r1; ++t) {
+    int slot = -1;
+    if (hv.row_nnz[t] > hv.k) {
+      if (rank < hv.s_max) {
+        slot = rank;
+        hv.spill_rows[rank] = static_cast<int32_t>(t);
+      }
+      ++rank;
+    }
+    hv.spill_slot[t] = slot;
+  }
+  if (tid == kPackThreads - 1) {
+    const int total = s_scan[tid];
+    *hv.n_spill = total;
+    if (diag) {
+      atomicAdd(reinterpret_cast<int*>(diag + SGE_DIAG_SPILL_ROWS), total);
+      if (total > hv.s_max) atomicAdd(reinterpret_cast<int*>(diag + SGE_DIAG_DROPPED_ROWS), total - hv.s_max);
+    }
+  }
+}
+
+// One warp per row: ELL rows get their entries in ascending column order
+// (padding kEllPad / 0); kept spill rows get a dense row of a.
+__global__ void __launch_bounds__(256) hybrid_fill_kernel(const uint8_t* __restrict__ count,
+                                                          const uint8_t* __restrict__ idx,
+                                                          const uint16_t* __restrict__ val,
+                                                          int nt, int tile, int cap, HybridView hv) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= hv.n) return;
+  const int nnz = hv.row_nnz[t];
+  const bool ell = nnz <= hv.k;
+  const int slot = hv.spill_slot[t];
+  if (!ell && slot < 0) return;  // dropped
+  uint16_t* dense = ell ? nullptr : hv.spill_a + static_cast<int64_t>(slot) * hv.f;
+  if (!ell) {
+    for (int j = lane * 8; j < hv.f; j += 32 * 8) *reinterpret_cast<uint4*>(dense + j) = make_uint4(0, 0, 0, 0);
+    __syncwarp();
+  }
+  const uint8_t* c = count + t * nt;
+  int base = 0;
+  for (int b0 = 0; b0 < nt; b0 += 32) {
+    const int b = b0 + lane;
+    const int cb = b < nt ? min(static_cast<int>(c[b]), cap) : 0;
+    int incl = cb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int off = base + incl - cb;
+    const int64_t seg = t * nt + b;
+    for (int s = 0; s < cb; ++s) {
+      const int j = b * tile + idx[seg * cap + s];
+      const uint16_t a = val[seg * cap + s];
+      if (ell) {
+        hv.ell_idx[t * hv.k + off + s] = static_cast<uint16_t>(j);
+        hv.ell_a[t * hv.k + off + s] = a;
+      } else {
+        dense[j] = a;
+      }
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (ell)
+    for (int e = nnz + lane; e < hv.k; e += 32) {
+      hv.ell_idx[t * hv.k + e] = kEllPad;
+      hv.ell_a[t * hv.k + e] = 0;
+    }
+}
+
+// ------------------------------------------------------- ELL forward
+
+constexpr int kEllThreads = 128;
+constexpr int kEllWarps = kEllThreads / 32;
+constexpr int kEllMaxK = 512;
+constexpr int kEllBatch = 4;
+
+struct EllFwdParams {
+  const uint16_t* x;
+  const uint16_t* wu_t;
+  const uint16_t* wd;
+  uint16_t* y;
+  HybridView hv;
+  int d;
+};
+
+// One CTA per token.  ELL rows: u for every entry (saved to ell_u, rounded
+// to bf16), h = bf16(a u), y = sum h W_down[j].  Dropped rows: y = 0.  Spill
+// rows are left to the spill GEMMs.
+template <int NV>
+__global__ void __launch_bounds__(kEllThreads) hybrid_ell_fwd_kernel(EllFwdParams p) {
+  using E = Elem<true>;
+  constexpr int VEC = E::VEC;
+  __shared__ int s_j[kEllMaxK];
+  __shared__ float s_h[kEllMaxK];
+  __shared__ float s_up[kEllWarps][kEllMaxK];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t t = blockIdx.x;
+  const int nvec = p.d / VEC;
+  const int64_t row_bytes = static_cast<int64_t>(p.d) * 2;
+  const int nnz = p.hv.row_nnz[t];
+  uint4* yrow = reinterpret_cast<uint4*>(p.y + t * p.d);
+  if (nnz > p.hv.k) {
+    if (p.hv.spill_slot[t] < 0)
+      for (int v = tid; v < nvec; v += kEllThreads) yrow[v] = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  uint4 xv[NV];
+  float acc[NV][VEC];
+  const uint4* xrow = reinterpret_cast<const uint4*>(p.x + t * p.d);
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int v = tid + k * kEllThreads;
+    xv[k] = v < nvec ? __ldg(xrow + v) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int q = 0; q < VEC; ++q) acc[k][q] = 0.0f;
+  }
+  for (int e = tid; e < nnz; e += kEllThreads) {
+    s_j[e] = p.hv.ell_idx[t * p.hv.k + e];
+    s_h[e] = __uint_as_float(static_cast<uint32_t>(p.hv.ell_a[t * p.hv.k + e]) << 16);
+  }
+  __syncthreads();
+  // phase U
+  for (int e0 = 0; e0 < nnz; e0 += kEllBatch) {
+    uint4 w[kEllBatch][NV];
+#pragma unroll
+    for (int u = 0; u < kEllBatch; ++u) {
+      const int e = e0 + u;
+      const int j = e < nnz ? s_j[e] : -1;
+      const uint4* row = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wu_t) + static_cast<int64_t>(j) * row_bytes);
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int v = tid + k * kEllThreads;
+        w[u][k] = (j >= 0 && v < nvec) ? __ldg(row + v) : make_uint4(0, 0, 0, 0);
+      }
+    }
+    float part[kEllBatch];
+#pragma unroll
+    for (int u = 0; u < kEllBatch; ++u) {
+      float s = 0.0f;
+#pragma unroll
+      for (int k = 0; k < NV; ++k) s = E::dot(xv[k], w[u][k], s);
+      part[u] = s;
+    }
+    const float tot = warp_reduce_multi<kEllBatch>(part, lane);
+    if ((lane & (32 / kEllBatch - 1)) == 0) {
+      const int e = e0 + multi_entry<kEllBatch>(lane);
+      if (e < nnz) s_up[warp][e] = tot;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < nnz; e += kEllThreads) {
+    float u = 0.0f;
+#pragma unroll
+    for (int w8 = 0; w8 < kEllWarps; ++w8) u += s_up[w8][e];
+    p.hv.ell_u[t * p.hv.k + e] = f32_to_bf16_bits(u);
+    s_h[e] = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_bits(s_h[e] * u)) << 16);
+  }
+  __syncthreads();
+  // phase D
+  for (int e0 = 0; e0 < nnz; e0 += kEllBatch) {
+    uint4 w[kEllBatch][NV];
+    uint16_t hb[kEllBatch];
+#pragma unroll
+    for (int u = 0; u < kEllBatch; ++u) {
+      const int e = e0 + u;
+      const int j = e < nnz ? s_j[e] : -1;
+      hb[u] = e < nnz ? static_cast<uint16_t>(__float_as_uint(s_h[e]) >> 16) : 0;
+      const uint4* row = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wd) + static_cast<int64_t>(j) * row_bytes);
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int v = tid + k * kEllThreads;
+        w[u][k] = (j >= 0 && v < nvec) ? __ldg(row + v) : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kEllBatch; ++u)
+#pragma unroll
+      for (int k = 0; k < NV; ++k) E::axpy(hb[u], w[u][k], acc[k]);
+  }
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int v = tid + k * kEllThreads;
+    if (v < nvec) yrow[v] = E::pack(acc[k]);
+  }
+}
+
+// ------------------------------------------------------ spill forward
+
+// X_s[r] = x[spill_rows[r]] for the kept spill rows, zero rows after them.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ src,
+                                                          const int32_t* __restrict__ rows,
+                                                          const int32_t* __restrict__ n_rows_dev,
+                                                          int cap_rows, int d, uint16_t* dst) {
+  const int r = blockIdx.x;
+  const int kept = min(*n_rows_dev, cap_rows);
+  uint4* out = reinterpret_cast<uint4*>(dst + static_cast<int64_t>(r) * d);
+  const int nvec = d / 8;
+  if (r < kept) {
+    const uint4* in = reinterpret_cast<const uint4*>(src + static_cast<int64_t>(rows[r]) * d);
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) out[v] = __ldg(in + v);
+  } else {
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) out[v] = make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Epilogue of U = X_s W_up: spill_u = bf16(u), h = bf16(a u) -> hs.  Rows
+// past the kept spill rows are left untouched (their outputs are ignored).
+struct EpiSpillUp {
+  const uint16_t* spill_a;
+  uint16_t* spill_u;
+  uint16_t* hs;
+  const int32_t* n_spill;
+  int s_max;
+  int n_cols;
+
+  template <int BN>
+  __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {
+    const int kept = min(*n_spill, s_max);
+#pragma unroll 1
+    for (int ch = 0; ch < BN / 32; ++ch) {
+      uint32_t r[32];
+      tmem_ld32(taddr + ch * 32, r);
+      tmem_ld_wait();
+      const int col0 = n_blk * BN + ch * 32;
+      if (row >= kept) continue;
+      const int64_t off = row * n_cols + col0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (col0 + q * 8 + 8 > n_cols) break;
+        const uint4 av = *reinterpret_cast<const uint4*>(spill_a + off + q * 8);
+        const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+        uint32_t uw[4], hw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float u0 = __uint_as_float(r[q * 8 + 2 * i]);
+          const float u1 = __uint_as_float(r[q * 8 + 2 * i + 1]);
+          const float a0 = __uint_as_float(aw[i] << 16), a1 = __uint_as_float(aw[i] & 0xFFFF0000u);
+          uw[i] = static_cast<uint32_t>(f32_to_bf16_bits(u0)) | (static_cast<uint32_t>(f32_to_bf16_bits(u1)) << 16);
+          hw[i] = static_cast<uint32_t>(f32_to_bf16_bits(a0 * u0)) |
+                  (static_cast<uint32_t>(f32_to_bf16_bits(a1 * u1)) << 16);
+        }
+        *reinterpret_cast<uint4*>(spill_u + off + q * 8) = make_uint4(uw[0], uw[1], uw[2], uw[3]);
+        *reinterpret_cast<uint4*>(hs + off + q * 8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      }
+    }
+  }
+};
+
+// Epilogue of Y_s = H_s W_down: row r of the tile goes to y[spill_rows[r]].
+struct EpiScatterRows {
+  uint16_t* y;
+  const int32_t* rows;
+  const int32_t* n_spill;
+  int s_max;
+  int n_cols;
+
+  template <int BN>
+  __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {
+    const int kept = min(*n_spill, s_max);
+    const int64_t t = row < kept ? rows[row] : -1;
+#pragma unroll 1
+    for (int ch = 0; ch < BN / 32; ++ch) {
+      uint32_t r[32];
+      tmem_ld32(taddr + ch * 32, r);
+      tmem_ld_wait();
+      const int col0 = n_blk * BN + ch * 32;
+      if (t < 0) continue;
+      uint16_t* o = y + t * n_cols + col0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (col0 + q * 8 + 8 > n_cols) break;
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          w[i] = static_cast<uint32_t>(f32_to_bf16_bits(__uint_as_float(r[q * 8 + 2 * i]))) |
+                 (static_cast<uint32_t>(f32_to_bf16_bits(__uint_as_float(r[q * 8 + 2 * i + 1]))) << 16);
+        *reinterpret_cast<uint4*>(o + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+};
+
+static HybridView view_of(const sge_hybrid* h) {
+  HybridView v;
+  v.n = h->n_tokens;
+  v.f = static_cast<int>(h->d_ff);
+  v.k = h->ell_cap;
+  v.s_max = h->s_max;
+  v.row_nnz = h->row_nnz;
+  v.spill_slot = h->spill_slot;
+  v.spill_rows = h->spill_rows;
+  v.n_spill = h->n_spill;
+  v.ell_idx = h->ell_idx;
+  v.ell_a = static_cast<uint16_t*>(h->ell_a);
+  v.ell_u = static_cast<uint16_t*>(h->ell_u);
+  v.spill_a = static_cast<uint16_t*>(h->spill_a);
+  v.spill_u = static_cast<uint16_t*>(h->spill_u);
+  return v;
+}
+
+static int check_hybrid(const sge_hybrid* h, const char* fn) {
+  if (!h) return fail(SGE_ERR_ARG, "%s: null hybrid descriptor", fn);
+  if (h->n_tokens < 0 || h->d_ff < 1 || h->d_ff > 65535 || h->d_ff % 8)
+    return fail(SGE_ERR_ARG, "%s: d_ff must be in [8, 65535] and a multiple of 8", fn);
+  if (h->ell_cap < 0 || h->ell_cap > kEllMaxK)
+    return fail(SGE_ERR_UNSUPPORTED, "%s: ELL capacity %d outside [0, %d]", fn, h->ell_cap, kEllMaxK);
+  if (h->s_max < 0) return fail(SGE_ERR_ARG, "%s: negative spill capacity", fn);
+  if (h->dtype != SGE_BF16) return fail(SGE_ERR_UNSUPPORTED, "%s: the hybrid path is bf16 only", fn);
+  if (h->n_tokens == 0) return SGE_OK;
+  if (!h->row_nnz || !h->spill_slot || !h->n_spill || !h->ell_idx || !h->ell_a ||
+      (h->s_max > 0 && (!h->spill_rows || !h->spill_a)))
+    return fail(SGE_ERR_ARG, "%s: null hybrid buffer", fn);
+  if (!aligned16(h->spill_a) || !aligned16(h->spill_u))
+    return fail(SGE_ERR_ARG, "%s: spill buffers must be 16-byte aligned", fn);
+  return SGE_OK;
+}
+
+}  // namespace sge
+
+using namespace sge;
+
+extern "C" int hybrid_pack(const uint8_t* count, const uint8_t* idx, const void* val, int tile,
+                           int cap, sge_hybrid* hy, int32_t* diag, void* stream) {
+  clear_error();
+  int rc = check_hybrid(hy, "hybrid_pack");
+  if (rc) return rc;
+  if (tile < 1 || tile > 255 || hy->d_ff % tile || cap < 1 || cap > tile)
+    return fail(SGE_ERR_ARG, "hybrid_pack: bad TwELL tile %d / capacity %d", tile, cap);
+  if (hy->n_tokens == 0) return SGE_OK;
+  if (!count || !idx || !val) return fail(SGE_ERR_ARG, "hybrid_pack: null TwELL buffer");
+  if (hy->s_max > 0 && !aligned16(hy->spill_a))
+    return fail(SGE_ERR_ARG, "hybrid_pack: spill_a must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const HybridView hv = view_of(hy);
+  const int nt = static_cast<int>(hy->d_ff / tile);
+  hybrid_route_kernel<<<1, kPackThreads, 0, st>>>(count, nt, cap, hv, diag);
+  rc = check_launch("hybrid_pack (route)");
+  if (rc) return rc;
+  hybrid_fill_kernel<<<static_cast<unsigned>((hy->n_tokens + 7) / 8), 256, 0, st>>>(
+      count, idx, static_cast<const uint16_t*>(val), nt, tile, cap, hv);
+  return check_launch("hybrid_pack (fill)");
+}
+
+extern "C" size_t hybrid_ffn_fwd_workspace_bytes(int64_t d_model, int64_t d_ff, int s_max) {
+  if (d_model < 0 || d_ff < 0 || s_max < 0) return 0;
+  return static_cast<size_t>(s_max) * static_cast<size_t>(d_model + d_ff) * 2 + 256;
+}
+
+template <int NV>
+static int launch_ell_fwd(const EllFwdParams& p, int64_t n, cudaStream_t st) {
+  hybrid_ell_fwd_kernel<NV><<<static_cast<unsigned>(n), kEllThreads, 0, st>>>(p);
+  return check_launch("hybrid_ffn_fwd (ELL rows)");
+}
+
+extern "C" int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* wu_t, const void* wd,
+                              const void* wd_t, void* y, int64_t d_model, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  clear_error();
+  int rc = check_hybrid(hy, "hybrid_ffn_fwd");
+  if (rc) return rc;
+  if (d_model < 8 || d_model % 8) return fail(SGE_ERR_ARG, "hybrid_ffn_fwd: d_model %% 8 != 0");
+  if (hy->n_tokens == 0) return SGE_OK;
+  if (!x || !wu_t || !wd || !y || !hy->ell_u || (hy->s_max > 0 && (!wd_t || !hy->spill_u)))
+    return fail(SGE_ERR_ARG, "hybrid_ffn_fwd: null pointer");
+  if (!aligned16(x) || !aligned16(wu_t) || !aligned16(wd) || !aligned16(y) ||
+      (wd_t && !aligned16(wd_t)))
+    return fail(SGE_ERR_ARG, "hybrid_ffn_fwd: pointer not 16-byte aligned");
+  const size_t need = hybrid_ffn_fwd_workspace_bytes(d_model, hy->d_ff, hy->s_max);
+  if (hy->s_max > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(SGE_ERR_ARG, "hybrid_ffn_fwd: workspace of %zu bytes, %zu needed (16-byte aligned)",
+                workspace_bytes, need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const HybridView hv = view_of(hy);
+  EllFwdParams p{static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(wu_t),
+                 static_cast<const uint16_t*>(wd), static_cast<uint16_t*>(y), hv,
+                 static_cast<int>(d_model)};
+  const int64_t nvec = d_model / 8;
+  if (nvec <= kEllThreads) rc = launch_ell_fwd<1>(p, hy->n_tokens, st);
+  else if (nvec <= 2 * kEllThreads) rc = launch_ell_fwd<2>(p, hy->n_tokens, st);
+  else if (nvec <= 3 * kEllThreads) rc = launch_ell_fwd<3>(p, hy->n_tokens, st);
+  else if (nvec <= 4 * kEllThreads) rc = launch_ell_fwd<4>(p, hy->n_tokens, st);
+  else return fail(SGE_ERR_UNSUPPORTED, "hybrid_ffn_fwd: d_model %lld > 4096", (long long)d_model);
+  if (rc || hy->s_max == 0) return rc;
+
+  // spill rows: X_s gathered, U = X_s W_up (epilogue: u saved, h = a u),
+  // Y_s = H_s W_down scattered to y.
+  uint16_t* xs = static_cast<uint16_t*>(workspace);
+  uint16_t* hs = xs + static_cast<size_t>(hy->s_max) * d_model;
+  gather_rows_kernel<<<hy->s_max, 256, 0, st>>>(static_cast<const uint16_t*>(x), hy->spill_rows,
+                                                 hy->n_spill, hy->s_max, static_cast<int>(d_model), xs);
+  if ((rc = check_launch("hybrid_ffn_fwd (gather)"))) return rc;
+  using S = TcPairShape<256, 1>;
+  CUtensorMap ma, mb, mh, md;
+  if ((rc = make_tmap_bf16(&ma, xs, hy->s_max, d_model, d_model, kBM))) return rc;
+  if ((rc = make_tmap_bf16(&mb, wu_t, hy->d_ff, d_model, d_model, S::BN / 2))) return rc;
+  EpiSpillUp e1{static_cast<const uint16_t*>(hy->spill_a), static_cast<uint16_t*>(hy->spill_u), hs,
+                hy->n_spill, hy->s_max, static_cast<int>(hy->d_ff)};
+  if ((rc = launch_tc_gemm_pair<S>(ma, mb, mb, hy->s_max, hy->d_ff, d_model, e1, nullptr, st,
+                                   "hybrid_ffn_fwd (spill up)")))
+    return rc;
+  if ((rc = make_tmap_bf16(&mh, hs, hy->s_max, hy->d_ff, hy->d_ff, kBM))) return rc;
+  if ((rc = make_tmap_bf16(&md, wd_t, d_model, hy->d_ff, hy->d_ff, S::BN / 2))) return rc;
+  EpiScatterRows e2{static_cast<uint16_t*>(y), hy->spill_rows, hy->n_spill, hy->s_max,
+                    static_cast<int>(d_model)};
+  return launch_tc_gemm_pair<S>(mh, md, md, hy->s_max, d_model, hy->d_ff, e2, nullptr, st,
+                                "hybrid_ffn_fwd (spill down)");
+}

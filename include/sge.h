@@ -183,6 +183,78 @@ int dense_ffn_fwd(const void* x, const void* wg_t, const void* wu_t, const void*
                   void* y, int64_t n_tokens, int64_t d_model, int64_t d_ff, int32_t* diag,
                   void* stream);
 
+/*
+ * Hybrid format for training ("Sparser, Faster, Lighter Transformer Language
+ * Models", pwwt.cn summary, section 03 and figure "routing of the
+ * hybrid-format sparse operator": tokens with few active gates go to a
+ * compressed ELL matrix, rare highly active tokens to a dense backup path on
+ * tensor cores; kongchang.com page, "custom CUDA kernels: fusion and
+ * compression": TwELL is compressed into this hybrid form).  bf16 only.
+ *
+ * All buffers are caller-owned device memory described by this struct:
+ *   row_nnz    int32 [N]          stored entries of row t (sum of min(count, C))
+ *   spill_slot int32 [N]          rank of row t among the spill rows if
+ *                                 row_nnz > K and that rank < S_max, else -1
+ *   spill_rows int32 [S_max]      token of each kept spill row (ascending)
+ *   n_spill    int32 [1]          number of rows with row_nnz > K (may
+ *                                 exceed S_max; rows ranked >= S_max are
+ *                                 dropped: their y, dx and dW contributions
+ *                                 are zero and diag reports them)
+ *   ell_idx    uint16 [N][K]      columns of an ELL row's entries, ascending,
+ *                                 0xFFFF after row_nnz (requires F <= 65535)
+ *   ell_a      bf16 [N][K]        a = ReLU(g) of those entries, 0 after row_nnz
+ *   ell_u      bf16 [N][K]        u = x . W_up[:, j], written by hybrid_ffn_fwd
+ *   spill_a    bf16 [S_max][F]    dense a of each kept spill row
+ *   spill_u    bf16 [S_max][F]    dense u of each kept spill row, written by
+ *                                 hybrid_ffn_fwd
+ * ELL rows are rows with row_nnz <= K (ties go to ELL).
+ */
+typedef struct sge_hybrid {
+  int64_t n_tokens;
+  int64_t d_ff;
+  int32_t ell_cap; /* K, 0 <= K <= 512 */
+  int32_t s_max;   /* spill capacity in rows, >= 0 */
+  int32_t dtype;   /* SGE_BF16 */
+  int32_t reserved;
+  int32_t* row_nnz;
+  int32_t* spill_slot;
+  int32_t* spill_rows;
+  int32_t* n_spill;
+  uint16_t* ell_idx;
+  void* ell_a;
+  void* ell_u;
+  void* spill_a;
+  void* spill_u;
+} sge_hybrid;
+
+/*
+ * hybrid_pack -- compress a TwELL (count/idx/val with tile T and capacity C,
+ * as written by twell_gate_pack) into the hybrid form described by `hy`
+ * (which names N, F, K, S_max and the output buffers).  Deterministic:
+ * spill ranks follow ascending token order.  diag (nullable) gains the
+ * number of spill rows in [SGE_DIAG_SPILL_ROWS] and of dropped rows in
+ * [SGE_DIAG_DROPPED_ROWS].
+ */
+int hybrid_pack(const uint8_t* count, const uint8_t* idx, const void* val, int tile, int cap,
+                sge_hybrid* hy, int32_t* diag, void* stream);
+
+/*
+ * hybrid_ffn_fwd -- the gated FFN forward from the hybrid form, saving u.
+ *   ELL rows: y[t] = sum_e bf16(a_e u_e) W_down[j_e], u_e = x[t] . W_up[:, j_e]
+ *             (fp32 accumulation; u_e saved to ell_u in bf16)
+ *   spill rows: U = X_s W_up (all F columns, tcgen05), saved to spill_u;
+ *             H = bf16(A (.) U); Y_s = H W_down (tcgen05), scattered to y.
+ *   dropped rows: y = 0.
+ *   x [N][d], y [N][d], wu_t [F][d], wd [F][d], wd_t [d][F] (W_down
+ *   transposed, the K-major operand of the spill GEMM; may be NULL when
+ *   S_max == 0); workspace >= hybrid_ffn_fwd_workspace_bytes(d, F, S_max).
+ */
+size_t hybrid_ffn_fwd_workspace_bytes(int64_t d_model, int64_t d_ff, int s_max);
+
+int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* wu_t, const void* wd,
+                   const void* wd_t, void* y, int64_t d_model, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

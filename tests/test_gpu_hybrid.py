@@ -1,0 +1,104 @@
+"""GPU parity of the hybrid training format (pack and forward) against the
+fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import activation_sparse_gated_epilogue_b200 as sge
+import oracle
+from activation_sparse_gated_epilogue_b200 import synth
+from tests._util import BF16_TOL, compare_twell_inexact, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _small_inputs(n=300, d=256, f=1024, seed=0):
+    cfg = synth.CONFIGS["train_1b_hybrid"].with_(n_tokens=n, d_model=d, d_ff=f, spill_frac=None,
+                                                 rho=0.02, seed=seed)
+    return synth.make_inputs(cfg)
+
+
+def _upload_twell(tw: oracle.TwELL, dev):
+    return sge.TwELL(torch.from_numpy(tw.count).to(dev), torch.from_numpy(tw.idx).to(dev),
+                     torch.from_numpy(tw.val).to(torch.bfloat16).to(dev), tw.tile, tw.cap)
+
+
+def _check_pack(hy: sge.Hybrid, ora: oracle.Hybrid):
+    np.testing.assert_array_equal(hy.row_nnz.cpu().numpy(), ora.row_nnz)
+    np.testing.assert_array_equal(hy.spill_slot.cpu().numpy(), ora.spill_slot)
+    assert int(hy.n_spill.item()) == ora.n_spill
+    kept = min(ora.n_spill, ora.s_max)
+    np.testing.assert_array_equal(hy.spill_rows.cpu().numpy()[:kept], ora.spill_rows[:kept])
+    k = ora.k
+    if k > 0:
+        ell = ora.row_nnz <= k
+        gidx = hy.ell_idx.cpu().numpy().astype(np.int64)[:, :k]
+        gidx[gidx == 0xFFFF] = -1
+        np.testing.assert_array_equal(gidx[ell], ora.ell_idx[ell])
+        np.testing.assert_array_equal(to_f64(hy.ell_a)[:, :k][ell], ora.ell_a[ell])
+    if kept:
+        np.testing.assert_array_equal(to_f64(hy.spill_a)[:kept], ora.spill_a[:kept])
+
+
+@pytest.mark.parametrize("k,s_max", [(16, 64), (16, 4), (0, 300), (512, 8), (40, 32)])
+def test_hybrid_pack_and_fwd_match_oracle(cuda_device, k, s_max):
+    inp = _small_inputs()
+    x, wg, wu, wd = (inp.as_f64(n) for n in ("x", "wg_t", "wu_t", "wd"))
+    x[:7, :-1] *= 3.0                                     # a few heavy rows
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    x = xb.double().numpy()
+    tw = oracle.twell_pack(oracle.gate_preact(x, wg), 128, 128, oracle.VAL_BF16)
+    ora = oracle.hybrid_pack(tw, k, s_max)
+    y_ora = oracle.hybrid_fwd(x, ora, wu, wd)
+
+    diag = sge.new_diag(cuda_device)
+    hy = sge.hybrid_pack(_upload_twell(tw, cuda_device), k, s_max, diag=diag)
+    torch.cuda.synchronize()
+    _check_pack(hy, ora)
+    assert int(diag[1]) == ora.n_spill
+    assert int(diag[2]) == ora.dropped
+
+    y = sge.hybrid_ffn_fwd(xb.to(cuda_device), hy, inp.wu_t.to(cuda_device), inp.wd.to(cuda_device))
+    torch.cuda.synchronize()
+    err = oracle.max_abs_rel(to_f64(y), y_ora)
+    assert err <= BF16_TOL, err
+    if k > 0:
+        ell = ora.row_nnz <= k
+        gu = to_f64(hy.ell_u)[:, :k][ell]
+        mask = np.arange(k)[None, :] < ora.row_nnz[ell][:, None]
+        assert oracle.max_abs_rel(gu[mask], ora.ell_u[ell][mask]) <= 1e-2
+    kept = min(ora.n_spill, s_max)
+    if kept:
+        assert oracle.max_abs_rel(to_f64(hy.spill_u)[:kept], ora.spill_u[:kept]) <= 1e-2
+    dropped = (ora.row_nnz > k) & (ora.spill_slot < 0)
+    assert np.all(to_f64(y)[dropped] == 0.0)
+
+
+def test_hybrid_train_workload_sampled(cuda_device):
+    """The full training-shaped workload (N=8192, d=2048, F=8192, K=128,
+    S_max=1024): gate GEMM + TwELL, hybrid pack, hybrid forward on the GPU;
+    the oracle checks sampled ELL and spill rows."""
+    cfg = synth.CONFIGS["train_1b_hybrid"]
+    inp = synth.make_inputs(cfg)
+    dev = cuda_device
+    x, wg, wu, wd = (getattr(inp, n).to(dev) for n in ("x", "wg_t", "wu_t", "wd"))
+    tw = sge.twell_gate_pack(x, wg, cfg.tile, cfg.cap)
+    diag = sge.new_diag(dev)
+    hy = sge.hybrid_pack(tw, cfg.ell_cap, cfg.s_max, diag=diag)
+    y = sge.hybrid_ffn_fwd(x, hy, wu, wd)
+    torch.cuda.synchronize()
+    n_spill = int(hy.n_spill.item())
+    assert 0 < n_spill <= cfg.s_max, n_spill        # a few % of rows spill, none dropped
+    nnz = hy.row_nnz.cpu().numpy()
+    spill_rows = np.flatnonzero(nnz > cfg.ell_cap)
+    ell_rows = np.flatnonzero(nnz <= cfg.ell_cap)
+    rows = np.unique(np.concatenate([spill_rows[:6], spill_rows[-2:], ell_rows[::512]]))
+    xf, wgf, wuf, wdf = (inp.as_f64(n) for n in ("x", "wg_t", "wu_t", "wd"))
+    y_ora, tw_ora, g = oracle.sparse_ffn(xf[rows], wgf, wuf, wdf, cfg.tile, cfg.cap, oracle.VAL_BF16)
+    abs_sum = np.abs(xf[rows]) @ np.abs(wgf).T
+    bad_rows, _ = compare_twell_inexact(tw, tw_ora, g, oracle.VAL_BF16, abs_sum, rows=rows)
+    ok = ~bad_rows
+    assert ok.sum() >= len(rows) - 2
+    err = oracle.max_abs_rel(to_f64(y)[rows][ok], y_ora[ok])
+    assert err <= BF16_TOL, err
+    print(f"train hybrid: {n_spill} spill rows, max-abs-rel {err:.2e} on {ok.sum()} rows")
