@@ -68,6 +68,9 @@ def library() -> ctypes.CDLL:
             "hybrid_ffn_fwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I]),
             "hybrid_ffn_fwd": (I, [P, ctypes.POINTER(_SgeHybrid), P, P, P, P, I64, P,
                                    ctypes.c_size_t, P]),
+            "hybrid_ffn_bwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I64, I, I]),
+            "hybrid_ffn_bwd": (I, [P, P, ctypes.POINTER(_SgeHybrid), P, P, P, P, P, P, P, I64, P,
+                                   ctypes.c_size_t, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -300,3 +303,31 @@ def hybrid_ffn_fwd(x: torch.Tensor, hy: Hybrid, wu_t: torch.Tensor, wd: torch.Te
     _call("hybrid_ffn_fwd", _ptr(x), ctypes.byref(cs), _ptr(wu_t), _ptr(wd), _ptr(wd_t), _ptr(y), d,
           _ptr(workspace), workspace.numel(), _stream(x.device, stream))
     return y
+
+
+def hybrid_bwd_workspace(n_tokens: int, d_model: int, d_ff: int, ell_cap: int, s_max: int,
+                         device) -> torch.Tensor:
+    nbytes = library().hybrid_ffn_bwd_workspace_bytes(n_tokens, d_model, d_ff, ell_cap, s_max)
+    # 256-byte alignment: the caching allocator hands out 512-byte aligned blocks
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def hybrid_ffn_bwd(x: torch.Tensor, dy: torch.Tensor, hy: Hybrid, wg_t: torch.Tensor,
+                   wu_t: torch.Tensor, wd: torch.Tensor, workspace: Optional[torch.Tensor] = None,
+                   stream=None):
+    """Returns (dx bf16 [N][d], dwg_t, dwu_t, dwd fp32 [F][d])."""
+    _check(x, "x", torch.bfloat16)
+    n, d = x.shape
+    f = hy.d_ff
+    _check(dy, "dy", torch.bfloat16, (n, d))
+    for name, w in (("wg_t", wg_t), ("wu_t", wu_t), ("wd", wd)):
+        _check(w, name, torch.bfloat16, (f, d))
+    dx = torch.empty_like(x)
+    grads = [torch.empty((f, d), dtype=torch.float32, device=x.device) for _ in range(3)]
+    if workspace is None:
+        workspace = hybrid_bwd_workspace(n, d, f, hy.ell_cap, hy.s_max, x.device)
+    cs = hy.c_struct()
+    _call("hybrid_ffn_bwd", _ptr(x), _ptr(dy), ctypes.byref(cs), _ptr(wg_t), _ptr(wu_t), _ptr(wd),
+          _ptr(dx), _ptr(grads[0]), _ptr(grads[1]), _ptr(grads[2]), d, _ptr(workspace),
+          workspace.numel(), _stream(x.device, stream))
+    return (dx, *grads)

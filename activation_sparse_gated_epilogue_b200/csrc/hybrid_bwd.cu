@@ -1,0 +1,675 @@
+// Backward pass of the gated FFN from the hybrid format.
+//
+// "Sparser, Faster, Lighter Transformer Language Models", pwwt.cn summary,
+// section 03: training routes low-activity tokens to the compact ELL matrix
+// and heavy tokens to a dense path on tensor cores, cutting dense compute and
+// activation storage.  The pages print no backward formulas; these are the
+// derivatives of y = sum_j a_j u_j W_down[j] with a_j = ReLU(g_j) > 0 at every
+// stored entry (so dReLU = 1 there and entries not stored contribute 0):
+//   dh_j = dy . W_down[j]     du_j = dh_j a_j     dg_j = dh_j u_j
+//   dx   = sum_j du_j W_up[:, j] + dg_j W_gate[:, j]
+//   dW_down[j] += a_j u_j dy   dW_up[:, j] += du_j x   dW_gate[:, j] += dg_j x
+//
+// ELL rows: one CTA per token computes dh (dot products with rows of
+// W_down), du, dg (kept in fp32 for the weight gradients) and dx.  Weight
+// gradients of the ELL entries are summed per hidden unit over its tokens in
+// ascending token order: entries are bucketed by column (counting sort) and
+// each column's bucket is ordered by token, so the result is deterministic.
+// Spill rows: dense tcgen05 GEMMs on the gathered rows,
+//   dH = dY_s W_down^T (epilogue: dU = dH a, dG = dH u [a > 0], H = a u),
+//   dX_s = [dU | dG] [W_up ; W_gate]^T (scattered to dx),
+//   dW_down += H^T dY_s,  [dW_up ; dW_gate] += [dU | dG]^T X_s,
+// with the small operands transposed in the workspace so that every GEMM
+// reads K-major tiles.
+#include "sparse_common.cuh"
+#include "tc_launch.cuh"
+
+namespace sge {
+
+constexpr int kBwdThreads = 128;
+constexpr int kBwdWarps = kBwdThreads / 32;
+constexpr int kBwdMaxK = 512;
+constexpr int kBwdBatch = 4;
+
+struct BwdHybrid {
+  int64_t n;
+  int f, k, s_max;
+  const int32_t* row_nnz;
+  const int32_t* spill_slot;
+  const int32_t* spill_rows;
+  const int32_t* n_spill;
+  const uint16_t* ell_idx;
+  const uint16_t* ell_a;
+  const uint16_t* ell_u;
+  const uint16_t* spill_a;
+  const uint16_t* spill_u;
+};
+
+// Workspace carve-up (each piece 256-byte aligned).
+struct BwdWs {
+  float* du;         // [N][K]
+  float* dg;         // [N][K]
+  int* col_count;    // [F]
+  int* col_start;    // [F + 1]
+  int* col_cursor;   // [F]
+  int2* csc;         // [N * K] (token, slot), bucketed by column
+  int2* csc_sorted;  // [N * K] same, ascending token within a column
+  uint16_t* dys;     // [Sp][d]   gathered dy of the kept spill rows
+  uint16_t* xs;      // [Sp][d]   gathered x
+  uint16_t* acat;    // [Sp][2F]  dU | dG
+  uint16_t* hs;      // [Sp][F]   H = a u
+  uint16_t* acat_t;  // [2F][Sp]
+  uint16_t* hs_t;    // [F][Sp]
+  uint16_t* dys_t;   // [d][Sp]
+  uint16_t* xs_t;    // [d][Sp]
+  uint16_t* bcat;    // [d][2F]   W_up | W_gate (row i = row i of W_up, W_gate)
+  size_t bytes;
+};
+
+static size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+static BwdWs carve(void* base, int64_t n, int64_t d, int64_t f, int k, int s_max) {
+  BwdWs w{};
+  const int64_t sp = (s_max + 63) / 64 * 64;  // spill rows padded for 16-byte TMA pitches
+  char* p = static_cast<char*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* q = p ? p + off : nullptr;
+    off += align256(bytes);
+    return q;
+  };
+  const size_t nk = static_cast<size_t>(n) * static_cast<size_t>(k > 0 ? k : 1);
+  w.du = reinterpret_cast<float*>(take(nk * 4));
+  w.dg = reinterpret_cast<float*>(take(nk * 4));
+  w.col_count = reinterpret_cast<int*>(take(f * 4));
+  w.col_start = reinterpret_cast<int*>(take((f + 1) * 4));
+  w.col_cursor = reinterpret_cast<int*>(take(f * 4));
+  w.csc = reinterpret_cast<int2*>(take(nk * 8));
+  w.csc_sorted = reinterpret_cast<int2*>(take(nk * 8));
+  if (s_max > 0) {
+    w.dys = reinterpret_cast<uint16_t*>(take(sp * d * 2));
+    w.xs = reinterpret_cast<uint16_t*>(take(sp * d * 2));
+    w.acat = reinterpret_cast<uint16_t*>(take(sp * 2 * f * 2));
+    w.hs = reinterpret_cast<uint16_t*>(take(sp * f * 2));
+    w.acat_t = reinterpret_cast<uint16_t*>(take(2 * f * sp * 2));
+    w.hs_t = reinterpret_cast<uint16_t*>(take(f * sp * 2));
+    w.dys_t = reinterpret_cast<uint16_t*>(take(d * sp * 2));
+    w.xs_t = reinterpret_cast<uint16_t*>(take(d * sp * 2));
+    w.bcat = reinterpret_cast<uint16_t*>(take(d * 2 * f * 2));
+  }
+  w.bytes = off;
+  return w;
+}
+
+// ---------------------------------------------------------- ELL rows
+
+struct EllBwdParams {
+  const uint16_t* x;
+  const uint16_t* dy;
+  const uint16_t* wg_t;
+  const uint16_t* wu_t;
+  const uint16_t* wd;
+  uint16_t* dx;
+  BwdHybrid hv;
+  BwdWs ws;
+  int d;
+};
+
+template <int NV>
+__global__ void __launch_bounds__(kBwdThreads) ell_bwd_kernel(EllBwdParams p) {
+  using E = Elem<true>;
+  constexpr int VEC = E::VEC;
+  __shared__ int s_j[kBwdMaxK];
+  __shared__ float s_c[2][kBwdMaxK];  // (a, u) -> (du, dg) rounded for dx
+  __shared__ float s_part[kBwdWarps][kBwdMaxK];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t t = blockIdx.x;
+  const int nvec = p.d / VEC;
+  const int64_t row_bytes = static_cast<int64_t>(p.d) * 2;
+  const int nnz = p.hv.row_nnz[t];
+  uint4* dxrow = reinterpret_cast<uint4*>(p.dx + t * p.d);
+  if (nnz > p.hv.k) {  // spill rows: dx from the spill GEMMs; dropped rows: 0
+    if (p.hv.spill_slot[t] < 0)
+      for (int v = tid; v < nvec; v += kBwdThreads) dxrow[v] = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  uint4 dyv[NV];
+  float acc[NV][VEC];
+  const uint4* dyrow = reinterpret_cast<const uint4*>(p.dy + t * p.d);
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int v = tid + k * kBwdThreads;
+    dyv[k] = v < nvec ? __ldg(dyrow + v) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int q = 0; q < VEC; ++q) acc[k][q] = 0.0f;
+  }
+  const int64_t rk = t * p.hv.k;
+  for (int e = tid; e < nnz; e += kBwdThreads) {
+    s_j[e] = p.hv.ell_idx[rk + e];
+    s_c[0][e] = __uint_as_float(static_cast<uint32_t>(p.hv.ell_a[rk + e]) << 16);
+    s_c[1][e] = __uint_as_float(static_cast<uint32_t>(p.hv.ell_u[rk + e]) << 16);
+  }
+  __syncthreads();
+  // dh_e = dy . W_down[j_e]
+  for (int e0 = 0; e0 < nnz; e0 += kBwdBatch) {
+    uint4 w[kBwdBatch][NV];
+#pragma unroll
+    for (int u = 0; u < kBwdBatch; ++u) {
+      const int e = e0 + u;
+      const int j = e < nnz ? s_j[e] : -1;
+      const uint4* row = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wd) + static_cast<int64_t>(j) * row_bytes);
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int v = tid + k * kBwdThreads;
+        w[u][k] = (j >= 0 && v < nvec) ? __ldg(row + v) : make_uint4(0, 0, 0, 0);
+      }
+    }
+    float part[kBwdBatch];
+#pragma unroll
+    for (int u = 0; u < kBwdBatch; ++u) {
+      float s = 0.0f;
+#pragma unroll
+      for (int k = 0; k < NV; ++k) s = E::dot(dyv[k], w[u][k], s);
+      part[u] = s;
+    }
+    const float tot = warp_reduce_multi<kBwdBatch>(part, lane);
+    if ((lane & (32 / kBwdBatch - 1)) == 0) {
+      const int e = e0 + multi_entry<kBwdBatch>(lane);
+      if (e < nnz) s_part[warp][e] = tot;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < nnz; e += kBwdThreads) {
+    float dh = 0.0f;
+#pragma unroll
+    for (int w8 = 0; w8 < kBwdWarps; ++w8) dh += s_part[w8][e];
+    const float du = dh * s_c[0][e], dg = dh * s_c[1][e];
+    p.ws.du[rk + e] = du;
+    p.ws.dg[rk + e] = dg;
+    s_c[0][e] = du;
+    s_c[1][e] = dg;
+  }
+  __syncthreads();
+  // dx = sum du W_up[:, j] + dg W_gate[:, j]  (coefficients rounded to bf16)
+  for (int e0 = 0; e0 < nnz; e0 += kBwdBatch) {
+    uint4 wu[kBwdBatch][NV], wg[kBwdBatch][NV];
+    uint16_t cu[kBwdBatch], cg[kBwdBatch];
+#pragma unroll
+    for (int u = 0; u < kBwdBatch; ++u) {
+      const int e = e0 + u;
+      const int j = e < nnz ? s_j[e] : -1;
+      cu[u] = e < nnz ? f32_to_bf16_bits(s_c[0][e]) : 0;
+      cg[u] = e < nnz ? f32_to_bf16_bits(s_c[1][e]) : 0;
+      const uint4* ru = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wu_t) + static_cast<int64_t>(j) * row_bytes);
+      const uint4* rg = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wg_t) + static_cast<int64_t>(j) * row_bytes);
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int v = tid + k * kBwdThreads;
+        const bool ok = j >= 0 && v < nvec;
+        wu[u][k] = ok ? __ldg(ru + v) : make_uint4(0, 0, 0, 0);
+        wg[u][k] = ok ? __ldg(rg + v) : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBwdBatch; ++u)
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        E::axpy(cu[u], wu[u][k], acc[k]);
+        E::axpy(cg[u], wg[u][k], acc[k]);
+      }
+  }
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int v = tid + k * kBwdThreads;
+    if (v < nvec) dxrow[v] = E::pack(acc[k]);
+  }
+}
+
+// ------------------------------------------------- column buckets (CSC)
+
+__global__ void __launch_bounds__(256) csc_count_kernel(BwdHybrid hv, int* col_count) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= hv.n) return;
+  const int nnz = hv.row_nnz[t];
+  if (nnz > hv.k) return;
+  for (int e = lane; e < nnz; e += 32) atomicAdd(&col_count[hv.ell_idx[t * hv.k + e]], 1);
+}
+
+// One CTA: exclusive scan of the column counts.
+__global__ void __launch_bounds__(1024) csc_scan_kernel(const int* col_count, int f, int* col_start,
+                                                        int* col_cursor) {
+  __shared__ int s[1024];
+  const int tid = threadIdx.x;
+  const int per = (f + 1023) / 1024;
+  const int c0 = tid * per, c1 = min(f, c0 + per);
+  int local = 0;
+  for (int c = c0; c < c1; ++c) local += col_count[c];
+  s[tid] = local;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {
+    const int v = tid >= o ? s[tid - o] : 0;
+    __syncthreads();
+    s[tid] += v;
+    __syncthreads();
+  }
+  int run = s[tid] - local;
+  for (int c = c0; c < c1; ++c) {
+    col_start[c] = run;
+    col_cursor[c] = run;
+    run += col_count[c];
+  }
+  if (tid == 1023) col_start[f] = s[1023];
+}
+
+__global__ void __launch_bounds__(256) csc_scatter_kernel(BwdHybrid hv, int* col_cursor, int2* csc) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= hv.n) return;
+  const int nnz = hv.row_nnz[t];
+  if (nnz > hv.k) return;
+  for (int e = lane; e < nnz; e += 32) {
+    const int pos = atomicAdd(&col_cursor[hv.ell_idx[t * hv.k + e]], 1);
+    csc[pos] = make_int2(static_cast<int>(t), e);
+  }
+}
+
+// Per column (one warp): order the bucket by token.  Tokens are unique in a
+// column, so an entry's position is the number of smaller tokens.
+__global__ void __launch_bounds__(256) csc_sort_kernel(const int* col_start, int f, const int2* csc,
+                                                       int2* sorted) {
+  const int c = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (c >= f) return;
+  const int s0 = col_start[c], n = col_start[c + 1] - s0;
+  for (int i = lane; i < n; i += 32) {
+    const int2 me = csc[s0 + i];
+    int rank = 0;
+    for (int m = 0; m < n; ++m) rank += csc[s0 + m].x < me.x;
+    sorted[s0 + rank] = me;
+  }
+}
+
+// Per column j (one CTA): weight-gradient rows from the ELL entries, summed
+// in ascending token order, written (overwriting) in fp32.
+struct DwParams {
+  const uint16_t* x;
+  const uint16_t* dy;
+  BwdHybrid hv;
+  BwdWs ws;
+  float* dwg_t;
+  float* dwu_t;
+  float* dwd;
+  int d;
+};
+
+template <int NV>
+__global__ void __launch_bounds__(kBwdThreads) dw_ell_kernel(DwParams p) {
+  constexpr int VEC = 8;
+  const int j = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int nvec = p.d / VEC;
+  float ad[NV][VEC], au[NV][VEC], ag[NV][VEC];
+#pragma unroll
+  for (int k = 0; k < NV; ++k)
+#pragma unroll
+    for (int q = 0; q < VEC; ++q) ad[k][q] = au[k][q] = ag[k][q] = 0.0f;
+  const int s0 = p.ws.col_start[j], s1 = p.ws.col_start[j + 1];
+  for (int i = s0; i < s1; ++i) {
+    const int2 te = p.ws.csc_sorted[i];
+    const int64_t rk = static_cast<int64_t>(te.x) * p.hv.k + te.y;
+    const float a = __uint_as_float(static_cast<uint32_t>(p.hv.ell_a[rk]) << 16);
+    const float u = __uint_as_float(static_cast<uint32_t>(p.hv.ell_u[rk]) << 16);
+    const float h = a * u, du = p.ws.du[rk], dg = p.ws.dg[rk];
+    const uint4* dyr = reinterpret_cast<const uint4*>(p.dy + static_cast<int64_t>(te.x) * p.d);
+    const uint4* xr = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(te.x) * p.d);
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+      const int v = tid + k * kBwdThreads;
+      if (v >= nvec) continue;
+      const uint4 yv = __ldg(dyr + v), xv = __ldg(xr + v);
+      const uint32_t ys[4] = {yv.x, yv.y, yv.z, yv.w}, xs[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float y0 = __uint_as_float(ys[q] << 16), y1 = __uint_as_float(ys[q] & 0xFFFF0000u);
+        const float x0 = __uint_as_float(xs[q] << 16), x1 = __uint_as_float(xs[q] & 0xFFFF0000u);
+        ad[k][2 * q] = fmaf(h, y0, ad[k][2 * q]);
+        ad[k][2 * q + 1] = fmaf(h, y1, ad[k][2 * q + 1]);
+        au[k][2 * q] = fmaf(du, x0, au[k][2 * q]);
+        au[k][2 * q + 1] = fmaf(du, x1, au[k][2 * q + 1]);
+        ag[k][2 * q] = fmaf(dg, x0, ag[k][2 * q]);
+        ag[k][2 * q + 1] = fmaf(dg, x1, ag[k][2 * q + 1]);
+      }
+    }
+  }
+  const int64_t base = static_cast<int64_t>(j) * p.d;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int v = tid + k * kBwdThreads;
+    if (v >= nvec) continue;
+    float4* od = reinterpret_cast<float4*>(p.dwd + base) + 2 * v;
+    float4* ou = reinterpret_cast<float4*>(p.dwu_t + base) + 2 * v;
+    float4* og = reinterpret_cast<float4*>(p.dwg_t + base) + 2 * v;
+    od[0] = make_float4(ad[k][0], ad[k][1], ad[k][2], ad[k][3]);
+    od[1] = make_float4(ad[k][4], ad[k][5], ad[k][6], ad[k][7]);
+    ou[0] = make_float4(au[k][0], au[k][1], au[k][2], au[k][3]);
+    ou[1] = make_float4(au[k][4], au[k][5], au[k][6], au[k][7]);
+    og[0] = make_float4(ag[k][0], ag[k][1], ag[k][2], ag[k][3]);
+    og[1] = make_float4(ag[k][4], ag[k][5], ag[k][6], ag[k][7]);
+  }
+}
+
+// -------------------------------------------------------- spill rows
+
+__global__ void __launch_bounds__(256) gather2_kernel(const uint16_t* __restrict__ a,
+                                                      const uint16_t* __restrict__ b,
+                                                      const int32_t* __restrict__ rows,
+                                                      const int32_t* __restrict__ n_rows_dev,
+                                                      int cap_rows, int d, uint16_t* da, uint16_t* db) {
+  const int r = blockIdx.x;
+  const int kept = min(*n_rows_dev, cap_rows);
+  const int nvec = d / 8;
+  uint4* oa = reinterpret_cast<uint4*>(da + static_cast<int64_t>(r) * d);
+  uint4* ob = reinterpret_cast<uint4*>(db + static_cast<int64_t>(r) * d);
+  if (r < kept) {
+    const uint4* ia = reinterpret_cast<const uint4*>(a + static_cast<int64_t>(rows[r]) * d);
+    const uint4* ib = reinterpret_cast<const uint4*>(b + static_cast<int64_t>(rows[r]) * d);
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      oa[v] = __ldg(ia + v);
+      ob[v] = __ldg(ib + v);
+    }
+  } else {
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      oa[v] = make_uint4(0, 0, 0, 0);
+      ob[v] = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
+// dst[c][col_off + r] = src[r][c] for r < rows, c < cols (bf16, 32x32 tiles).
+__global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restrict__ src, int rows,
+                                                        int cols, int64_t src_pitch, uint16_t* dst,
+                                                        int64_t dst_pitch, int col_off) {
+  __shared__ uint16_t tile[32][33];
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int i = ty; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + tx;
+    tile[i][tx] = (r < rows && c < cols) ? src[static_cast<int64_t>(r) * src_pitch + c] : 0;
+  }
+  __syncthreads();
+  for (int i = ty; i < 32; i += 8) {
+    const int c = c0 + i, r = r0 + tx;
+    if (c < cols && r < rows) dst[static_cast<int64_t>(c) * dst_pitch + col_off + r] = tile[tx][i];
+  }
+}
+
+// Epilogue of dH = dY_s W_down^T: dU = dH a, dG = dH u [a > 0] -> acat
+// (dU in columns [0, F), dG in [F, 2F)), H = a u -> hs; zero rows past the
+// kept spill rows so that they add nothing in the later GEMMs.
+struct EpiBwdSpill {
+  const uint16_t* spill_a;
+  const uint16_t* spill_u;
+  uint16_t* acat;
+  uint16_t* hs;
+  const int32_t* n_spill;
+  int s_max;
+  int f;
+  int64_t m_rows;  // rows of the padded spill buffers
+
+  template <int BN>
+  __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {
+    const int kept = min(*n_spill, s_max);
+#pragma unroll 1
+    for (int ch = 0; ch < BN / 32; ++ch) {
+      uint32_t r[32];
+      tmem_ld32(taddr + ch * 32, r);
+      tmem_ld_wait();
+      if (row >= m_rows) continue;
+      const int col0 = n_blk * BN + ch * 32;
+      const int64_t off = row * f + col0;
+      const int64_t offc = row * 2 * f + col0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (col0 + q * 8 + 8 > f) break;
+        uint32_t du[4] = {0, 0, 0, 0}, dg[4] = {0, 0, 0, 0}, hw[4] = {0, 0, 0, 0};
+        if (row < kept) {
+          const uint4 av = *reinterpret_cast<const uint4*>(spill_a + off + q * 8);
+          const uint4 uv = *reinterpret_cast<const uint4*>(spill_u + off + q * 8);
+          const uint32_t aw[4] = {av.x, av.y, av.z, av.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float o[2][3];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float dh = __uint_as_float(r[q * 8 + 2 * i + h]);
+              const float a = __uint_as_float(h ? (aw[i] & 0xFFFF0000u) : (aw[i] << 16));
+              const float u = __uint_as_float(h ? (uw[i] & 0xFFFF0000u) : (uw[i] << 16));
+              o[h][0] = dh * a;
+              o[h][1] = a > 0.0f ? dh * u : 0.0f;
+              o[h][2] = a * u;
+            }
+            du[i] = static_cast<uint32_t>(f32_to_bf16_bits(o[0][0])) | (static_cast<uint32_t>(f32_to_bf16_bits(o[1][0])) << 16);
+            dg[i] = static_cast<uint32_t>(f32_to_bf16_bits(o[0][1])) | (static_cast<uint32_t>(f32_to_bf16_bits(o[1][1])) << 16);
+            hw[i] = static_cast<uint32_t>(f32_to_bf16_bits(o[0][2])) | (static_cast<uint32_t>(f32_to_bf16_bits(o[1][2])) << 16);
+          }
+        }
+        *reinterpret_cast<uint4*>(acat + offc + q * 8) = make_uint4(du[0], du[1], du[2], du[3]);
+        *reinterpret_cast<uint4*>(acat + offc + f + q * 8) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+        *reinterpret_cast<uint4*>(hs + off + q * 8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      }
+    }
+  }
+};
+
+// Epilogue: out[row] += D (fp32).  Rows [0, split) go to out0, rows
+// [split, 2 split) to out1 (row - split).
+struct EpiAddF32 {
+  float* out0;
+  float* out1;
+  int64_t split;
+  int n_cols;
+
+  template <int BN>
+  __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {
+    float* out = row < split ? out0 + row * n_cols : (out1 ? out1 + (row - split) * n_cols : nullptr);
+    if (row >= 2 * split) out = nullptr;
+#pragma unroll 1
+    for (int ch = 0; ch < BN / 32; ++ch) {
+      uint32_t r[32];
+      tmem_ld32(taddr + ch * 32, r);
+      tmem_ld_wait();
+      const int col0 = n_blk * BN + ch * 32;
+      if (!out) continue;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (col0 + q * 4 + 4 > n_cols) break;
+        float4* o = reinterpret_cast<float4*>(out + col0 + q * 4);
+        float4 v = *o;
+        v.x += __uint_as_float(r[q * 4]);
+        v.y += __uint_as_float(r[q * 4 + 1]);
+        v.z += __uint_as_float(r[q * 4 + 2]);
+        v.w += __uint_as_float(r[q * 4 + 3]);
+        *o = v;
+      }
+    }
+  }
+};
+
+// Epilogue: row r of D goes to dst[rows[r]] (bf16) for the kept rows.
+struct EpiScatterRowsBwd {
+  uint16_t* dst;
+  const int32_t* rows;
+  const int32_t* n_spill;
+  int s_max;
+  int n_cols;
+
+  template <int BN>
+  __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {
+    const int kept = min(*n_spill, s_max);
+    const int64_t t = row < kept ? rows[row] : -1;
+#pragma unroll 1
+    for (int ch = 0; ch < BN / 32; ++ch) {
+      uint32_t r[32];
+      tmem_ld32(taddr + ch * 32, r);
+      tmem_ld_wait();
+      const int col0 = n_blk * BN + ch * 32;
+      if (t < 0) continue;
+      uint16_t* o = dst + t * n_cols + col0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (col0 + q * 8 + 8 > n_cols) break;
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          w[i] = static_cast<uint32_t>(f32_to_bf16_bits(__uint_as_float(r[q * 8 + 2 * i]))) |
+                 (static_cast<uint32_t>(f32_to_bf16_bits(__uint_as_float(r[q * 8 + 2 * i + 1]))) << 16);
+        *reinterpret_cast<uint4*>(o + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+};
+
+static int launch_transpose(const uint16_t* src, int rows, int cols, int64_t src_pitch,
+                            uint16_t* dst, int64_t dst_pitch, int col_off, cudaStream_t st) {
+  dim3 grid((cols + 31) / 32, (rows + 31) / 32);
+  transpose_kernel<<<grid, 256, 0, st>>>(src, rows, cols, src_pitch, dst, dst_pitch, col_off);
+  return check_launch("hybrid_ffn_bwd (transpose)");
+}
+
+template <int NV>
+static int launch_ell_bwd(const EllBwdParams& p, int64_t n, cudaStream_t st) {
+  ell_bwd_kernel<NV><<<static_cast<unsigned>(n), kBwdThreads, 0, st>>>(p);
+  return check_launch("hybrid_ffn_bwd (ELL rows)");
+}
+
+template <int NV>
+static int launch_dw(const DwParams& q, int f, cudaStream_t st) {
+  dw_ell_kernel<NV><<<f, kBwdThreads, 0, st>>>(q);
+  return check_launch("hybrid_ffn_bwd (weight gradients)");
+}
+
+}  // namespace sge
+
+using namespace sge;
+
+extern "C" size_t hybrid_ffn_bwd_workspace_bytes(int64_t n_tokens, int64_t d_model, int64_t d_ff,
+                                                 int ell_cap, int s_max) {
+  if (n_tokens < 0 || d_model < 0 || d_ff < 0 || ell_cap < 0 || s_max < 0) return 0;
+  return carve(nullptr, n_tokens, d_model, d_ff, ell_cap, s_max).bytes;
+}
+
+extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* hy,
+                              const void* wg_t, const void* wu_t, const void* wd, void* dx,
+                              float* dwg_t, float* dwu_t, float* dwd, int64_t d_model,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  clear_error();
+  if (!hy) return fail(SGE_ERR_ARG, "hybrid_ffn_bwd: null hybrid descriptor");
+  if (hy->dtype != SGE_BF16) return fail(SGE_ERR_UNSUPPORTED, "hybrid_ffn_bwd: bf16 only");
+  if (hy->n_tokens < 0 || hy->d_ff < 8 || hy->d_ff > 65535 || hy->d_ff % 8 || hy->ell_cap < 0 ||
+      hy->ell_cap > kBwdMaxK || hy->s_max < 0)
+    return fail(SGE_ERR_ARG, "hybrid_ffn_bwd: bad hybrid sizes");
+  if (d_model < 8 || d_model % 8) return fail(SGE_ERR_ARG, "hybrid_ffn_bwd: d_model %% 8 != 0");
+  if (d_model > 4 * kBwdThreads * 8)
+    return fail(SGE_ERR_UNSUPPORTED, "hybrid_ffn_bwd: d_model %lld > 4096", (long long)d_model);
+  const int64_t n = hy->n_tokens, f = hy->d_ff, d = d_model;
+  const int k = hy->ell_cap, s_max = hy->s_max;
+  if (!x || !dy || !wg_t || !wu_t || !wd || !dx || !dwg_t || !dwu_t || !dwd)
+    return fail(SGE_ERR_ARG, "hybrid_ffn_bwd: null pointer");
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(wg_t) || !aligned16(wu_t) || !aligned16(wd) ||
+      !aligned16(dx) || !aligned16(dwg_t) || !aligned16(dwu_t) || !aligned16(dwd))
+    return fail(SGE_ERR_ARG, "hybrid_ffn_bwd: pointer not 16-byte aligned");
+  const BwdWs need = carve(nullptr, n, d, f, k, s_max);
+  if (!workspace || workspace_bytes < need.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return fail(SGE_ERR_ARG, "hybrid_ffn_bwd: workspace of %zu bytes, %zu needed (256-byte aligned)",
+                workspace_bytes, need.bytes);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const BwdWs ws = carve(workspace, n, d, f, k, s_max);
+  BwdHybrid hv{n, static_cast<int>(f), k, s_max, hy->row_nnz, hy->spill_slot, hy->spill_rows,
+               hy->n_spill, hy->ell_idx, static_cast<const uint16_t*>(hy->ell_a),
+               static_cast<const uint16_t*>(hy->ell_u), static_cast<const uint16_t*>(hy->spill_a),
+               static_cast<const uint16_t*>(hy->spill_u)};
+  const auto* xb = static_cast<const uint16_t*>(x);
+  const auto* dyb = static_cast<const uint16_t*>(dy);
+  int rc;
+  if (n > 0) {
+    // ---- ELL rows: dh, du, dg, dx
+    EllBwdParams p{xb, dyb, static_cast<const uint16_t*>(wg_t), static_cast<const uint16_t*>(wu_t),
+                   static_cast<const uint16_t*>(wd), static_cast<uint16_t*>(dx), hv, ws,
+                   static_cast<int>(d)};
+    DwParams q{xb, dyb, hv, ws, dwg_t, dwu_t, dwd, static_cast<int>(d)};
+    const int64_t nvec = d / 8;
+    if (nvec <= kBwdThreads) rc = launch_ell_bwd<1>(p, n, st);
+    else if (nvec <= 2 * kBwdThreads) rc = launch_ell_bwd<2>(p, n, st);
+    else if (nvec <= 3 * kBwdThreads) rc = launch_ell_bwd<3>(p, n, st);
+    else rc = launch_ell_bwd<4>(p, n, st);
+    if (rc) return rc;
+    // ---- column buckets of the ELL entries, ordered by token
+    cudaError_t e = cudaMemsetAsync(ws.col_count, 0, sizeof(int) * f, st);
+    if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "hybrid_ffn_bwd: %s", cudaGetErrorString(e));
+    const unsigned rb = static_cast<unsigned>((n + 7) / 8);
+    csc_count_kernel<<<rb, 256, 0, st>>>(hv, ws.col_count);
+    csc_scan_kernel<<<1, 1024, 0, st>>>(ws.col_count, static_cast<int>(f), ws.col_start, ws.col_cursor);
+    csc_scatter_kernel<<<rb, 256, 0, st>>>(hv, ws.col_cursor, ws.csc);
+    csc_sort_kernel<<<static_cast<unsigned>((f + 7) / 8), 256, 0, st>>>(ws.col_start, static_cast<int>(f),
+                                                                       ws.csc, ws.csc_sorted);
+    if ((rc = check_launch("hybrid_ffn_bwd (column buckets)"))) return rc;
+    // ---- weight gradients of the ELL entries (overwrite)
+    if (nvec <= kBwdThreads) rc = launch_dw<1>(q, static_cast<int>(f), st);
+    else if (nvec <= 2 * kBwdThreads) rc = launch_dw<2>(q, static_cast<int>(f), st);
+    else if (nvec <= 3 * kBwdThreads) rc = launch_dw<3>(q, static_cast<int>(f), st);
+    else rc = launch_dw<4>(q, static_cast<int>(f), st);
+    if (rc) return rc;
+  } else {
+    cudaMemsetAsync(dwg_t, 0, sizeof(float) * f * d, st);
+    cudaMemsetAsync(dwu_t, 0, sizeof(float) * f * d, st);
+    cudaMemsetAsync(dwd, 0, sizeof(float) * f * d, st);
+    return SGE_OK;
+  }
+  if (s_max == 0) return SGE_OK;
+
+  // ---- spill rows on tensor cores
+  const int sp = (s_max + 63) / 64 * 64;
+  gather2_kernel<<<sp, 256, 0, st>>>(dyb, xb, hy->spill_rows, hy->n_spill, s_max, static_cast<int>(d),
+                                      ws.dys, ws.xs);
+  if ((rc = check_launch("hybrid_ffn_bwd (gather)"))) return rc;
+  using S = TcPairShape<256, 1>;
+  CUtensorMap m1a, m1b;
+  if ((rc = make_tmap_bf16(&m1a, ws.dys, sp, d, d, kBM))) return rc;
+  if ((rc = make_tmap_bf16(&m1b, wd, f, d, d, S::BN / 2))) return rc;
+  EpiBwdSpill e1{hv.spill_a, hv.spill_u, ws.acat, ws.hs, hy->n_spill, s_max, static_cast<int>(f), sp};
+  if ((rc = launch_tc_gemm_pair<S>(m1a, m1b, m1b, sp, f, d, e1, nullptr, st, "hybrid_ffn_bwd (dH)")))
+    return rc;
+  // operands of the remaining GEMMs, K-major
+  if ((rc = launch_transpose(ws.acat, sp, static_cast<int>(2 * f), 2 * f, ws.acat_t, sp, 0, st))) return rc;
+  if ((rc = launch_transpose(ws.hs, sp, static_cast<int>(f), f, ws.hs_t, sp, 0, st))) return rc;
+  if ((rc = launch_transpose(ws.dys, sp, static_cast<int>(d), d, ws.dys_t, sp, 0, st))) return rc;
+  if ((rc = launch_transpose(ws.xs, sp, static_cast<int>(d), d, ws.xs_t, sp, 0, st))) return rc;
+  if ((rc = launch_transpose(static_cast<const uint16_t*>(wu_t), static_cast<int>(f), static_cast<int>(d), d,
+                             ws.bcat, 2 * f, 0, st)))
+    return rc;
+  if ((rc = launch_transpose(static_cast<const uint16_t*>(wg_t), static_cast<int>(f), static_cast<int>(d), d,
+                             ws.bcat, 2 * f, static_cast<int>(f), st)))
+    return rc;
+  // dX_s = [dU | dG] [W_up ; W_gate]^T  -> dx rows
+  CUtensorMap m2a, m2b;
+  if ((rc = make_tmap_bf16(&m2a, ws.acat, sp, 2 * f, 2 * f, kBM))) return rc;
+  if ((rc = make_tmap_bf16(&m2b, ws.bcat, d, 2 * f, 2 * f, S::BN / 2))) return rc;
+  EpiScatterRowsBwd e2{static_cast<uint16_t*>(dx), hy->spill_rows, hy->n_spill, s_max, static_cast<int>(d)};
+  if ((rc = launch_tc_gemm_pair<S>(m2a, m2b, m2b, sp, d, 2 * f, e2, nullptr, st, "hybrid_ffn_bwd (dX)")))
+    return rc;
+  // dW_down += H^T dY_s
+  CUtensorMap m3a, m3b;
+  if ((rc = make_tmap_bf16(&m3a, ws.hs_t, f, sp, sp, kBM))) return rc;
+  if ((rc = make_tmap_bf16(&m3b, ws.dys_t, d, sp, sp, S::BN / 2))) return rc;
+  EpiAddF32 e3{dwd, nullptr, f, static_cast<int>(d)};
+  if ((rc = launch_tc_gemm_pair<S>(m3a, m3b, m3b, f, d, sp, e3, nullptr, st, "hybrid_ffn_bwd (dW_down)")))
+    return rc;
+  // [dW_up ; dW_gate] += [dU | dG]^T X_s
+  CUtensorMap m4a, m4b;
+  if ((rc = make_tmap_bf16(&m4a, ws.acat_t, 2 * f, sp, sp, kBM))) return rc;
+  if ((rc = make_tmap_bf16(&m4b, ws.xs_t, d, sp, sp, S::BN / 2))) return rc;
+  EpiAddF32 e4{dwu_t, dwg_t, f, static_cast<int>(d)};
+  return launch_tc_gemm_pair<S>(m4a, m4b, m4b, 2 * f, d, sp, e4, nullptr, st,
+                                "hybrid_ffn_bwd (dW_up, dW_gate)");
+}

@@ -255,6 +255,32 @@ int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* wu_t, const 
                    const void* wd_t, void* y, int64_t d_model, void* workspace,
                    size_t workspace_bytes, void* stream);
 
+/*
+ * hybrid_ffn_bwd -- gradients of the gated FFN from the hybrid form (after
+ * hybrid_ffn_fwd filled ell_u / spill_u).  The pages print no backward
+ * formulas; these are the derivatives of y = sum_j a_j u_j W_down[j] over the
+ * stored entries (a_j > 0, so dReLU = 1 there; other entries contribute 0):
+ *   dh = dy . W_down[j], du = dh a, dg = dh u,
+ *   dx = sum_j du W_up[:, j] + dg W_gate[:, j],
+ *   dW_down[j] = sum_t a u dy_t, dW_up[:, j] = sum_t du x_t,
+ *   dW_gate[:, j] = sum_t dg x_t.
+ * ELL rows run on CUDA cores (weight gradients summed per hidden unit in
+ * ascending token order); spill rows run as tcgen05 GEMMs whose results are
+ * added to the same fp32 rows.  Deterministic.
+ *   x, dy, dx [N][d] bf16; wg_t, wu_t, wd [F][d] bf16;
+ *   dwg_t, dwu_t [F][d] fp32 (neuron-major like the weights), dwd [F][d] fp32,
+ *   all overwritten; dropped rows get dx = 0 and add nothing.
+ *   workspace >= hybrid_ffn_bwd_workspace_bytes(N, d, F, K, S_max) bytes,
+ *   256-byte aligned.
+ */
+size_t hybrid_ffn_bwd_workspace_bytes(int64_t n_tokens, int64_t d_model, int64_t d_ff, int ell_cap,
+                                      int s_max);
+
+int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* hy, const void* wg_t,
+                   const void* wu_t, const void* wd, void* dx, float* dwg_t, float* dwu_t,
+                   float* dwd, int64_t d_model, void* workspace, size_t workspace_bytes,
+                   void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -102,3 +102,77 @@ def test_hybrid_train_workload_sampled(cuda_device):
     err = oracle.max_abs_rel(to_f64(y)[rows][ok], y_ora[ok])
     assert err <= BF16_TOL, err
     print(f"train hybrid: {n_spill} spill rows, max-abs-rel {err:.2e} on {ok.sum()} rows")
+
+
+@pytest.mark.parametrize("k,s_max", [(16, 64), (16, 4), (0, 300), (512, 8), (40, 32)])
+def test_hybrid_bwd_matches_oracle(cuda_device, k, s_max):
+    inp = _small_inputs(seed=1)
+    x, wg, wu, wd = (inp.as_f64(n) for n in ("x", "wg_t", "wu_t", "wd"))
+    x[:7, :-1] *= 3.0
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    x = xb.double().numpy()
+    dyb = torch.from_numpy(np.random.default_rng(5).standard_normal(x.shape)).to(torch.bfloat16)
+    dy = dyb.double().numpy()
+    tw = oracle.twell_pack(oracle.gate_preact(x, wg), 128, 128, oracle.VAL_BF16)
+    ora = oracle.hybrid_pack(tw, k, s_max)
+    oracle.hybrid_fwd(x, ora, wu, wd)
+    want = oracle.hybrid_bwd(x, dy, ora, wg, wu, wd)
+
+    dev = cuda_device
+    hy = sge.hybrid_pack(_upload_twell(tw, dev), k, s_max)
+    w_dev = [getattr(inp, n).to(dev) for n in ("wg_t", "wu_t", "wd")]
+    sge.hybrid_ffn_fwd(xb.to(dev), hy, w_dev[1], w_dev[2])
+    got = sge.hybrid_ffn_bwd(xb.to(dev), dyb.to(dev), hy, *w_dev)
+    torch.cuda.synchronize()
+    for name, a, b in zip(("dx", "dW_gate", "dW_up", "dW_down"), got, want):
+        err = oracle.max_abs_rel(to_f64(a), b)
+        assert err <= BF16_TOL, (name, err)
+    dropped = (ora.row_nnz > k) & (ora.spill_slot < 0)
+    assert np.all(to_f64(got[0])[dropped] == 0.0)
+
+
+def test_hybrid_bwd_is_deterministic(cuda_device):
+    inp = _small_inputs(seed=2)
+    dev = cuda_device
+    x, wg, wu, wd = (getattr(inp, n).to(dev) for n in ("x", "wg_t", "wu_t", "wd"))
+    dy = torch.randn(x.shape, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16).to(dev)
+    tw = sge.twell_gate_pack(x, wg, 128, 128)
+    hy = sge.hybrid_pack(tw, 16, 64)
+    sge.hybrid_ffn_fwd(x, hy, wu, wd)
+    a = sge.hybrid_ffn_bwd(x, dy, hy, wg, wu, wd)
+    b = sge.hybrid_ffn_bwd(x, dy, hy, wg, wu, wd)
+    torch.cuda.synchronize()
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)
+
+
+def test_hybrid_bwd_train_workload_sampled_dx(cuda_device):
+    """Full training-shaped backward; dx of sampled ELL and spill rows
+    against the oracle (each row's dx depends only on its own entries)."""
+    cfg = synth.CONFIGS["train_1b_hybrid"]
+    inp = synth.make_inputs(cfg)
+    dev = cuda_device
+    x, wg, wu, wd, dy = (getattr(inp, n).to(dev) for n in ("x", "wg_t", "wu_t", "wd", "dy"))
+    tw = sge.twell_gate_pack(x, wg, cfg.tile, cfg.cap)
+    hy = sge.hybrid_pack(tw, cfg.ell_cap, cfg.s_max)
+    sge.hybrid_ffn_fwd(x, hy, wu, wd)
+    dx, dwg, dwu, dwd = sge.hybrid_ffn_bwd(x, dy, hy, wg, wu, wd)
+    torch.cuda.synchronize()
+    assert all(torch.isfinite(t).all() for t in (dx, dwg, dwu, dwd))
+    nnz = hy.row_nnz.cpu().numpy()
+    spill_rows = np.flatnonzero(nnz > cfg.ell_cap)
+    ell_rows = np.flatnonzero(nnz <= cfg.ell_cap)
+    rows = np.unique(np.concatenate([spill_rows[:5], ell_rows[::700]]))
+    xf, wgf, wuf, wdf, dyf = (inp.as_f64(n) for n in ("x", "wg_t", "wu_t", "wd", "dy"))
+    g = oracle.gate_preact(xf[rows], wgf)
+    tw_ora = oracle.twell_pack(g, cfg.tile, cfg.cap, oracle.VAL_BF16)
+    abs_sum = np.abs(xf[rows]) @ np.abs(wgf).T
+    bad_rows, _ = compare_twell_inexact(tw, tw_ora, g, oracle.VAL_BF16, abs_sum, rows=rows)
+    # route the sampled rows as the GPU did (K, and no drops at this size)
+    ora = oracle.hybrid_pack(tw_ora, cfg.ell_cap, len(rows))
+    oracle.hybrid_fwd(xf[rows], ora, wuf, wdf)
+    dx_ora = oracle.hybrid_bwd(xf[rows], dyf[rows], ora, wgf, wuf, wdf)[0]
+    ok = ~bad_rows
+    err = oracle.max_abs_rel(to_f64(dx)[rows][ok], dx_ora[ok])
+    assert err <= BF16_TOL, err
+    print(f"train hybrid bwd: dx max-abs-rel {err:.2e} on {ok.sum()} rows")
