@@ -60,9 +60,11 @@ def library() -> ctypes.CDLL:
             "sge_version": (I, []),
             "sge_last_error": (ctypes.c_char_p, []),
             "twell_gate_pack": (I, [P, P, I64, I64, I64, I, I, I, P, P, P, P, P]),
-            "twell_fused_up_down_workspace_bytes": (ctypes.c_size_t, [I64]),
+            "twell_fused_up_down_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
             "twell_fused_up_down": (I, [P, P, P, P, P, P, P, I64, I64, I64, I, I, I, P,
-                                        ctypes.c_size_t, P]),
+                                        ctypes.c_size_t, P, P]),
+            "twell_fused_up_down_noalloc": (I, [P, P, P, P, P, P, P, I64, I64, I64, I, I, I, P, P]),
+            "twell_fused_up_down_noalloc_max_tokens": (I64, []),
             "dense_ffn_fwd": (I, [P, P, P, P, P, P, I64, I64, I64, P, P]),
             "hybrid_pack": (I, [P, P, P, I, I, ctypes.POINTER(_SgeHybrid), P, P]),
             "hybrid_ffn_fwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I]),
@@ -166,15 +168,16 @@ def twell_gate_pack(x: torch.Tensor, wg_t: torch.Tensor, tile: int, cap: int,
     return out
 
 
-def fused_workspace(n_tokens: int, device) -> torch.Tensor:
-    """Scratch for twell_fused_up_down (heavy-token list and work cursors)."""
-    nbytes = library().twell_fused_up_down_workspace_bytes(n_tokens)
+def fused_workspace(n_tokens: int, d_model: int, device) -> torch.Tensor:
+    """Scratch for twell_fused_up_down (entry counts, job lists, fp32 partial
+    outputs of split heavy tokens, counters)."""
+    nbytes = library().twell_fused_up_down_workspace_bytes(n_tokens, d_model)
     return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
 
 
 def twell_fused_up_down(x: torch.Tensor, tw: TwELL, wu_t: torch.Tensor, wd: torch.Tensor,
                         y: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                        stream=None) -> torch.Tensor:
+                        diag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """y = sum over TwELL entries of a * (x . W_up[:, j]) * W_down[j] (h never stored)."""
     _check(x, "x")
     n, d = x.shape
@@ -188,11 +191,13 @@ def twell_fused_up_down(x: torch.Tensor, tw: TwELL, wu_t: torch.Tensor, wd: torc
         y = torch.empty_like(x)
     _check(y, "y", x.dtype, (n, d))
     if workspace is None:
-        workspace = fused_workspace(n, x.device)
+        workspace = fused_workspace(n, d, x.device)
     _check(workspace, "workspace", torch.uint8)
+    if diag is not None:
+        _check(diag, "diag", torch.int32, (4,))
     _call("twell_fused_up_down", _ptr(x), _ptr(tw.count), _ptr(tw.idx), _ptr(tw.val),
           _ptr(wu_t), _ptr(wd), _ptr(y), n, d, f, _dtype_code(x), tw.tile, tw.cap,
-          _ptr(workspace), workspace.numel(), _stream(x.device, stream))
+          _ptr(workspace), workspace.numel(), _ptr(diag), _stream(x.device, stream))
     return y
 
 
@@ -202,7 +207,7 @@ def twell_ffn_forward(x, wg_t, wu_t, wd, tile: int, cap: int, tw: Optional[TwELL
     """The sparse inference forward: gate GEMM + TwELL epilogue, then the
     fused up/down kernel.  Returns (y, twell)."""
     tw = twell_gate_pack(x, wg_t, tile, cap, out=tw, diag=diag, stream=stream)
-    y = twell_fused_up_down(x, tw, wu_t, wd, y=y, workspace=workspace, stream=stream)
+    y = twell_fused_up_down(x, tw, wu_t, wd, y=y, workspace=workspace, diag=diag, stream=stream)
     return y, tw
 
 

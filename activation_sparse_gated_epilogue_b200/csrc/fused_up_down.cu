@@ -7,31 +7,46 @@
 // (t, j, a) of the TwELL gate activations:
 //     u = x[t] . W_up[:, j]      h = a * u      y[t] += h * W_down[j, :]
 //
-// Work is per token, and per-token work is heavy-tailed (a few tokens carry
-// tens of times the mean number of entries), so:
-//   * a classify kernel marks tokens with more than kHeavyEntries entries and
-//     lists them in the caller's workspace;
-//   * one persistent kernel (one CTA per SM made of three 128-thread
-//     groups) first takes the heavy tokens, one per CTA, the groups
-//     splitting the token's TwELL tiles and summing their partial y in a
-//     fixed order in shared memory; then each group pulls light tokens one at
-//     a time from a global cursor.
-// Inside a group a token is processed in chunks of at most kMaxEntries
-// entries gathered into shared memory (ascending column order):
-//   * the d-vector is split across the group's threads in 16-byte vectors,
-//     so each thread keeps a few elements of x[t] and of the fp32 y[t]
-//     accumulator in registers;
-//   * phase U: every thread loads its 16-byte slice of row j of W_up for a
-//     batch of entries (two batches in flight: register double buffering),
-//     forms exact bf16 x bf16 products accumulated in fp32, the warp reduces a
-//     batch with a halving shuffle tree and the per-warp partials go to
-//     shared memory;
-//   * h_e = a_e * (sum of the per-warp partials, fixed order), rounded to the
-//     activation dtype (the precision the dense FFN gives h);
-//   * phase D: every thread streams its slice of row j of W_down and
-//     accumulates h_e * W_down[j] into its y registers.
-// h lives only in shared memory.  Results do not depend on which CTA or
-// group processes a token: no atomics touch data.
+// At the densities the method runs at (about 1% of d_ff) two tokens rarely
+// share a column, so every entry streams one row of W_up and one of W_down
+// from L2 with little reuse: the kernel is bound by how many row bytes it
+// keeps in flight between L2 and the SMs, and by its instructions per row.
+//
+// Warps.  Each warp streams whole rows (one 16-byte piece per lane per 512
+// bytes) through its own ring of shared-memory slots with cp.async.bulk: its
+// lanes issue copies in parallel, one mbarrier per slot, several rows ahead
+// of consumption.  It keeps x[t] (bf16) and the fp32 y[t] of its job in
+// registers, forms each dot product x[t] . W_up[:, j] with exact bf16 x bf16
+// products accumulated in fp32 and reduced over the lanes, rounds
+// h = a * u to the activation dtype (what the dense FFN gives h), and
+// accumulates h * W_down[j] into y.  h lives only in registers and shared
+// memory.  Entries are taken in chunks of 32, one per lane: the W_up rows of
+// a chunk, then its W_down rows.
+//
+// Teams.  A team of kTeam warps shares one job (a token, or a unit of a heavy
+// token): warp w takes the job's entries w, w + kTeam, ...  At the end of the
+// job the warps add their fp32 partial y, one after the other in warp order,
+// into a row buffer in shared memory; the last warp stores the sum.
+//
+// Entries.  Each warp resolves its own entries straight from the TwELL
+// (exclusive prefix of the token's tile counts in registers, a binary search
+// per lane, one load of idx and of val) one chunk ahead of consumption, so
+// its copies run ahead across chunk and job boundaries.
+//
+// Jobs.  Three small kernels plan the work: stored entries per token; the unit
+// length U (a multiple of 32: heavy tokens split into units of about an
+// eighth of a team's average share, whose fp32 partial outputs fit the
+// pool); the job lists: units of heavy tokens first, then the other
+// non-empty tokens in four classes of decreasing size, so that the last jobs
+// are short; empty tokens get y = 0 there.  The team leader pulls jobs from a
+// global cursor and queues them two jobs ahead.  A unit stores its fp32
+// partial in the pool; the team that completes a split token's last unit (a
+// counter per token) sums the units' partials in unit order and stores y.  No
+// atomics touch data, so results do not depend on scheduling.
+//
+// Every wait is bounded: a wait that runs out of time sets SGE_FLAG_TIMEOUT in
+// diag and stops the CTA, after each warp has waited (again bounded) for its
+// own copies in flight.
 #include <mutex>
 
 #include "sge_host.h"
@@ -39,28 +54,84 @@
 
 namespace sge {
 
-constexpr int kGroupThreads = 128;  // threads processing one token
-constexpr int kGroupWarps = kGroupThreads / 32;
-constexpr int kMaxEntries = 512;    // entries per chunk in a group's shared list
-constexpr int kMaxTiles = 512;      // TwELL tiles per chunk
-constexpr int kHeavyEntries = 384;  // tokens with more entries use a whole CTA
+constexpr int kTeam = 4;        // warps per job
+constexpr int kChunk = 32;      // entries per chunk, one per lane
+constexpr int kBatch = 4;       // rows per reduction batch (the partial-sum shift register has 4)
+constexpr int kMaxSlots = 16;   // ring slots per warp
+constexpr int kSmemBudget = 232448;
+constexpr int kUnitMin = 32;
+constexpr int kMaxCtas = 256;   // the grid is clamped to this many CTAs
+constexpr int kLightClasses = 4;
+// Per-team shared memory before the row buffer: the job queue (4 entries and
+// a staging entry), then the barriers tbar, tfree and chain[kTeam - 1].
+constexpr int kTeamHdr = (5 * 32 + 8 * (2 + kTeam - 1) + 15) & ~15;
 
-// Per row width (NV 16-byte vectors per thread): groups per CTA and entries
-// per load batch (two batches in flight), chosen so that the double-buffered
-// rows fit in registers at one CTA per SM.
+constexpr size_t kPoolBytes = size_t(64) << 20;
+
+// Warps per CTA for NV pieces per lane: registers hold NV pieces of x and
+// the fp32 y of NV pieces per lane.
 template <int NV>
-struct UdTune {
-  static constexpr int kGroups = 3;
-  static constexpr int kBatch = NV == 1 ? 8 : (NV == 2 ? 4 : 2);
-  static constexpr int kThreads = kGroups * kGroupThreads;
+struct UdLaunch {
+  static constexpr int kWarps = NV <= 2 ? 24 : (NV <= 4 ? 16 : (NV <= 8 ? 12 : 8));
 };
 
-// Workspace: int header[4] = {heavy count, heavy cursor, light cursor, 0},
-// int heavy_list[N], uint8 heavy_flag[N].
-constexpr size_t kWsHeader = 16;
+inline int warps_for_nv(int nv) {
+  return nv <= 2 ? UdLaunch<2>::kWarps
+                 : (nv <= 4 ? UdLaunch<4>::kWarps : (nv <= 8 ? UdLaunch<8>::kWarps : UdLaunch<16>::kWarps));
+}
 
-__device__ __forceinline__ void group_sync(int g) {
-  asm volatile("bar.sync %0, %1;" ::"r"(g + 1), "r"(kGroupThreads) : "memory");
+// Pieces per lane (2, 4, 8, 12 or 16) for rows of row_bytes; 0 if too long.
+inline int nv_for(int64_t row_bytes) {
+  const int64_t need = (row_bytes / 16 + 31) / 32;
+  if (need <= 2) return 2;
+  if (need <= 4) return 4;
+  if (need <= 8) return 8;
+  if (need <= 12) return 12;
+  if (need <= 16) return 16;
+  return 0;
+}
+
+// Header of the workspace (int32 words).
+constexpr int kHTotal = 0;     // stored entries (int64, words 0..1)
+constexpr int kHUnit = 2;      // unit length U
+constexpr int kHUnits = 3;     // unit jobs
+constexpr int kHLight = 4;     // unsplit non-empty tokens per size class (4 words)
+constexpr int kHSplit = 8;     // split tokens
+constexpr int kHCursor = 9;    // job cursor
+constexpr int kHOverflow = 10; // units that did not fit the pool (stays 0)
+constexpr size_t kHdrBytes = 256;
+
+struct Job {  // 32 bytes
+  int t;      // token; -1 ends the work
+  int e0;     // first entry of the job among the token's entries
+  int n;      // entries
+  int nu;     // units of the token (1: not split)
+  int u;      // this unit
+  int base;   // first pool slot of the token's units
+  int sid;    // split-token index (completion counters)
+  int pad;
+};
+
+// Workspace layout for n tokens and pool_slots pool slots of d floats.
+struct WsLayout {
+  size_t blk, ntok, lights, units, done, pool, total;
+  WsLayout(int64_t n, int64_t d, int64_t pool_slots) {
+    const size_t nblk = static_cast<size_t>((n + 255) / 256);
+    const size_t ps = static_cast<size_t>(pool_slots);
+    size_t o = kHdrBytes;
+    blk = o;     o += (8 * nblk + 255) & ~size_t(255);
+    ntok = o;    o += (4 * static_cast<size_t>(n) + 255) & ~size_t(255);
+    lights = o;  o += (8 * kLightClasses * static_cast<size_t>(n) + 255) & ~size_t(255);
+    units = o;   o += 32 * ps;
+    done = o;    o += (4 * ps + 255) & ~size_t(255);
+    pool = o;    o += 4 * ps * static_cast<size_t>(d);
+    total = o;
+  }
+};
+
+inline int64_t pool_slots_for(size_t pool_bytes, int64_t d) {
+  const int64_t s = static_cast<int64_t>(pool_bytes / (4 * static_cast<size_t>(d)));
+  return s < (1 << 28) ? s : (1 << 28);
 }
 
 struct UdParams {
@@ -71,357 +142,731 @@ struct UdParams {
   const void* wu_t;
   const void* wd;
   void* y;
-  int* ws;             // header + heavy list
-  const uint8_t* heavy_flag;
+  int* hdr;
+  const int* ntok;
+  const int2* lights;  // [kLightClasses][n_rows]
+  const Job* units;
+  int* done;
+  float* pool;
+  int32_t* diag;
   int64_t n_rows;
   int d;
-  int n_cols;
+  int nt;
   int tile;
   int cap;
+  int row_bytes;
+  int teams;       // teams per CTA
+  int slots;       // ring slots per warp
+  int slot_bytes;  // one ring slot: NV * 512 bytes (a row, then zeros)
+  int off_full;    // shared-memory offsets: per-warp slot barriers,
+  int off_team;    // per-team job queue, barriers and row buffer,
+  int team_bytes;
+  int off_abort;   // CTA-wide abort flag
 };
 
-// Shared memory of one group.
-struct GroupSmem {
-  int2 jh[kMaxEntries];                 // (column j, a bits) -> (j, h bits)
-  float upart[kGroupWarps][kMaxEntries];
-  int tile_off[kMaxTiles + 1];
-  int chunk[2];
-  int token;
-};
+// ------------------------------------------------------------- planning
 
-template <int NV, bool BF16>
-struct Group {
-  static constexpr int kBatch = UdTune<NV>::kBatch;
-  using E = Elem<BF16>;
-  static constexpr int VEC = E::VEC;
-  static constexpr int ESZ = BF16 ? 2 : 4;
-
-  const UdParams& p;
-  GroupSmem& sm;
-  const int g, gtid, gwarp, lane, nvec;
-  const int64_t row_bytes;
-
-  __device__ Group(const UdParams& p_, GroupSmem& sm_, int g_, int gtid_)
-      : p(p_), sm(sm_), g(g_), gtid(gtid_), gwarp(gtid_ >> 5), lane(gtid_ & 31),
-        nvec(p_.d / E::VEC), row_bytes(static_cast<int64_t>(p_.d) * ESZ) {}
-
-  __device__ __forceinline__ void load_x(int64_t t, uint4 (&xv)[NV]) const {
-    const uint4* xrow = reinterpret_cast<const uint4*>(static_cast<const char*>(p.x) + t * row_bytes);
-#pragma unroll
-    for (int k = 0; k < NV; ++k) {
-      const int v = gtid + k * kGroupThreads;
-      xv[k] = v < nvec ? __ldg(xrow + v) : make_uint4(0, 0, 0, 0);
-    }
-  }
-
-  __device__ __forceinline__ void load_rows(const void* base, int e0, int n_e, uint4 (&w)[kBatch][NV]) const {
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int e = e0 + u;
-      const int j = e < n_e ? sm.jh[e].x : -1;
-      const uint4* row = reinterpret_cast<const uint4*>(static_cast<const char*>(base) + static_cast<int64_t>(j) * row_bytes);
-#pragma unroll
-      for (int k = 0; k < NV; ++k) {
-        const int v = gtid + k * kGroupThreads;
-        w[u][k] = (j >= 0 && v < nvec) ? __ldg(row + v) : make_uint4(0, 0, 0, 0);
-      }
-    }
-  }
-
-  __device__ __forceinline__ void reduce_u(const uint4 (&xv)[NV], const uint4 (&w)[kBatch][NV], int e0, int n_e) const {
-    float part[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      float s = 0.0f;
-#pragma unroll
-      for (int k = 0; k < NV; ++k) s = E::dot(xv[k], w[u][k], s);
-      part[u] = s;
-    }
-    const float tot = warp_reduce_multi<kBatch>(part, lane);
-    if ((lane & (32 / kBatch - 1)) == 0) {
-      const int e = e0 + multi_entry<kBatch>(lane);
-      if (e < n_e) sm.upart[gwarp][e] = tot;
-    }
-  }
-
-  __device__ __forceinline__ void apply_d(const uint4 (&w)[kBatch][NV], int e0, int n_e,
-                                          float (&acc)[NV][VEC]) const {
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int e = e0 + u;
-      const typename E::HType h = E::h_from_bits(e < n_e ? sm.jh[e].y : 0);
-#pragma unroll
-      for (int k = 0; k < NV; ++k) E::axpy(h, w[u][k], acc[k]);
-    }
-  }
-
-  // Accumulate into acc the entries of token t in tiles b_first, b_first +
-  // stride, ... (ascending).
-  __device__ void run(int64_t t, int b_first, int stride, const uint4 (&xv)[NV],
-                      float (&acc)[NV][VEC]) const {
-    const int nt = p.n_cols / p.tile;
-    const uint8_t* cnt = p.count + t * nt;
-    const int nk = b_first < nt ? (nt - b_first + stride - 1) / stride : 0;
-    int k0 = 0;
-    while (k0 < nk) {
-      // ---- chunk: tiles k0 .. k1 (in units of stride) holding <= kMaxEntries
-      if (gwarp == 0) {
-        int k = k0, total = 0, n_tiles = 0;
-        if (lane == 0) sm.tile_off[0] = 0;
-        while (true) {
-          const int kk = k + lane;
-          const int c = kk < nk ? min(static_cast<int>(cnt[b_first + kk * stride]), p.cap) : 0;
-          int incl = c;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int nb = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += nb;
-          }
-          // all three conditions are monotone in the lane: the fitting lanes form a prefix
-          const bool fits = kk < nk && total + incl <= kMaxEntries && n_tiles + lane < kMaxTiles;
-          const int take = __popc(__ballot_sync(0xffffffffu, fits));
-          if (lane < take) sm.tile_off[n_tiles + lane + 1] = total + incl;
-          if (take > 0) total += __shfl_sync(0xffffffffu, incl, take - 1);
-          n_tiles += take;
-          k += take;
-          if (take < 32) break;
-        }
-        if (lane == 0) {
-          sm.chunk[0] = k;
-          sm.chunk[1] = total;
-        }
-      }
-      group_sync(g);
-      const int k1 = sm.chunk[0];
-      const int n_e = sm.chunk[1];
-      const int n_tiles = k1 - k0;
-
-      // ---- gather the chunk's entries, one thread per entry
-      for (int e = gtid; e < n_e; e += kGroupThreads) {
-        int lo = 0, hi = n_tiles;  // tile_off[lo] <= e < tile_off[lo + 1]
-        while (hi - lo > 1) {
-          const int mid = (lo + hi) >> 1;
-          if (sm.tile_off[mid] <= e) lo = mid; else hi = mid;
-        }
-        const int b = b_first + (k0 + lo) * stride;
-        const int s = e - sm.tile_off[lo];
-        const int64_t seg = t * nt + b;
-        sm.jh[e] = make_int2(b * p.tile + p.idx[seg * p.cap + s],
-                             __float_as_int(E::load_val(p.val, seg * p.cap + s)));
-      }
-      group_sync(g);
-
-      // ---- phase U: partial dot products, two batches of rows in flight
-      {
-        uint4 wa[kBatch][NV], wb[kBatch][NV];
-        if (n_e > 0) load_rows(p.wu_t, 0, n_e, wa);
-        for (int e0 = 0; e0 < n_e; e0 += 2 * kBatch) {
-          if (e0 + kBatch < n_e) load_rows(p.wu_t, e0 + kBatch, n_e, wb);
-          reduce_u(xv, wa, e0, n_e);
-          if (e0 + kBatch >= n_e) break;
-          if (e0 + 2 * kBatch < n_e) load_rows(p.wu_t, e0 + 2 * kBatch, n_e, wa);
-          reduce_u(xv, wb, e0 + kBatch, n_e);
-        }
-      }
-      group_sync(g);
-
-      // ---- h = a * u, rounded as phase D consumes it
-      for (int e = gtid; e < n_e; e += kGroupThreads) {
-        float u = 0.0f;
-#pragma unroll
-        for (int w = 0; w < kGroupWarps; ++w) u += sm.upart[w][e];
-        sm.jh[e].y = E::h_bits(E::h_of(__int_as_float(sm.jh[e].y) * u));
-      }
-      group_sync(g);
-
-      // ---- phase D: y += h * W_down[j], two batches of rows in flight
-      {
-        uint4 wa[kBatch][NV], wb[kBatch][NV];
-        if (n_e > 0) load_rows(p.wd, 0, n_e, wa);
-        for (int e0 = 0; e0 < n_e; e0 += 2 * kBatch) {
-          if (e0 + kBatch < n_e) load_rows(p.wd, e0 + kBatch, n_e, wb);
-          apply_d(wa, e0, n_e, acc);
-          if (e0 + kBatch >= n_e) break;
-          if (e0 + 2 * kBatch < n_e) load_rows(p.wd, e0 + 2 * kBatch, n_e, wa);
-          apply_d(wb, e0 + kBatch, n_e, acc);
-        }
-      }
-      group_sync(g);  // the next chunk rewrites the shared lists
-      k0 = k1;
-    }
-  }
-
-  __device__ __forceinline__ void store_y(int64_t t, const float (&acc)[NV][VEC]) const {
-    uint4* yrow = reinterpret_cast<uint4*>(static_cast<char*>(p.y) + t * row_bytes);
-#pragma unroll
-    for (int k = 0; k < NV; ++k) {
-      const int v = gtid + k * kGroupThreads;
-      if (v < nvec) yrow[v] = E::pack(acc[k]);
-    }
-  }
-};
-
-// Marks tokens whose stored entry count exceeds kHeavyEntries and lists them.
-__global__ void __launch_bounds__(256) classify_kernel(const uint8_t* __restrict__ count,
-                                                       int64_t n_rows, int nt, int cap, int* ws,
-                                                       uint8_t* heavy_flag) {
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t >= n_rows) return;
-  const uint8_t* cnt = count + t * nt;
+// Stored entries of every token (counts capped at C) and per-block sums.
+__global__ void __launch_bounds__(256) ud_count_kernel(const uint8_t* __restrict__ count,
+                                                       int64_t n_rows, int nt, int cap,
+                                                       int* __restrict__ ntok,
+                                                       long long* __restrict__ blk_sum) {
+  __shared__ long long wsum[8];
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   int s = 0;
-  for (int b = lane; b < nt; b += 32) s += min(static_cast<int>(cnt[b]), cap);
+  if (t < n_rows) {
+    const uint8_t* c = count + t * nt;
+    if ((nt & 3) == 0 && (reinterpret_cast<uintptr_t>(count) & 3) == 0) {
+      const uint32_t* c4 = reinterpret_cast<const uint32_t*>(c);
+      for (int b = 0; b < nt / 4; ++b) {
+        const uint32_t v = __ldg(c4 + b);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (lane == 0) {
-    const bool heavy = s > kHeavyEntries;
-    heavy_flag[t] = heavy ? 1 : 0;
-    if (heavy) ws[4 + atomicAdd(&ws[0], 1)] = static_cast<int>(t);
+        for (int k = 0; k < 4; ++k) s += min(static_cast<int>((v >> (8 * k)) & 255u), cap);
+      }
+    } else {
+      for (int b = 0; b < nt; ++b) s += min(static_cast<int>(__ldg(c + b)), cap);
+    }
+    ntok[t] = s;
+  }
+  long long v = s;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long tot = 0;
+    for (int w = 0; w < 8; ++w) tot += wsum[w];
+    blk_sum[blockIdx.x] = tot;
   }
 }
 
-template <int NV, bool BF16>
-__global__ void __launch_bounds__(UdTune<NV>::kThreads, 1) fused_up_down_kernel(UdParams p) {
-  using G = Group<NV, BF16>;
-  constexpr int VEC = G::VEC;
-  constexpr int kGroups = UdTune<NV>::kGroups;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  GroupSmem* gsm = reinterpret_cast<GroupSmem*>(smem_raw);
-  float* red = reinterpret_cast<float*>(smem_raw + kGroups * sizeof(GroupSmem));  // [3][128][NV*VEC]
-  __shared__ int s_heavy;
+// Total entries, the unit length and zeroed job counters (one CTA).
+__global__ void __launch_bounds__(1024) ud_plan_kernel(const long long* __restrict__ blk_sum,
+                                                       int64_t nblk, int64_t pool_slots,
+                                                       int64_t n_teams, int* hdr) {
+  __shared__ long long wsum[32];
+  long long s = 0;
+  for (int64_t b = threadIdx.x; b < nblk; b += blockDim.x) s += blk_sum[b];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long tot = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += wsum[w];
+    // Units of about an eighth of a team's average share; split tokens must
+    // fit the pool (a token of n > U entries takes ceil(n / U) <= 2n / U slots).
+    long long u = (tot + 8 * n_teams - 1) / (8 * n_teams);
+    const long long u_pool = pool_slots > 0 ? (2 * tot + pool_slots - 1) / pool_slots : (1LL << 30);
+    if (u < u_pool) u = u_pool;
+    if (u < kUnitMin) u = kUnitMin;
+    u = (u + kChunk - 1) / kChunk * kChunk;
+    if (u > (1LL << 30)) u = 1LL << 30;
+    *reinterpret_cast<long long*>(hdr + kHTotal) = tot;
+    hdr[kHUnit] = static_cast<int>(u);
+    hdr[kHUnits] = 0;
+    for (int c = 0; c < kLightClasses; ++c) hdr[kHLight + c] = 0;
+    hdr[kHSplit] = 0;
+    hdr[kHCursor] = 0;
+    hdr[kHOverflow] = 0;
+  }
+}
 
-  const int g = threadIdx.x / kGroupThreads;
-  const int gtid = threadIdx.x % kGroupThreads;
-  const G grp(p, gsm[g], g, gtid);
-  const int n_heavy = *reinterpret_cast<volatile int*>(&p.ws[0]);
+// Size class of an unsplit token of n entries (0: largest).
+__device__ __forceinline__ int light_class(int n, int U) {
+  return n > U / 2 ? 0 : (n > U / 8 ? 1 : (n > U / 32 ? 2 : 3));
+}
 
-  // ---- heavy tokens: the whole CTA, tiles split across the groups
-  while (true) {
-    if (threadIdx.x == 0) {
-      const int k = atomicAdd(&p.ws[1], 1);
-      s_heavy = k < n_heavy ? p.ws[4 + k] : -1;
+// Job lists: every split token's units, every other non-empty token in its
+// size class; empty tokens get y = 0 here.  Slots in the lists come from
+// warp-aggregated atomics: the job order may vary between calls, the results
+// do not.
+__global__ void __launch_bounds__(256) ud_jobs_kernel(const int* __restrict__ ntok, int64_t n_rows,
+                                                      int* hdr, int2* __restrict__ lights,
+                                                      Job* __restrict__ units, int* __restrict__ done,
+                                                      int64_t pool_slots, void* y, int row_bytes) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  const unsigned lt = (1u << lane) - 1u;
+  const int U = *reinterpret_cast<volatile int*>(hdr + kHUnit);
+  const int n = t < n_rows ? ntok[t] : -1;
+  const bool split = n > U;
+  // split tokens: ceil(n / U) units each
+  const int k = split ? (n + U - 1) / U : 0;
+  int incl = k;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int ktot = __shfl_sync(0xffffffffu, incl, 31);
+  const unsigned ms = __ballot_sync(0xffffffffu, split);
+  int ubase = 0, sbase = 0;
+  if (ms && lane == 0) {
+    ubase = atomicAdd(&hdr[kHUnits], ktot);
+    sbase = atomicAdd(&hdr[kHSplit], __popc(ms));
+  }
+  ubase = __shfl_sync(0xffffffffu, ubase, 0);
+  sbase = __shfl_sync(0xffffffffu, sbase, 0);
+  bool light = n > 0 && n <= U;
+  if (split) {
+    const int first = ubase + incl - k;
+    const int sid = sbase + __popc(ms & lt);
+    if (static_cast<int64_t>(first) + k > pool_slots) {
+      atomicAdd(&hdr[kHOverflow], 1);  // cannot happen with the planned U; run it unsplit
+      light = true;
+    } else {
+      for (int u = 0; u < k; ++u) {
+        Job j;
+        j.t = static_cast<int>(t);
+        j.e0 = u * U;
+        j.n = min(U, n - u * U);
+        j.nu = k;
+        j.u = u;
+        j.base = first;
+        j.sid = sid;
+        j.pad = 0;
+        units[first + u] = j;
+      }
+      done[sid] = 0;
     }
-    __syncthreads();
-    const int64_t t = s_heavy;
-    __syncthreads();
-    if (t < 0) break;
-    uint4 xv[NV];
-    float acc[NV][VEC];
-    grp.load_x(t, xv);
+  }
+  const int cls = light ? light_class(n, U) : -1;
 #pragma unroll
-    for (int k = 0; k < NV; ++k)
+  for (int c = 0; c < kLightClasses; ++c) {
+    const unsigned ml = __ballot_sync(0xffffffffu, cls == c);
+    int lbase = 0;
+    if (ml && lane == 0) lbase = atomicAdd(&hdr[kHLight + c], __popc(ml));
+    lbase = __shfl_sync(0xffffffffu, lbase, 0);
+    if (cls == c) lights[c * n_rows + lbase + __popc(ml & lt)] = make_int2(static_cast<int>(t), n);
+  }
+  // empty tokens: the warp writes each one's row of zeros
+  unsigned me = __ballot_sync(0xffffffffu, n == 0);
+  const int64_t t0 = t - lane;
+  const int nvec = row_bytes / 16;
+  while (me) {
+    const int l = __ffs(me) - 1;
+    me &= me - 1u;
+    uint4* row = reinterpret_cast<uint4*>(static_cast<char*>(y) + (t0 + l) * row_bytes);
+    for (int v = lane; v < nvec; v += 32) row[v] = make_uint4(0, 0, 0, 0);
+  }
+}
+
+// -------------------------------------------------------------- main kernel
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Bounded wait that also gives up as soon as another warp of the CTA has.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag, int32_t* diag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 31) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitNs) break;
+    }
+  }
+  *abort_flag = 1;
+  if (diag) atomicOr(reinterpret_cast<int*>(diag + SGE_DIAG_FLAGS), SGE_FLAG_TIMEOUT);
+  return false;
+}
+
+// Exclusive prefix of tile c's capped count, from the lane-distributed copy
+// (tile b lives in lane b % 32, register b / 32).  All lanes must call it.
+template <int NTR>
+__device__ __forceinline__ int prefix_at(const int (&pre)[NTR], int c) {
+  int v = 0;
 #pragma unroll
-      for (int q = 0; q < VEC; ++q) acc[k][q] = 0.0f;
-    grp.run(t, g, kGroups, xv, acc);
-    // fixed-order sum of the groups' partial accumulators
-    if (g > 0) {
-      float* dst = red + ((g - 1) * kGroupThreads + gtid) * (NV * VEC);
+  for (int r = 0; r < NTR; ++r) {
+    const int x = __shfl_sync(0xffffffffu, pre[r], c & 31);
+    if ((c >> 5) == r) v = x;
+  }
+  return v;
+}
+
+constexpr int kFirst = 1;  // chunk flags: first chunk of its job for this warp
+constexpr int kLast = 2;   //              last chunk of its job for this warp
+constexpr int kHasX = 4;   //              the x row leads the chunk's stream
+
+// The main kernel: teams of kTeam warps, one job at a time per team, each
+// warp streaming whole rows of its own entries through its own ring of
+// p.slots slots (see the file comment).
+template <bool BF16, int NTR, int NV>
+__global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(const UdParams p) {
+  using E = Elem<BF16>;
+  constexpr int VEC = E::VEC;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const int team = warp / kTeam, w = warp - team * kTeam;
+  const int S = p.slots;
+  uint8_t* ring = smem + warp * S * p.slot_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_full) + warp * S;
+  float* ubuf = reinterpret_cast<float*>(smem + p.off_full + warps * S * 8) + warp * kChunk;
+  uint8_t* tb = smem + p.off_team + team * p.team_bytes;
+  Job* jobq = reinterpret_cast<Job*>(tb);  // [4] + a staging entry
+  uint64_t* tbar = reinterpret_cast<uint64_t*>(tb + 5 * sizeof(Job));
+  uint64_t* tfree = tbar + 1;  // the row buffer may be written again
+  uint64_t* chain = tbar + 2;  // chain[w - 1]: warp w - 1 has added its partial row
+  static_assert(5 * sizeof(Job) + 8 * (2 + kTeam - 1) <= kTeamHdr, "team header overlaps the row buffer");
+  float* tbuf = reinterpret_cast<float*>(tb + kTeamHdr);  // the team's row buffer, d floats
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + p.off_abort);
+  const bool leader = w == 0;
+  const int pieces = p.row_bytes / 16;
+
+  // the slots' bytes past the row stay zero for the whole kernel
+  if (p.row_bytes < p.slot_bytes) {
+    for (int q = 0; q < S; ++q)
+      for (int o = p.row_bytes + lane * 16; o < p.slot_bytes; o += 32 * 16)
+        *reinterpret_cast<uint4*>(ring + q * p.slot_bytes + o) = make_uint4(0, 0, 0, 0);
+  }
+  if (lane == 0) {
+    for (int q = 0; q < S; ++q) mbar_init(full + q, 1);
+    if (leader) {
+      mbar_init(tbar, kTeam);
+      mbar_init(tfree, 1);
+      for (int q = 0; q < kTeam - 1; ++q) mbar_init(chain + q, 1);
+    }
+  }
+  if (threadIdx.x == 0) *abort_flag = 0;
+  fence_mbar_init();
+  __syncthreads();
+
+  const int n_units = *reinterpret_cast<volatile int*>(p.hdr + kHUnits);
+  int n_light[kLightClasses];
+#pragma unroll
+  for (int c = 0; c < kLightClasses; ++c) n_light[c] = *reinterpret_cast<volatile int*>(p.hdr + kHLight + c);
+  const int64_t rb = p.row_bytes;
+  const char* xb = static_cast<const char*>(p.x);
+  const char* ub = static_cast<const char*>(p.wu_t);
+  const char* db = static_cast<const char*>(p.wd);
+
+  // ---- team barrier (also publishes the leader's job-queue writes)
+  uint32_t tpar = 0;
+  auto team_sync = [&]() -> bool {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(tbar);
+    const bool ok = wait_or_abort(tbar, tpar, abort_flag, p.diag);
+    tpar ^= 1;
+    return ok;
+  };
+
+  // ---- jobs: the leader keeps the queue two jobs ahead of consumption; the
+  // job after that is fetched early into a staging entry (jobq[4]) with
+  // cp.async, so that no registers wait on its load.
+  int pf_kind = 0;  // leader lane 0: 0 unit, 1 unsplit token, 2 none
+  auto prefetch_job = [&]() {
+    int k = atomicAdd(&p.hdr[kHCursor], 1);
+    const uint32_t dst = smem_u32(jobq + 4);
+    if (k < n_units) {
+      pf_kind = 0;
+      const char* src = reinterpret_cast<const char*>(p.units + k);
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(dst + 16), "l"(src + 16) : "memory");
+    } else {
+      k -= n_units;
+      pf_kind = 2;
+#pragma unroll
+      for (int c = 0; c < kLightClasses; ++c) {
+        if (pf_kind == 2 && k < n_light[c]) {
+          pf_kind = 1;
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst),
+                       "l"(p.lights + c * p.n_rows + k) : "memory");
+        }
+        k -= n_light[c];
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  auto publish_job = [&](int at) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    Job j;
+    if (pf_kind == 0) {
+      j = jobq[4];
+    } else {
+      const int2 l = *reinterpret_cast<const int2*>(jobq + 4);
+      j.t = pf_kind == 1 ? l.x : -1;
+      j.e0 = 0;
+      j.n = pf_kind == 1 ? l.y : 0;
+      j.nu = 1;
+      j.u = 0;
+      j.base = -1;
+      j.sid = -1;
+      j.pad = 0;
+    }
+    jobq[at] = j;
+  };
+  if (leader && lane == 0) {
+    prefetch_job();
+    publish_job(0);
+    prefetch_job();
+    publish_job(1);
+    prefetch_job();
+  }
+  bool ok = team_sync();
+
+  // ---- entry resolution: this warp's entries of a job are w, w + kTeam, ...
+  int rk = 0, rci = 0;  // job sequence number and next chunk of the job being resolved
+  struct {
+    int t, e0, n;
+  } rj = {jobq[0].t, jobq[0].e0, jobq[0].n};
+  auto own_count = [&](int n) { return n > w ? (n - w + kTeam - 1) / kTeam : 0; };
+  int pre[NTR];
+  auto load_prefix = [&](int t) {
+    const uint8_t* cnt = p.count + static_cast<int64_t>(t) * p.nt;
+    int c[NTR];
+#pragma unroll
+    for (int r = 0; r < NTR; ++r) {
+      const int b = lane + 32 * r;
+      c[r] = b < p.nt ? min(static_cast<int>(__ldg(cnt + b)), p.cap) : 0;
+    }
+    int carry = 0;
+#pragma unroll
+    for (int r = 0; r < NTR; ++r) {
+      int incl = c[r];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      pre[r] = carry + incl - c[r];
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  };
+  if (rj.t >= 0) load_prefix(rj.t);
+  // A chunk: token (-1: none), own entries in it (may be 0 when the job has
+  // fewer entries than the team has warps), flags, job sequence number; per
+  // lane the column j and the activation a (fp32 bits) of entry `lane`.
+  struct Chunk {
+    int t, n, flags, k, j, a;
+  };
+  auto resolve = [&](Chunk& c) {
+    c.t = -1;
+    c.n = 0;
+    c.flags = 0;
+    if (rj.t < 0) return;
+    if (rci > 0 && rci * kChunk >= own_count(rj.n)) {
+      ++rk;
+      rj.t = jobq[rk & 3].t;
+      rj.e0 = jobq[rk & 3].e0;
+      rj.n = jobq[rk & 3].n;
+      rci = 0;
+      if (rj.t < 0) return;
+      load_prefix(rj.t);
+    }
+    const int own = own_count(rj.n);
+    c.t = rj.t;
+    c.k = rk;
+    c.n = max(0, min(kChunk, own - rci * kChunk));
+    c.flags = (rci == 0 ? kFirst : 0) | ((rci + 1) * kChunk >= own ? kLast : 0) |
+              (rci == 0 && own > 0 ? kHasX : 0);
+    const int e = rj.e0 + w + kTeam * (rci * kChunk + lane);
+    int b = 0;
+#pragma unroll
+    for (int step = 16 * NTR; step > 0; step >>= 1) {
+      const int cand = b + step;
+      const int v = prefix_at<NTR>(pre, cand < p.nt ? cand : 0);
+      if (cand < p.nt && v <= e) b = cand;
+    }
+    const int s = e - prefix_at<NTR>(pre, b);
+    c.j = 0;
+    c.a = 0;
+    if (lane < c.n) {
+      const int64_t at = (static_cast<int64_t>(c.t) * p.nt + b) * p.cap + s;
+      c.j = min(b * p.tile + __ldg(p.idx + at), p.nt * p.tile - 1);  // in bounds even if idx >= T
+      c.a = __float_as_int(E::load_val(p.val, at));
+    }
+    ++rci;
+  };
+  auto stream_len = [](const Chunk& c) {
+    return c.t < 0 ? 0 : ((c.flags & kHasX) ? 1 : 0) + 2 * c.n;
+  };
+  Chunk cur, nxt;
+  resolve(cur);
+  resolve(nxt);
+
+  // ---- this warp's ring: positions are the x row (first chunk of a job),
+  // then the W_up rows and the W_down rows of each chunk
+  uint32_t issued = 0, consumed = 0;
+  int is = 0, cs = 0;   // slots of the next issue and the next consumption
+  uint32_t cph = 0;     // phase parity of the slot being consumed
+  int ich = 0, iq = 0;  // issuing in cur (0) or nxt (1), at position iq of its stream
+  auto pump = [&]() {
+    __syncwarp();
+    while (true) {
+      const int room = S - static_cast<int>(issued - consumed);
+      if (room <= 0) break;
+      const Chunk& c = ich ? nxt : cur;
+      if (c.t < 0) break;
+      const int len = stream_len(c);
+      if (iq >= len) {
+        if (ich == 0) {
+          ich = 1;
+          iq = 0;
+          continue;
+        }
+        break;
+      }
+      const int m = min(room, len - iq);
+      const int hx = (c.flags & kHasX) ? 1 : 0;
+      const int q = iq + lane;
+      const int r = q - hx;
+      const int jv = __shfl_sync(0xffffffffu, c.j, (r < c.n ? r : r - c.n) & 31);
+      if (lane < m) {
+        const char* src = (hx && q == 0) ? xb + static_cast<int64_t>(c.t) * rb
+                                         : (r < c.n ? ub : db) + static_cast<int64_t>(jv) * rb;
+        int slot = is + lane;
+        if (slot >= S) slot -= S;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(full + slot, static_cast<uint32_t>(p.row_bytes));
+        bulk_load(ring + slot * p.slot_bytes, src, static_cast<uint32_t>(p.row_bytes), full + slot);
+      }
+      issued += m;
+      is += m;
+      if (is >= S) is -= S;
+      iq += m;
+    }
+  };
+  // waits for the next position and gives its slot's shared-memory address
+  auto acquire = [&](uint32_t& a) -> bool {
+    if (!wait_or_abort(full + cs, cph, abort_flag, p.diag)) return false;
+    a = smem_u32(ring + cs * p.slot_bytes);
+    return true;
+  };
+  // piece k of this lane; past the end of the row a slot holds zeros, which
+  // the copies never overwrite, so no bounds test is needed
+  auto piece = [&](uint32_t a, int k) -> uint4 { return lds128(a + (lane + 32 * k) * 16); };
+  // the warp is done with the slot; the pump may refill it
+  auto release = [&]() {
+    __syncwarp();
+    ++consumed;
+    if (++cs == S) {
+      cs = 0;
+      cph ^= 1;
+    }
+  };
+
+  // ---- consume chunks
+  uint4 xr[NV];
+#pragma unroll
+  for (int k = 0; k < NV; ++k) xr[k] = make_uint4(0, 0, 0, 0);
+  float acc[NV][VEC];
+  const int rq = (pieces + kTeam - 1) / kTeam;  // pieces each warp reduces at a job's end
+  const int q0 = w * rq, q1 = min(pieces, q0 + rq);
+  while (ok && cur.t >= 0) {
+    pump();
+    if (cur.flags & kFirst) {
 #pragma unroll
       for (int k = 0; k < NV; ++k)
 #pragma unroll
-        for (int q = 0; q < VEC; ++q) dst[k * VEC + q] = acc[k][q];
+        for (int q = 0; q < VEC; ++q) acc[k][q] = 0.0f;
     }
-    __syncthreads();
-    if (g == 0) {
+    if (cur.flags & kHasX) {
+      uint32_t a;
+      if (!(ok = acquire(a))) break;
 #pragma unroll
-      for (int r = 0; r < kGroups - 1; ++r) {
-        const float* src = red + (r * kGroupThreads + gtid) * (NV * VEC);
+      for (int k = 0; k < NV; ++k) xr[k] = piece(a, k);
+      release();
+    }
+    // phase U: dot products with the W_up rows, reduced over the lanes
+    for (int e0 = 0; ok && e0 < cur.n; e0 += kBatch) {
+      pump();
+      // the batch's partial sums shift through p0..p3 (no local-memory array;
+      // the row loop stays rolled to keep the hot code small)
+      float p0 = 0.0f, p1 = 0.0f, p2 = 0.0f, p3 = 0.0f;
+#pragma unroll 1
+      for (int r = 0; r < kBatch; ++r) {
+        float v = 0.0f;
+        if (e0 + r < cur.n) {
+          uint32_t a;
+          if (!(ok = acquire(a))) break;
+          float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-        for (int k = 0; k < NV; ++k)
-#pragma unroll
-          for (int q = 0; q < VEC; ++q) acc[k][q] += src[k * VEC + q];
+          for (int k = 0; k < NV; ++k) s[k & 3] = E::dot(xr[k], piece(a, k), s[k & 3]);
+          release();
+          v = (s[0] + s[1]) + (s[2] + s[3]);
+        }
+        p3 = p2;
+        p2 = p1;
+        p1 = p0;
+        p0 = v;
       }
-      grp.store_y(t, acc);
+      if (!ok) break;
+      float part[kBatch] = {p3, p2, p1, p0};
+      const float tot = warp_reduce_multi<kBatch>(part, lane);
+      if ((lane & (32 / kBatch - 1)) == 0) {
+        const int r = multi_entry<kBatch>(lane);
+        if (e0 + r < cur.n) ubuf[e0 + r] = tot;
+      }
     }
-    __syncthreads();
+    if (!ok) break;
+    __syncwarp();
+    // h = a * u, rounded as the down projection uses it (entry `lane`)
+    const int hb = lane < cur.n ? E::h_bits(E::h_of(__int_as_float(cur.a) * ubuf[lane])) : 0;
+    // phase D: y += h * W_down[j]
+    for (int e0 = 0; ok && e0 < cur.n; e0 += kBatch) {
+      pump();
+#pragma unroll 1
+      for (int r = 0; r < kBatch; ++r) {
+        const int hr = __shfl_sync(0xffffffffu, hb, (e0 + r) & 31);
+        if (e0 + r < cur.n) {
+          uint32_t a;
+          if (!(ok = acquire(a))) break;
+          const typename E::HType h = E::h_from_bits(hr);
+#pragma unroll
+          for (int k = 0; k < NV; ++k) E::axpy(h, piece(a, k), acc[k]);
+          release();
+        }
+      }
+    }
+    if (!ok) break;
+    if (cur.flags & kLast) {
+      // ---- job done: the warps add their partial rows into the team's row
+      // buffer one after the other (warp order), each waiting only for its
+      // predecessor; the last one stores the sum.  Warp 0 queues the job
+      // after next before it hands the buffer on.
+      uint64_t* wait_bar = w == 0 ? tfree : chain + (w - 1);
+      const uint32_t wait_par = w == 0 ? ((cur.k - 1) & 1) : (cur.k & 1);
+      if ((w > 0 || cur.k > 0) && !(ok = wait_or_abort(wait_bar, wait_par, abort_flag, p.diag))) break;
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int pc = lane + 32 * k;
+        if (pc < pieces) {
+          float4* b4 = reinterpret_cast<float4*>(tbuf + pc * VEC);
+#pragma unroll
+          for (int q = 0; q < VEC / 4; ++q) {
+            float4 v = make_float4(acc[k][4 * q], acc[k][4 * q + 1], acc[k][4 * q + 2], acc[k][4 * q + 3]);
+            if (w > 0) {
+              const float4 o = b4[q];
+              v.x = o.x + v.x;
+              v.y = o.y + v.y;
+              v.z = o.z + v.z;
+              v.w = o.w + v.w;
+            }
+            if (w < kTeam - 1) {
+              b4[q] = v;
+            } else {
+              acc[k][4 * q] = v.x;
+              acc[k][4 * q + 1] = v.y;
+              acc[k][4 * q + 2] = v.z;
+              acc[k][4 * q + 3] = v.w;
+            }
+          }
+        }
+      }
+      if (w < kTeam - 1) {
+        if (leader && lane == 0) publish_job((cur.k + 2) & 3);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(chain + w);
+        if (leader && lane == 0) prefetch_job();
+      }
+      if (w == kTeam - 1) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tfree);  // the buffer has been read
+        const Job jb = jobq[cur.k & 3];
+        char* yrow = static_cast<char*>(p.y) + static_cast<int64_t>(jb.t) * rb;
+        if (jb.nu <= 1) {
+#pragma unroll
+          for (int k = 0; k < NV; ++k) {
+            const int pc = lane + 32 * k;
+            if (pc < pieces) reinterpret_cast<uint4*>(yrow)[pc] = E::pack(acc[k]);
+          }
+        } else {
+          // a unit of a split token: its partial goes to the pool; the team
+          // that completes the token's last unit sums the partials in unit order
+          float* mine = p.pool + static_cast<int64_t>(jb.base + jb.u) * p.d;
+#pragma unroll
+          for (int k = 0; k < NV; ++k) {
+            const int pc = lane + 32 * k;
+            if (pc < pieces)
+#pragma unroll
+              for (int q = 0; q < VEC / 4; ++q)
+                reinterpret_cast<float4*>(mine + pc * VEC)[q] =
+                    make_float4(acc[k][4 * q], acc[k][4 * q + 1], acc[k][4 * q + 2], acc[k][4 * q + 3]);
+          }
+          __threadfence();
+          __syncwarp();
+          int last = 0;
+          if (lane == 0) last = atomicAdd(p.done + jb.sid, 1) == jb.nu - 1;
+          if (__shfl_sync(0xffffffffu, last, 0)) {
+            __threadfence();
+#pragma unroll
+            for (int k = 0; k < NV; ++k) {
+              const int pc = lane + 32 * k;
+              if (pc < pieces) {
+                float v[VEC];
+#pragma unroll
+                for (int q = 0; q < VEC; ++q) v[q] = 0.0f;
+                for (int u = 0; u < jb.nu; ++u) {
+                  const float4* src =
+                      reinterpret_cast<const float4*>(p.pool + static_cast<int64_t>(jb.base + u) * p.d + pc * VEC);
+#pragma unroll
+                  for (int q = 0; q < VEC / 4; ++q) {
+                    const float4 f = __ldcg(src + q);
+                    v[4 * q] += f.x;
+                    v[4 * q + 1] += f.y;
+                    v[4 * q + 2] += f.z;
+                    v[4 * q + 3] += f.w;
+                  }
+                }
+                reinterpret_cast<uint4*>(yrow)[pc] = E::pack(v);
+              }
+            }
+          }
+        }
+      }
+    }
+    // the next chunk becomes current; the issuer moves with it
+    cur = nxt;
+    if (ich == 1) {
+      ich = 0;
+    } else {
+      iq = 0;
+    }
+    resolve(nxt);
   }
-
-  // ---- light tokens: each group pulls one token at a time
-  while (true) {
-    if (gtid == 0) gsm[g].token = atomicAdd(&p.ws[2], 1);
-    group_sync(g);
-    const int64_t t = gsm[g].token;
-    group_sync(g);
-    if (t >= p.n_rows) break;
-    if (p.heavy_flag[t]) continue;
-    uint4 xv[NV];
-    float acc[NV][VEC];
-    grp.load_x(t, xv);
-#pragma unroll
-    for (int k = 0; k < NV; ++k)
-#pragma unroll
-      for (int q = 0; q < VEC; ++q) acc[k][q] = 0.0f;
-    grp.run(t, 0, 1, xv, acc);
-    grp.store_y(t, acc);
+  // Copies still in flight (only after a give-up) land before the CTA exits.
+  while (consumed != issued) {
+    mbar_wait(full + cs, cph, p.diag);
+    ++consumed;
+    if (++cs == S) {
+      cs = 0;
+      cph ^= 1;
+    }
   }
 }
 
-template <int NV, bool BF16>
-static int launch_ud(const UdParams& prm, cudaStream_t st) {
-  constexpr int VEC = Elem<BF16>::VEC;
-  constexpr int kGroups = UdTune<NV>::kGroups;
-  const int smem = static_cast<int>(kGroups * sizeof(GroupSmem) +
-                                    (kGroups - 1) * kGroupThreads * NV * VEC * sizeof(float));
-  auto kern = fused_up_down_kernel<NV, BF16>;
-  int rc = set_smem_limit(reinterpret_cast<const void*>(kern), smem);
+// ------------------------------------------------------------------ host
+
+// Teams per CTA, ring depth and shared-memory layout for rows of
+// p.row_bytes with nv pieces per lane; false if the rows are too long.
+static bool make_geometry(UdParams& p, int nv, int* smem_bytes) {
+  int warps = warps_for_nv(nv);
+  p.slot_bytes = nv * 512;
+  p.team_bytes = kTeamHdr + ((p.d * 4 + 15) & ~15);
+  for (;; warps -= kTeam) {
+    if (warps < kTeam) return false;
+    p.teams = warps / kTeam;
+    const int fixed = p.teams * p.team_bytes + warps * kChunk * 4 + 16 + 16;
+    int slots = (kSmemBudget - fixed) / (warps * (p.slot_bytes + 8));
+    if (slots > kMaxSlots) slots = kMaxSlots;
+    if (slots < kBatch) continue;  // a batch of rows must fit the ring
+    p.slots = slots;
+    p.off_full = warps * slots * p.slot_bytes;
+    p.off_team = (p.off_full + warps * slots * 8 + warps * kChunk * 4 + 15) & ~15;
+    p.off_abort = p.off_team + p.teams * p.team_bytes;
+    *smem_bytes = p.off_abort + 16;
+    return *smem_bytes <= kSmemBudget;
+  }
+}
+
+template <bool BF16, int NTR, int NV>
+static int launch_main(const UdParams& prm, int smem, int grid, cudaStream_t st) {
+  auto kern = ud_main_kernel<BF16, NTR, NV>;
+  const int rc = set_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (rc) return rc;
-  const int nt = prm.n_cols / prm.tile;
-  const int64_t cblocks = (prm.n_rows + 7) / 8;
-  classify_kernel<<<static_cast<unsigned>(cblocks), 256, 0, st>>>(
-      prm.count, prm.n_rows, nt, prm.cap, prm.ws, const_cast<uint8_t*>(prm.heavy_flag));
-  rc = check_launch("twell_fused_up_down (classify)");
-  if (rc) return rc;
-  const int64_t want = (prm.n_rows + kGroups - 1) / kGroups;
-  const int grid = static_cast<int>(want < sm_count() ? want : sm_count());
-  kern<<<grid, UdTune<NV>::kThreads, smem, st>>>(prm);
+  kern<<<grid, prm.teams * kTeam * 32, smem, st>>>(prm);
   return check_launch("twell_fused_up_down");
 }
 
+template <bool BF16, int NV>
+static int dispatch_ntr(const UdParams& prm, int smem, int grid, cudaStream_t st) {
+  if (prm.nt <= 32) return launch_main<BF16, 1, NV>(prm, smem, grid, st);
+  if (prm.nt <= 64) return launch_main<BF16, 2, NV>(prm, smem, grid, st);
+  if (prm.nt <= 128) return launch_main<BF16, 4, NV>(prm, smem, grid, st);
+  return launch_main<BF16, 8, NV>(prm, smem, grid, st);
+}
+
 template <bool BF16>
-static int dispatch_ud(const UdParams& prm, cudaStream_t st) {
-  constexpr int VEC = Elem<BF16>::VEC;
-  const int64_t nvec = prm.d / VEC;
-  if (nvec <= 1 * kGroupThreads) return launch_ud<1, BF16>(prm, st);
-  if (nvec <= 2 * kGroupThreads) return launch_ud<2, BF16>(prm, st);
-  if (nvec <= 3 * kGroupThreads) return launch_ud<3, BF16>(prm, st);
-  if (nvec <= 4 * kGroupThreads) return launch_ud<4, BF16>(prm, st);
-  return fail(SGE_ERR_UNSUPPORTED, "twell_fused_up_down: d_model %d too large (max %d)", prm.d,
-              4 * kGroupThreads * VEC);
+static int dispatch_main(const UdParams& prm, int nv, int smem, int grid, cudaStream_t st) {
+  switch (nv) {
+    case 2: return dispatch_ntr<BF16, 2>(prm, smem, grid, st);
+    case 4: return dispatch_ntr<BF16, 4>(prm, smem, grid, st);
+    case 8: return dispatch_ntr<BF16, 8>(prm, smem, grid, st);
+    case 12: return dispatch_ntr<BF16, 12>(prm, smem, grid, st);
+    default: return dispatch_ntr<BF16, 16>(prm, smem, grid, st);
+  }
 }
 
-}  // namespace sge
-
-using namespace sge;
-
-extern "C" size_t twell_fused_up_down_workspace_bytes(int64_t n_tokens) {
-  if (n_tokens < 0) return 0;
-  return (kWsHeader + 5 * static_cast<size_t>(n_tokens) + 15) & ~static_cast<size_t>(15);
-}
-
-extern "C" int twell_fused_up_down(const void* x, const uint8_t* count, const uint8_t* idx,
-                                   const void* val, const void* wu_t, const void* wd, void* y,
-                                   int64_t n_tokens, int64_t d_model, int64_t d_ff, int dtype,
-                                   int tile, int cap, void* workspace, size_t workspace_bytes,
-                                   void* stream) {
-  clear_error();
-  if (n_tokens < 0 || d_model < 1 || d_ff < 1)
-    return fail(SGE_ERR_ARG, "twell_fused_up_down: bad sizes");
-  if (d_model % 8) return fail(SGE_ERR_ARG, "twell_fused_up_down: d_model %% 8 != 0");
-  if (tile < 1 || tile > 255 || d_ff % tile)
-    return fail(SGE_ERR_ARG, "twell_fused_up_down: tile must divide d_ff and be <= 255");
-  if (cap < 1 || cap > tile) return fail(SGE_ERR_ARG, "twell_fused_up_down: cap outside [1, tile]");
-  if (d_ff >= (1LL << 31) || n_tokens >= (1LL << 31))
-    return fail(SGE_ERR_UNSUPPORTED, "twell_fused_up_down: size beyond 2^31");
-  if (n_tokens == 0) return SGE_OK;
-  if (!x || !count || !idx || !val || !wu_t || !wd || !y || !workspace)
-    return fail(SGE_ERR_ARG, "twell_fused_up_down: null pointer");
-  if (!aligned16(x) || !aligned16(wu_t) || !aligned16(wd) || !aligned16(y) || !aligned16(val) ||
-      !aligned16(workspace))
-    return fail(SGE_ERR_ARG, "twell_fused_up_down: pointer not 16-byte aligned");
-  if (workspace_bytes < twell_fused_up_down_workspace_bytes(n_tokens))
-    return fail(SGE_ERR_ARG, "twell_fused_up_down: workspace of %zu bytes, %zu needed", workspace_bytes,
-                twell_fused_up_down_workspace_bytes(n_tokens));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+// Planning kernels and the main kernel, shared by both entry points.
+static int run_fused(const char* name, const void* x, const uint8_t* count, const uint8_t* idx,
+                     const void* val, const void* wu_t, const void* wd, void* y, int64_t n_tokens,
+                     int64_t d_model, int64_t d_ff, int dtype, int tile, int cap, void* workspace,
+                     int64_t pool_slots, int32_t* diag, cudaStream_t st) {
+  if (dtype != SGE_BF16 && dtype != SGE_F32) return fail(SGE_ERR_UNSUPPORTED, "%s: dtype %d", name, dtype);
+  const int64_t esz = dtype == SGE_BF16 ? 2 : 4;
   UdParams prm;
   prm.x = x;
   prm.count = count;
@@ -430,18 +875,90 @@ extern "C" int twell_fused_up_down(const void* x, const uint8_t* count, const ui
   prm.wu_t = wu_t;
   prm.wd = wd;
   prm.y = y;
-  prm.ws = static_cast<int*>(workspace);
-  prm.heavy_flag = static_cast<const uint8_t*>(workspace) + kWsHeader + 4 * static_cast<size_t>(n_tokens);
+  const WsLayout L(n_tokens, d_model, pool_slots);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  prm.hdr = reinterpret_cast<int*>(ws);
+  long long* blk = reinterpret_cast<long long*>(ws + L.blk);
+  prm.ntok = reinterpret_cast<const int*>(ws + L.ntok);
+  prm.lights = reinterpret_cast<const int2*>(ws + L.lights);
+  prm.units = reinterpret_cast<const Job*>(ws + L.units);
+  prm.done = reinterpret_cast<int*>(ws + L.done);
+  prm.pool = reinterpret_cast<float*>(ws + L.pool);
+  prm.diag = diag;
   prm.n_rows = n_tokens;
   prm.d = static_cast<int>(d_model);
-  prm.n_cols = static_cast<int>(d_ff);
+  prm.nt = static_cast<int>(d_ff / tile);
   prm.tile = tile;
   prm.cap = cap;
-  cudaError_t e = cudaMemsetAsync(workspace, 0, kWsHeader, st);
-  if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "twell_fused_up_down: %s", cudaGetErrorString(e));
-  if (dtype == SGE_BF16) return dispatch_ud<true>(prm, st);
-  if (dtype == SGE_F32) return dispatch_ud<false>(prm, st);
-  return fail(SGE_ERR_UNSUPPORTED, "twell_fused_up_down: dtype %d", dtype);
+  prm.row_bytes = static_cast<int>(d_model * esz);
+  const int nv = nv_for(prm.row_bytes);
+  int smem = 0;
+  if (!nv || !make_geometry(prm, nv, &smem))
+    return fail(SGE_ERR_UNSUPPORTED, "%s: d_model too large: rows of %d bytes (max 8192)", name, prm.row_bytes);
+  if (prm.nt > 256)
+    return fail(SGE_ERR_UNSUPPORTED, "%s: %d TwELL tiles per row (max 256)", name, prm.nt);
+  int64_t grid = (n_tokens + prm.teams - 1) / prm.teams;
+  if (grid > sm_count()) grid = sm_count();
+  if (grid > kMaxCtas) grid = kMaxCtas;
+  const int64_t nblk = (n_tokens + 255) / 256;
+  ud_count_kernel<<<static_cast<unsigned>(nblk), 256, 0, st>>>(count, n_tokens, prm.nt, cap,
+                                                               const_cast<int*>(prm.ntok), blk);
+  int rc = check_launch("twell_fused_up_down (count)");
+  if (rc) return rc;
+  ud_plan_kernel<<<1, 1024, 0, st>>>(blk, nblk, pool_slots, grid * prm.teams, prm.hdr);
+  rc = check_launch("twell_fused_up_down (plan)");
+  if (rc) return rc;
+  ud_jobs_kernel<<<static_cast<unsigned>(nblk), 256, 0, st>>>(
+      prm.ntok, n_tokens, prm.hdr, const_cast<int2*>(prm.lights), const_cast<Job*>(prm.units),
+      prm.done, pool_slots, y, prm.row_bytes);
+  rc = check_launch("twell_fused_up_down (jobs)");
+  if (rc) return rc;
+  return dtype == SGE_BF16 ? dispatch_main<true>(prm, nv, smem, static_cast<int>(grid), st)
+                           : dispatch_main<false>(prm, nv, smem, static_cast<int>(grid), st);
+}
+
+static int check_args(const char* name, int64_t n_tokens, int64_t d_model, int64_t d_ff, int tile,
+                      int cap) {
+  if (n_tokens < 0 || d_model < 1 || d_ff < 1) return fail(SGE_ERR_ARG, "%s: bad sizes", name);
+  if (d_model % 8) return fail(SGE_ERR_ARG, "%s: d_model %% 8 != 0", name);
+  if (tile < 1 || tile > 255 || d_ff % tile)
+    return fail(SGE_ERR_ARG, "%s: tile must divide d_ff and be <= 255", name);
+  if (cap < 1 || cap > tile) return fail(SGE_ERR_ARG, "%s: cap outside [1, tile]", name);
+  if (d_ff >= (1LL << 31) || n_tokens >= (1LL << 31))
+    return fail(SGE_ERR_UNSUPPORTED, "%s: size beyond the supported range", name);
+  return SGE_OK;
+}
+
+}  // namespace sge
+
+using namespace sge;
+
+extern "C" size_t twell_fused_up_down_workspace_bytes(int64_t n_tokens, int64_t d_model) {
+  if (n_tokens < 0 || d_model < 1) return 0;
+  return WsLayout(n_tokens, d_model, pool_slots_for(kPoolBytes, d_model)).total;
+}
+
+extern "C" int twell_fused_up_down(const void* x, const uint8_t* count, const uint8_t* idx,
+                                   const void* val, const void* wu_t, const void* wd, void* y,
+                                   int64_t n_tokens, int64_t d_model, int64_t d_ff, int dtype,
+                                   int tile, int cap, void* workspace, size_t workspace_bytes,
+                                   int32_t* diag, void* stream) {
+  static const char* kName = "twell_fused_up_down";
+  clear_error();
+  int rc = check_args(kName, n_tokens, d_model, d_ff, tile, cap);
+  if (rc) return rc;
+  if (n_tokens == 0) return SGE_OK;
+  if (!x || !count || !idx || !val || !wu_t || !wd || !y || !workspace)
+    return fail(SGE_ERR_ARG, "%s: null pointer", kName);
+  if (!aligned16(x) || !aligned16(wu_t) || !aligned16(wd) || !aligned16(y) || !aligned16(val) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(SGE_ERR_ARG, "%s: pointer not 16-byte aligned (workspace: 256)", kName);
+  const size_t need = twell_fused_up_down_workspace_bytes(n_tokens, d_model);
+  if (workspace_bytes < need)
+    return fail(SGE_ERR_ARG, "%s: workspace of %zu bytes, %zu needed", kName, workspace_bytes, need);
+  return run_fused(kName, x, count, idx, val, wu_t, wd, y, n_tokens, d_model, d_ff, dtype, tile, cap,
+                   workspace, pool_slots_for(kPoolBytes, d_model), diag,
+                   static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------
@@ -453,14 +970,19 @@ extern "C" int twell_fused_up_down(const void* x, const uint8_t* count, const ui
 // handed all device memory to its own pools, a plugin that receives only the
 // tensors it works on).  For them the workspace of twell_fused_up_down lives
 // in this file-scope device array instead, sized for at most
-// kNoAllocMaxTokens tokens; every GPU that loads the library holds it until
-// the process exits.  In host code `g_fused_scratch` names a host-side stand-in,
+// kNoAllocMaxTokens tokens and a smaller pool for the partial outputs of
+// split heavy tokens; every GPU that loads the library holds it until the
+// process exits.  In host code `g_fused_scratch` names a host-side stand-in,
 // not a device address, so its device address is looked up per device with
 // cudaGetSymbolAddress, once, with that device current.
 
-constexpr int64_t kNoAllocMaxTokens = 262144;
+constexpr int64_t kNoAllocMaxTokens = 65536;
+constexpr int64_t kNoAllocPoolSlots = 1024;
+constexpr size_t kNoAllocPoolBytes = size_t(4) << 20;
 constexpr size_t kNoAllocScratchBytes =
-    (kWsHeader + 5 * static_cast<size_t>(kNoAllocMaxTokens) + 15) & ~static_cast<size_t>(15);
+    kHdrBytes + ((8 * static_cast<size_t>((kNoAllocMaxTokens + 255) / 256) + 255) & ~size_t(255)) +
+    4 * static_cast<size_t>(kNoAllocMaxTokens) + 8 * kLightClasses * static_cast<size_t>(kNoAllocMaxTokens) +
+    static_cast<size_t>(kNoAllocPoolSlots) * (32 + 4) + kNoAllocPoolBytes + 1024;
 
 static __device__ __align__(256) uint8_t g_fused_scratch[kNoAllocScratchBytes];
 
@@ -498,50 +1020,31 @@ extern "C" int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, 
                                            const void* val, const void* wu_t, const void* wd,
                                            void* y, int64_t n_tokens, int64_t d_model,
                                            int64_t d_ff, int dtype, int tile, int cap,
-                                           void* stream) {
+                                           int32_t* diag, void* stream) {
+  static const char* kName = "twell_fused_up_down_noalloc";
   clear_error();
-  if (n_tokens < 0 || d_model < 1 || d_ff < 1)
-    return fail(SGE_ERR_ARG, "twell_fused_up_down_noalloc: bad sizes");
   if (n_tokens > kNoAllocMaxTokens)
     return fail(SGE_ERR_UNSUPPORTED,
-                "twell_fused_up_down_noalloc: %lld tokens exceed the built-in scratch limit of %lld; "
+                "%s: %lld tokens exceed the built-in scratch limit of %lld; "
                 "use twell_fused_up_down with a workspace",
-                (long long)n_tokens, (long long)kNoAllocMaxTokens);
-  if (d_model % 8) return fail(SGE_ERR_ARG, "twell_fused_up_down_noalloc: d_model %% 8 != 0");
-  if (tile < 1 || tile > 255 || d_ff % tile)
-    return fail(SGE_ERR_ARG, "twell_fused_up_down_noalloc: tile must divide d_ff and be <= 255");
-  if (cap < 1 || cap > tile)
-    return fail(SGE_ERR_ARG, "twell_fused_up_down_noalloc: cap outside [1, tile]");
-  if (d_ff >= (1LL << 31)) return fail(SGE_ERR_UNSUPPORTED, "twell_fused_up_down_noalloc: d_ff beyond 2^31");
+                kName, (long long)n_tokens, (long long)kNoAllocMaxTokens);
+  int rc = check_args(kName, n_tokens, d_model, d_ff, tile, cap);
+  if (rc) return rc;
   if (n_tokens == 0) return SGE_OK;
   if (!x || !count || !idx || !val || !wu_t || !wd || !y)
-    return fail(SGE_ERR_ARG, "twell_fused_up_down_noalloc: null pointer");
+    return fail(SGE_ERR_ARG, "%s: null pointer", kName);
   if (!aligned16(x) || !aligned16(wu_t) || !aligned16(wd) || !aligned16(y) || !aligned16(val))
-    return fail(SGE_ERR_ARG, "twell_fused_up_down_noalloc: pointer not 16-byte aligned");
+    return fail(SGE_ERR_ARG, "%s: pointer not 16-byte aligned", kName);
+  int64_t slots = pool_slots_for(kNoAllocPoolBytes, d_model);
+  if (slots > kNoAllocPoolSlots) slots = kNoAllocPoolSlots;
+  if (WsLayout(n_tokens, d_model, slots).total > kNoAllocScratchBytes)
+    return fail(SGE_ERR_UNSUPPORTED, "%s: built-in scratch too small for this shape", kName);
   void* scratch = nullptr;
-  int rc = scratch_address(&scratch);
+  rc = scratch_address(&scratch);
   if (rc) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  UdParams prm;
-  prm.x = x;
-  prm.count = count;
-  prm.idx = idx;
-  prm.val = val;
-  prm.wu_t = wu_t;
-  prm.wd = wd;
-  prm.y = y;
-  prm.ws = static_cast<int*>(scratch);
-  prm.heavy_flag = static_cast<const uint8_t*>(scratch) + kWsHeader + 4 * static_cast<size_t>(n_tokens);
-  prm.n_rows = n_tokens;
-  prm.d = static_cast<int>(d_model);
-  prm.n_cols = static_cast<int>(d_ff);
-  prm.tile = tile;
-  prm.cap = cap;
-  // the array keeps the previous call's contents: the cursors start at zero
-  cudaError_t e = cudaMemsetAsync(scratch, 0, kWsHeader, st);
-  if (e != cudaSuccess)
-    return fail(SGE_ERR_CUDA, "twell_fused_up_down_noalloc: %s", cudaGetErrorString(e));
-  if (dtype == SGE_BF16) return dispatch_ud<true>(prm, st);
-  if (dtype == SGE_F32) return dispatch_ud<false>(prm, st);
-  return fail(SGE_ERR_UNSUPPORTED, "twell_fused_up_down_noalloc: dtype %d", dtype);
+  // The array keeps the previous call's contents; the planning kernels reset
+  // every counter the call relies on (job counters and cursor, and the
+  // completion counter of each split token).
+  return run_fused(kName, x, count, idx, val, wu_t, wd, y, n_tokens, d_model, d_ff, dtype, tile, cap,
+                   scratch, slots, diag, static_cast<cudaStream_t>(stream));
 }

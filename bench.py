@@ -158,7 +158,7 @@ def run_own(args, rank, world, local_rank):
     h = torch.empty((n, f), dtype=x.dtype, device=dev)
     y_dense = torch.empty_like(x)
     diag = sge.new_diag(dev)
-    ws = sge.fused_workspace(n, dev)
+    ws = sge.fused_workspace(n, d, dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 

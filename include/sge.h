@@ -122,19 +122,27 @@ int twell_gate_pack(const void* x, const void* wg_t, int64_t n_tokens, int64_t d
  *   x [N][d], wu_t [F][d], wd [F][d], y [N][d] in dtype; count/idx/val the
  *   TwELL produced by twell_gate_pack with the same T and C.
  *   workspace  device scratch of at least
- *              twell_fused_up_down_workspace_bytes(N) bytes, 16-byte aligned,
- *              owned by the caller; it holds the list of heavy tokens (those
- *              processed by a whole SM) and work cursors, and must not be
- *              shared by calls that may run concurrently.
- * Errors: as twell_gate_pack; SGE_ERR_ARG for a missing or short workspace;
- * SGE_ERR_UNSUPPORTED for d > 4096 (bf16) or d > 2048 (fp32).
+ *              twell_fused_up_down_workspace_bytes(N, d) bytes (N-proportional
+ *              lists plus a pool of about 64 MiB), 256-byte aligned, owned by
+ *              the caller; it holds per-token entry counts, the job lists,
+ *              the fp32 partial outputs of the units that heavy tokens are
+ *              split into, and counters; it must not be shared by calls that
+ *              may run concurrently.  Empty tokens get y = 0.
+ *   tile       T, with F / T <= 256 TwELL tiles per row.
+ *   diag       nullable int32[4]; diag[SGE_DIAG_FLAGS] gets SGE_FLAG_TIMEOUT
+ *              if a pipeline wait gave up (y is then invalid).
+ * Results are deterministic: repeated calls on the same inputs give the same
+ * bits, whatever the scheduling.
+ * Errors: as twell_gate_pack; SGE_ERR_ARG for a missing, short or misaligned
+ * workspace; SGE_ERR_UNSUPPORTED for d > 4096 or
+ * F / T > 256.
  */
-size_t twell_fused_up_down_workspace_bytes(int64_t n_tokens);
+size_t twell_fused_up_down_workspace_bytes(int64_t n_tokens, int64_t d_model);
 
 int twell_fused_up_down(const void* x, const uint8_t* count, const uint8_t* idx, const void* val,
                         const void* wu_t, const void* wd, void* y, int64_t n_tokens,
                         int64_t d_model, int64_t d_ff, int dtype, int tile, int cap,
-                        void* workspace, size_t workspace_bytes, void* stream);
+                        void* workspace, size_t workspace_bytes, int32_t* diag, void* stream);
 
 /*
  * twell_fused_up_down_noalloc -- twell_fused_up_down for callers that cannot
@@ -148,22 +156,24 @@ int twell_fused_up_down(const void* x, const uint8_t* count, const uint8_t* idx,
  * workspace and allocates nothing (no cudaMalloc, no cudaFree, no allocating
  * library routine).  Its scratch is a fixed device array built into the
  * library, sized for at most twell_fused_up_down_noalloc_max_tokens()
- * tokens (262144; about 1.3 MB, held on every GPU that loads the library
+ * tokens (262144; about 7.2 MB, held on every GPU that loads the library
  * until the process exits).  Larger N is rejected with SGE_ERR_UNSUPPORTED.
  *
  * The first call on a device looks up the array's device address on that
  * device (cudaGetSymbolAddress); make that first call before any stream
  * capture.  Every call shares the one array, so calls that may overlap on
  * the GPU (different streams, or different host threads on the same device)
- * race and must be serialised by the caller.  Results equal those of
- * twell_fused_up_down.
+ * race and must be serialised by the caller.  Results agree with those of
+ * twell_fused_up_down up to fp32 rounding order: the array's smaller pool for
+ * partial outputs splits the heaviest tokens into fewer, longer units, which
+ * also makes heavy-tailed batches slower than with a workspace.
  */
 int64_t twell_fused_up_down_noalloc_max_tokens(void);
 
 int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, const uint8_t* idx,
                                 const void* val, const void* wu_t, const void* wd, void* y,
                                 int64_t n_tokens, int64_t d_model, int64_t d_ff, int dtype,
-                                int tile, int cap, void* stream);
+                                int tile, int cap, int32_t* diag, void* stream);
 
 /*
  * dense_ffn_fwd -- the dense gated FFN the method is compared against

@@ -74,22 +74,27 @@ def test_bad_arguments_are_rejected_on_host(lib):
 def test_empty_input_is_a_no_op(lib):
     assert _gate(lib, n=0) == 0
     assert lib.twell_fused_up_down(None, None, None, None, None, None, None, 0, 64, 256,
-                                   sge.SGE_BF16, 128, 128, None, 0, None) == 0
+                                   sge.SGE_BF16, 128, 128, None, 0, None, None) == 0
     assert lib.dense_ffn_fwd(None, None, None, None, None, None, 0, 64, 256, None, None) == 0
 
 
 def test_fused_rejects_bad_arguments(lib):
     assert lib.twell_fused_up_down(None, None, None, None, None, None, None, 8, 12, 256,
-                                   sge.SGE_BF16, 128, 128, None, 0, None) == 1
+                                   sge.SGE_BF16, 128, 128, None, 0, None, None) == 1
     assert lib.twell_fused_up_down(None, None, None, None, None, None, None, 8, 64, 256,
-                                   sge.SGE_BF16, 128, 128, None, 0, None) == 1
+                                   sge.SGE_BF16, 128, 128, None, 0, None, None) == 1
     p = ctypes.c_void_p(16)
     # a workspace smaller than the query's answer is rejected
     assert lib.twell_fused_up_down(p, p, p, p, p, p, p, 1000, 64, 256, sge.SGE_BF16, 128, 128,
-                                   p, 64, None) == 1
+                                   p, 64, None, None) == 1
     assert b"workspace" in lib.sge_last_error()
-    assert lib.twell_fused_up_down_workspace_bytes(1000) >= 16 + 5 * 1000
-    assert lib.twell_fused_up_down_workspace_bytes(1000) % 16 == 0
+    assert lib.twell_fused_up_down_workspace_bytes(1000, 64) >= 16 + 5 * 1000
+    assert lib.twell_fused_up_down_workspace_bytes(1000, 64) % 256 == 0
+    # the workspace must be 256-byte aligned
+    ws = lib.twell_fused_up_down_workspace_bytes(1000, 64)
+    assert lib.twell_fused_up_down(p, p, p, p, p, p, p, 1000, 64, 256, sge.SGE_BF16, 128, 128,
+                                   ctypes.c_void_p(4096 + 16), ws, None, None) == 1
+    assert b"aligned" in lib.sge_last_error()
     assert lib.dense_ffn_fwd(None, None, None, None, None, None, 8, 64, 100, None, None) == 1
 
 

@@ -95,7 +95,7 @@ def test_gate_pack_gaussian_sign_flips(cuda_device, name, cap):
 def test_fused_up_down_matches_oracle(cuda_device, dtype, tol, n, d, f, tile, cap):
     """Both sides get the same TwELL (the oracle's pack of its fp64 G)."""
     if dtype == torch.float32 and d > 2048:
-        pytest.skip("fp32 rows are limited to d_model <= 2048 (test_fused_fp32_d_limit)")
+        pytest.skip("fp32 rows are limited to d_model <= 2048 (test_fused_d_limit)")
     inp = synth.make_inputs(synth.CONFIGS["ffn_0p5b_bf16"].with_(
         n_tokens=n, d_model=d, d_ff=f, dtype="bf16" if dtype == torch.bfloat16 else "f32",
         rho=0.05))
@@ -108,11 +108,13 @@ def test_fused_up_down_matches_oracle(cuda_device, dtype, tol, n, d, f, tile, ca
     assert err <= tol, err
 
 
-def test_fused_fp32_d_limit(cuda_device):
-    """fp32 rows are held as 16-byte vectors over 128 threads, at most 4 each."""
-    x = torch.zeros(4, 2056, dtype=torch.float32, device=cuda_device)
-    w = torch.zeros(128, 2056, dtype=torch.float32, device=cuda_device)
-    tw = sge.TwELL.empty(4, 128, 128, 128, torch.float32, cuda_device)
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 4104), (torch.float32, 2056)])
+def test_fused_d_limit(cuda_device, dtype, d):
+    """A warp keeps at most 16 sixteen-byte pieces of a row per lane: rows of
+    at most 8 KB (bf16 d <= 4096, fp32 d <= 2048); longer rows are rejected."""
+    x = torch.zeros(4, d, dtype=dtype, device=cuda_device)
+    w = torch.zeros(128, d, dtype=dtype, device=cuda_device)
+    tw = sge.TwELL.empty(4, 128, 128, 128, dtype, cuda_device)
     tw.count.zero_()
     with pytest.raises(sge.LibraryError, match="too large"):
         sge.twell_fused_up_down(x, tw, w, w)
@@ -120,8 +122,8 @@ def test_fused_fp32_d_limit(cuda_device):
 
 @pytest.mark.parametrize("dtype,tol", [(torch.bfloat16, BF16_TOL), (torch.float32, F32_TOL)])
 def test_fused_heavy_and_light_tokens(cuda_device, dtype, tol):
-    """Tokens above the heavy threshold (processed by a whole CTA, tiles split
-    across its groups, several shared-memory chunks each) mixed with light
+    """Tokens far above the mean (split into units whose fp32 partial outputs
+    are summed in unit order, several 32-entry chunks each) mixed with light
     ones; every row is checked."""
     n, d, f = 200, 264, 4096
     inp = synth.make_inputs(synth.CONFIGS["ffn_0p5b_bf16"].with_(
