@@ -38,23 +38,35 @@ struct HybridView {
 
 // ---------------------------------------------------------------- pack
 
-// One CTA: per-row stored entry counts, routing, and the ascending ranks of
-// the spill rows (block-wide exclusive scan over contiguous row ranges).
-__global__ void __launch_bounds__(kPackThreads)
-    hybrid_route_kernel(const uint8_t* __restrict__ count, int nt, int cap, HybridView hv,
-                        int32_t* diag) {
+// Stored entries per row (counts capped at C), one thread per row.
+__global__ void __launch_bounds__(256) hybrid_nnz_kernel(const uint8_t* __restrict__ count, int nt,
+                                                         int cap, HybridView hv) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  if (t >= hv.n) return;
+  const uint8_t* c = count + t * nt;
+  int nnz = 0;
+  if ((nt & 3) == 0 && (reinterpret_cast<uintptr_t>(count) & 3) == 0) {
+    const uint32_t* c4 = reinterpret_cast<const uint32_t*>(c);
+    for (int b = 0; b < nt / 4; ++b) {
+      const uint32_t v = __ldg(c4 + b);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) nnz += min(static_cast<int>((v >> (8 * k)) & 255u), cap);
+    }
+  } else {
+    for (int b = 0; b < nt; ++b) nnz += min(static_cast<int>(__ldg(c + b)), cap);
+  }
+  hv.row_nnz[t] = nnz;
+}
+
+// One CTA: routing and the ascending ranks of the spill rows (block-wide
+// exclusive scan over contiguous row ranges of the per-row counts).
+__global__ void __launch_bounds__(kPackThreads) hybrid_route_kernel(HybridView hv, int32_t* diag) {
   __shared__ int s_scan[kPackThreads];
   const int tid = threadIdx.x;
   const int64_t per = (hv.n + kPackThreads - 1) / kPackThreads;
   const int64_t r0 = tid * per, r1 = min(hv.n, r0 + per);
   int local = 0;
-  for (int64_t t = r0; t < r1; ++t) {
-    const uint8_t* c = count + t * nt;
-    int nnz = 0;
-    for (int b = 0; b < nt; ++b) nnz += min(static_cast<int>(c[b]), cap);
-    hv.row_nnz[t] = nnz;
-    local += nnz > hv.k;
-  }
+  for (int64_t t = r0; t < r1; ++t) local += hv.row_nnz[t] > hv.k;
   s_scan[tid] = local;
   __syncthreads();
   for (int o = 1; o < kPackThreads; o <<= 1) {  // inclusive Hillis-Steele scan
@@ -401,7 +413,10 @@ extern "C" int hybrid_pack(const uint8_t* count, const uint8_t* idx, const void*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const HybridView hv = view_of(hy);
   const int nt = static_cast<int>(hy->d_ff / tile);
-  hybrid_route_kernel<<<1, kPackThreads, 0, st>>>(count, nt, cap, hv, diag);
+  hybrid_nnz_kernel<<<static_cast<unsigned>((hy->n_tokens + 255) / 256), 256, 0, st>>>(count, nt, cap, hv);
+  rc = check_launch("hybrid_pack (count)");
+  if (rc) return rc;
+  hybrid_route_kernel<<<1, kPackThreads, 0, st>>>(hv, diag);
   rc = check_launch("hybrid_pack (route)");
   if (rc) return rc;
   hybrid_fill_kernel<<<static_cast<unsigned>((hy->n_tokens + 7) / 8), 256, 0, st>>>(
