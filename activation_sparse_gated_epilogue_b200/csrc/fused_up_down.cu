@@ -238,13 +238,13 @@ __device__ __forceinline__ int light_class(int n, int U) {
 }
 
 // Job lists: every split token's units, every other non-empty token in its
-// size class; empty tokens get y = 0 here.  Slots in the lists come from
+// size class.  Slots in the lists come from
 // warp-aggregated atomics: the job order may vary between calls, the results
 // do not.
 __global__ void __launch_bounds__(256) ud_jobs_kernel(const int* __restrict__ ntok, int64_t n_rows,
                                                       int* hdr, int2* __restrict__ lights,
                                                       Job* __restrict__ units, int* __restrict__ done,
-                                                      int64_t pool_slots, void* y, int row_bytes) {
+                                                      int64_t pool_slots) {
   const int lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   const unsigned lt = (1u << lane) - 1u;
@@ -300,16 +300,16 @@ __global__ void __launch_bounds__(256) ud_jobs_kernel(const int* __restrict__ nt
     lbase = __shfl_sync(0xffffffffu, lbase, 0);
     if (cls == c) lights[c * n_rows + lbase + __popc(ml & lt)] = make_int2(static_cast<int>(t), n);
   }
-  // empty tokens: the warp writes each one's row of zeros
-  unsigned me = __ballot_sync(0xffffffffu, n == 0);
-  const int64_t t0 = t - lane;
-  const int nvec = row_bytes / 16;
-  while (me) {
-    const int l = __ffs(me) - 1;
-    me &= me - 1u;
-    uint4* row = reinterpret_cast<uint4*>(static_cast<char*>(y) + (t0 + l) * row_bytes);
-    for (int v = lane; v < nvec; v += 32) row[v] = make_uint4(0, 0, 0, 0);
-  }
+}
+
+// y = 0 for tokens without stored entries: a thread per 16 bytes of y
+// (grid-stride).
+__global__ void __launch_bounds__(256) ud_zero_kernel(const int* __restrict__ ntok, int64_t n_rows,
+                                                      int nvec, void* y) {
+  const int64_t total = n_rows * nvec;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * 256)
+    if (ntok[i / nvec] == 0) reinterpret_cast<uint4*>(y)[i] = make_uint4(0, 0, 0, 0);
 }
 
 // -------------------------------------------------------------- main kernel
@@ -910,8 +910,15 @@ static int run_fused(const char* name, const void* x, const uint8_t* count, cons
   if (rc) return rc;
   ud_jobs_kernel<<<static_cast<unsigned>(nblk), 256, 0, st>>>(
       prm.ntok, n_tokens, prm.hdr, const_cast<int2*>(prm.lights), const_cast<Job*>(prm.units),
-      prm.done, pool_slots, y, prm.row_bytes);
+      prm.done, pool_slots);
   rc = check_launch("twell_fused_up_down (jobs)");
+  if (rc) return rc;
+  const int64_t nvec = prm.row_bytes / 16;
+  int64_t zblocks = (n_tokens * nvec + 255) / 256;
+  if (zblocks > 32 * 1024) zblocks = 32 * 1024;
+  ud_zero_kernel<<<static_cast<unsigned>(zblocks), 256, 0, st>>>(
+      prm.ntok, n_tokens, static_cast<int>(nvec), y);
+  rc = check_launch("twell_fused_up_down (zero rows)");
   if (rc) return rc;
   return dtype == SGE_BF16 ? dispatch_main<true>(prm, nv, smem, static_cast<int>(grid), st)
                            : dispatch_main<false>(prm, nv, smem, static_cast<int>(grid), st);

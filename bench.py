@@ -38,6 +38,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "source": "fallback"}
 # fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flop x 1.965 GHz
 FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# ELL capacity of the hybrid format when it serves inference (tokens with more
+# stored entries run on the tensor-core spill GEMMs)
+HYB_INFER_K = 64
 
 # DRAM bytes (read + write) per launch from the committed ncu captures
 # (profiles/*.md), keyed by the source hash of the kernel they were taken on;
@@ -242,6 +245,34 @@ def run_own(args, rank, world, local_rank):
     e2e_value = n * world * e2e_steps / (e2e_ms / 1e3)
     diag_host = diag.tolist()
 
+    # ---- the hybrid format used for inference (a further row of the method,
+    # not the step above): rows with more than K stored entries go through the
+    # dense spill GEMMs on tensor cores, the others through the ELL kernel
+    hyb = None
+    if x.dtype == torch.bfloat16:
+        hk, hs = HYB_INFER_K, max(128, (n // 4 + 127) // 128 * 128)
+        hy = sge.Hybrid.empty(n, f, hk, hs, dev)
+        hws = sge.hybrid_fwd_workspace(d, f, hs, dev)
+        y_h = torch.empty_like(x)
+        hdiag = sge.new_diag(dev)
+        hpack = lambda: sge.hybrid_pack(tw, hk, hs, out=hy, diag=hdiag)
+        hfwd = lambda: sge.hybrid_ffn_fwd(x, hy, wu, wd, wd_t=wd_t, y=y_h, workspace=hws)
+        hsteps = min(args.steps, 100)
+        timed([gate, hpack, hfwd], 0, 3)
+        barrier()
+        evh = timed([gate, hpack, hfwd], hsteps, 0)
+        barrier()
+        h_ms = reduce_max(sum(e[0].elapsed_time(e[3]) for e in evh)) / hsteps
+        dropped = int(hdiag[2].item())
+        err = float(((y_h.float() - y.float()).abs().max() / y.float().abs().max()).item())
+        hyb = {"value": round(n * world / (h_ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(h_ms, 4),
+               "ell_cap_K": hk, "s_max": hs, "spill_rows": int(hy.n_spill.item()), "dropped_rows": dropped,
+               "ms_parts": {"gate": round(statistics.mean(e[0].elapsed_time(e[1]) for e in evh), 4),
+                            "hybrid_pack": round(statistics.mean(e[1].elapsed_time(e[2]) for e in evh), 4),
+                            "hybrid_ffn_fwd": round(statistics.mean(e[2].elapsed_time(e[3]) for e in evh), 4)},
+               "max_abs_rel_vs_fused": round(err, 6),
+               "note": "gate GEMM + TwELL, hybrid_pack, hybrid_ffn_fwd (spill rows' h goes through HBM)"}
+
     if rank != 0:
         return None
 
@@ -257,7 +288,7 @@ def run_own(args, rank, world, local_rank):
     # (at most all of W_up and W_down), TwELL entries and counts, y
     bytes_fused = (2 * n * d + 2 * 2 * f * d + 3 * nnz + n * (f // tile) + 2 * n * d)
     gate_src = src_hash("gate_pack.cu", "tc_gemm.cuh", "sge_common.cuh")
-    fused_src = src_hash("fused_up_down.cu", "sge_common.cuh")
+    fused_src = src_hash("fused_up_down.cu", "sparse_common.cuh", "sge_common.cuh")
     tr_gate = TRAFFIC.get(gate_src)
     tr_fused = TRAFFIC.get(fused_src)
     tr_gate = None if tr_gate is None else int(tr_gate)
@@ -268,7 +299,7 @@ def run_own(args, rank, world, local_rank):
               "ms": round(mg, 4), "share": round(mg / (mg + mf), 3),
               "algorithmic": f"2*N*d*F = {flops_gate:.3e} flop per launch",
               "peak_note": "bf16_tflops (burst) of measured peaks: the step keeps SM clocks at max"}
-    k_fused = {"kernel": "twell_fused_up_down (classify + persistent fused kernel)", "bound": "alu", "achieved": round(fused_tf, 2),
+    k_fused = {"kernel": "twell_fused_up_down (3 planning kernels + persistent main kernel)", "bound": "alu", "achieved": round(fused_tf, 2),
                "peak": round(FP32_SIMT_TFLOPS, 1), "unit": "TFLOP/s",
                "frac": round(fused_tf / FP32_SIMT_TFLOPS, 4), "traffic": tr_fused,
                "ms": round(mf, 4), "share": round(mf / (mg + mf), 3),
@@ -299,8 +330,9 @@ def run_own(args, rank, world, local_rank):
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
                 "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
-        "gpu_launches": 3 * args.steps,
-        "launches_note": "per step: gate GEMM + TwELL epilogue, heavy-token classify, fused up/down",
+        "gpu_launches": 6 * args.steps,
+        "launches_note": "per step: gate GEMM + TwELL epilogue; fused up/down = count, plan, jobs, zero rows, main kernel",
+        "hybrid_inference": hyb,
         "clocks": clocks,
         "diag": diag_host,
         "gpu": torch.cuda.get_device_name(dev),

@@ -156,7 +156,7 @@ int twell_fused_up_down(const void* x, const uint8_t* count, const uint8_t* idx,
  * workspace and allocates nothing (no cudaMalloc, no cudaFree, no allocating
  * library routine).  Its scratch is a fixed device array built into the
  * library, sized for at most twell_fused_up_down_noalloc_max_tokens()
- * tokens (262144; about 7.2 MB, held on every GPU that loads the library
+ * tokens (65536; about 6.6 MB, held on every GPU that loads the library
  * until the process exits).  Larger N is rejected with SGE_ERR_UNSUPPORTED.
  *
  * The first call on a device looks up the array's device address on that
