@@ -47,7 +47,7 @@ HYB_INFER_K = 64
 # a kernel whose source changed since gets null.
 TRAFFIC = {
     "c5973eaffc07627f": 80.4e6,   # gate GEMM + TwELL, profiles/gate_gemm_twell_ffn_1b_bf16.md
-    "fe89ac0e242a0959": 364.4e6,  # fused up/down, profiles/fused_up_down_ffn_1b_bf16.md
+    "7567d00c4e88d7fb": 427.2e6,  # fused up/down main kernel, profiles/fused_up_down_ffn_1b_bf16.md
 }
 
 
