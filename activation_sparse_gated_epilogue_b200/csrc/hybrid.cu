@@ -293,6 +293,9 @@ struct EpiSpillUp {
   int s_max;
   int n_cols;
 
+  // only the kept spill rows are computed
+  __device__ __forceinline__ int m_limit(int m) const { return min(m, min(*n_spill, s_max)); }
+
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {
     const int kept = min(*n_spill, s_max);
@@ -333,6 +336,9 @@ struct EpiScatterRows {
   const int32_t* n_spill;
   int s_max;
   int n_cols;
+
+  // only the kept spill rows are computed
+  __device__ __forceinline__ int m_limit(int m) const { return min(m, min(*n_spill, s_max)); }
 
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {

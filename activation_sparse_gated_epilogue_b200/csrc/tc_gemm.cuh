@@ -49,6 +49,21 @@ struct TileCoord {
   int m_blk, n_blk;
 };
 
+// Rows of A an epilogue needs: an epilogue may bound M by a count that only
+// the device knows (Epi::m_limit); tiles past it are skipped.
+template <class E>
+__device__ __forceinline__ auto epi_m_limit_impl(const E& e, int m, int) -> decltype(e.m_limit(m)) {
+  return e.m_limit(m);
+}
+template <class E>
+__device__ __forceinline__ int epi_m_limit_impl(const E&, int m, long) {
+  return m;
+}
+template <class E>
+__device__ __forceinline__ int epi_m_limit(const E& e, int m) {
+  return epi_m_limit_impl(e, m, 0);
+}
+
 __device__ __forceinline__ TileCoord tile_coord(int tile, int m_blocks) {
   return TileCoord{tile % m_blocks, tile / m_blocks};
 }
@@ -88,7 +103,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m_blocks = (M + kBM - 1) / kBM;
+  const int m_blocks = (epi_m_limit(epi, M) + kBM - 1) / kBM;
   const int n_blocks = (N + BN - 1) / BN;
   const int num_tiles = m_blocks * n_blocks;
   const int k_blocks = (K + kBK - 1) / kBK;
@@ -271,7 +286,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const bool leader = rank == 0;
   const int pair = static_cast<int>(cluster_id_x());
   const int n_pairs = static_cast<int>(cluster_count_x());
-  const int m_blocks = (M + Shape::BM - 1) / Shape::BM;
+  const int m_blocks = (epi_m_limit(epi, M) + Shape::BM - 1) / Shape::BM;
   const int n_blocks = (N + BN - 1) / BN;
   const int num_tiles = m_blocks * n_blocks;
   const int k_blocks = (K + kBK - 1) / kBK;
