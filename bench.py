@@ -59,6 +59,8 @@ def parse():
     p.add_argument("--workload", default="ffn_1b_bf16")
     p.add_argument("--impl", default="own", choices=["own", "reference"])
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    p.add_argument("--sweep", action="store_true",
+                   help="density sweep of the workload (0.25%%..5%%): one JSON line per density")
     p.add_argument("--profile", action="store_true",
                    help="run only warmup + steps of the sparse step (for ncu captures); no JSON")
     return p.parse_args()
@@ -341,6 +343,90 @@ def run_own(args, rank, world, local_rank):
     return out
 
 
+# ------------------------------------------------------- density sweep
+
+SWEEP_RHO = (0.0025, 0.005, 0.01, 0.02, 0.05)
+
+
+def run_sweep(args, local_rank):
+    """The workload's shape at mean densities 0.25%..5%: the gate bias
+    (last input row of W_gate, times the constant last feature of x) is the
+    only input that changes, so W_gate's bias column is rewritten on the GPU
+    for each density.  Per density: the sparse step (gate GEMM + TwELL, fused
+    up/down), the hybrid inference path, and the dense FFNs."""
+    import activation_sparse_gated_epilogue_b200 as sge
+    from activation_sparse_gated_epilogue_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = synth.CONFIGS[args.workload]
+    inp = synth.make_inputs(cfg)
+    n, d, f, tile, cap = cfg.n_tokens, cfg.d_model, cfg.d_ff, cfg.tile, cfg.cap
+    x, wg, wu, wd = (getattr(inp, k).to(dev) for k in ("x", "wg_t", "wu_t", "wd"))
+    wd_t = wd.t().contiguous()
+    tw = sge.TwELL.empty(n, f, tile, cap, x.dtype, dev)
+    y = torch.empty_like(x)
+    ws = sge.fused_workspace(n, d, dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    steps = min(args.steps, 50)
+
+    def timed(fns, steps, warm):
+        evs = []
+        for s_ in range(warm + steps):
+            flush.zero_()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+            e[0].record(stream)
+            for i, fn in enumerate(fns):
+                fn()
+                e[i + 1].record(stream)
+            if s_ >= warm:
+                evs.append(e)
+        torch.cuda.synchronize(dev)
+        return [[e[i].elapsed_time(e[i + 1]) for i in range(len(fns))] for e in evs]
+
+    h = torch.empty((n, f), dtype=x.dtype, device=dev)
+    y_dense = torch.empty_like(x)
+    dense_ms = statistics.mean(t[0] for t in timed([lambda: sge.dense_ffn_fwd(x, wg, wu, wd_t, h=h, y=y_dense)],
+                                                   steps, 3))
+    pk = peaks()
+    out = []
+    for rho in SWEEP_RHO:
+        tau = synth.solve_tau_density(rho, cfg.sigma, d)
+        wg[:, d - 1] = -tau                      # rounded to the weight dtype
+        gate = lambda: sge.twell_gate_pack(x, wg, tile, cap, out=tw)
+        fused = lambda: sge.twell_fused_up_down(x, tw, wu, wd, y=y, workspace=ws)
+        t = timed([gate, fused], steps, 3)
+        mg = statistics.mean(a for a, _ in t)
+        mf = statistics.mean(b for _, b in t)
+        nnz = int(torch.minimum(tw.count.to(torch.int64), torch.tensor(cap, device=dev)).sum().item())
+        per_tok = torch.minimum(tw.count.to(torch.int64), torch.tensor(cap, device=dev)).sum(1)
+        hk = HYB_INFER_K
+        hs = max(128, (int((per_tok > hk).sum().item()) + 127) // 128 * 128)
+        hy = sge.Hybrid.empty(n, f, hk, hs, dev)
+        hws = sge.hybrid_fwd_workspace(d, f, hs, dev)
+        y_h = torch.empty_like(x)
+        th = timed([gate, lambda: sge.hybrid_pack(tw, hk, hs, out=hy),
+                    lambda: sge.hybrid_ffn_fwd(x, hy, wu, wd, wd_t=wd_t, y=y_h, workspace=hws)], steps, 3)
+        hms = statistics.mean(sum(r) for r in th)
+        flops_gate, flops_fused = 2.0 * n * d * f, 4.0 * nnz * d
+        roof_ms = flops_gate / (pk["bf16_tflops"] * 1e12) * 1e3 + flops_fused / (FP32_SIMT_TFLOPS * 1e12) * 1e3
+        step = mg + mf
+        out.append({
+            "sweep": f"{cfg.name} N={n} d={d} F={f} T={tile} C={cap}", "target_density": rho,
+            "realised_density": round(nnz / (n * f), 5), "nnz": nnz, "tau": round(-float(wg[0, d - 1].item()), 5),
+            "gate_ms": round(mg, 4), "fused_ms": round(mf, 4), "step_ms": round(step, 4),
+            "tokens_per_s": round(n / (step / 1e3), 1),
+            "fused_tflops": round(flops_fused / (mf / 1e3) / 1e12, 2),
+            "fused_l2_row_tbs": round(4.0 * nnz * d / (mf / 1e3) / 1e12, 2),
+            "step_roofline_ms": round(roof_ms, 4), "step_roofline_frac": round(roof_ms / step, 4),
+            "dense_own_ms": round(dense_ms, 4), "speedup_vs_own_dense": round(dense_ms / step, 3),
+            "hybrid_inference_ms": round(hms, 4), "hybrid_speedup_vs_own_dense": round(dense_ms / hms, 3),
+            "hybrid_K": hk, "hybrid_spill_rows": int((per_tok > hk).sum().item()),
+        })
+    return out
+
+
 # ------------------------------------------------ training step (hybrid)
 
 def run_train(args, local_rank):
@@ -506,6 +592,11 @@ def main():
     if args.workload == "train_1b_hybrid":
         if rank == 0:
             print(json.dumps(run_train(args, local_rank)), flush=True)
+        return
+    if args.sweep:
+        if rank == 0:
+            for line in run_sweep(args, local_rank):
+                print(json.dumps(line), flush=True)
         return
     out = run_own(args, rank, world, local_rank)
     if rank == 0 and out is not None:
