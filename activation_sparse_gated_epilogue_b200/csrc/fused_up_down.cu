@@ -897,8 +897,8 @@ static int run_fused(const char* name, const void* x, const uint8_t* count, cons
     return fail(SGE_ERR_UNSUPPORTED, "%s: d_model too large: rows of %d bytes (max 8192)", name, prm.row_bytes);
   if (prm.nt > 256)
     return fail(SGE_ERR_UNSUPPORTED, "%s: %d TwELL tiles per row (max 256)", name, prm.nt);
-  int64_t grid = (n_tokens + prm.teams - 1) / prm.teams;
-  if (grid > sm_count()) grid = sm_count();
+  // every SM gets a CTA (small batches split their tokens into more units)
+  int64_t grid = sm_count();
   if (grid > kMaxCtas) grid = kMaxCtas;
   const int64_t nblk = (n_tokens + 255) / 256;
   ud_count_kernel<<<static_cast<unsigned>(nblk), 256, 0, st>>>(count, n_tokens, prm.nt, cap,

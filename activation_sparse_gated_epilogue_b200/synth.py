@@ -71,6 +71,8 @@ CONFIGS = {
     "ffn_0p5b_bf16": Config("ffn_0p5b_bf16", 4096, 1024, 4096, "bf16", 128, 128, 0.5, rho=0.02),
     "ffn_1b_bf16": Config("ffn_1b_bf16", 8192, 2048, 8192, "bf16", 128, 128, 0.7, rho=0.01),
     "ffn_2b_bf16": Config("ffn_2b_bf16", 16384, 2560, 10240, "bf16", 128, 128, 0.5, rho=0.01),
+    # decode-shaped: a small batch of tokens against the 1B FFN's weights
+    "decode_1b_bf16": Config("decode_1b_bf16", 64, 2048, 8192, "bf16", 128, 128, 0.7, rho=0.01),
     "train_1b_hybrid": Config("train_1b_hybrid", 8192, 2048, 8192, "bf16", 128, 128, 1.0,
                               ell_cap=128, spill_frac=0.02, s_max=1024),
 }
