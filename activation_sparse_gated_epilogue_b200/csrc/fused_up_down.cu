@@ -34,8 +34,8 @@
 // its copies run ahead across chunk and job boundaries.
 //
 // Jobs.  Three small kernels plan the work: stored entries per token; the unit
-// length U (a multiple of 32: heavy tokens split into units of about an
-// eighth of a team's average share, whose fp32 partial outputs fit the
+// length U (a multiple of 32: heavy tokens split into units of about a
+// quarter of a team's average share, whose fp32 partial outputs fit the
 // pool); the job lists: units of heavy tokens first, then the other
 // non-empty tokens in four classes of decreasing size, so that the last jobs
 // are short; empty tokens get y = 0 there.  The team leader pulls jobs from a
@@ -214,9 +214,11 @@ __global__ void __launch_bounds__(1024) ud_plan_kernel(const long long* __restri
   if (threadIdx.x == 0) {
     long long tot = 0;
     for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += wsum[w];
-    // Units of about an eighth of a team's average share; split tokens must
-    // fit the pool (a token of n > U entries takes ceil(n / U) <= 2n / U slots).
-    long long u = (tot + 8 * n_teams - 1) / (8 * n_teams);
+    // Units of about a quarter of a team's average share (measured on the 1B
+    // workload: an eighth costs more job overhead, a half more imbalance);
+    // split tokens must fit the pool (a token of n > U entries takes
+    // ceil(n / U) <= 2n / U slots).
+    long long u = (tot + 4 * n_teams - 1) / (4 * n_teams);
     const long long u_pool = pool_slots > 0 ? (2 * tot + pool_slots - 1) / pool_slots : (1LL << 30);
     if (u < u_pool) u = u_pool;
     if (u < kUnitMin) u = kUnitMin;
