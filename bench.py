@@ -46,8 +46,8 @@ HYB_INFER_K = 64
 # (profiles/*.md), keyed by the source hash of the kernel they were taken on;
 # a kernel whose source changed since gets null.
 TRAFFIC = {
-    "c5973eaffc07627f": 80.4e6,   # gate GEMM + TwELL, profiles/gate_gemm_twell_ffn_1b_bf16.md
-    "7567d00c4e88d7fb": 427.2e6,  # fused up/down main kernel, profiles/fused_up_down_ffn_1b_bf16.md
+    "6a2687f5a38d2d10": 79.3e6,   # gate GEMM + TwELL, profiles/gate_gemm_twell_ffn_1b_bf16.md
+    "f09b286e5d436fcd": 346.2e6,  # fused up/down main kernel, profiles/fused_up_down_ffn_1b_bf16.md
 }
 
 
