@@ -654,11 +654,12 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
         if (e0 + r < cur.n) {
           uint32_t a;
           if (!(ok = acquire(a))) break;
-          float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          // eight independent accumulator chains
+          float s[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-          for (int k = 0; k < NV; ++k) s[k & 3] = E::dot(xr[k], piece(a, k), s[k & 3]);
+          for (int k = 0; k < NV; ++k) E::dot2(xr[k], piece(a, k), s[2 * (k & 3)], s[2 * (k & 3) + 1]);
           release();
-          v = (s[0] + s[1]) + (s[2] + s[3]);
+          v = ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
         }
         p3 = p2;
         p2 = p1;
@@ -810,6 +811,330 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
   }
 }
 
+// ---------------------------------------------------------- small batches
+//
+// With few tokens (decode-sized batches) the persistent kernel's per-warp row
+// streams are short and its latency chain (five launches, the job queue, a
+// ring a few rows deep) dominates.  The small-batch path splits every token
+// into units of E entries (E = 8, doubled until the split tokens' partial
+// outputs fit the pool), gives each unit one CTA of kSmWarps warps and each
+// warp one entry at a time: the warp loads x[t], the W_up row and the W_down
+// row with plain 16-byte loads issued together, so a unit costs one memory
+// round trip.  The warps' partial rows are summed in warp order in shared
+// memory; a token of one unit stores y directly, the others store fp32
+// partials in the pool and the CTA that completes a token's last unit (a
+// counter per token) sums them in unit order.  Results do not depend on
+// scheduling.
+
+constexpr int kSmallTokens = 64;   // tokens at most for the small-batch path (measured: it
+                                   // loses to the persistent kernel from about 128 tokens)
+constexpr int kSmWarps = 8;        // warps per CTA (the smallest unit length)
+
+// Exclusive prefix sum over the kSmallTokens threads of one CTA; returns the
+// exclusive value of this thread and writes the total to *total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* tmp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) tmp[warp] = incl;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int s = 0;
+    for (int w = 0; w < kSmallTokens / 32; ++w) {
+      const int c = tmp[w];
+      tmp[w] = s;
+      s += c;
+    }
+    tmp[kSmallTokens / 32] = s;
+  }
+  __syncthreads();
+  const int r = tmp[warp] + incl - v;
+  *total = tmp[kSmallTokens / 32];
+  __syncthreads();
+  return r;
+}
+
+// Entries per token, the unit length E, every token's first unit (ufirst,
+// n_rows + 1 entries) and first pool slot (pbase), zeroed completion
+// counters.  One CTA of kSmallTokens threads, a thread per token.
+__global__ void __launch_bounds__(kSmallTokens) us_plan_kernel(const uint8_t* __restrict__ count,
+                                                              int64_t n_rows, int nt, int cap,
+                                                              int64_t pool_slots, int* hdr,
+                                                              int* __restrict__ ntok,
+                                                              int* __restrict__ ufirst,
+                                                              int* __restrict__ pbase,
+                                                              int* __restrict__ done) {
+  __shared__ int tmp[kSmallTokens / 32 + 1];
+  const int t = threadIdx.x;
+  int n = 0;
+  if (t < n_rows) {
+    const uint8_t* c = count + static_cast<int64_t>(t) * nt;
+    if ((nt & 15) == 0 && (reinterpret_cast<uintptr_t>(count) & 15) == 0) {
+      // 16 counts per load, all loads in flight together
+      for (int b = 0; b < nt; b += 16) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(c + b));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) n += min(static_cast<int>((w[q] >> (8 * k)) & 255u), cap);
+      }
+    } else {
+      for (int b = 0; b < nt; ++b) n += min(static_cast<int>(__ldg(c + b)), cap);
+    }
+    ntok[t] = n;
+    done[t] = 0;
+  }
+  // the smallest E (kSmWarps times a power of two) whose split tokens fit the pool
+  int E = kSmWarps;
+  for (;;) {
+    const int nu = t < n_rows ? max(1, (n + E - 1) / E) : 0;
+    int split = 0;
+    block_exclusive_scan(nu > 1 ? nu : 0, tmp, &split);
+    if (split <= pool_slots || E >= (1 << 24)) break;
+    E *= 2;
+  }
+  const int nu = t < n_rows ? max(1, (n + E - 1) / E) : 0;
+  int units = 0, split = 0;
+  const int uf = block_exclusive_scan(nu, tmp, &units);
+  const int pb = block_exclusive_scan(nu > 1 ? nu : 0, tmp, &split);
+  if (t < n_rows) {
+    ufirst[t] = uf;
+    pbase[t] = pb;
+  }
+  if (t == 0) {
+    ufirst[n_rows] = units;
+    hdr[kHUnit] = E;
+    hdr[kHUnits] = units;
+    hdr[kHOverflow] = split > pool_slots ? 1 : 0;
+  }
+}
+
+struct UsParams {
+  const void* x;
+  const uint8_t* count;
+  const uint8_t* idx;
+  const void* val;
+  const void* wu_t;
+  const void* wd;
+  void* y;
+  const int* hdr;
+  const int* ntok;
+  const int* ufirst;
+  const int* pbase;
+  int* done;
+  float* pool;
+  int64_t n_rows;
+  int d;
+  int nt;
+  int tile;
+  int cap;
+  int pieces;  // 16-byte pieces per row
+};
+
+// One CTA per unit (grid-stride over the units), kSmWarps warps; NV pieces
+// of a row per lane.
+template <bool BF16, int NTR, int NV>
+__global__ void __launch_bounds__(kSmWarps * 32, 1) us_main_kernel(const UsParams p) {
+  using E = Elem<BF16>;
+  constexpr int VEC = E::VEC;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  float* red = reinterpret_cast<float*>(smem);  // [kSmWarps][d]
+  int* uf = reinterpret_cast<int*>(smem + kSmWarps * p.d * 4);  // [n_rows + 1]
+  __shared__ int last_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i <= p.n_rows; i += blockDim.x) uf[i] = p.ufirst[i];
+  __syncthreads();
+  const int EU = p.hdr[kHUnit];
+  const int n_units = p.hdr[kHUnits];
+  const int64_t rb = static_cast<int64_t>(p.pieces) * 16;
+  for (int k = blockIdx.x; k < n_units; k += gridDim.x) {
+    // the unit's token: the last t with uf[t] <= k
+    int lo = 0, hi = static_cast<int>(p.n_rows) - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (uf[mid] <= k) lo = mid; else hi = mid - 1;
+    }
+    const int t = lo;
+    const int u = k - uf[t];
+    const int nu = uf[t + 1] - uf[t];
+    const int n = p.ntok[t];
+    const int e_end = min(n, (u + 1) * EU);
+    float acc[NV][VEC];
+#pragma unroll
+    for (int q = 0; q < NV; ++q)
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[q][v] = 0.0f;
+    int e = u * EU + warp;
+    if (e < e_end) {
+      // exclusive prefix of the token's capped tile counts (tile b: lane b % 32, register b / 32)
+      int pre[NTR];
+      {
+        const uint8_t* cnt = p.count + static_cast<int64_t>(t) * p.nt;
+        int c[NTR];
+#pragma unroll
+        for (int r = 0; r < NTR; ++r) {
+          const int b = lane + 32 * r;
+          c[r] = b < p.nt ? min(static_cast<int>(__ldg(cnt + b)), p.cap) : 0;
+        }
+        int carry = 0;
+#pragma unroll
+        for (int r = 0; r < NTR; ++r) {
+          int incl = c[r];
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+          }
+          pre[r] = carry + incl - c[r];
+          carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+      }
+      uint4 xr[NV];
+      const uint4* xrow = reinterpret_cast<const uint4*>(static_cast<const char*>(p.x) + t * rb);
+#pragma unroll
+      for (int q = 0; q < NV; ++q) {
+        const int pc = lane + 32 * q;
+        xr[q] = pc < p.pieces ? __ldg(xrow + pc) : make_uint4(0, 0, 0, 0);
+      }
+      // this warp's entries e, e + kSmWarps, ...: 32 resolved at a time, one per lane
+      for (; e < e_end; e += 32 * kSmWarps) {
+        const int my = e + kSmWarps * lane;
+        const int er = my < e_end ? my : e;
+        int b = 0;
+#pragma unroll
+        for (int step = 16 * NTR; step > 0; step >>= 1) {
+          const int cand = b + step;
+          const int v = prefix_at<NTR>(pre, cand < p.nt ? cand : 0);
+          if (cand < p.nt && v <= er) b = cand;
+        }
+        const int s = er - prefix_at<NTR>(pre, b);
+        int j = 0;
+        float a = 0.0f;
+        if (my < e_end) {
+          const int64_t at = (static_cast<int64_t>(t) * p.nt + b) * p.cap + s;
+          j = min(b * p.tile + static_cast<int>(__ldg(p.idx + at)), p.nt * p.tile - 1);
+          a = E::load_val(p.val, at);
+        }
+        const int cnt = min(32, (e_end - e + kSmWarps - 1) / kSmWarps);
+        for (int i = 0; i < cnt; ++i) {
+          const int ji = __shfl_sync(0xffffffffu, j, i);
+          const float ai = __shfl_sync(0xffffffffu, a, i);
+          const uint4* ur = reinterpret_cast<const uint4*>(static_cast<const char*>(p.wu_t) + ji * rb);
+          const uint4* dr = reinterpret_cast<const uint4*>(static_cast<const char*>(p.wd) + ji * rb);
+          uint4 wu[NV], wdv[NV];
+#pragma unroll
+          for (int q = 0; q < NV; ++q) {
+            const int pc = lane + 32 * q;
+            wu[q] = pc < p.pieces ? __ldg(ur + pc) : make_uint4(0, 0, 0, 0);
+            wdv[q] = pc < p.pieces ? __ldg(dr + pc) : make_uint4(0, 0, 0, 0);
+          }
+          float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+          for (int q = 0; q < NV; ++q) s4[q & 3] = E::dot(xr[q], wu[q], s4[q & 3]);
+          float dot = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+          const typename E::HType h = E::h_of(ai * dot);
+#pragma unroll
+          for (int q = 0; q < NV; ++q) E::axpy(h, wdv[q], acc[q]);
+        }
+      }
+    }
+    // the warps' partial rows, summed in warp order
+    float* mine = red + warp * p.d;
+#pragma unroll
+    for (int q = 0; q < NV; ++q) {
+      const int pc = lane + 32 * q;
+      if (pc < p.pieces)
+#pragma unroll
+        for (int v = 0; v < VEC / 4; ++v)
+          reinterpret_cast<float4*>(mine + pc * VEC)[v] =
+              make_float4(acc[q][4 * v], acc[q][4 * v + 1], acc[q][4 * v + 2], acc[q][4 * v + 3]);
+    }
+    __syncthreads();
+    char* yrow = static_cast<char*>(p.y) + static_cast<int64_t>(t) * rb;
+    float* slot = nu > 1 ? p.pool + static_cast<int64_t>(p.pbase[t] + u) * p.d : nullptr;
+    for (int pc = threadIdx.x; pc < p.pieces; pc += blockDim.x) {
+      float v[VEC];
+#pragma unroll
+      for (int q = 0; q < VEC; ++q) v[q] = 0.0f;
+      for (int w = 0; w < kSmWarps; ++w)
+#pragma unroll
+        for (int q = 0; q < VEC / 4; ++q) {
+          const float4 f = reinterpret_cast<const float4*>(red + w * p.d + pc * VEC)[q];
+          v[4 * q] += f.x;
+          v[4 * q + 1] += f.y;
+          v[4 * q + 2] += f.z;
+          v[4 * q + 3] += f.w;
+        }
+      if (nu == 1) {
+        reinterpret_cast<uint4*>(yrow)[pc] = E::pack(v);
+      } else {
+#pragma unroll
+        for (int q = 0; q < VEC / 4; ++q)
+          reinterpret_cast<float4*>(slot + pc * VEC)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      }
+    }
+    if (nu > 1) {
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) last_flag = atomicAdd(p.done + t, 1) == nu - 1;
+      __syncthreads();
+      if (last_flag) {
+        __threadfence();
+        const float* base = p.pool + static_cast<int64_t>(p.pbase[t]) * p.d;
+        for (int pc = threadIdx.x; pc < p.pieces; pc += blockDim.x) {
+          float v[VEC];
+#pragma unroll
+          for (int q = 0; q < VEC; ++q) v[q] = 0.0f;
+          for (int w = 0; w < nu; ++w)
+#pragma unroll
+            for (int q = 0; q < VEC / 4; ++q) {
+              const float4 f = __ldcg(reinterpret_cast<const float4*>(base + static_cast<int64_t>(w) * p.d + pc * VEC) + q);
+              v[4 * q] += f.x;
+              v[4 * q + 1] += f.y;
+              v[4 * q + 2] += f.z;
+              v[4 * q + 3] += f.w;
+            }
+          reinterpret_cast<uint4*>(yrow)[pc] = E::pack(v);
+        }
+      }
+    }
+    __syncthreads();  // red is written again by the next unit
+  }
+}
+
+template <bool BF16, int NTR, int NV>
+static int launch_small(const UsParams& prm, int smem, int grid, cudaStream_t st) {
+  auto kern = us_main_kernel<BF16, NTR, NV>;
+  const int rc = set_smem_limit(reinterpret_cast<const void*>(kern), smem);
+  if (rc) return rc;
+  kern<<<grid, kSmWarps * 32, smem, st>>>(prm);
+  return check_launch("twell_fused_up_down (small batch)");
+}
+
+template <bool BF16, int NV>
+static int small_ntr(const UsParams& prm, int smem, int grid, cudaStream_t st) {
+  if (prm.nt <= 32) return launch_small<BF16, 1, NV>(prm, smem, grid, st);
+  if (prm.nt <= 64) return launch_small<BF16, 2, NV>(prm, smem, grid, st);
+  if (prm.nt <= 128) return launch_small<BF16, 4, NV>(prm, smem, grid, st);
+  return launch_small<BF16, 8, NV>(prm, smem, grid, st);
+}
+
+template <bool BF16>
+static int small_nv(const UsParams& prm, int nv, int smem, int grid, cudaStream_t st) {
+  switch (nv) {
+    case 2: return small_ntr<BF16, 2>(prm, smem, grid, st);
+    case 4: return small_ntr<BF16, 4>(prm, smem, grid, st);
+    default: return small_ntr<BF16, 8>(prm, smem, grid, st);
+  }
+}
+
 // ------------------------------------------------------------------ host
 
 // Teams per CTA, ring depth and shared-memory layout for rows of
@@ -862,6 +1187,39 @@ static int dispatch_main(const UdParams& prm, int nv, int smem, int grid, cudaSt
   }
 }
 
+// The small-batch path: its planning kernel and its main kernel.
+static int run_small(const UdParams& prm, const WsLayout& L, uint8_t* ws, int64_t pool_slots, int nv,
+                     bool bf16, cudaStream_t st) {
+  UsParams up;
+  up.x = prm.x;
+  up.count = prm.count;
+  up.idx = prm.idx;
+  up.val = prm.val;
+  up.wu_t = prm.wu_t;
+  up.wd = prm.wd;
+  up.y = prm.y;
+  up.hdr = prm.hdr;
+  up.ntok = prm.ntok;
+  int* ufirst = reinterpret_cast<int*>(ws + L.lights);  // n + 1 words, then pbase (n words)
+  int* pbase = ufirst + prm.n_rows + 1;
+  up.ufirst = ufirst;
+  up.pbase = pbase;
+  up.done = prm.done;
+  up.pool = prm.pool;
+  up.n_rows = prm.n_rows;
+  up.d = prm.d;
+  up.nt = prm.nt;
+  up.tile = prm.tile;
+  up.cap = prm.cap;
+  up.pieces = prm.row_bytes / 16;
+  us_plan_kernel<<<1, kSmallTokens, 0, st>>>(prm.count, prm.n_rows, prm.nt, prm.cap, pool_slots, prm.hdr,
+                                             const_cast<int*>(prm.ntok), ufirst, pbase, prm.done);
+  const int rc = check_launch("twell_fused_up_down (small-batch plan)");
+  if (rc) return rc;
+  const int smem = (kSmWarps * prm.d * 4 + 4 * static_cast<int>(prm.n_rows + 1) + 15) & ~15;
+  return bf16 ? small_nv<true>(up, nv, smem, sm_count(), st) : small_nv<false>(up, nv, smem, sm_count(), st);
+}
+
 // Planning kernels and the main kernel, shared by both entry points.
 static int run_fused(const char* name, const void* x, const uint8_t* count, const uint8_t* idx,
                      const void* val, const void* wu_t, const void* wd, void* y, int64_t n_tokens,
@@ -899,6 +1257,8 @@ static int run_fused(const char* name, const void* x, const uint8_t* count, cons
     return fail(SGE_ERR_UNSUPPORTED, "%s: d_model too large: rows of %d bytes (max 8192)", name, prm.row_bytes);
   if (prm.nt > 256)
     return fail(SGE_ERR_UNSUPPORTED, "%s: %d TwELL tiles per row (max 256)", name, prm.nt);
+  if (n_tokens <= kSmallTokens && nv <= 8 && pool_slots >= n_tokens)
+    return run_small(prm, L, ws, pool_slots, nv, dtype == SGE_BF16, st);
   // every SM gets a CTA (small batches split their tokens into more units)
   int64_t grid = sm_count();
   if (grid > kMaxCtas) grid = kMaxCtas;

@@ -30,6 +30,20 @@ struct Elem<true> {
           : "r"(xs[i]), "r"(ws[i]));
     return acc;
   }
+  // two accumulators: acc0 += the products of even elements, acc1 += the odd ones
+  __device__ __forceinline__ static void dot2(const uint4& x, const uint4& w, float& acc0, float& acc1) {
+    const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      asm("{\n\t.reg .b16 xl, xh, wl, wh;\n\t"
+          "mov.b32 {xl, xh}, %2;\n\t"
+          "mov.b32 {wl, wh}, %3;\n\t"
+          "fma.rn.f32.bf16 %0, xl, wl, %0;\n\t"
+          "fma.rn.f32.bf16 %1, xh, wh, %1;\n\t}"
+          : "+f"(acc0), "+f"(acc1)
+          : "r"(xs[i]), "r"(ws[i]));
+  }
   // y += h * w with h already rounded to bf16, exact products
   __device__ __forceinline__ static void axpy(HType hb, const uint4& w, float (&y)[8]) {
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -68,6 +82,12 @@ struct Elem<false> {
     acc = fmaf(__uint_as_float(x.z), __uint_as_float(w.z), acc);
     acc = fmaf(__uint_as_float(x.w), __uint_as_float(w.w), acc);
     return acc;
+  }
+  __device__ __forceinline__ static void dot2(const uint4& x, const uint4& w, float& acc0, float& acc1) {
+    acc0 = fmaf(__uint_as_float(x.x), __uint_as_float(w.x), acc0);
+    acc1 = fmaf(__uint_as_float(x.y), __uint_as_float(w.y), acc1);
+    acc0 = fmaf(__uint_as_float(x.z), __uint_as_float(w.z), acc0);
+    acc1 = fmaf(__uint_as_float(x.w), __uint_as_float(w.w), acc1);
   }
   __device__ __forceinline__ static void axpy(HType h, const uint4& w, float (&y)[4]) {
     y[0] = fmaf(h, __uint_as_float(w.x), y[0]);

@@ -146,6 +146,84 @@ def test_fused_heavy_and_light_tokens(cuda_device, dtype, tol):
         assert err <= tol, (rows[:3], err)
 
 
+# Batches of at most 64 tokens take the small-batch path (units of E entries
+# per CTA, one memory round trip per entry); these cases cover its row widths
+# (2, 4 and 8 sixteen-byte pieces per lane), its tile-count widths (1 to 8
+# registers of 32 tiles), truncated tiles and tokens split over many units.
+@pytest.mark.parametrize("n,d,f,tile,cap,dt", [
+    (1, 2048, 8192, 128, 128, "bf16"),   # one token, 8 pieces per lane
+    (7, 264, 640, 64, 64, "f32"),        # ragged row: 66 pieces
+    (33, 520, 768, 32, 6, "bf16"),       # truncated tiles
+    (64, 1024, 8192, 32, 32, "bf16"),    # 256 tiles per row
+    (40, 1024, 2048, 64, 64, "f32"),     # 4 KB fp32 rows
+])
+def test_fused_small_batch_matches_oracle(cuda_device, n, d, f, tile, cap, dt):
+    dtype = torch.bfloat16 if dt == "bf16" else torch.float32
+    tol = BF16_TOL if dt == "bf16" else F32_TOL
+    inp = synth.make_inputs(synth.CONFIGS["ffn_0p5b_bf16"].with_(
+        n_tokens=n, d_model=d, d_ff=f, dtype=dt, rho=0.05))
+    xf, wgf, wuf, wdf = _f64(inp)
+    ora_tw = oracle.twell_pack(oracle.gate_preact(xf, wgf), tile, cap, KIND[dtype])
+    x, _, wu, wd = _dev(inp, cuda_device)
+    y = sge.twell_fused_up_down(x, _upload_twell(ora_tw, dtype, cuda_device), wu, wd)
+    want = oracle.fused_up_down(xf, ora_tw, wuf, wdf)
+    err = oracle.max_abs_rel(to_f64(y), want)
+    assert err <= tol, err
+
+
+@pytest.mark.parametrize("dtype,tol", [(torch.bfloat16, BF16_TOL), (torch.float32, F32_TOL)])
+def test_fused_small_batch_heavy_tokens(cuda_device, dtype, tol):
+    """A 16-token batch whose heavy tokens hold thousands of entries: each is
+    split into hundreds of units whose fp32 partials are summed in unit order
+    by the CTA that completes the last one; every row is checked."""
+    n, d, f = 16, 264, 4096
+    inp = synth.make_inputs(synth.CONFIGS["ffn_0p5b_bf16"].with_(
+        n_tokens=n, d_model=d, d_ff=f, dtype="bf16" if dtype == torch.bfloat16 else "f32",
+        rho=0.01))
+    x = inp.x.clone()
+    heavy = [0, 5, 15]
+    x[heavy, :-1] *= 25.0
+    xf = x.double().numpy()
+    wgf, wuf, wdf = inp.as_f64("wg_t"), inp.as_f64("wu_t"), inp.as_f64("wd")
+    ora_tw = oracle.twell_pack(oracle.gate_preact(xf, wgf), 128, 128, KIND[dtype])
+    nnz = np.minimum(ora_tw.count, 128).sum(1)
+    assert nnz[heavy].min() > 600
+    y = sge.twell_fused_up_down(x.to(cuda_device), _upload_twell(ora_tw, dtype, cuda_device),
+                                inp.wu_t.to(cuda_device), inp.wd.to(cuda_device))
+    want = oracle.fused_up_down(xf, ora_tw, wuf, wdf)
+    got = to_f64(y)
+    for rows in (heavy, [r for r in range(n) if r not in heavy]):
+        err = oracle.max_abs_rel(got[rows], want[rows])
+        assert err <= tol, (rows[:3], err)
+
+
+def test_fused_small_batch_full_density(cuda_device):
+    """64 tokens with every gate active: 4096 entries per token, more split
+    units than the pool holds at the smallest unit length, so the planner
+    doubles the unit length until the partials fit; the result is the dense
+    FFN."""
+    n, d, f = 64, 2048, 4096
+    inp = synth.make_inputs(synth.CONFIGS["ffn_0p5b_bf16"].with_(n_tokens=n, d_model=d, d_ff=f),
+                            tau=-1e3)
+    x, wg, wu, wd = _dev(inp, cuda_device)
+    y, tw = sge.twell_ffn_forward(x, wg, wu, wd, 128, 128)
+    want = oracle.dense_ffn(*_f64(inp))
+    torch.cuda.synchronize()
+    assert int(tw.count.sum()) == n * f
+    assert oracle.max_abs_rel(to_f64(y), want) <= BF16_TOL
+
+
+def test_fused_small_batch_repeat_is_deterministic(cuda_device):
+    cfg = synth.CONFIGS["decode_1b_bf16"]
+    inp = synth.make_inputs(cfg)
+    x, wg, wu, wd = _dev(inp, cuda_device)
+    tw = sge.twell_gate_pack(x, wg, cfg.tile, cfg.cap)
+    y1 = sge.twell_fused_up_down(x, tw, wu, wd)
+    y2 = sge.twell_fused_up_down(x, tw, wu, wd)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
 def test_fused_up_down_repeat_is_deterministic(cuda_device):
     """Work is handed out dynamically; the result must not depend on it."""
     cfg = synth.CONFIGS["ffn_0p5b_bf16"]

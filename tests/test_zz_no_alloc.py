@@ -66,3 +66,24 @@ def test_noalloc_rejects_more_tokens_than_its_scratch_holds(cuda_device):
     rc = fn(p, p, p, p, p, p, p, limit + 1, 64, 256, sge.SGE_BF16, 128, 128, None, None)
     assert rc == 2
     assert b"scratch limit" in lib.sge_last_error()
+
+
+def test_noalloc_small_batch_full_density(cuda_device):
+    """The built-in pool holds 512 fp32 partial rows at d_model = 2048; a
+    64-token batch with every gate active needs units of 512 entries for its
+    partials to fit, and still equals the dense FFN."""
+    lib, fn = _noalloc_fn()
+    n, d, f = 64, 2048, 4096
+    inp = synth.make_inputs(synth.CONFIGS["ffn_0p5b_bf16"].with_(n_tokens=n, d_model=d, d_ff=f),
+                            tau=-1e3)
+    x, wg, wu, wd = (getattr(inp, k).to(cuda_device) for k in ("x", "wg_t", "wu_t", "wd"))
+    tw = sge.twell_gate_pack(x, wg, 128, 128)
+    stream = ctypes.c_void_p(torch.cuda.current_stream(cuda_device).cuda_stream)
+    y = torch.full_like(x, float("nan"))
+    rc = fn(_ptr(x), _ptr(tw.count), _ptr(tw.idx), _ptr(tw.val), _ptr(wu), _ptr(wd), _ptr(y),
+            n, d, f, sge.SGE_BF16, tw.tile, tw.cap, None, stream)
+    assert rc == 0, lib.sge_last_error()
+    torch.cuda.synchronize()
+    assert int(tw.count.sum()) == n * f
+    want = oracle.dense_ffn(*[inp.as_f64(k) for k in ("x", "wg_t", "wu_t", "wd")])
+    assert oracle.max_abs_rel(y.double().cpu().numpy(), want) <= BF16_TOL
