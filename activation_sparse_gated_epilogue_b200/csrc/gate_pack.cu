@@ -189,6 +189,11 @@ __global__ void __launch_bounds__(256) gate_pack_f32_kernel(const float* __restr
 
 // ----------------------------------------------------------- launchers
 
+// Batches of at most this many tokens run on single-CTA 128 x 128 tiles:
+// with few rows, the CTA pair's 256-row tiles are mostly padding, and the
+// tensor-core time of that padding (not the W_gate bytes) sets the time.
+constexpr int64_t kSmallGateRows = 256;
+
 template <int T>
 static int launch_bf16(const void* x, const void* wg_t, int64_t n, int64_t d, int64_t f, int cap,
                        uint8_t* count, uint8_t* idx, void* val, int32_t* diag, cudaStream_t st) {
@@ -196,6 +201,14 @@ static int launch_bf16(const void* x, const void* wg_t, int64_t n, int64_t d, in
   CUtensorMap ma, mb;
   int rc = make_tmap_bf16(&ma, x, n, d, d, kBM);
   if (rc) return rc;
+  if (n <= kSmallGateRows) {
+    using Small = TcShape<128, 1>;
+    rc = make_tmap_bf16(&mb, wg_t, f, d, d, Small::BN);
+    if (rc) return rc;
+    EpiTwell<T> epi{count, idx, static_cast<uint16_t*>(val), n, static_cast<int>(f), cap, diag};
+    return launch_tc_gemm<Small>(ma, mb, mb, n, f, d, epi, diag, st,
+                                 "twell_gate_pack (bf16 tcgen05, small batch)");
+  }
   rc = make_tmap_bf16(&mb, wg_t, f, d, d, Shape::BN / 2);
   if (rc) return rc;
   EpiTwell<T> epi{count, idx, static_cast<uint16_t*>(val), n, static_cast<int>(f), cap, diag};

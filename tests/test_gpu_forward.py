@@ -37,6 +37,8 @@ def _upload_twell(tw: oracle.TwELL, dtype, dev):
     (128, 64, 256, 32, 5),        # overflow
     (520, 264, 768, 16, 16),
     (64, 512, 1024, 128, 12),
+    (1, 136, 512, 128, 128),      # one token (batches of <= 256 rows: single-CTA tiles)
+    (200, 264, 384, 64, 64),      # ragged rows inside one 128-row tile
 ])
 def test_gate_pack_exact_on_grid_inputs(cuda_device, dtype, n, d, f, tile, cap):
     """Grid inputs make G exact in fp32, so counts, indices and values are
