@@ -147,6 +147,24 @@ class ClockSampler:
 
 # ------------------------------------------------------------- own arm
 
+def reduce_max_over_ranks(v: float, device) -> float:
+    """Max over the ranks of the default process group of a per-rank time
+    (each rank's CUDA-event total); v itself with no group or one rank."""
+    if not torch.distributed.is_available() or not torch.distributed.is_initialized():
+        return v
+    if torch.distributed.get_world_size() == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_tokens_per_s(n_tokens: int, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput of `world` replicas that each processed
+    n_tokens per step for `steps` steps, timed as the slowest rank's max_ms."""
+    return n_tokens * world * steps / (max_ms / 1e3)
+
+
 def run_own(args, rank, world, local_rank):
     import activation_sparse_gated_epilogue_b200 as sge
     from activation_sparse_gated_epilogue_b200 import synth
@@ -188,11 +206,7 @@ def run_own(args, rank, world, local_rank):
         return evs
 
     def reduce_max(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max_over_ranks(v, dev)
 
     gate = lambda: sge.twell_gate_pack(x, wg, tile, cap, out=tw, diag=diag)
     fused = lambda: sge.twell_fused_up_down(x, tw, wu, wd, y=y, workspace=ws)
@@ -214,7 +228,7 @@ def run_own(args, rank, world, local_rank):
     t_fused = [e[1].elapsed_time(e[2]) for e in evs]
     total_ms = reduce_max(sum(a + b for a, b in zip(t_gate, t_fused)))
     ms_step = total_ms / args.steps
-    value = n * world * args.steps / (total_ms / 1e3)
+    value = replica_tokens_per_s(n, world, args.steps, total_ms)
 
     nnz = int(tw.count.to(torch.int64).sum().item())
     density = nnz / (n * f)
@@ -244,7 +258,7 @@ def run_own(args, rank, world, local_rank):
     eve = timed([e2e], e2e_steps, 3)
     barrier()
     e2e_ms = reduce_max(sum(e[0].elapsed_time(e[1]) for e in eve))
-    e2e_value = n * world * e2e_steps / (e2e_ms / 1e3)
+    e2e_value = replica_tokens_per_s(n, world, e2e_steps, e2e_ms)
     diag_host = diag.tolist()
 
     # ---- the hybrid format used for inference (a further row of the method,
@@ -267,7 +281,7 @@ def run_own(args, rank, world, local_rank):
         h_ms = reduce_max(sum(e[0].elapsed_time(e[3]) for e in evh)) / hsteps
         dropped = int(hdiag[2].item())
         err = float(((y_h.float() - y.float()).abs().max() / y.float().abs().max()).item())
-        hyb = {"value": round(n * world / (h_ms / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(h_ms, 4),
+        hyb = {"value": round(replica_tokens_per_s(n, world, 1, h_ms), 1), "unit": "tokens/s", "ms_per_step": round(h_ms, 4),
                "ell_cap_K": hk, "s_max": hs, "spill_rows": int(hy.n_spill.item()), "dropped_rows": dropped,
                "ms_parts": {"gate": round(statistics.mean(e[0].elapsed_time(e[1]) for e in evh), 4),
                             "hybrid_pack": round(statistics.mean(e[1].elapsed_time(e[2]) for e in evh), 4),
