@@ -190,8 +190,12 @@ void oracle_dense_ffn(const double* x, const double* wg_t, const double* wu_t,
 /* ------------------------------------------------------------ hybrid pack */
 
 /* Compress TwELL into the hybrid form.  Row t's nonzero count is the number
- * of stored entries, sum over tiles of min(count, C).  Rows with count <= K
- * are ELL rows: their entries, in ascending global column, fill
+ * of stored entries, sum over tiles of min(count, C); a row with a tile whose
+ * count exceeds C has lost entries to the capacity and cannot be an exact ELL
+ * row, so if its stored count is <= K it is set to K + 1 and the row goes to
+ * the spill (the dense backup path, where a forward given W_gate recomputes
+ * it: the pages' dense path for the rows that do not fit the compact
+ * format).  Rows with count <= K are ELL rows: their entries, in ascending global column, fill
  * ell_idx / ell_a [t][0 .. count) (the rest of the row is -1 / 0).  Rows with
  * count > K are spill rows, numbered in ascending t; the first S_max of them
  * get a dense row of spill_a (zero where inactive) and spill_slot[t] = rank;
@@ -205,10 +209,13 @@ int64_t oracle_hybrid_pack(const uint8_t* count, const uint8_t* idx, const doubl
     int64_t n_spill = 0, dropped = 0;
     for (int64_t t = 0; t < n; ++t) {
         int64_t nnz = 0;
+        int over = 0;
         for (int64_t b = 0; b < nt; ++b) {
             const int c = count[t * nt + b];
             nnz += c < cap ? c : cap;
+            if (c > cap) over = 1;
         }
+        if (over && nnz <= k) nnz = k + 1;
         row_nnz[t] = (int32_t)nnz;
         for (int s = 0; s < k; ++s) { ell_idx[t * k + s] = -1; ell_a[t * k + s] = 0.0; }
         if (nnz <= k) {

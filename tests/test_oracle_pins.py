@@ -244,6 +244,36 @@ def test_hybrid_pack_invariants(k, s_max):
         assert hy.n_spill == (nnz > 0).sum()
 
 
+def test_hybrid_pack_routes_overflowing_rows_to_spill():
+    """Capacity C below the tile width: a row with a tile holding more than C
+    active gates has lost entries and goes to the spill even when its stored
+    count fits K (its row_nnz is then K + 1); rows without overflow route by
+    their count as before; the spill row holds the stored (first C per tile)
+    entries."""
+    tile, cap, k = 8, 2, 6
+    f = 32
+    g = np.full((4, f), -1.0)
+    g[0, [1, 5]] = [0.5, 0.25]            # 2 entries in tile 0: fits C, ELL
+    g[1, [0, 1, 2]] = [1.0, 2.0, 3.0]     # 3 entries in tile 0 > C: spill, K + 1
+    g[2, [0, 9, 17, 25]] = 1.5            # 4 entries, one per tile: ELL
+    g[3, :] = 0.75                        # every gate: 4 tiles x 8 > C: spill
+    tw = oracle.twell_pack(g, tile, cap, oracle.VAL_F64)
+    assert tw.overflow == 2 * 0 + 1 + 4
+    hy = oracle.hybrid_pack(tw, k, 8)
+    np.testing.assert_array_equal(hy.row_nnz, [2, k + 1, 4, 8])
+    np.testing.assert_array_equal(hy.spill_slot, [-1, 0, -1, 1])
+    np.testing.assert_array_equal(hy.spill_rows, [1, 3])
+    assert hy.n_spill == 2 and hy.dropped == 0
+    want1 = np.zeros(f); want1[[0, 1]] = [1.0, 2.0]     # the first C of tile 0
+    np.testing.assert_array_equal(hy.spill_a[0], want1)
+    want3 = np.zeros(f)
+    for b in range(f // tile):
+        want3[b * tile:b * tile + cap] = 0.75
+    np.testing.assert_array_equal(hy.spill_a[1], want3)
+    np.testing.assert_array_equal(hy.ell_idx[0, :2], [1, 5])
+    np.testing.assert_array_equal(hy.ell_idx[2, :4], [0, 9, 17, 25])
+
+
 def _hy_inputs(seed, n=24, d=16, f=64, shift=1.2):
     rng = np.random.default_rng(seed)
     x, wg, wu, wd = _rand(rng, n, d), _rand(rng, f, d), _rand(rng, f, d), _rand(rng, f, d)
