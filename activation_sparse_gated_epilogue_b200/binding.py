@@ -68,7 +68,7 @@ def library() -> ctypes.CDLL:
             "dense_ffn_fwd": (I, [P, P, P, P, P, P, I64, I64, I64, P, P]),
             "hybrid_pack": (I, [P, P, P, I, I, ctypes.POINTER(_SgeHybrid), P, P]),
             "hybrid_ffn_fwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I]),
-            "hybrid_ffn_fwd": (I, [P, ctypes.POINTER(_SgeHybrid), P, P, P, P, I64, P,
+            "hybrid_ffn_fwd": (I, [P, ctypes.POINTER(_SgeHybrid), P, P, P, P, P, I64, P,
                                    ctypes.c_size_t, P]),
             "hybrid_ffn_bwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I64, I, I]),
             "hybrid_ffn_bwd": (I, [P, P, ctypes.POINTER(_SgeHybrid), P, P, P, P, P, P, P, I64, P,
@@ -290,8 +290,12 @@ def hybrid_fwd_workspace(d_model: int, d_ff: int, s_max: int, device) -> torch.T
 
 def hybrid_ffn_fwd(x: torch.Tensor, hy: Hybrid, wu_t: torch.Tensor, wd: torch.Tensor,
                    wd_t: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
-                   workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """y from the hybrid form; fills hy.ell_u and hy.spill_u."""
+                   workspace: Optional[torch.Tensor] = None, stream=None,
+                   wg_t: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y from the hybrid form; fills hy.ell_u and hy.spill_u.  With wg_t the
+    spill rows' activations are recomputed from the gate (and written to
+    hy.spill_a), so rows that reached the spill through an overflowing
+    TwELL tile come out exact."""
     _check(x, "x", torch.bfloat16)
     n, d = x.shape
     f = hy.d_ff
@@ -300,12 +304,15 @@ def hybrid_ffn_fwd(x: torch.Tensor, hy: Hybrid, wu_t: torch.Tensor, wd: torch.Te
     if wd_t is None:
         wd_t = wd.t().contiguous()
     _check(wd_t, "wd_t", torch.bfloat16, (d, f))
+    if wg_t is not None:
+        _check(wg_t, "wg_t", torch.bfloat16, (f, d))
     if y is None:
         y = torch.empty_like(x)
     if workspace is None:
         workspace = hybrid_fwd_workspace(d, f, hy.s_max, x.device)
     cs = hy.c_struct()
-    _call("hybrid_ffn_fwd", _ptr(x), ctypes.byref(cs), _ptr(wu_t), _ptr(wd), _ptr(wd_t), _ptr(y), d,
+    _call("hybrid_ffn_fwd", _ptr(x), ctypes.byref(cs), _ptr(wu_t), _ptr(wd), _ptr(wd_t),
+          _ptr(wg_t) if wg_t is not None else None, _ptr(y), d,
           _ptr(workspace), workspace.numel(), _stream(x.device, stream))
     return y
 

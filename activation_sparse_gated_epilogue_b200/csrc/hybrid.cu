@@ -7,9 +7,10 @@
 // kongchang.com page ("定制CUDA内核：融合与压缩") adds that TwELL is compressed
 // into this hybrid form to minimise activation storage.
 //
-//   hybrid_pack     TwELL -> row nnz, routing (nnz <= K: ELL row, else spill
-//                   row, spill rows numbered in ascending token order), ELL
-//                   columns and values, dense spill rows of a.
+//   hybrid_pack     TwELL -> row nnz, routing (nnz <= K and no tile past its
+//                   capacity: ELL row, else spill row, spill rows numbered in
+//                   ascending token order), ELL columns and values, dense
+//                   spill rows of a.
 //   hybrid_ffn_fwd  ELL rows: the fused sparse up/down (u saved for the
 //                   backward pass); spill rows: gathered and run as tcgen05
 //                   GEMMs, U = X_s W_up (u saved, h = a (.) u), Y_s = H_s W_down,
@@ -38,24 +39,36 @@ struct HybridView {
 
 // ---------------------------------------------------------------- pack
 
-// Stored entries per row (counts capped at C), one thread per row.
+// Stored entries per row (counts capped at C), one thread per row.  A row
+// that lost entries to the capacity (a tile with count > C) and would fit
+// the ELL gets K + 1: it goes to the spill, where the forward can recompute
+// it from the gate.
 __global__ void __launch_bounds__(256) hybrid_nnz_kernel(const uint8_t* __restrict__ count, int nt,
                                                          int cap, HybridView hv) {
   const int64_t t = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   if (t >= hv.n) return;
   const uint8_t* c = count + t * nt;
   int nnz = 0;
+  bool over = false;
   if ((nt & 3) == 0 && (reinterpret_cast<uintptr_t>(count) & 3) == 0) {
     const uint32_t* c4 = reinterpret_cast<const uint32_t*>(c);
     for (int b = 0; b < nt / 4; ++b) {
       const uint32_t v = __ldg(c4 + b);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) nnz += min(static_cast<int>((v >> (8 * k)) & 255u), cap);
+      for (int k = 0; k < 4; ++k) {
+        const int cb = static_cast<int>((v >> (8 * k)) & 255u);
+        nnz += min(cb, cap);
+        over |= cb > cap;
+      }
     }
   } else {
-    for (int b = 0; b < nt; ++b) nnz += min(static_cast<int>(__ldg(c + b)), cap);
+    for (int b = 0; b < nt; ++b) {
+      const int cb = __ldg(c + b);
+      nnz += min(cb, cap);
+      over |= cb > cap;
+    }
   }
-  hv.row_nnz[t] = nnz;
+  hv.row_nnz[t] = over && nnz <= hv.k ? hv.k + 1 : nnz;
 }
 
 // One CTA: routing and the ascending ranks of the spill rows (block-wide
@@ -329,6 +342,57 @@ struct EpiSpillUp {
   }
 };
 
+// Epilogue of [G | U] = X_s [W_gate | W_up] (two B operands): the spill
+// rows' activations recomputed from the gate, a = bf16(ReLU(g)) -> spill_a,
+// spill_u = bf16(u), h = bf16(a u) -> hs (the same roundings as the packed
+// path).  Rows past the kept spill rows are left untouched.
+struct EpiSpillGateUp {
+  uint16_t* spill_a;
+  uint16_t* spill_u;
+  uint16_t* hs;
+  const int32_t* n_spill;
+  int s_max;
+  int n_cols;
+
+  __device__ __forceinline__ int m_limit(int m) const { return min(m, min(*n_spill, s_max)); }
+
+  template <int BN>
+  __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {
+    const int kept = min(*n_spill, s_max);
+#pragma unroll 1
+    for (int ch = 0; ch < BN / 32; ++ch) {
+      uint32_t g[32], u[32];
+      tmem_ld32(taddr + ch * 32, g);
+      tmem_ld32(taddr + BN + ch * 32, u);
+      tmem_ld_wait();
+      const int col0 = n_blk * BN + ch * 32;
+      if (row >= kept) continue;
+      const int64_t off = row * n_cols + col0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (col0 + q * 8 + 8 > n_cols) break;
+        uint32_t aw[4], uw[4], hw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int k = q * 8 + 2 * i;
+          const uint16_t a0b = f32_to_bf16_bits(fmaxf(__uint_as_float(g[k]), 0.0f));
+          const uint16_t a1b = f32_to_bf16_bits(fmaxf(__uint_as_float(g[k + 1]), 0.0f));
+          const float a0 = __uint_as_float(static_cast<uint32_t>(a0b) << 16);
+          const float a1 = __uint_as_float(static_cast<uint32_t>(a1b) << 16);
+          const float u0 = __uint_as_float(u[k]), u1 = __uint_as_float(u[k + 1]);
+          aw[i] = static_cast<uint32_t>(a0b) | (static_cast<uint32_t>(a1b) << 16);
+          uw[i] = static_cast<uint32_t>(f32_to_bf16_bits(u0)) | (static_cast<uint32_t>(f32_to_bf16_bits(u1)) << 16);
+          hw[i] = static_cast<uint32_t>(f32_to_bf16_bits(a0 * u0)) |
+                  (static_cast<uint32_t>(f32_to_bf16_bits(a1 * u1)) << 16);
+        }
+        *reinterpret_cast<uint4*>(spill_a + off + q * 8) = make_uint4(aw[0], aw[1], aw[2], aw[3]);
+        *reinterpret_cast<uint4*>(spill_u + off + q * 8) = make_uint4(uw[0], uw[1], uw[2], uw[3]);
+        *reinterpret_cast<uint4*>(hs + off + q * 8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      }
+    }
+  }
+};
+
 // Epilogue of Y_s = H_s W_down: row r of the tile goes to y[spill_rows[r]].
 struct EpiScatterRows {
   uint16_t* y;
@@ -442,8 +506,8 @@ static int launch_ell_fwd(const EllFwdParams& p, int64_t n, cudaStream_t st) {
 }
 
 extern "C" int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* wu_t, const void* wd,
-                              const void* wd_t, void* y, int64_t d_model, void* workspace,
-                              size_t workspace_bytes, void* stream) {
+                              const void* wd_t, const void* wg_t, void* y, int64_t d_model,
+                              void* workspace, size_t workspace_bytes, void* stream) {
   clear_error();
   int rc = check_hybrid(hy, "hybrid_ffn_fwd");
   if (rc) return rc;
@@ -452,7 +516,7 @@ extern "C" int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* w
   if (!x || !wu_t || !wd || !y || !hy->ell_u || (hy->s_max > 0 && (!wd_t || !hy->spill_u)))
     return fail(SGE_ERR_ARG, "hybrid_ffn_fwd: null pointer");
   if (!aligned16(x) || !aligned16(wu_t) || !aligned16(wd) || !aligned16(y) ||
-      (wd_t && !aligned16(wd_t)))
+      (wd_t && !aligned16(wd_t)) || (wg_t && !aligned16(wg_t)))
     return fail(SGE_ERR_ARG, "hybrid_ffn_fwd: pointer not 16-byte aligned");
   const size_t need = hybrid_ffn_fwd_workspace_bytes(d_model, hy->d_ff, hy->s_max);
   if (hy->s_max > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
@@ -481,12 +545,25 @@ extern "C" int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* w
   using S = TcPairShape<256, 1>;
   CUtensorMap ma, mb, mh, md;
   if ((rc = make_tmap_bf16(&ma, xs, hy->s_max, d_model, d_model, kBM))) return rc;
-  if ((rc = make_tmap_bf16(&mb, wu_t, hy->d_ff, d_model, d_model, S::BN / 2))) return rc;
-  EpiSpillUp e1{static_cast<const uint16_t*>(hy->spill_a), static_cast<uint16_t*>(hy->spill_u), hs,
-                hy->n_spill, hy->s_max, static_cast<int>(hy->d_ff)};
-  if ((rc = launch_tc_gemm_pair<S>(ma, mb, mb, hy->s_max, hy->d_ff, d_model, e1, nullptr, st,
-                                   "hybrid_ffn_fwd (spill up)")))
-    return rc;
+  if (wg_t) {
+    // the gate recomputed with the up projection: [G | U] = X_s [W_gate | W_up]
+    using S1 = TcPairShape<128, 2>;
+    CUtensorMap mg;
+    if ((rc = make_tmap_bf16(&mg, wg_t, hy->d_ff, d_model, d_model, S1::BN / 2))) return rc;
+    if ((rc = make_tmap_bf16(&mb, wu_t, hy->d_ff, d_model, d_model, S1::BN / 2))) return rc;
+    EpiSpillGateUp e1{static_cast<uint16_t*>(hy->spill_a), static_cast<uint16_t*>(hy->spill_u), hs,
+                      hy->n_spill, hy->s_max, static_cast<int>(hy->d_ff)};
+    if ((rc = launch_tc_gemm_pair<S1>(ma, mg, mb, hy->s_max, hy->d_ff, d_model, e1, nullptr, st,
+                                      "hybrid_ffn_fwd (spill gate and up)")))
+      return rc;
+  } else {
+    if ((rc = make_tmap_bf16(&mb, wu_t, hy->d_ff, d_model, d_model, S::BN / 2))) return rc;
+    EpiSpillUp e1{static_cast<const uint16_t*>(hy->spill_a), static_cast<uint16_t*>(hy->spill_u), hs,
+                  hy->n_spill, hy->s_max, static_cast<int>(hy->d_ff)};
+    if ((rc = launch_tc_gemm_pair<S>(ma, mb, mb, hy->s_max, hy->d_ff, d_model, e1, nullptr, st,
+                                     "hybrid_ffn_fwd (spill up)")))
+      return rc;
+  }
   if ((rc = make_tmap_bf16(&mh, hs, hy->s_max, hy->d_ff, hy->d_ff, kBM))) return rc;
   if ((rc = make_tmap_bf16(&md, wd_t, d_model, hy->d_ff, hy->d_ff, S::BN / 2))) return rc;
   EpiScatterRows e2{static_cast<uint16_t*>(y), hy->spill_rows, hy->n_spill, hy->s_max,

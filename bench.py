@@ -61,6 +61,9 @@ def parse():
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--sweep", action="store_true",
                    help="density sweep of the workload (0.25%%..5%%): one JSON line per density")
+    p.add_argument("--cap-sweep", action="store_true",
+                   help="TwELL capacity C in {T/4, T/2, T}: footprint, overflow, truncation error, "
+                        "and the hybrid path that recomputes overflowing rows: one JSON line per C")
     p.add_argument("--profile", action="store_true",
                    help="run only warmup + steps of the sparse step (for ncu captures); no JSON")
     return p.parse_args()
@@ -441,6 +444,91 @@ def run_sweep(args, local_rank):
     return out
 
 
+def run_cap_sweep(args, local_rank):
+    """TwELL capacity C below the tile width T (C in {T/4, T/2, T}) on the
+    workload: footprint of the TwELL against the tiles and rows that overflow
+    C; the TwELL step at that C (overflowing tiles keep their first C
+    entries, so those rows are truncated) and its error against C = T; and
+    the hybrid inference path with the safety valve: rows with an
+    overflowing tile go to the spill and the spill rows are recomputed from
+    the gate (hybrid_ffn_fwd given W_gate), so the result is the C = T one."""
+    import activation_sparse_gated_epilogue_b200 as sge
+    from activation_sparse_gated_epilogue_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = synth.CONFIGS[args.workload]
+    inp = synth.make_inputs(cfg)
+    n, d, f, tile = cfg.n_tokens, cfg.d_model, cfg.d_ff, cfg.tile
+    x, wg, wu, wd = (getattr(inp, k).to(dev) for k in ("x", "wg_t", "wu_t", "wd"))
+    wd_t = wd.t().contiguous()
+    ws = sge.fused_workspace(n, d, dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    steps = min(args.steps, 50)
+
+    def timed(fns, steps, warm):
+        evs = []
+        for s_ in range(warm + steps):
+            flush.zero_()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+            e[0].record(stream)
+            for fn in fns:
+                fn()
+            e[-1].record(stream)
+            if s_ >= warm:
+                evs.append(e)
+        torch.cuda.synchronize(dev)
+        return statistics.mean(e[0].elapsed_time(e[-1]) for e in evs)
+
+    def rel(a, b):
+        return float(((a.float() - b.float()).abs().max() / b.float().abs().max()).item())
+
+    # the full-capacity result every C is compared with
+    tw_full = sge.twell_gate_pack(x, wg, tile, tile)
+    y_full = sge.twell_fused_up_down(x, tw_full, wu, wd, workspace=ws)
+    torch.cuda.synchronize(dev)
+    out = []
+    for cap in (tile // 4, tile // 2, tile):
+        tw = sge.TwELL.empty(n, f, tile, cap, x.dtype, dev)
+        diag = sge.new_diag(dev)
+        y = torch.empty_like(x)
+        gate = lambda: sge.twell_gate_pack(x, wg, tile, cap, out=tw)
+        fused = lambda: sge.twell_fused_up_down(x, tw, wu, wd, y=y, workspace=ws)
+        sge.twell_gate_pack(x, wg, tile, cap, out=tw, diag=diag)
+        torch.cuda.synchronize(dev)
+        cnt = tw.count.to(torch.int64)
+        over_rows = int((cnt > cap).any(1).sum().item())
+        stored = torch.minimum(cnt, torch.tensor(cap, device=dev)).sum(1)
+        step_ms = timed([gate, fused], steps, 3)
+        err = rel(y, y_full)
+        rows_differ = int(((y.float() - y_full.float()).abs().amax(1) > 0).sum().item())
+        # hybrid with the safety valve
+        hk = HYB_INFER_K
+        n_sp = int(((stored > hk) | (cnt > cap).any(1)).sum().item())
+        hs = max(128, (n_sp + 127) // 128 * 128)
+        hy = sge.Hybrid.empty(n, f, hk, hs, dev)
+        hws = sge.hybrid_fwd_workspace(d, f, hs, dev)
+        y_h = torch.empty_like(x)
+        hdiag = sge.new_diag(dev)
+        hpack = lambda: sge.hybrid_pack(tw, hk, hs, out=hy, diag=hdiag)
+        hfwd = lambda: sge.hybrid_ffn_fwd(x, hy, wu, wd, wd_t=wd_t, y=y_h, workspace=hws, wg_t=wg)
+        h_ms = timed([gate, hpack, hfwd], steps, 3)
+        out.append({
+            "cap_sweep": f"{cfg.name} N={n} d={d} F={f} T={tile}", "C": cap,
+            "twell_bytes": int(n * (f // tile) * (1 + 3 * cap)),
+            "overflow_tiles": int(diag[0].item()), "rows_with_overflow": over_rows,
+            "stored_entries": int(stored.sum().item()),
+            "twell_step_ms": round(step_ms, 4), "twell_tokens_per_s": round(n / (step_ms / 1e3), 1),
+            "twell_max_abs_rel_vs_full_capacity": round(err, 6), "twell_rows_differing": rows_differ,
+            "hybrid_valve_ms": round(h_ms, 4), "hybrid_valve_tokens_per_s": round(n / (h_ms / 1e3), 1),
+            "hybrid_K": hk, "hybrid_spill_rows": int(hy.n_spill.item()), "hybrid_s_max": hs,
+            "hybrid_dropped_rows": int(hdiag[2].item()),
+            "hybrid_max_abs_rel_vs_full_capacity": round(rel(y_h, y_full), 6),
+        })
+    return out
+
+
 # ------------------------------------------------ training step (hybrid)
 
 def run_train(args, local_rank):
@@ -610,6 +698,11 @@ def main():
     if args.sweep:
         if rank == 0:
             for line in run_sweep(args, local_rank):
+                print(json.dumps(line), flush=True)
+        return
+    if args.cap_sweep:
+        if rank == 0:
+            for line in run_cap_sweep(args, local_rank):
                 print(json.dumps(line), flush=True)
         return
     out = run_own(args, rank, world, local_rank)

@@ -202,7 +202,12 @@ int dense_ffn_fwd(const void* x, const void* wg_t, const void* wu_t, const void*
  * compression": TwELL is compressed into this hybrid form).  bf16 only.
  *
  * All buffers are caller-owned device memory described by this struct:
- *   row_nnz    int32 [N]          stored entries of row t (sum of min(count, C))
+ *   row_nnz    int32 [N]          stored entries of row t (sum of min(count, C));
+ *                                 a row with a tile whose count exceeds C
+ *                                 (entries lost to the capacity) and at most
+ *                                 K stored entries gets K + 1 instead, so that
+ *                                 it goes to the spill (where hybrid_ffn_fwd
+ *                                 can recompute it exactly)
  *   spill_slot int32 [N]          rank of row t among the spill rows if
  *                                 row_nnz > K and that rank < S_max, else -1
  *   spill_rows int32 [S_max]      token of each kept spill row (ascending)
@@ -254,15 +259,23 @@ int hybrid_pack(const uint8_t* count, const uint8_t* idx, const void* val, int t
  *             (fp32 accumulation; u_e saved to ell_u in bf16)
  *   spill rows: U = X_s W_up (all F columns, tcgen05), saved to spill_u;
  *             H = bf16(A (.) U); Y_s = H W_down (tcgen05), scattered to y.
+ *             With wg_t given, A is first recomputed from the gate,
+ *             A = bf16(ReLU(X_s W_gate)) (one tcgen05 GEMM with two B
+ *             operands, W_gate and W_up) and written to spill_a: the rows
+ *             that went to the spill because a TwELL tile overflowed its
+ *             capacity C then come out as if C = T (the safety valve of a
+ *             capacity below the tile width).  With wg_t NULL the spill rows
+ *             use spill_a as packed.
  *   dropped rows: y = 0.
  *   x [N][d], y [N][d], wu_t [F][d], wd [F][d], wd_t [d][F] (W_down
  *   transposed, the K-major operand of the spill GEMM; may be NULL when
- *   S_max == 0); workspace >= hybrid_ffn_fwd_workspace_bytes(d, F, S_max).
+ *   S_max == 0), wg_t [F][d] or NULL; workspace >=
+ *   hybrid_ffn_fwd_workspace_bytes(d, F, S_max).
  */
 size_t hybrid_ffn_fwd_workspace_bytes(int64_t d_model, int64_t d_ff, int s_max);
 
 int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* wu_t, const void* wd,
-                   const void* wd_t, void* y, int64_t d_model, void* workspace,
+                   const void* wd_t, const void* wg_t, void* y, int64_t d_model, void* workspace,
                    size_t workspace_bytes, void* stream);
 
 /*

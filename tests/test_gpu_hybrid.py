@@ -74,6 +74,57 @@ def test_hybrid_pack_and_fwd_match_oracle(cuda_device, k, s_max):
     assert np.all(to_f64(y)[dropped] == 0.0)
 
 
+@pytest.mark.parametrize("cap", [32, 16])
+def test_hybrid_capacity_below_tile(cuda_device, cap):
+    """TwELL with a capacity C below the tile width T: rows with a tile past
+    C go to the spill (row_nnz = K + 1 when their stored count fits K), and
+    the pack matches the oracle bit for bit.  Given W_gate, the forward
+    recomputes the spill rows from the gate and equals the full-capacity
+    (C = T) sparse FFN; without it the spill rows use the truncated
+    activations, as the oracle's forward of the same pack does."""
+    n, d, f, tile, k, s_max = 300, 256, 1024, 128, 64, 300
+    inp = _small_inputs(n, d, f)
+    x, wg, wu, wd = (inp.as_f64(nm) for nm in ("x", "wg_t", "wu_t", "wd"))
+    x[:9, :-1] *= 5.0                                     # heavy rows: tiles past C, > K entries
+    # rows 10..19 switch on 40 gates of tile 0 through feature 0: a tile past
+    # C in a row whose stored entries still fit K
+    x[:, 0] = 0.0
+    x[10:20, 0] = 4.0
+    wg = wg.copy()
+    wg[:40, 0] = 2.0
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    x = xb.double().numpy()
+    wgb = torch.from_numpy(wg).to(torch.bfloat16)
+    wg = wgb.double().numpy()
+    g = oracle.gate_preact(x, wg)
+    tw_c = oracle.twell_pack(g, tile, cap, oracle.VAL_BF16)
+    assert tw_c.overflow > 0
+    ora = oracle.hybrid_pack(tw_c, k, s_max)
+    assert np.any(ora.row_nnz == k + 1)                   # spilled only through the capacity
+    dev = cuda_device
+    wg_d = wgb.to(dev)
+    wu_d, wd_d = (getattr(inp, nm).to(dev) for nm in ("wu_t", "wd"))
+
+    hy = sge.hybrid_pack(_upload_twell(tw_c, dev), k, s_max)
+    torch.cuda.synchronize()
+    _check_pack(hy, ora)
+    y = sge.hybrid_ffn_fwd(xb.to(dev), hy, wu_d, wd_d, wg_t=wg_d)
+    want = oracle.fused_up_down(x, oracle.twell_pack(g, tile, tile, oracle.VAL_BF16), wu, wd)
+    torch.cuda.synchronize()
+    err = oracle.max_abs_rel(to_f64(y), want)
+    assert err <= BF16_TOL, err
+    # the recomputed activations of the kept spill rows are the full ReLU(g)
+    kept = min(ora.n_spill, s_max)
+    full_a = oracle.round_array(np.maximum(g[ora.spill_rows[:kept]], 0.0), oracle.VAL_BF16)
+    assert oracle.max_abs_rel(to_f64(hy.spill_a)[:kept], full_a) <= 1e-2
+
+    hy2 = sge.hybrid_pack(_upload_twell(tw_c, dev), k, s_max)
+    y2 = sge.hybrid_ffn_fwd(xb.to(dev), hy2, wu_d, wd_d)
+    torch.cuda.synchronize()
+    err2 = oracle.max_abs_rel(to_f64(y2), oracle.hybrid_fwd(x, ora, wu, wd))
+    assert err2 <= BF16_TOL, err2
+
+
 def test_hybrid_train_workload_sampled(cuda_device):
     """The full training-shaped workload (N=8192, d=2048, F=8192, K=128,
     S_max=1024): gate GEMM + TwELL, hybrid pack, hybrid forward on the GPU;
