@@ -132,7 +132,10 @@ int twell_gate_pack(const void* x, const void* wg_t, int64_t n_tokens, int64_t d
  *   diag       nullable int32[4]; diag[SGE_DIAG_FLAGS] gets SGE_FLAG_TIMEOUT
  *              if a pipeline wait gave up (y is then invalid).
  * Results are deterministic: repeated calls on the same inputs give the same
- * bits, whatever the scheduling.
+ * bits, whatever the scheduling.  Batches of at most 64 tokens (with rows of
+ * at most 4 KB) run a small-batch kernel whose fp32 sums are ordered
+ * differently from the larger batches' kernel: a token's y can differ between
+ * the two in the last bits.
  * Errors: as twell_gate_pack; SGE_ERR_ARG for a missing, short or misaligned
  * workspace; SGE_ERR_UNSUPPORTED for d > 4096 or
  * F / T > 256.
