@@ -66,6 +66,7 @@ def library() -> ctypes.CDLL:
             "twell_fused_up_down_noalloc": (I, [P, P, P, P, P, P, P, I64, I64, I64, I, I, I, P, P]),
             "twell_fused_up_down_noalloc_max_tokens": (I64, []),
             "dense_ffn_fwd": (I, [P, P, P, P, P, P, I64, I64, I64, P, P]),
+            "sge_l2_gather_probe": (I, [P, I64, I, P, I64, P, P, P]),
             "hybrid_pack": (I, [P, P, P, I, I, ctypes.POINTER(_SgeHybrid), P, P]),
             "hybrid_ffn_fwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I]),
             "hybrid_ffn_fwd": (I, [P, ctypes.POINTER(_SgeHybrid), P, P, P, P, P, I64, P,
@@ -230,6 +231,20 @@ def dense_ffn_fwd(x: torch.Tensor, wg_t: torch.Tensor, wu_t: torch.Tensor, wd_t:
     _call("dense_ffn_fwd", _ptr(x), _ptr(wg_t), _ptr(wu_t), _ptr(wd_t), _ptr(h), _ptr(y),
           n, d, f, _ptr(diag), _stream(x.device, stream))
     return y
+
+
+def l2_gather_probe(table: torch.Tensor, ids: torch.Tensor, sink: torch.Tensor,
+                    diag: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Stream rows ids of table (2-D, contiguous) into shared memory on every
+    SM, the way the fused up/down kernel streams its weight rows (a
+    measurement helper; time it with CUDA events)."""
+    if table.dim() != 2 or not table.is_contiguous():
+        raise ValueError("table must be a contiguous 2-D tensor")
+    if ids.dtype != torch.int32 or not ids.is_contiguous():
+        raise ValueError("ids must be contiguous int32")
+    row_bytes = table.shape[1] * table.element_size()
+    _call("sge_l2_gather_probe", _ptr(table), table.shape[0], row_bytes, _ptr(ids), ids.numel(),
+          _ptr(sink), _ptr(diag), _stream(table.device, stream))
 
 
 @dataclass

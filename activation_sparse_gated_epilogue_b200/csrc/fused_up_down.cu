@@ -331,13 +331,16 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // Bounded wait that also gives up as soon as another warp of the CTA has.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
                                               volatile int* abort_flag, int32_t* diag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  uint64_t t0 = 0;  // the clock is read only once a wait has lasted kWaitSpins tries
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitNs) break;
+      if ((i & (kWaitSpins - 1)) == 0) {
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) t0 = now;
+        else if (now - t0 > kWaitNs) break;
+      }
     }
   }
   *abort_flag = 1;

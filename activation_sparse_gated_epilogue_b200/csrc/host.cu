@@ -39,10 +39,29 @@ int sm_count() {
   return cached[dev];
 }
 
+// The dynamic shared-memory limit of each (device, kernel) is set once and
+// only raised afterwards: setting the attribute on every launch is not free.
 int set_smem_limit(const void* kernel, int bytes) {
+  struct Entry {
+    int dev;
+    const void* kernel;
+    int bytes;
+  };
+  static Entry table[256];
+  static int used = 0;
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  std::lock_guard<std::mutex> lock(mu);
+  Entry* hit = nullptr;
+  for (int i = 0; i < used; ++i)
+    if (table[i].dev == dev && table[i].kernel == kernel) hit = &table[i];
+  if (hit && hit->bytes >= bytes) return SGE_OK;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess)
     return fail(SGE_ERR_CUDA, "cudaFuncSetAttribute(smem=%d): %s", bytes, cudaGetErrorString(e));
+  if (hit) hit->bytes = bytes;
+  else if (used < 256) table[used++] = Entry{dev, kernel, bytes};
   return SGE_OK;
 }
 

@@ -22,6 +22,8 @@ namespace sge {
 // legitimate wait in this library is microseconds; four seconds means the
 // pipeline is broken, and the kernel gives up instead of hanging the GPU.
 constexpr uint64_t kWaitNs = 4000000000ull;
+// Tries of an mbarrier wait between two reads of %globaltimer (a power of two).
+constexpr uint32_t kWaitSpins = 1024;
 
 SGE_DEV uint64_t globaltimer_ns() {
   uint64_t t;
@@ -68,11 +70,16 @@ SGE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for the phase of `bar` with the given parity to complete.  Returns
 // false (and flags a timeout in diag) if it does not within kWaitNs.
 SGE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* diag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  // the clock is read only once a wait has lasted kWaitSpins tries: most
+  // waits end sooner and never pay for reading it
+  uint64_t t0 = 0;
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 0 && globaltimer_ns() - t0 > kWaitNs) break;
+    if ((i & (kWaitSpins - 1)) == 0) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > kWaitNs) break;
+    }
   }
   if (diag) atomicOr(reinterpret_cast<int*>(diag + SGE_DIAG_FLAGS), SGE_FLAG_TIMEOUT);
   return false;

@@ -71,12 +71,15 @@ __device__ __forceinline__ TileCoord tile_coord(int tile, int m_blocks) {
 // Bounded wait that also gives up when another role of the CTA aborted.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
                                               volatile int* abort_flag, int32_t* diag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  uint64_t t0 = 0;  // the clock is read only once a wait has lasted kWaitSpins tries
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if ((i & 63) == 0 && globaltimer_ns() - t0 > kWaitNs) break;
+    if ((i & (kWaitSpins - 1)) == 0) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > kWaitNs) break;
+    }
   }
   if (diag) atomicOr(reinterpret_cast<int*>(diag + SGE_DIAG_FLAGS), SGE_FLAG_TIMEOUT);
   *abort_flag = 1;

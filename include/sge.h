@@ -197,6 +197,23 @@ int dense_ffn_fwd(const void* x, const void* wg_t, const void* wu_t, const void*
                   void* stream);
 
 /*
+ * sge_l2_gather_probe -- measurement helper, not part of the FFN: streams the
+ * rows ids[0 .. n_ids) of `table` (table_rows rows of row_bytes bytes,
+ * row-major, 16-byte aligned) from memory into shared memory the way the
+ * fused up/down kernel streams its W_up and W_down rows (bulk copies of whole
+ * rows through per-warp rings, every row read back), on every SM.  With a
+ * table that fits L2 and random ids, bytes / time is the L2-to-SM row
+ * gather rate that bounds twell_fused_up_down.  Asynchronous on `stream`;
+ * the caller times it with events.  ids outside [0, table_rows) are clamped.
+ *   sink  device uint32[1] the kernel may write (keeps the reads live)
+ *   diag  nullable int32[4]; SGE_FLAG_TIMEOUT if a wait gave up
+ * Errors: SGE_ERR_ARG for bad sizes, a null or misaligned pointer;
+ * SGE_ERR_UNSUPPORTED for rows too long for the rings (> about 100 KB).
+ */
+int sge_l2_gather_probe(const void* table, int64_t table_rows, int row_bytes, const int32_t* ids,
+                        int64_t n_ids, uint32_t* sink, int32_t* diag, void* stream);
+
+/*
  * Hybrid format for training ("Sparser, Faster, Lighter Transformer Language
  * Models", pwwt.cn summary, section 03 and figure "routing of the
  * hybrid-format sparse operator": tokens with few active gates go to a

@@ -360,3 +360,16 @@ def test_library_errors_raise(cuda_device):
     w = torch.zeros(200, 64, dtype=torch.bfloat16, device=cuda_device)
     with pytest.raises(sge.LibraryError):
         sge.twell_gate_pack(x, w, 64, 64)          # 64 does not divide 200
+
+
+def test_l2_gather_probe_runs(cuda_device):
+    """The measurement helper behind the bench's row-gather ceiling streams
+    random rows of a table without giving up, for a few row widths."""
+    for d in (1024, 2048):
+        table = torch.empty((16 * 1024 * 1024) // (2 * d), d, dtype=torch.bfloat16, device=cuda_device)
+        ids = torch.randint(-5, table.shape[0] + 5, (50000,), dtype=torch.int32, device=cuda_device)
+        sink = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+        diag = sge.new_diag(cuda_device)
+        sge.l2_gather_probe(table, ids, sink, diag=diag)
+        torch.cuda.synchronize()
+        assert int(diag[3]) == 0
