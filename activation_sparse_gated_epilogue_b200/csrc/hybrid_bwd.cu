@@ -389,18 +389,43 @@ __global__ void __launch_bounds__(256) gather2_kernel(const uint16_t* __restrict
 // dst[c][col_off + r] = src[r][c] for r < rows, c < cols (bf16, 32x32 tiles).
 __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restrict__ src, int rows,
                                                         int cols, int64_t src_pitch, uint16_t* dst,
-                                                        int64_t dst_pitch, int col_off) {
-  __shared__ uint16_t tile[32][33];
-  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int i = ty; i < 32; i += 8) {
-    const int r = r0 + i, c = c0 + tx;
-    tile[i][tx] = (r < rows && c < cols) ? src[static_cast<int64_t>(r) * src_pitch + c] : 0;
+                                                        int64_t dst_pitch, int col_off,
+                                                        const int32_t* rows_dev, int rows_cap) {
+  // 64 x 64 tiles moved with 16-byte loads and stores (rows, cols, pitches,
+  // col_off and the row limit are multiples of 8); the shared tile's row
+  // pitch of 66 elements keeps the column reads off one bank
+  __shared__ uint16_t tile[64][66];
+  const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
+  // with rows_dev, only the first min(*rows_dev, rows_cap) rows rounded up to
+  // 64 are transposed (the K that the later GEMMs read)
+  if (rows_dev) rows = min(rows, (min(*rows_dev, rows_cap) + 63) / 64 * 64);
+  if (r0 >= rows) return;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int id = threadIdx.x + 256 * h;
+    const int r = id >> 3, c8 = (id & 7) * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r0 + r < rows && c0 + c8 < cols)
+      v = *reinterpret_cast<const uint4*>(src + static_cast<int64_t>(r0 + r) * src_pitch + c0 + c8);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      tile[r][c8 + 2 * k] = static_cast<uint16_t>(w[k] & 0xFFFFu);
+      tile[r][c8 + 2 * k + 1] = static_cast<uint16_t>(w[k] >> 16);
+    }
   }
   __syncthreads();
-  for (int i = ty; i < 32; i += 8) {
-    const int c = c0 + i, r = r0 + tx;
-    if (c < cols && r < rows) dst[static_cast<int64_t>(c) * dst_pitch + col_off + r] = tile[tx][i];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int id = threadIdx.x + 256 * h;
+    const int c = id >> 3, r8 = (id & 7) * 8;  // destination row c0 + c, columns r0 + r8 ..
+    if (c0 + c >= cols || r0 + r8 >= rows) continue;
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      w[k] = static_cast<uint32_t>(tile[r8 + 2 * k][c]) | (static_cast<uint32_t>(tile[r8 + 2 * k + 1][c]) << 16);
+    *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(c0 + c) * dst_pitch + col_off + r0 + r8) =
+        make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -416,6 +441,13 @@ struct EpiBwdSpill {
   int s_max;
   int f;
   int64_t m_rows;  // rows of the padded spill buffers
+
+  // rows up to the kept spill rows rounded up to 64 (the K the later GEMMs
+  // read): the zero rows past the kept ones matter only that far
+  __device__ __forceinline__ int m_limit(int m) const {
+    const int c = min(*n_spill, s_max);
+    return min(m, (c + 63) / 64 * 64);
+  }
 
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {
@@ -469,29 +501,60 @@ struct EpiAddF32 {
   float* out1;
   int64_t split;
   int n_cols;
+  const int32_t* k_count;  // nullable: K is the kept spill rows, rounded up to 64
+  int k_cap;
+
+  __device__ __forceinline__ int k_limit(int k) const {
+    if (!k_count) return k;
+    const int c = min(*k_count, k_cap);
+    return min(k, (c + 63) / 64 * 64);
+  }
 
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {
-    float* out = row < split ? out0 + row * n_cols : (out1 ? out1 + (row - split) * n_cols : nullptr);
-    if (row >= 2 * split) out = nullptr;
+    // the warp's 32 rows pass through shared memory so that each row is
+    // added with contiguous 128-byte accesses (a thread per row would add 16
+    // bytes at a time to 32 different rows)
+    __shared__ __align__(16) float stage[4][32][36];
+    float(*buf)[36] = stage[(threadIdx.x >> 5) & 3];
+    const int64_t row0 = row - lane;
+    const int rr = lane >> 3, c4 = (lane & 7) * 4;
 #pragma unroll 1
     for (int ch = 0; ch < BN / 32; ++ch) {
       uint32_t r[32];
       tmem_ld32(taddr + ch * 32, r);
       tmem_ld_wait();
       const int col0 = n_blk * BN + ch * 32;
-      if (!out) continue;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (col0 + q * 4 + 4 > n_cols) break;
-        float4* o = reinterpret_cast<float4*>(out + col0 + q * 4);
-        float4 v = *o;
-        v.x += __uint_as_float(r[q * 4]);
-        v.y += __uint_as_float(r[q * 4 + 1]);
-        v.z += __uint_as_float(r[q * 4 + 2]);
-        v.w += __uint_as_float(r[q * 4 + 3]);
-        *o = v;
+      for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<float4*>(&buf[lane][4 * q]) =
+            make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                        __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+      __syncwarp();
+      if (col0 + c4 + 4 <= n_cols) {
+        // all 8 rows' loads in flight before any add
+        float4* o[8];
+        float4 v[8];
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int64_t g = row0 + rr + 4 * it;
+          float* out = g < split ? out0 + g * n_cols
+                                 : (out1 && g < 2 * split ? out1 + (g - split) * n_cols : nullptr);
+          o[it] = out ? reinterpret_cast<float4*>(out + col0 + c4) : nullptr;
+          v[it] = o[it] ? *o[it] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          if (!o[it]) continue;
+          const float4 add = *reinterpret_cast<const float4*>(&buf[rr + 4 * it][c4]);
+          v[it].x += add.x;
+          v[it].y += add.y;
+          v[it].z += add.z;
+          v[it].w += add.w;
+          *o[it] = v[it];
+        }
       }
+      __syncwarp();
     }
   }
 };
@@ -534,9 +597,11 @@ struct EpiScatterRowsBwd {
 };
 
 static int launch_transpose(const uint16_t* src, int rows, int cols, int64_t src_pitch,
-                            uint16_t* dst, int64_t dst_pitch, int col_off, cudaStream_t st) {
-  dim3 grid((cols + 31) / 32, (rows + 31) / 32);
-  transpose_kernel<<<grid, 256, 0, st>>>(src, rows, cols, src_pitch, dst, dst_pitch, col_off);
+                            uint16_t* dst, int64_t dst_pitch, int col_off, cudaStream_t st,
+                            const int32_t* rows_dev = nullptr, int rows_cap = 0) {
+  dim3 grid((cols + 63) / 64, (rows + 63) / 64);
+  transpose_kernel<<<grid, 256, 0, st>>>(src, rows, cols, src_pitch, dst, dst_pitch, col_off, rows_dev,
+                                         rows_cap);
   return check_launch("hybrid_ffn_bwd (transpose)");
 }
 
@@ -644,10 +709,12 @@ extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* h
   if ((rc = launch_tc_gemm_pair<S>(m1a, m1b, m1b, sp, f, d, e1, nullptr, st, "hybrid_ffn_bwd (dH)")))
     return rc;
   // operands of the remaining GEMMs, K-major
-  if ((rc = launch_transpose(ws.acat, sp, static_cast<int>(2 * f), 2 * f, ws.acat_t, sp, 0, st))) return rc;
-  if ((rc = launch_transpose(ws.hs, sp, static_cast<int>(f), f, ws.hs_t, sp, 0, st))) return rc;
-  if ((rc = launch_transpose(ws.dys, sp, static_cast<int>(d), d, ws.dys_t, sp, 0, st))) return rc;
-  if ((rc = launch_transpose(ws.xs, sp, static_cast<int>(d), d, ws.xs_t, sp, 0, st))) return rc;
+  // (spill-row operands: only as many rows as the weight-gradient GEMMs read)
+  if ((rc = launch_transpose(ws.acat, sp, static_cast<int>(2 * f), 2 * f, ws.acat_t, sp, 0, st, hy->n_spill, s_max)))
+    return rc;
+  if ((rc = launch_transpose(ws.hs, sp, static_cast<int>(f), f, ws.hs_t, sp, 0, st, hy->n_spill, s_max))) return rc;
+  if ((rc = launch_transpose(ws.dys, sp, static_cast<int>(d), d, ws.dys_t, sp, 0, st, hy->n_spill, s_max))) return rc;
+  if ((rc = launch_transpose(ws.xs, sp, static_cast<int>(d), d, ws.xs_t, sp, 0, st, hy->n_spill, s_max))) return rc;
   if ((rc = launch_transpose(static_cast<const uint16_t*>(wu_t), static_cast<int>(f), static_cast<int>(d), d,
                              ws.bcat, 2 * f, 0, st)))
     return rc;
@@ -665,14 +732,14 @@ extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* h
   CUtensorMap m3a, m3b;
   if ((rc = make_tmap_bf16(&m3a, ws.hs_t, f, sp, sp, kBM))) return rc;
   if ((rc = make_tmap_bf16(&m3b, ws.dys_t, d, sp, sp, S::BN / 2))) return rc;
-  EpiAddF32 e3{dwd, nullptr, f, static_cast<int>(d)};
+  EpiAddF32 e3{dwd, nullptr, f, static_cast<int>(d), hy->n_spill, s_max};
   if ((rc = launch_tc_gemm_pair<S>(m3a, m3b, m3b, f, d, sp, e3, nullptr, st, "hybrid_ffn_bwd (dW_down)")))
     return rc;
   // [dW_up ; dW_gate] += [dU | dG]^T X_s
   CUtensorMap m4a, m4b;
   if ((rc = make_tmap_bf16(&m4a, ws.acat_t, 2 * f, sp, sp, kBM))) return rc;
   if ((rc = make_tmap_bf16(&m4b, ws.xs_t, d, sp, sp, S::BN / 2))) return rc;
-  EpiAddF32 e4{dwu_t, dwg_t, f, static_cast<int>(d)};
+  EpiAddF32 e4{dwu_t, dwg_t, f, static_cast<int>(d), hy->n_spill, s_max};
   return launch_tc_gemm_pair<S>(m4a, m4b, m4b, 2 * f, d, sp, e4, nullptr, st,
                                 "hybrid_ffn_bwd (dW_up, dW_gate)");
 }

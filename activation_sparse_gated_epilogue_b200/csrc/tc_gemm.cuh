@@ -64,6 +64,23 @@ __device__ __forceinline__ int epi_m_limit(const E& e, int m) {
   return epi_m_limit_impl(e, m, 0);
 }
 
+// K an epilogue needs: an epilogue may bound K by a device-side count
+// (Epi::k_limit, returning a multiple of kBK or K itself); K-blocks past it
+// are skipped, and with no K-block left every tile is skipped (its product
+// is zero: only epilogues that add D to their output may bound K).
+template <class E>
+__device__ __forceinline__ auto epi_k_limit_impl(const E& e, int k, int) -> decltype(e.k_limit(k)) {
+  return e.k_limit(k);
+}
+template <class E>
+__device__ __forceinline__ int epi_k_limit_impl(const E&, int k, long) {
+  return k;
+}
+template <class E>
+__device__ __forceinline__ int epi_k_limit(const E& e, int k) {
+  return epi_k_limit_impl(e, k, 0);
+}
+
 __device__ __forceinline__ TileCoord tile_coord(int tile, int m_blocks) {
   return TileCoord{tile % m_blocks, tile / m_blocks};
 }
@@ -108,8 +125,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int lane = threadIdx.x & 31;
   const int m_blocks = (epi_m_limit(epi, M) + kBM - 1) / kBM;
   const int n_blocks = (N + BN - 1) / BN;
-  const int num_tiles = m_blocks * n_blocks;
-  const int k_blocks = (K + kBK - 1) / kBK;
+  const int k_blocks = (epi_k_limit(epi, K) + kBK - 1) / kBK;
+  const int num_tiles = k_blocks > 0 ? m_blocks * n_blocks : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -291,8 +308,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int n_pairs = static_cast<int>(cluster_count_x());
   const int m_blocks = (epi_m_limit(epi, M) + Shape::BM - 1) / Shape::BM;
   const int n_blocks = (N + BN - 1) / BN;
-  const int num_tiles = m_blocks * n_blocks;
-  const int k_blocks = (K + kBK - 1) / kBK;
+  const int k_blocks = (epi_k_limit(epi, K) + kBK - 1) / kBK;
+  const int num_tiles = k_blocks > 0 ? m_blocks * n_blocks : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {

@@ -606,6 +606,9 @@ def run_train(args, local_rank):
         torch.cuda.synchronize(dev)
         return [a.elapsed_time(b) for a, b in ts]
 
+    if args.profile:
+        timed(step, args.steps, args.warmup)
+        return None
     with ClockSampler(local_rank) as clk:
         t_sparse = timed(step, args.steps, args.warmup)
     t_dense = timed(dense_step, min(args.steps, 50), 3)
@@ -718,7 +721,9 @@ def main():
                                              device_id=torch.device("cuda", local_rank))
     if args.workload == "train_1b_hybrid":
         if rank == 0:
-            print(json.dumps(run_train(args, local_rank)), flush=True)
+            out = run_train(args, local_rank)
+            if out is not None:
+                print(json.dumps(out), flush=True)
         return
     if args.sweep:
         if rank == 0:
