@@ -212,18 +212,24 @@ __global__ void __launch_bounds__(kEllThreads) hybrid_ell_fwd_kernel(EllFwdParam
     s_h[e] = __uint_as_float(static_cast<uint32_t>(p.hv.ell_a[t * p.hv.k + e]) << 16);
   }
   __syncthreads();
-  // phase U
+  // batches of kEllBatch entries: the W_up and the W_down rows of a batch are
+  // loaded together (one memory round trip per batch), u is summed over the
+  // warps' parts of d, then h = bf16(a u) feeds the down projection
   for (int e0 = 0; e0 < nnz; e0 += kEllBatch) {
-    uint4 w[kEllBatch][NV];
+    uint4 wu[kEllBatch][NV], wdv[kEllBatch][NV];
 #pragma unroll
     for (int u = 0; u < kEllBatch; ++u) {
       const int e = e0 + u;
       const int j = e < nnz ? s_j[e] : -1;
-      const uint4* row = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wu_t) + static_cast<int64_t>(j) * row_bytes);
+      const int64_t off = static_cast<int64_t>(j) * row_bytes;
+      const uint4* ur = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wu_t) + off);
+      const uint4* dr = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wd) + off);
 #pragma unroll
       for (int k = 0; k < NV; ++k) {
         const int v = tid + k * kEllThreads;
-        w[u][k] = (j >= 0 && v < nvec) ? __ldg(row + v) : make_uint4(0, 0, 0, 0);
+        const bool in = j >= 0 && v < nvec;
+        wu[u][k] = in ? __ldg(ur + v) : make_uint4(0, 0, 0, 0);
+        wdv[u][k] = in ? __ldg(dr + v) : make_uint4(0, 0, 0, 0);
       }
     }
     float part[kEllBatch];
@@ -231,7 +237,7 @@ __global__ void __launch_bounds__(kEllThreads) hybrid_ell_fwd_kernel(EllFwdParam
     for (int u = 0; u < kEllBatch; ++u) {
       float s = 0.0f;
 #pragma unroll
-      for (int k = 0; k < NV; ++k) s = E::dot(xv[k], w[u][k], s);
+      for (int k = 0; k < NV; ++k) s = E::dot(xv[k], wu[u][k], s);
       part[u] = s;
     }
     const float tot = warp_reduce_multi<kEllBatch>(part, lane);
@@ -239,36 +245,23 @@ __global__ void __launch_bounds__(kEllThreads) hybrid_ell_fwd_kernel(EllFwdParam
       const int e = e0 + multi_entry<kEllBatch>(lane);
       if (e < nnz) s_up[warp][e] = tot;
     }
-  }
-  __syncthreads();
-  for (int e = tid; e < nnz; e += kEllThreads) {
-    float u = 0.0f;
+    __syncthreads();
+    if (tid < kEllBatch && e0 + tid < nnz) {
+      const int e = e0 + tid;
+      float u = 0.0f;
 #pragma unroll
-    for (int w8 = 0; w8 < kEllWarps; ++w8) u += s_up[w8][e];
-    p.hv.ell_u[t * p.hv.k + e] = f32_to_bf16_bits(u);
-    s_h[e] = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_bits(s_h[e] * u)) << 16);
-  }
-  __syncthreads();
-  // phase D
-  for (int e0 = 0; e0 < nnz; e0 += kEllBatch) {
-    uint4 w[kEllBatch][NV];
-    uint16_t hb[kEllBatch];
+      for (int w8 = 0; w8 < kEllWarps; ++w8) u += s_up[w8][e];
+      p.hv.ell_u[t * p.hv.k + e] = f32_to_bf16_bits(u);
+      s_h[e] = __uint_as_float(static_cast<uint32_t>(f32_to_bf16_bits(s_h[e] * u)) << 16);
+    }
+    __syncthreads();
 #pragma unroll
     for (int u = 0; u < kEllBatch; ++u) {
       const int e = e0 + u;
-      const int j = e < nnz ? s_j[e] : -1;
-      hb[u] = e < nnz ? static_cast<uint16_t>(__float_as_uint(s_h[e]) >> 16) : 0;
-      const uint4* row = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wd) + static_cast<int64_t>(j) * row_bytes);
+      const uint16_t hb = e < nnz ? static_cast<uint16_t>(__float_as_uint(s_h[e]) >> 16) : 0;
 #pragma unroll
-      for (int k = 0; k < NV; ++k) {
-        const int v = tid + k * kEllThreads;
-        w[u][k] = (j >= 0 && v < nvec) ? __ldg(row + v) : make_uint4(0, 0, 0, 0);
-      }
+      for (int k = 0; k < NV; ++k) E::axpy(hb, wdv[u][k], acc[k]);
     }
-#pragma unroll
-    for (int u = 0; u < kEllBatch; ++u)
-#pragma unroll
-      for (int k = 0; k < NV; ++k) E::axpy(hb[u], w[u][k], acc[k]);
   }
 #pragma unroll
   for (int k = 0; k < NV; ++k) {
