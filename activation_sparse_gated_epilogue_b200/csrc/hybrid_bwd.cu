@@ -150,18 +150,28 @@ __global__ void __launch_bounds__(kBwdThreads) ell_bwd_kernel(EllBwdParams p) {
     s_c[1][e] = __uint_as_float(static_cast<uint32_t>(p.hv.ell_u[rk + e]) << 16);
   }
   __syncthreads();
-  // dh_e = dy . W_down[j_e]
+  // batches of kBwdBatch entries: the W_down, W_up and W_gate rows of a
+  // batch are loaded together (one memory round trip per batch);
+  // dh_e = dy . W_down[j_e] is summed over the warps' parts of d, then
+  // du = dh a, dg = dh u and dx += du W_up[:, j] + dg W_gate[:, j]
+  // (coefficients rounded to bf16)
   for (int e0 = 0; e0 < nnz; e0 += kBwdBatch) {
-    uint4 w[kBwdBatch][NV];
+    uint4 wdv[kBwdBatch][NV], wu[kBwdBatch][NV], wg[kBwdBatch][NV];
 #pragma unroll
     for (int u = 0; u < kBwdBatch; ++u) {
       const int e = e0 + u;
       const int j = e < nnz ? s_j[e] : -1;
-      const uint4* row = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wd) + static_cast<int64_t>(j) * row_bytes);
+      const int64_t off = static_cast<int64_t>(j) * row_bytes;
+      const uint4* rd = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wd) + off);
+      const uint4* ru = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wu_t) + off);
+      const uint4* rg = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wg_t) + off);
 #pragma unroll
       for (int k = 0; k < NV; ++k) {
         const int v = tid + k * kBwdThreads;
-        w[u][k] = (j >= 0 && v < nvec) ? __ldg(row + v) : make_uint4(0, 0, 0, 0);
+        const bool ok = j >= 0 && v < nvec;
+        wdv[u][k] = ok ? __ldg(rd + v) : make_uint4(0, 0, 0, 0);
+        wu[u][k] = ok ? __ldg(ru + v) : make_uint4(0, 0, 0, 0);
+        wg[u][k] = ok ? __ldg(rg + v) : make_uint4(0, 0, 0, 0);
       }
     }
     float part[kBwdBatch];
@@ -169,7 +179,7 @@ __global__ void __launch_bounds__(kBwdThreads) ell_bwd_kernel(EllBwdParams p) {
     for (int u = 0; u < kBwdBatch; ++u) {
       float s = 0.0f;
 #pragma unroll
-      for (int k = 0; k < NV; ++k) s = E::dot(dyv[k], w[u][k], s);
+      for (int k = 0; k < NV; ++k) s = E::dot(dyv[k], wdv[u][k], s);
       part[u] = s;
     }
     const float tot = warp_reduce_multi<kBwdBatch>(part, lane);
@@ -177,46 +187,30 @@ __global__ void __launch_bounds__(kBwdThreads) ell_bwd_kernel(EllBwdParams p) {
       const int e = e0 + multi_entry<kBwdBatch>(lane);
       if (e < nnz) s_part[warp][e] = tot;
     }
-  }
-  __syncthreads();
-  for (int e = tid; e < nnz; e += kBwdThreads) {
-    float dh = 0.0f;
+    __syncthreads();
+    if (tid < kBwdBatch && e0 + tid < nnz) {
+      const int e = e0 + tid;
+      float dh = 0.0f;
 #pragma unroll
-    for (int w8 = 0; w8 < kBwdWarps; ++w8) dh += s_part[w8][e];
-    const float du = dh * s_c[0][e], dg = dh * s_c[1][e];
-    p.ws.du[rk + e] = du;
-    p.ws.dg[rk + e] = dg;
-    s_c[0][e] = du;
-    s_c[1][e] = dg;
-  }
-  __syncthreads();
-  // dx = sum du W_up[:, j] + dg W_gate[:, j]  (coefficients rounded to bf16)
-  for (int e0 = 0; e0 < nnz; e0 += kBwdBatch) {
-    uint4 wu[kBwdBatch][NV], wg[kBwdBatch][NV];
-    uint16_t cu[kBwdBatch], cg[kBwdBatch];
+      for (int w8 = 0; w8 < kBwdWarps; ++w8) dh += s_part[w8][e];
+      const float du = dh * s_c[0][e], dg = dh * s_c[1][e];
+      p.ws.du[rk + e] = du;
+      p.ws.dg[rk + e] = dg;
+      s_c[0][e] = du;
+      s_c[1][e] = dg;
+    }
+    __syncthreads();
 #pragma unroll
     for (int u = 0; u < kBwdBatch; ++u) {
       const int e = e0 + u;
-      const int j = e < nnz ? s_j[e] : -1;
-      cu[u] = e < nnz ? f32_to_bf16_bits(s_c[0][e]) : 0;
-      cg[u] = e < nnz ? f32_to_bf16_bits(s_c[1][e]) : 0;
-      const uint4* ru = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wu_t) + static_cast<int64_t>(j) * row_bytes);
-      const uint4* rg = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.wg_t) + static_cast<int64_t>(j) * row_bytes);
+      const uint16_t cu = e < nnz ? f32_to_bf16_bits(s_c[0][e]) : 0;
+      const uint16_t cg = e < nnz ? f32_to_bf16_bits(s_c[1][e]) : 0;
 #pragma unroll
       for (int k = 0; k < NV; ++k) {
-        const int v = tid + k * kBwdThreads;
-        const bool ok = j >= 0 && v < nvec;
-        wu[u][k] = ok ? __ldg(ru + v) : make_uint4(0, 0, 0, 0);
-        wg[u][k] = ok ? __ldg(rg + v) : make_uint4(0, 0, 0, 0);
+        E::axpy(cu, wu[u][k], acc[k]);
+        E::axpy(cg, wg[u][k], acc[k]);
       }
     }
-#pragma unroll
-    for (int u = 0; u < kBwdBatch; ++u)
-#pragma unroll
-      for (int k = 0; k < NV; ++k) {
-        E::axpy(cu[u], wu[u][k], acc[k]);
-        E::axpy(cg[u], wg[u][k], acc[k]);
-      }
   }
 #pragma unroll
   for (int k = 0; k < NV; ++k) {
