@@ -46,8 +46,8 @@ HYB_INFER_K = 64
 # (profiles/*.md), keyed by the source hash of the kernel they were taken on;
 # a kernel whose source changed since gets null.
 TRAFFIC = {
-    "593c4f4534efd102": 81.0e6,   # gate GEMM + TwELL, profiles/gate_gemm_twell_ffn_1b_bf16.md
-    "1d65e94c7498b4e5": 339.7e6,  # fused up/down main kernel, profiles/fused_up_down_ffn_1b_bf16.md
+    "2eebdb20775a495c": 80.1e6,   # gate GEMM + TwELL, profiles/gate_gemm_twell_ffn_1b_bf16.md
+    "6033b28ca36d3085": 341.5e6,  # fused up/down main kernel, profiles/fused_up_down_ffn_1b_bf16.md
 }
 
 
