@@ -698,9 +698,14 @@ extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* h
   using S = TcPairShape<256, 1>;
   CUtensorMap m1a, m1b;
   if ((rc = make_tmap_bf16(&m1a, ws.dys, sp, d, d, kBM))) return rc;
-  if ((rc = make_tmap_bf16(&m1b, wd, f, d, d, S::BN / 2))) return rc;
+  // tile widths for few spill rows: N = F in 128-wide tiles (dH), N = d in
+  // 64-wide tiles (dX), so that the GEMMs with one or two row tiles still
+  // spread over the SMs
+  using Sh = TcPairShape<128, 1>;
+  using Sx = TcPairShape<64, 1>;
+  if ((rc = make_tmap_bf16(&m1b, wd, f, d, d, Sh::BN / 2))) return rc;
   EpiBwdSpill e1{hv.spill_a, hv.spill_u, ws.acat, ws.hs, hy->n_spill, s_max, static_cast<int>(f), sp};
-  if ((rc = launch_tc_gemm_pair<S>(m1a, m1b, m1b, sp, f, d, e1, nullptr, st, "hybrid_ffn_bwd (dH)")))
+  if ((rc = launch_tc_gemm_pair<Sh>(m1a, m1b, m1b, sp, f, d, e1, nullptr, st, "hybrid_ffn_bwd (dH)")))
     return rc;
   // operands of the remaining GEMMs, K-major
   // (spill-row operands: only as many rows as the weight-gradient GEMMs read)
@@ -718,9 +723,9 @@ extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* h
   // dX_s = [dU | dG] [W_up ; W_gate]^T  -> dx rows
   CUtensorMap m2a, m2b;
   if ((rc = make_tmap_bf16(&m2a, ws.acat, sp, 2 * f, 2 * f, kBM))) return rc;
-  if ((rc = make_tmap_bf16(&m2b, ws.bcat, d, 2 * f, 2 * f, S::BN / 2))) return rc;
+  if ((rc = make_tmap_bf16(&m2b, ws.bcat, d, 2 * f, 2 * f, Sx::BN / 2))) return rc;
   EpiScatterRowsBwd e2{static_cast<uint16_t*>(dx), hy->spill_rows, hy->n_spill, s_max, static_cast<int>(d)};
-  if ((rc = launch_tc_gemm_pair<S>(m2a, m2b, m2b, sp, d, 2 * f, e2, nullptr, st, "hybrid_ffn_bwd (dX)")))
+  if ((rc = launch_tc_gemm_pair<Sx>(m2a, m2b, m2b, sp, d, 2 * f, e2, nullptr, st, "hybrid_ffn_bwd (dX)")))
     return rc;
   // dW_down += H^T dY_s
   CUtensorMap m3a, m3b;
