@@ -61,9 +61,11 @@ def library() -> ctypes.CDLL:
             "sge_last_error": (ctypes.c_char_p, []),
             "twell_gate_pack": (I, [P, P, I64, I64, I64, I, I, I, P, P, P, P, P]),
             "twell_fused_up_down_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
-            "twell_fused_up_down": (I, [P, P, P, P, P, P, P, I64, I64, I64, I, I, I, P,
+            "twell_fused_up_down": (I, [P, P, P, P, P, P, I64, P, I64, I64, I64, I, I, I, P,
                                         ctypes.c_size_t, P, P]),
-            "twell_fused_up_down_noalloc": (I, [P, P, P, P, P, P, P, I64, I64, I64, I, I, I, P, P]),
+            "twell_fused_up_down_noalloc": (I, [P, P, P, P, P, P, I64, P, I64, I64, I64, I, I, I,
+                                                P, P]),
+            "sge_interleave_up_down": (I, [P, P, P, I64, I64, I, P]),
             "twell_fused_up_down_noalloc_max_tokens": (I64, []),
             "dense_ffn_fwd": (I, [P, P, P, P, P, P, I64, I64, I64, P, P]),
             "sge_l2_gather_probe": (I, [P, I64, I, P, I64, P, P, P]),
@@ -104,6 +106,20 @@ def _check(t: torch.Tensor, name: str, dtype=None, shape=None) -> torch.Tensor:
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     return t
+
+
+def _check_rows(t: torch.Tensor, name: str, dtype, shape) -> int:
+    """A 2-D matrix of `shape` whose rows are contiguous (any row stride);
+    returns the row stride in elements."""
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.stride(1) != 1 and t.shape[1] > 1:
+        raise ValueError(f"{name} must have contiguous rows")
+    return t.stride(0) if t.shape[0] > 1 else t.shape[1]
 
 
 def _stream(dev: torch.device, stream) -> ctypes.c_void_p:
@@ -176,15 +192,32 @@ def fused_workspace(n_tokens: int, d_model: int, device) -> torch.Tensor:
     return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
 
 
+def interleave_up_down(wu_t: torch.Tensor, wd: torch.Tensor, stream=None):
+    """The interleaved weight layout twell_fused_up_down streams fastest:
+    returns (w_ud, wu_view, wd_view), w_ud [F][2d] with row j = wu_t[j] then
+    wd[j], and the two [F][d] views of it (row stride 2d) to pass as wu_t and
+    wd.  A weight-loading step, done once."""
+    _check(wu_t, "wu_t")
+    f, d = wu_t.shape
+    _check(wd, "wd", wu_t.dtype, (f, d))
+    w_ud = torch.empty((f, 2 * d), dtype=wu_t.dtype, device=wu_t.device)
+    _call("sge_interleave_up_down", _ptr(wu_t), _ptr(wd), _ptr(w_ud), f, d, _dtype_code(wu_t),
+          _stream(wu_t.device, stream))
+    return w_ud, w_ud[:, :d], w_ud[:, d:]
+
+
 def twell_fused_up_down(x: torch.Tensor, tw: TwELL, wu_t: torch.Tensor, wd: torch.Tensor,
                         y: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                         diag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """y = sum over TwELL entries of a * (x . W_up[:, j]) * W_down[j] (h never stored)."""
+    """y = sum over TwELL entries of a * (x . W_up[:, j]) * W_down[j] (h never stored).
+    wu_t and wd may be row-strided views with one row stride, e.g. the two
+    halves of interleave_up_down's matrix."""
     _check(x, "x")
     n, d = x.shape
     f = wu_t.shape[0]
-    _check(wu_t, "wu_t", x.dtype, (f, d))
-    _check(wd, "wd", x.dtype, (f, d))
+    ldw = _check_rows(wu_t, "wu_t", x.dtype, (f, d))
+    if _check_rows(wd, "wd", x.dtype, (f, d)) != ldw:
+        raise ValueError("wu_t and wd must have the same row stride")
     _check(tw.count, "count", torch.uint8, (n, f // tw.tile))
     _check(tw.idx, "idx", torch.uint8, (n, f // tw.tile, tw.cap))
     _check(tw.val, "val", x.dtype, (n, f // tw.tile, tw.cap))
@@ -197,7 +230,7 @@ def twell_fused_up_down(x: torch.Tensor, tw: TwELL, wu_t: torch.Tensor, wd: torc
     if diag is not None:
         _check(diag, "diag", torch.int32, (4,))
     _call("twell_fused_up_down", _ptr(x), _ptr(tw.count), _ptr(tw.idx), _ptr(tw.val),
-          _ptr(wu_t), _ptr(wd), _ptr(y), n, d, f, _dtype_code(x), tw.tile, tw.cap,
+          _ptr(wu_t), _ptr(wd), ldw, _ptr(y), n, d, f, _dtype_code(x), tw.tile, tw.cap,
           _ptr(workspace), workspace.numel(), _ptr(diag), _stream(x.device, stream))
     return y
 

@@ -10,18 +10,20 @@
 // At the densities the method runs at (about 1% of d_ff) two tokens rarely
 // share a column, so every entry streams one row of W_up and one of W_down
 // from L2 with little reuse: the kernel is bound by how many row bytes it
-// keeps in flight between L2 and the SMs, and by its instructions per row.
+// keeps in flight between L2 and the SMs, by the copies and waits per byte,
+// and by its instructions per row.
 //
-// Warps.  Each warp streams whole rows (one 16-byte piece per lane per 512
-// bytes) through its own ring of shared-memory slots with cp.async.bulk: its
-// lanes issue copies in parallel, one mbarrier per slot, several rows ahead
-// of consumption.  It keeps x[t] (bf16) and the fp32 y[t] of its job in
-// registers, forms each dot product x[t] . W_up[:, j] with exact bf16 x bf16
-// products accumulated in fp32 and reduced over the lanes, rounds
-// h = a * u to the activation dtype (what the dense FFN gives h), and
-// accumulates h * W_down[j] into y.  h lives only in registers and shared
-// memory.  Entries are taken in chunks of 32, one per lane: the W_up rows of
-// a chunk, then its W_down rows.
+// Warps.  Each warp streams its entries through its own ring of
+// shared-memory slots with cp.async.bulk: one slot holds an entry's W_up row
+// and its W_down row (one copy when the caller interleaves the two matrices
+// row by row, two copies on the same mbarrier otherwise); its lanes issue the
+// copies of several slots in parallel, ahead of consumption.  It keeps x[t]
+// (bf16) and the fp32 y[t] of its job in registers.  For each entry it forms
+// the dot product x[t] . W_up[:, j] with exact bf16 x bf16 products
+// accumulated in fp32, reduces it over the lanes, rounds h = a * u to the
+// activation dtype (what the dense FFN gives h), and accumulates
+// h * W_down[j] into y.  h lives only in registers.  Entries are resolved in
+// chunks of 32, one per lane.
 //
 // Teams.  A team of kTeam warps shares one job (a token, or a unit of a heavy
 // token): warp w takes the job's entries w, w + kTeam, ...  At the end of the
@@ -56,8 +58,7 @@ namespace sge {
 
 constexpr int kTeam = 4;        // warps per job
 constexpr int kChunk = 32;      // entries per chunk, one per lane
-constexpr int kBatch = 4;       // rows per reduction batch (the partial-sum shift register has 4)
-constexpr int kMaxSlots = 16;   // ring slots per warp
+constexpr int kMaxSlots = 8;    // ring slots per warp
 constexpr int kSmemBudget = 232448;
 constexpr int kUnitMin = 32;
 constexpr int kMaxCtas = 256;   // the grid is clamped to this many CTAs
@@ -157,7 +158,9 @@ struct UdParams {
   int row_bytes;
   int teams;       // teams per CTA
   int slots;       // ring slots per warp
-  int slot_bytes;  // one ring slot: NV * 512 bytes (a row, then zeros)
+  int slot_bytes;  // one ring slot: two halves of NV * 512 bytes (a row, then zeros)
+  int64_t w_ld;    // row stride of wu_t and wd in bytes
+  int w_one;       // each wd row directly follows its wu_t row and fills a half: one copy per entry
   int off_full;    // shared-memory offsets: per-warp slot barriers,
   int off_team;    // per-team job queue, barriers and row buffer,
   int team_bytes;
@@ -379,7 +382,6 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
   const int S = p.slots;
   uint8_t* ring = smem + warp * S * p.slot_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_full) + warp * S;
-  float* ubuf = reinterpret_cast<float*>(smem + p.off_full + warps * S * 8) + warp * kChunk;
   uint8_t* tb = smem + p.off_team + team * p.team_bytes;
   Job* jobq = reinterpret_cast<Job*>(tb);  // [4] + a staging entry
   uint64_t* tbar = reinterpret_cast<uint64_t*>(tb + 5 * sizeof(Job));
@@ -391,11 +393,12 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
   const bool leader = w == 0;
   const int pieces = p.row_bytes / 16;
 
-  // the slots' bytes past the row stay zero for the whole kernel
-  if (p.row_bytes < p.slot_bytes) {
-    for (int q = 0; q < S; ++q)
-      for (int o = p.row_bytes + lane * 16; o < p.slot_bytes; o += 32 * 16)
-        *reinterpret_cast<uint4*>(ring + q * p.slot_bytes + o) = make_uint4(0, 0, 0, 0);
+  // the bytes of each half slot past the row stay zero for the whole kernel
+  const int half = p.slot_bytes / 2;
+  if (p.row_bytes < half) {
+    for (int q = 0; q < 2 * S; ++q)
+      for (int o = p.row_bytes + lane * 16; o < half; o += 32 * 16)
+        *reinterpret_cast<uint4*>(ring + q * half + o) = make_uint4(0, 0, 0, 0);
   }
   if (lane == 0) {
     for (int q = 0; q < S; ++q) mbar_init(full + q, 1);
@@ -413,7 +416,7 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
   int n_light[kLightClasses];
 #pragma unroll
   for (int c = 0; c < kLightClasses; ++c) n_light[c] = *reinterpret_cast<volatile int*>(p.hdr + kHLight + c);
-  const int64_t rb = p.row_bytes;
+  const int64_t rb = p.row_bytes, wl = p.w_ld;
   const char* xb = static_cast<const char*>(p.x);
   const char* ub = static_cast<const char*>(p.wu_t);
   const char* db = static_cast<const char*>(p.wd);
@@ -556,14 +559,15 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
     ++rci;
   };
   auto stream_len = [](const Chunk& c) {
-    return c.t < 0 ? 0 : ((c.flags & kHasX) ? 1 : 0) + 2 * c.n;
+    return c.t < 0 ? 0 : ((c.flags & kHasX) ? 1 : 0) + c.n;
   };
   Chunk cur, nxt;
   resolve(cur);
   resolve(nxt);
 
   // ---- this warp's ring: positions are the x row (first chunk of a job),
-  // then the W_up rows and the W_down rows of each chunk
+  // then one per entry of each chunk (its W_up row in the first half of the
+  // slot, its W_down row in the second)
   uint32_t issued = 0, consumed = 0;
   int is = 0, cs = 0;   // slots of the next issue and the next consumption
   uint32_t cph = 0;     // phase parity of the slot being consumed
@@ -587,16 +591,25 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
       const int m = min(room, len - iq);
       const int hx = (c.flags & kHasX) ? 1 : 0;
       const int q = iq + lane;
-      const int r = q - hx;
-      const int jv = __shfl_sync(0xffffffffu, c.j, (r < c.n ? r : r - c.n) & 31);
+      const int jv = __shfl_sync(0xffffffffu, c.j, (q - hx) & 31);
       if (lane < m) {
-        const char* src = (hx && q == 0) ? xb + static_cast<int64_t>(c.t) * rb
-                                         : (r < c.n ? ub : db) + static_cast<int64_t>(jv) * rb;
         int slot = is + lane;
         if (slot >= S) slot -= S;
+        uint8_t* dst = ring + slot * p.slot_bytes;
+        const uint32_t rb32 = static_cast<uint32_t>(p.row_bytes);
         fence_proxy_async_smem();
-        mbar_arrive_expect_tx(full + slot, static_cast<uint32_t>(p.row_bytes));
-        bulk_load(ring + slot * p.slot_bytes, src, static_cast<uint32_t>(p.row_bytes), full + slot);
+        if (hx && q == 0) {
+          mbar_arrive_expect_tx(full + slot, rb32);
+          bulk_load(dst, xb + static_cast<int64_t>(c.t) * rb, rb32, full + slot);
+        } else {
+          mbar_arrive_expect_tx(full + slot, 2 * rb32);
+          if (p.w_one) {
+            bulk_load(dst, ub + static_cast<int64_t>(jv) * wl, 2 * rb32, full + slot);
+          } else {
+            bulk_load(dst, ub + static_cast<int64_t>(jv) * wl, rb32, full + slot);
+            bulk_load(dst + half, db + static_cast<int64_t>(jv) * wl, rb32, full + slot);
+          }
+        }
       }
       issued += m;
       is += m;
@@ -644,58 +657,26 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
 #pragma unroll
       for (int k = 0; k < NV; ++k) xr[k] = piece(a, k);
       release();
-    }
-    // phase U: dot products with the W_up rows, reduced over the lanes
-    for (int e0 = 0; ok && e0 < cur.n; e0 += kBatch) {
       pump();
-      // the batch's partial sums shift through p0..p3 (no local-memory array;
-      // the row loop stays rolled to keep the hot code small)
-      float p0 = 0.0f, p1 = 0.0f, p2 = 0.0f, p3 = 0.0f;
-#pragma unroll 1
-      for (int r = 0; r < kBatch; ++r) {
-        float v = 0.0f;
-        if (e0 + r < cur.n) {
-          uint32_t a;
-          if (!(ok = acquire(a))) break;
-          // eight independent accumulator chains
-          float s[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-          for (int k = 0; k < NV; ++k) E::dot2(xr[k], piece(a, k), s[2 * (k & 3)], s[2 * (k & 3) + 1]);
-          release();
-          v = ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
-        }
-        p3 = p2;
-        p2 = p1;
-        p1 = p0;
-        p0 = v;
-      }
-      if (!ok) break;
-      float part[kBatch] = {p3, p2, p1, p0};
-      const float tot = warp_reduce_multi<kBatch>(part, lane);
-      if ((lane & (32 / kBatch - 1)) == 0) {
-        const int r = multi_entry<kBatch>(lane);
-        if (e0 + r < cur.n) ubuf[e0 + r] = tot;
-      }
     }
-    if (!ok) break;
-    __syncwarp();
-    // h = a * u, rounded as the down projection uses it (entry `lane`)
-    const int hb = lane < cur.n ? E::h_bits(E::h_of(__int_as_float(cur.a) * ubuf[lane])) : 0;
-    // phase D: y += h * W_down[j]
-    for (int e0 = 0; ok && e0 < cur.n; e0 += kBatch) {
-      pump();
-#pragma unroll 1
-      for (int r = 0; r < kBatch; ++r) {
-        const int hr = __shfl_sync(0xffffffffu, hb, (e0 + r) & 31);
-        if (e0 + r < cur.n) {
-          uint32_t a;
-          if (!(ok = acquire(a))) break;
-          const typename E::HType h = E::h_from_bits(hr);
+    // each entry: u = x . W_up[:, j] reduced over the lanes, h = a * u
+    // rounded as the down projection uses it, y += h * W_down[j]
+    for (int e = 0; e < cur.n; ++e) {
+      const float ae = __int_as_float(__shfl_sync(0xffffffffu, cur.a, e & 31));
+      uint32_t a;
+      if (!(ok = acquire(a))) break;
+      // eight independent accumulator chains
+      float s[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-          for (int k = 0; k < NV; ++k) E::axpy(h, piece(a, k), acc[k]);
-          release();
-        }
-      }
+      for (int k = 0; k < NV; ++k) E::dot2(xr[k], piece(a, k), s[2 * (k & 3)], s[2 * (k & 3) + 1]);
+      float u = ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
+      const typename E::HType h = E::h_of(ae * u);
+#pragma unroll
+      for (int k = 0; k < NV; ++k) E::axpy(h, piece(a + half, k), acc[k]);
+      release();
+      pump();
     }
     if (!ok) break;
     if (cur.flags & kLast) {
@@ -936,7 +917,8 @@ struct UsParams {
   int nt;
   int tile;
   int cap;
-  int pieces;  // 16-byte pieces per row
+  int pieces;    // 16-byte pieces per row
+  int64_t w_ld;  // row stride of wu_t and wd in bytes
 };
 
 // One CTA per unit (grid-stride over the units), kSmWarps warps; NV pieces
@@ -1027,8 +1009,8 @@ __global__ void __launch_bounds__(kSmWarps * 32, 1) us_main_kernel(const UsParam
         for (int i = 0; i < cnt; ++i) {
           const int ji = __shfl_sync(0xffffffffu, j, i);
           const float ai = __shfl_sync(0xffffffffu, a, i);
-          const uint4* ur = reinterpret_cast<const uint4*>(static_cast<const char*>(p.wu_t) + ji * rb);
-          const uint4* dr = reinterpret_cast<const uint4*>(static_cast<const char*>(p.wd) + ji * rb);
+          const uint4* ur = reinterpret_cast<const uint4*>(static_cast<const char*>(p.wu_t) + ji * p.w_ld);
+          const uint4* dr = reinterpret_cast<const uint4*>(static_cast<const char*>(p.wd) + ji * p.w_ld);
           uint4 wu[NV], wdv[NV];
 #pragma unroll
           for (int q = 0; q < NV; ++q) {
@@ -1144,18 +1126,18 @@ static int small_nv(const UsParams& prm, int nv, int smem, int grid, cudaStream_
 // p.row_bytes with nv pieces per lane; false if the rows are too long.
 static bool make_geometry(UdParams& p, int nv, int* smem_bytes) {
   int warps = warps_for_nv(nv);
-  p.slot_bytes = nv * 512;
+  p.slot_bytes = 2 * nv * 512;
   p.team_bytes = kTeamHdr + ((p.d * 4 + 15) & ~15);
   for (;; warps -= kTeam) {
     if (warps < kTeam) return false;
     p.teams = warps / kTeam;
-    const int fixed = p.teams * p.team_bytes + warps * kChunk * 4 + 16 + 16;
+    const int fixed = p.teams * p.team_bytes + 16 + 16;
     int slots = (kSmemBudget - fixed) / (warps * (p.slot_bytes + 8));
     if (slots > kMaxSlots) slots = kMaxSlots;
-    if (slots < kBatch) continue;  // a batch of rows must fit the ring
+    if (slots < 2) continue;  // one slot in flight while the other is read
     p.slots = slots;
     p.off_full = warps * slots * p.slot_bytes;
-    p.off_team = (p.off_full + warps * slots * 8 + warps * kChunk * 4 + 15) & ~15;
+    p.off_team = (p.off_full + warps * slots * 8 + 15) & ~15;
     p.off_abort = p.off_team + p.teams * p.team_bytes;
     *smem_bytes = p.off_abort + 16;
     return *smem_bytes <= kSmemBudget;
@@ -1215,6 +1197,7 @@ static int run_small(const UdParams& prm, const WsLayout& L, uint8_t* ws, int64_
   up.tile = prm.tile;
   up.cap = prm.cap;
   up.pieces = prm.row_bytes / 16;
+  up.w_ld = prm.w_ld;
   us_plan_kernel<<<1, kSmallTokens, 0, st>>>(prm.count, prm.n_rows, prm.nt, prm.cap, pool_slots, prm.hdr,
                                              const_cast<int*>(prm.ntok), ufirst, pbase, prm.done);
   const int rc = check_launch("twell_fused_up_down (small-batch plan)");
@@ -1225,7 +1208,7 @@ static int run_small(const UdParams& prm, const WsLayout& L, uint8_t* ws, int64_
 
 // Planning kernels and the main kernel, shared by both entry points.
 static int run_fused(const char* name, const void* x, const uint8_t* count, const uint8_t* idx,
-                     const void* val, const void* wu_t, const void* wd, void* y, int64_t n_tokens,
+                     const void* val, const void* wu_t, const void* wd, int64_t ldw, void* y, int64_t n_tokens,
                      int64_t d_model, int64_t d_ff, int dtype, int tile, int cap, void* workspace,
                      int64_t pool_slots, int32_t* diag, cudaStream_t st) {
   if (dtype != SGE_BF16 && dtype != SGE_F32) return fail(SGE_ERR_UNSUPPORTED, "%s: dtype %d", name, dtype);
@@ -1254,10 +1237,15 @@ static int run_fused(const char* name, const void* x, const uint8_t* count, cons
   prm.tile = tile;
   prm.cap = cap;
   prm.row_bytes = static_cast<int>(d_model * esz);
+  prm.w_ld = ldw * esz;
   const int nv = nv_for(prm.row_bytes);
   int smem = 0;
   if (!nv || !make_geometry(prm, nv, &smem))
     return fail(SGE_ERR_UNSUPPORTED, "%s: d_model too large: rows of %d bytes (max 8192)", name, prm.row_bytes);
+  // one copy per entry brings both rows when each wd row directly follows
+  // its wu_t row and a row fills half a slot exactly
+  prm.w_one = static_cast<const char*>(wd) == static_cast<const char*>(wu_t) + prm.row_bytes &&
+              prm.w_ld == 2 * static_cast<int64_t>(prm.row_bytes) && 2 * prm.row_bytes == prm.slot_bytes;
   if (prm.nt > 256)
     return fail(SGE_ERR_UNSUPPORTED, "%s: %d TwELL tiles per row (max 256)", name, prm.nt);
   if (n_tokens <= kSmallTokens && nv <= 8 && pool_slots >= n_tokens)
@@ -1289,10 +1277,12 @@ static int run_fused(const char* name, const void* x, const uint8_t* count, cons
                            : dispatch_main<false>(prm, nv, smem, static_cast<int>(grid), st);
 }
 
-static int check_args(const char* name, int64_t n_tokens, int64_t d_model, int64_t d_ff, int tile,
-                      int cap) {
+static int check_args(const char* name, int64_t n_tokens, int64_t d_model, int64_t d_ff, int64_t ldw,
+                      int tile, int cap) {
   if (n_tokens < 0 || d_model < 1 || d_ff < 1) return fail(SGE_ERR_ARG, "%s: bad sizes", name);
   if (d_model % 8) return fail(SGE_ERR_ARG, "%s: d_model %% 8 != 0", name);
+  if (ldw < d_model || ldw % 8 || ldw >= (1LL << 40))
+    return fail(SGE_ERR_ARG, "%s: ldw %lld must be a multiple of 8 and >= d_model", name, (long long)ldw);
   if (tile < 1 || tile > 255 || d_ff % tile)
     return fail(SGE_ERR_ARG, "%s: tile must divide d_ff and be <= 255", name);
   if (cap < 1 || cap > tile) return fail(SGE_ERR_ARG, "%s: cap outside [1, tile]", name);
@@ -1311,13 +1301,13 @@ extern "C" size_t twell_fused_up_down_workspace_bytes(int64_t n_tokens, int64_t 
 }
 
 extern "C" int twell_fused_up_down(const void* x, const uint8_t* count, const uint8_t* idx,
-                                   const void* val, const void* wu_t, const void* wd, void* y,
-                                   int64_t n_tokens, int64_t d_model, int64_t d_ff, int dtype,
-                                   int tile, int cap, void* workspace, size_t workspace_bytes,
-                                   int32_t* diag, void* stream) {
+                                   const void* val, const void* wu_t, const void* wd, int64_t ldw,
+                                   void* y, int64_t n_tokens, int64_t d_model, int64_t d_ff,
+                                   int dtype, int tile, int cap, void* workspace,
+                                   size_t workspace_bytes, int32_t* diag, void* stream) {
   static const char* kName = "twell_fused_up_down";
   clear_error();
-  int rc = check_args(kName, n_tokens, d_model, d_ff, tile, cap);
+  int rc = check_args(kName, n_tokens, d_model, d_ff, ldw, tile, cap);
   if (rc) return rc;
   if (n_tokens == 0) return SGE_OK;
   if (!x || !count || !idx || !val || !wu_t || !wd || !y || !workspace)
@@ -1328,7 +1318,7 @@ extern "C" int twell_fused_up_down(const void* x, const uint8_t* count, const ui
   const size_t need = twell_fused_up_down_workspace_bytes(n_tokens, d_model);
   if (workspace_bytes < need)
     return fail(SGE_ERR_ARG, "%s: workspace of %zu bytes, %zu needed", kName, workspace_bytes, need);
-  return run_fused(kName, x, count, idx, val, wu_t, wd, y, n_tokens, d_model, d_ff, dtype, tile, cap,
+  return run_fused(kName, x, count, idx, val, wu_t, wd, ldw, y, n_tokens, d_model, d_ff, dtype, tile, cap,
                    workspace, pool_slots_for(kPoolBytes, d_model), diag,
                    static_cast<cudaStream_t>(stream));
 }
@@ -1390,7 +1380,7 @@ extern "C" int64_t twell_fused_up_down_noalloc_max_tokens(void) { return kNoAllo
 
 extern "C" int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, const uint8_t* idx,
                                            const void* val, const void* wu_t, const void* wd,
-                                           void* y, int64_t n_tokens, int64_t d_model,
+                                           int64_t ldw, void* y, int64_t n_tokens, int64_t d_model,
                                            int64_t d_ff, int dtype, int tile, int cap,
                                            int32_t* diag, void* stream) {
   static const char* kName = "twell_fused_up_down_noalloc";
@@ -1400,7 +1390,7 @@ extern "C" int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, 
                 "%s: %lld tokens exceed the built-in scratch limit of %lld; "
                 "use twell_fused_up_down with a workspace",
                 kName, (long long)n_tokens, (long long)kNoAllocMaxTokens);
-  int rc = check_args(kName, n_tokens, d_model, d_ff, tile, cap);
+  int rc = check_args(kName, n_tokens, d_model, d_ff, ldw, tile, cap);
   if (rc) return rc;
   if (n_tokens == 0) return SGE_OK;
   if (!x || !count || !idx || !val || !wu_t || !wd || !y)
@@ -1417,6 +1407,36 @@ extern "C" int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, 
   // The array keeps the previous call's contents; the planning kernels reset
   // every counter the call relies on (job counters and cursor, and the
   // completion counter of each split token).
-  return run_fused(kName, x, count, idx, val, wu_t, wd, y, n_tokens, d_model, d_ff, dtype, tile, cap,
+  return run_fused(kName, x, count, idx, val, wu_t, wd, ldw, y, n_tokens, d_model, d_ff, dtype, tile, cap,
                    scratch, slots, diag, static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// The interleaved weight layout: row j of w_ud is wu_t[j] then wd[j].
+
+extern "C" int sge_interleave_up_down(const void* wu_t, const void* wd, void* w_ud, int64_t d_ff,
+                                      int64_t d_model, int dtype, void* stream) {
+  static const char* kName = "sge_interleave_up_down";
+  clear_error();
+  if (dtype != SGE_BF16 && dtype != SGE_F32) return fail(SGE_ERR_UNSUPPORTED, "%s: dtype %d", kName, dtype);
+  if (d_ff < 0 || d_model < 1 || d_model >= (1LL << 31) || d_ff >= (1LL << 31))
+    return fail(SGE_ERR_ARG, "%s: bad sizes", kName);
+  if (d_ff == 0) return SGE_OK;
+  if (!wu_t || !wd || !w_ud) return fail(SGE_ERR_ARG, "%s: null pointer", kName);
+  const size_t rb = static_cast<size_t>(d_model) * (dtype == SGE_BF16 ? 2 : 4);
+  const size_t n = rb * static_cast<size_t>(d_ff);
+  const char* o = static_cast<const char*>(w_ud);
+  auto overlaps = [&](const void* a, size_t na) {
+    const char* c = static_cast<const char*>(a);
+    return c < o + 2 * n && o < c + na;
+  };
+  if (overlaps(wu_t, n) || overlaps(wd, n)) return fail(SGE_ERR_ARG, "%s: w_ud overlaps an input", kName);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpy2DAsync(w_ud, 2 * rb, wu_t, rb, rb, static_cast<size_t>(d_ff),
+                                    cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpy2DAsync(static_cast<char*>(w_ud) + rb, 2 * rb, wd, rb, rb, static_cast<size_t>(d_ff),
+                          cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "%s: %s", kName, cudaGetErrorString(e));
+  return SGE_OK;
 }

@@ -179,6 +179,8 @@ def run_own(args, rank, world, local_rank):
     n, d, f, tile, cap = cfg.n_tokens, cfg.d_model, cfg.d_ff, cfg.tile, cfg.cap
     x, wg, wu, wd = (getattr(inp, k).to(dev) for k in ("x", "wg_t", "wu_t", "wd"))
     wd_t = wd.t().contiguous()
+    # the fused kernel's weights: W_up^T and W_down interleaved row by row
+    _w_ud, wu_i, wd_i = sge.interleave_up_down(wu, wd)
     tw = sge.TwELL.empty(n, f, tile, cap, x.dtype, dev)
     y = torch.empty_like(x)
     h = torch.empty((n, f), dtype=x.dtype, device=dev)
@@ -212,7 +214,7 @@ def run_own(args, rank, world, local_rank):
         return reduce_max_over_ranks(v, dev)
 
     gate = lambda: sge.twell_gate_pack(x, wg, tile, cap, out=tw, diag=diag)
-    fused = lambda: sge.twell_fused_up_down(x, tw, wu, wd, y=y, workspace=ws)
+    fused = lambda: sge.twell_fused_up_down(x, tw, wu_i, wd_i, y=y, workspace=ws)
     dense = lambda: sge.dense_ffn_fwd(x, wg, wu, wd_t, h=h, y=y_dense)
 
     if args.profile:
@@ -272,7 +274,7 @@ def run_own(args, rank, world, local_rank):
     def e2e():
         x_dev2.copy_(x_host, non_blocking=True)
         sge.twell_gate_pack(x_dev2, wg, tile, cap, out=tw, diag=diag)
-        sge.twell_fused_up_down(x_dev2, tw, wu, wd, y=y, workspace=ws)
+        sge.twell_fused_up_down(x_dev2, tw, wu_i, wd_i, y=y, workspace=ws)
         y_host.copy_(y, non_blocking=True)
     e2e_steps = min(args.steps, 50)
     barrier()
@@ -363,6 +365,7 @@ def run_own(args, rank, world, local_rank):
                                f"target density {cfg.rho} sigma={cfg.sigma}",
                    "realised_density": round(density, 5), "nnz": nnz,
                    "l2": "flushed between steps (256 MB write outside the step events)",
+                   "weights": "fused kernel reads W_up^T and W_down interleaved row by row ([F][2d], built once)",
                    "parallelism": f"replicas x{world} (token batches independent)"},
         "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")},
         "kernels": [dominant, rest],
@@ -406,6 +409,8 @@ def run_sweep(args, local_rank):
     n, d, f, tile, cap = cfg.n_tokens, cfg.d_model, cfg.d_ff, cfg.tile, cfg.cap
     x, wg, wu, wd = (getattr(inp, k).to(dev) for k in ("x", "wg_t", "wu_t", "wd"))
     wd_t = wd.t().contiguous()
+    # the fused kernel's weights: W_up^T and W_down interleaved row by row
+    _w_ud, wu_i, wd_i = sge.interleave_up_down(wu, wd)
     tw = sge.TwELL.empty(n, f, tile, cap, x.dtype, dev)
     y = torch.empty_like(x)
     ws = sge.fused_workspace(n, d, dev)
@@ -437,7 +442,7 @@ def run_sweep(args, local_rank):
         tau = synth.solve_tau_density(rho, cfg.sigma, d)
         wg[:, d - 1] = -tau                      # rounded to the weight dtype
         gate = lambda: sge.twell_gate_pack(x, wg, tile, cap, out=tw)
-        fused = lambda: sge.twell_fused_up_down(x, tw, wu, wd, y=y, workspace=ws)
+        fused = lambda: sge.twell_fused_up_down(x, tw, wu_i, wd_i, y=y, workspace=ws)
         t = timed([gate, fused], steps, 3)
         mg = statistics.mean(a for a, _ in t)
         mf = statistics.mean(b for _, b in t)
@@ -487,6 +492,8 @@ def run_cap_sweep(args, local_rank):
     n, d, f, tile = cfg.n_tokens, cfg.d_model, cfg.d_ff, cfg.tile
     x, wg, wu, wd = (getattr(inp, k).to(dev) for k in ("x", "wg_t", "wu_t", "wd"))
     wd_t = wd.t().contiguous()
+    # the fused kernel's weights: W_up^T and W_down interleaved row by row
+    _w_ud, wu_i, wd_i = sge.interleave_up_down(wu, wd)
     ws = sge.fused_workspace(n, d, dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -511,7 +518,7 @@ def run_cap_sweep(args, local_rank):
 
     # the full-capacity result every C is compared with
     tw_full = sge.twell_gate_pack(x, wg, tile, tile)
-    y_full = sge.twell_fused_up_down(x, tw_full, wu, wd, workspace=ws)
+    y_full = sge.twell_fused_up_down(x, tw_full, wu_i, wd_i, workspace=ws)
     torch.cuda.synchronize(dev)
     out = []
     for cap in (tile // 4, tile // 2, tile):
@@ -519,7 +526,7 @@ def run_cap_sweep(args, local_rank):
         diag = sge.new_diag(dev)
         y = torch.empty_like(x)
         gate = lambda: sge.twell_gate_pack(x, wg, tile, cap, out=tw)
-        fused = lambda: sge.twell_fused_up_down(x, tw, wu, wd, y=y, workspace=ws)
+        fused = lambda: sge.twell_fused_up_down(x, tw, wu_i, wd_i, y=y, workspace=ws)
         sge.twell_gate_pack(x, wg, tile, cap, out=tw, diag=diag)
         torch.cuda.synchronize(dev)
         cnt = tw.count.to(torch.int64)

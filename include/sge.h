@@ -119,8 +119,16 @@ int twell_gate_pack(const void* x, const void* wg_t, int64_t n_tokens, int64_t d
  *   before the down projection (the precision the dense bf16 FFN gives h).
  *   y is written in `dtype`.
  *
- *   x [N][d], wu_t [F][d], wd [F][d], y [N][d] in dtype; count/idx/val the
- *   TwELL produced by twell_gate_pack with the same T and C.
+ *   x [N][d], y [N][d] in dtype; count/idx/val the TwELL produced by
+ *   twell_gate_pack with the same T and C.
+ *   wu_t, wd   F rows of d elements each (row j of wu_t is column j of W_up),
+ *              rows ldw elements apart in both (ldw >= d, a multiple of 8).
+ *              ldw = d: two separate [F][d] matrices.  The fastest layout
+ *              interleaves them: one [F][2d] matrix whose row j holds
+ *              W_up[:, j] then W_down[j, :], passed as wu_t = its start,
+ *              wd = wu_t + d elements and ldw = 2d (sge_interleave_up_down
+ *              builds it).  When d * element size is a multiple of 512 bytes,
+ *              one copy then brings both rows of an entry.
  *   workspace  device scratch of at least
  *              twell_fused_up_down_workspace_bytes(N, d) bytes (N-proportional
  *              lists plus a pool of about 64 MiB), 256-byte aligned, owned by
@@ -137,13 +145,13 @@ int twell_gate_pack(const void* x, const void* wg_t, int64_t n_tokens, int64_t d
  * differently from the larger batches' kernel: a token's y can differ between
  * the two in the last bits.
  * Errors: as twell_gate_pack; SGE_ERR_ARG for a missing, short or misaligned
- * workspace; SGE_ERR_UNSUPPORTED for d > 4096 or
+ * workspace or a bad ldw; SGE_ERR_UNSUPPORTED for d > 4096 or
  * F / T > 256.
  */
 size_t twell_fused_up_down_workspace_bytes(int64_t n_tokens, int64_t d_model);
 
 int twell_fused_up_down(const void* x, const uint8_t* count, const uint8_t* idx, const void* val,
-                        const void* wu_t, const void* wd, void* y, int64_t n_tokens,
+                        const void* wu_t, const void* wd, int64_t ldw, void* y, int64_t n_tokens,
                         int64_t d_model, int64_t d_ff, int dtype, int tile, int cap,
                         void* workspace, size_t workspace_bytes, int32_t* diag, void* stream);
 
@@ -174,9 +182,21 @@ int twell_fused_up_down(const void* x, const uint8_t* count, const uint8_t* idx,
 int64_t twell_fused_up_down_noalloc_max_tokens(void);
 
 int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, const uint8_t* idx,
-                                const void* val, const void* wu_t, const void* wd, void* y,
-                                int64_t n_tokens, int64_t d_model, int64_t d_ff, int dtype,
-                                int tile, int cap, int32_t* diag, void* stream);
+                                const void* val, const void* wu_t, const void* wd, int64_t ldw,
+                                void* y, int64_t n_tokens, int64_t d_model, int64_t d_ff,
+                                int dtype, int tile, int cap, int32_t* diag, void* stream);
+
+/*
+ * sge_interleave_up_down -- builds the interleaved weight layout that
+ * twell_fused_up_down streams fastest: w_ud [F][2d], row j = wu_t[j] (d
+ * elements) then wd[j] (d elements).  A layout step for loading weights, done
+ * once; it is not part of the forward pass.
+ *   wu_t [F][d], wd [F][d] contiguous; w_ud [F][2d] caller-allocated, not
+ *   overlapping them; dtype SGE_BF16 or SGE_F32.  Stream-ordered copies.
+ * Errors: SGE_ERR_ARG for null pointers or bad sizes; SGE_ERR_CUDA.
+ */
+int sge_interleave_up_down(const void* wu_t, const void* wd, void* w_ud, int64_t d_ff,
+                           int64_t d_model, int dtype, void* stream);
 
 /*
  * dense_ffn_fwd -- the dense gated FFN the method is compared against

@@ -73,29 +73,47 @@ def test_bad_arguments_are_rejected_on_host(lib):
 
 def test_empty_input_is_a_no_op(lib):
     assert _gate(lib, n=0) == 0
-    assert lib.twell_fused_up_down(None, None, None, None, None, None, None, 0, 64, 256,
+    assert lib.twell_fused_up_down(None, None, None, None, None, None, 64, None, 0, 64, 256,
                                    sge.SGE_BF16, 128, 128, None, 0, None, None) == 0
     assert lib.dense_ffn_fwd(None, None, None, None, None, None, 0, 64, 256, None, None) == 0
 
 
 def test_fused_rejects_bad_arguments(lib):
-    assert lib.twell_fused_up_down(None, None, None, None, None, None, None, 8, 12, 256,
+    assert lib.twell_fused_up_down(None, None, None, None, None, None, 12, None, 8, 12, 256,
                                    sge.SGE_BF16, 128, 128, None, 0, None, None) == 1
-    assert lib.twell_fused_up_down(None, None, None, None, None, None, None, 8, 64, 256,
+    assert lib.twell_fused_up_down(None, None, None, None, None, None, 64, None, 8, 64, 256,
                                    sge.SGE_BF16, 128, 128, None, 0, None, None) == 1
     p = ctypes.c_void_p(16)
     # a workspace smaller than the query's answer is rejected
-    assert lib.twell_fused_up_down(p, p, p, p, p, p, p, 1000, 64, 256, sge.SGE_BF16, 128, 128,
+    assert lib.twell_fused_up_down(p, p, p, p, p, p, 64, p, 1000, 64, 256, sge.SGE_BF16, 128, 128,
                                    p, 64, None, None) == 1
     assert b"workspace" in lib.sge_last_error()
     assert lib.twell_fused_up_down_workspace_bytes(1000, 64) >= 16 + 5 * 1000
     assert lib.twell_fused_up_down_workspace_bytes(1000, 64) % 256 == 0
     # the workspace must be 256-byte aligned
     ws = lib.twell_fused_up_down_workspace_bytes(1000, 64)
-    assert lib.twell_fused_up_down(p, p, p, p, p, p, p, 1000, 64, 256, sge.SGE_BF16, 128, 128,
+    assert lib.twell_fused_up_down(p, p, p, p, p, p, 64, p, 1000, 64, 256, sge.SGE_BF16, 128, 128,
                                    ctypes.c_void_p(4096 + 16), ws, None, None) == 1
     assert b"aligned" in lib.sge_last_error()
+    # the weights' row stride: at least d_model, a multiple of 8
+    for ldw in (32, 60, 68):
+        assert lib.twell_fused_up_down(p, p, p, p, p, p, ldw, p, 1000, 64, 256, sge.SGE_BF16, 128,
+                                       128, ctypes.c_void_p(4096), ws, None, None) == 1
+        assert b"ldw" in lib.sge_last_error()
     assert lib.dense_ffn_fwd(None, None, None, None, None, None, 8, 64, 100, None, None) == 1
+
+
+def test_interleave_rejects_bad_arguments(lib):
+    p = ctypes.c_void_p(4096)
+    assert lib.sge_interleave_up_down(None, None, None, 0, 64, sge.SGE_BF16, None) == 0  # F = 0
+    assert lib.sge_interleave_up_down(None, p, p, 8, 64, sge.SGE_BF16, None) == 1
+    assert b"null" in lib.sge_last_error()
+    assert lib.sge_interleave_up_down(p, p, p, 8, 0, sge.SGE_BF16, None) == 1
+    assert lib.sge_interleave_up_down(p, p, p, 8, 64, 7, None) == 2
+    # the output may not overlap an input
+    assert lib.sge_interleave_up_down(ctypes.c_void_p(4096), ctypes.c_void_p(1 << 20),
+                                      ctypes.c_void_p(4096 + 512), 8, 64, sge.SGE_BF16, None) == 1
+    assert b"overlaps" in lib.sge_last_error()
 
 
 def test_binding_refuses_cpu_tensors():

@@ -110,6 +110,53 @@ def test_fused_up_down_matches_oracle(cuda_device, dtype, tol, n, d, f, tile, ca
     assert err <= tol, err
 
 
+@pytest.mark.parametrize("dtype,tol", [(torch.bfloat16, BF16_TOL), (torch.float32, F32_TOL)])
+@pytest.mark.parametrize("n,d,f", [
+    (300, 1024, 2048),            # rows of 512-byte multiples: one copy per entry when interleaved
+    (300, 264, 640),              # ragged rows: two copies per entry in every layout
+    (40, 512, 1024),              # the small-batch kernel
+])
+def test_fused_weight_layouts(cuda_device, dtype, tol, n, d, f):
+    """W_up^T and W_down as separate matrices, interleaved row by row (one
+    [F][2d] matrix), and with padded rows give the same bits, and match the
+    oracle."""
+    inp = synth.make_inputs(synth.CONFIGS["ffn_0p5b_bf16"].with_(
+        n_tokens=n, d_model=d, d_ff=f, dtype="bf16" if dtype == torch.bfloat16 else "f32",
+        rho=0.05))
+    _, wgf, wuf, wdf = _f64(inp)
+    x, _, wu, wd = _dev(inp, cuda_device)
+    if n > 64:
+        x[:3, :-1] *= 6.0          # heavy tokens: split units in the large-batch kernel
+    xf = to_f64(x)
+    ora_tw = oracle.twell_pack(oracle.gate_preact(xf, wgf), 128, 32, KIND[dtype])
+    tw = _upload_twell(ora_tw, dtype, cuda_device)
+    y_sep = sge.twell_fused_up_down(x, tw, wu, wd)
+    w_ud, wu_i, wd_i = sge.interleave_up_down(wu, wd)
+    assert torch.equal(w_ud[:, :d], wu) and torch.equal(w_ud[:, d:], wd)
+    y_int = sge.twell_fused_up_down(x, tw, wu_i, wd_i)
+    pad = torch.zeros((f, d + 40), dtype=dtype, device=cuda_device)
+    pad2 = torch.zeros((f, d + 40), dtype=dtype, device=cuda_device)
+    pad[:, :d] = wu
+    pad2[:, :d] = wd
+    y_pad = sge.twell_fused_up_down(x, tw, pad[:, :d], pad2[:, :d])
+    torch.cuda.synchronize()
+    assert torch.equal(y_sep, y_int)
+    assert torch.equal(y_sep, y_pad)
+    want = oracle.fused_up_down(xf, ora_tw, wuf, wdf)
+    err = oracle.max_abs_rel(to_f64(y_int), want)
+    assert err <= tol, err
+
+
+def test_fused_rejects_mismatched_weight_strides(cuda_device):
+    x = torch.zeros(4, 64, dtype=torch.bfloat16, device=cuda_device)
+    w = torch.zeros(128, 64, dtype=torch.bfloat16, device=cuda_device)
+    w2 = torch.zeros(128, 72, dtype=torch.bfloat16, device=cuda_device)
+    tw = sge.TwELL.empty(4, 128, 128, 128, torch.bfloat16, cuda_device)
+    tw.count.zero_()
+    with pytest.raises(ValueError, match="row stride"):
+        sge.twell_fused_up_down(x, tw, w, w2[:, :64])
+
+
 @pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 4104), (torch.float32, 2056)])
 def test_fused_d_limit(cuda_device, dtype, d):
     """A warp keeps at most 16 sixteen-byte pieces of a row per lane: rows of

@@ -26,7 +26,7 @@ def _noalloc_fn():
     fn = lib.twell_fused_up_down_noalloc
     P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
     fn.restype = I
-    fn.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I, I, I, P, P]
+    fn.argtypes = [P, P, P, P, P, P, I64, P, I64, I64, I64, I, I, I, P, P]
     lib.twell_fused_up_down_noalloc_max_tokens.restype = I64
     return lib, fn
 
@@ -49,7 +49,7 @@ def test_noalloc_matches_workspace_entry_point(cuda_device):
     want = y_ref.double().cpu().numpy()
     for call in range(2):           # the second call reuses the array's old contents
         y = torch.full_like(x, float("nan"))
-        rc = fn(_ptr(x), _ptr(tw.count), _ptr(tw.idx), _ptr(tw.val), _ptr(wu), _ptr(wd), _ptr(y),
+        rc = fn(_ptr(x), _ptr(tw.count), _ptr(tw.idx), _ptr(tw.val), _ptr(wu), _ptr(wd), d, _ptr(y),
                 n, d, f, sge.SGE_BF16, tw.tile, tw.cap, None, stream)
         assert rc == 0, lib.sge_last_error()
         torch.cuda.synchronize()
@@ -63,7 +63,7 @@ def test_noalloc_rejects_more_tokens_than_its_scratch_holds(cuda_device):
     limit = lib.twell_fused_up_down_noalloc_max_tokens()
     assert limit >= 8192
     p = ctypes.c_void_p(16)
-    rc = fn(p, p, p, p, p, p, p, limit + 1, 64, 256, sge.SGE_BF16, 128, 128, None, None)
+    rc = fn(p, p, p, p, p, p, 64, p, limit + 1, 64, 256, sge.SGE_BF16, 128, 128, None, None)
     assert rc == 2
     assert b"scratch limit" in lib.sge_last_error()
 
@@ -80,7 +80,7 @@ def test_noalloc_small_batch_full_density(cuda_device):
     tw = sge.twell_gate_pack(x, wg, 128, 128)
     stream = ctypes.c_void_p(torch.cuda.current_stream(cuda_device).cuda_stream)
     y = torch.full_like(x, float("nan"))
-    rc = fn(_ptr(x), _ptr(tw.count), _ptr(tw.idx), _ptr(tw.val), _ptr(wu), _ptr(wd), _ptr(y),
+    rc = fn(_ptr(x), _ptr(tw.count), _ptr(tw.idx), _ptr(tw.val), _ptr(wu), _ptr(wd), d, _ptr(y),
             n, d, f, sge.SGE_BF16, tw.tile, tw.cap, None, stream)
     assert rc == 0, lib.sge_last_error()
     torch.cuda.synchronize()
