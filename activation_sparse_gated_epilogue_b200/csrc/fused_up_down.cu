@@ -35,12 +35,13 @@
 // per lane, one load of idx and of val) one chunk ahead of consumption, so
 // its copies run ahead across chunk and job boundaries.
 //
-// Jobs.  Three small kernels plan the work: stored entries per token; the unit
-// length U (a multiple of 32: heavy tokens split into units of about a
+// Jobs.  Two small kernels plan the work: stored entries per token; then the
+// unit length U (a multiple of 32: heavy tokens split into units of about a
 // quarter of a team's average share, whose fp32 partial outputs fit the
-// pool); the job lists: units of heavy tokens first, then the other
+// pool) and the job lists: units of heavy tokens first, then the other
 // non-empty tokens in four classes of decreasing size, so that the last jobs
-// are short; empty tokens get y = 0 there.  The team leader pulls jobs from a
+// are short.  The main kernel's warps first store y = 0 for the empty tokens
+// of an equal share of the batch each.  The team leader pulls jobs from a
 // global cursor and queues them two jobs ahead.  A unit stores its fp32
 // partial in the pool; the team that completes a split token's last unit (a
 // counter per token) sums the units' partials in unit order and stores y.  No
@@ -169,13 +170,18 @@ struct UdParams {
 
 // ------------------------------------------------------------- planning
 
-// Stored entries of every token (counts capped at C) and per-block sums.
+// Stored entries of every token (counts capped at C) and per-block sums;
+// block 0 also zeroes the job counters that the job-list kernel fills.
 __global__ void __launch_bounds__(256) ud_count_kernel(const uint8_t* __restrict__ count,
                                                        int64_t n_rows, int nt, int cap,
                                                        int* __restrict__ ntok,
-                                                       long long* __restrict__ blk_sum) {
+                                                       long long* __restrict__ blk_sum, int* hdr) {
   __shared__ long long wsum[8];
   const int64_t t = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  if (blockIdx.x == 0 && threadIdx.x < 16) {
+    const int w = threadIdx.x;
+    if (w >= kHUnits && w <= kHOverflow) hdr[w] = 0;
+  }
   int s = 0;
   if (t < n_rows) {
     const uint8_t* c = count + t * nt;
@@ -203,11 +209,13 @@ __global__ void __launch_bounds__(256) ud_count_kernel(const uint8_t* __restrict
   }
 }
 
-// Total entries, the unit length and zeroed job counters (one CTA).
-__global__ void __launch_bounds__(1024) ud_plan_kernel(const long long* __restrict__ blk_sum,
-                                                       int64_t nblk, int64_t pool_slots,
-                                                       int64_t n_teams, int* hdr) {
-  __shared__ long long wsum[32];
+// Total entries (summed from the per-block sums by the calling CTA; every
+// CTA gets the same value) and the unit length U.  All threads must call it.
+__device__ int plan_unit(const long long* __restrict__ blk_sum, int64_t nblk, int64_t pool_slots,
+                         int64_t n_teams, long long* total) {
+  __shared__ long long wsum[8];
+  __shared__ int u_sh;
+  __shared__ long long tot_sh;
   long long s = 0;
   for (int64_t b = threadIdx.x; b < nblk; b += blockDim.x) s += blk_sum[b];
 #pragma unroll
@@ -227,14 +235,12 @@ __global__ void __launch_bounds__(1024) ud_plan_kernel(const long long* __restri
     if (u < kUnitMin) u = kUnitMin;
     u = (u + kChunk - 1) / kChunk * kChunk;
     if (u > (1LL << 30)) u = 1LL << 30;
-    *reinterpret_cast<long long*>(hdr + kHTotal) = tot;
-    hdr[kHUnit] = static_cast<int>(u);
-    hdr[kHUnits] = 0;
-    for (int c = 0; c < kLightClasses; ++c) hdr[kHLight + c] = 0;
-    hdr[kHSplit] = 0;
-    hdr[kHCursor] = 0;
-    hdr[kHOverflow] = 0;
+    u_sh = static_cast<int>(u);
+    tot_sh = tot;
   }
+  __syncthreads();
+  *total = tot_sh;
+  return u_sh;
 }
 
 // Size class of an unsplit token of n entries (0: largest).
@@ -243,17 +249,25 @@ __device__ __forceinline__ int light_class(int n, int U) {
 }
 
 // Job lists: every split token's units, every other non-empty token in its
-// size class.  Slots in the lists come from
+// size class.  Each CTA first derives the unit length from the count
+// kernel's per-block sums (CTA 0 records it).  Slots in the lists come from
 // warp-aggregated atomics: the job order may vary between calls, the results
 // do not.
 __global__ void __launch_bounds__(256) ud_jobs_kernel(const int* __restrict__ ntok, int64_t n_rows,
+                                                      const long long* __restrict__ blk_sum,
+                                                      int64_t nblk, int64_t n_teams,
                                                       int* hdr, int2* __restrict__ lights,
                                                       Job* __restrict__ units, int* __restrict__ done,
                                                       int64_t pool_slots) {
   const int lane = threadIdx.x & 31;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   const unsigned lt = (1u << lane) - 1u;
-  const int U = *reinterpret_cast<volatile int*>(hdr + kHUnit);
+  long long total = 0;
+  const int U = plan_unit(blk_sum, nblk, pool_slots, n_teams, &total);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *reinterpret_cast<long long*>(hdr + kHTotal) = total;
+    hdr[kHUnit] = U;
+  }
   const int n = t < n_rows ? ntok[t] : -1;
   const bool split = n > U;
   // split tokens: ceil(n / U) units each
@@ -305,16 +319,6 @@ __global__ void __launch_bounds__(256) ud_jobs_kernel(const int* __restrict__ nt
     lbase = __shfl_sync(0xffffffffu, lbase, 0);
     if (cls == c) lights[c * n_rows + lbase + __popc(ml & lt)] = make_int2(static_cast<int>(t), n);
   }
-}
-
-// y = 0 for tokens without stored entries: a thread per 16 bytes of y
-// (grid-stride).
-__global__ void __launch_bounds__(256) ud_zero_kernel(const int* __restrict__ ntok, int64_t n_rows,
-                                                      int nvec, void* y) {
-  const int64_t total = n_rows * nvec;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * 256)
-    if (ntok[i / nvec] == 0) reinterpret_cast<uint4*>(y)[i] = make_uint4(0, 0, 0, 0);
 }
 
 // -------------------------------------------------------------- main kernel
@@ -412,6 +416,23 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
   fence_mbar_init();
   __syncthreads();
 
+  // y = 0 for tokens without stored entries: each warp takes an equal share
+  // of the tokens; its stores drain while it starts its first job
+  {
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * warps + warp;
+    const int64_t ngw = static_cast<int64_t>(gridDim.x) * warps;
+    const int64_t per = (p.n_rows + ngw - 1) / ngw;
+    const int64_t t0 = gw * per, t1 = min(p.n_rows, t0 + per);
+    for (int64_t tb = t0; tb < t1; tb += 32) {
+      unsigned m = __ballot_sync(0xffffffffu, tb + lane < t1 && p.ntok[tb + lane] == 0);
+      while (m) {
+        const int i = __ffs(m) - 1;
+        m &= m - 1;
+        uint4* row = reinterpret_cast<uint4*>(static_cast<char*>(p.y) + (tb + i) * p.row_bytes);
+        for (int pc = lane; pc < pieces; pc += 32) row[pc] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
   const int n_units = *reinterpret_cast<volatile int*>(p.hdr + kHUnits);
   int n_light[kLightClasses];
 #pragma unroll
@@ -1255,23 +1276,13 @@ static int run_fused(const char* name, const void* x, const uint8_t* count, cons
   if (grid > kMaxCtas) grid = kMaxCtas;
   const int64_t nblk = (n_tokens + 255) / 256;
   ud_count_kernel<<<static_cast<unsigned>(nblk), 256, 0, st>>>(count, n_tokens, prm.nt, cap,
-                                                               const_cast<int*>(prm.ntok), blk);
+                                                               const_cast<int*>(prm.ntok), blk, prm.hdr);
   int rc = check_launch("twell_fused_up_down (count)");
   if (rc) return rc;
-  ud_plan_kernel<<<1, 1024, 0, st>>>(blk, nblk, pool_slots, grid * prm.teams, prm.hdr);
-  rc = check_launch("twell_fused_up_down (plan)");
-  if (rc) return rc;
   ud_jobs_kernel<<<static_cast<unsigned>(nblk), 256, 0, st>>>(
-      prm.ntok, n_tokens, prm.hdr, const_cast<int2*>(prm.lights), const_cast<Job*>(prm.units),
-      prm.done, pool_slots);
+      prm.ntok, n_tokens, blk, nblk, grid * prm.teams, prm.hdr, const_cast<int2*>(prm.lights),
+      const_cast<Job*>(prm.units), prm.done, pool_slots);
   rc = check_launch("twell_fused_up_down (jobs)");
-  if (rc) return rc;
-  const int64_t nvec = prm.row_bytes / 16;
-  int64_t zblocks = (n_tokens * nvec + 255) / 256;
-  if (zblocks > 32 * 1024) zblocks = 32 * 1024;
-  ud_zero_kernel<<<static_cast<unsigned>(zblocks), 256, 0, st>>>(
-      prm.ntok, n_tokens, static_cast<int>(nvec), y);
-  rc = check_launch("twell_fused_up_down (zero rows)");
   if (rc) return rc;
   return dtype == SGE_BF16 ? dispatch_main<true>(prm, nv, smem, static_cast<int>(grid), st)
                            : dispatch_main<false>(prm, nv, smem, static_cast<int>(grid), st);

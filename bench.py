@@ -377,8 +377,8 @@ def run_own(args, rank, world, local_rank):
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
                 "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
-        "gpu_launches": 6 * args.steps,
-        "launches_note": "per step: gate GEMM + TwELL epilogue; fused up/down = count, plan, jobs, zero rows, main kernel",
+        "gpu_launches": 4 * args.steps,
+        "launches_note": "per step: gate GEMM + TwELL epilogue; fused up/down = count, jobs, main kernel",
         "hybrid_inference": hyb,
         "clocks": clocks,
         "diag": diag_host,
