@@ -536,10 +536,14 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
   };
   if (rj.t >= 0) load_prefix(rj.t);
   // A chunk: token (-1: none), own entries in it (may be 0 when the job has
-  // fewer entries than the team has warps), flags, job sequence number; per
-  // lane the column j and the activation a (fp32 bits) of entry `lane`.
+  // fewer entries than the team has warps), flags (bits 0..2) and the job
+  // sequence number (the bits above); per
+  // lane, for entry `lane`, the first column of its tile, its index in the
+  // tile and its activation as loaded (raw bits).  The raw loads are first
+  // used a chunk later, so their latency hides behind the current chunk.
   struct Chunk {
-    int t, n, flags, k, j, a;
+    int t, n, flags, jb, ji;
+    uint32_t a;
   };
   auto resolve = [&](Chunk& c) {
     c.t = -1;
@@ -557,10 +561,9 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
     }
     const int own = own_count(rj.n);
     c.t = rj.t;
-    c.k = rk;
     c.n = max(0, min(kChunk, own - rci * kChunk));
     c.flags = (rci == 0 ? kFirst : 0) | ((rci + 1) * kChunk >= own ? kLast : 0) |
-              (rci == 0 && own > 0 ? kHasX : 0);
+              (rci == 0 && own > 0 ? kHasX : 0) | (rk << 3);
     const int e = rj.e0 + w + kTeam * (rci * kChunk + lane);
     int b = 0;
 #pragma unroll
@@ -570,12 +573,13 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
       if (cand < p.nt && v <= e) b = cand;
     }
     const int s = e - prefix_at<NTR>(pre, b);
-    c.j = 0;
+    c.jb = b * p.tile;
+    c.ji = 0;
     c.a = 0;
     if (lane < c.n) {
       const int64_t at = (static_cast<int64_t>(c.t) * p.nt + b) * p.cap + s;
-      c.j = min(b * p.tile + __ldg(p.idx + at), p.nt * p.tile - 1);  // in bounds even if idx >= T
-      c.a = __float_as_int(E::load_val(p.val, at));
+      c.ji = __ldg(p.idx + at);
+      c.a = E::load_raw(p.val, at);
     }
     ++rci;
   };
@@ -612,13 +616,15 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
       const int m = min(room, len - iq);
       const int hx = (c.flags & kHasX) ? 1 : 0;
       const int q = iq + lane;
-      const int jv = __shfl_sync(0xffffffffu, c.j, (q - hx) & 31);
+      // the column, kept in bounds even if a stored index is >= T
+      const int jv = min(__shfl_sync(0xffffffffu, c.jb + c.ji, (q - hx) & 31), p.nt * p.tile - 1);
       if (lane < m) {
         int slot = is + lane;
         if (slot >= S) slot -= S;
         uint8_t* dst = ring + slot * p.slot_bytes;
         const uint32_t rb32 = static_cast<uint32_t>(p.row_bytes);
-        fence_proxy_async_smem();
+        // a W row slot's earlier contents were consumed by FMAs that have
+        // issued, so its reads are complete; an x slot is fenced when read
         if (hx && q == 0) {
           mbar_arrive_expect_tx(full + slot, rb32);
           bulk_load(dst, xb + static_cast<int64_t>(c.t) * rb, rb32, full + slot);
@@ -677,13 +683,16 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
       if (!(ok = acquire(a))) break;
 #pragma unroll
       for (int k = 0; k < NV; ++k) xr[k] = piece(a, k);
+      // x stays unused for a while: order these reads before the slot's
+      // next copy
+      fence_proxy_async_smem();
       release();
       pump();
     }
     // each entry: u = x . W_up[:, j] reduced over the lanes, h = a * u
     // rounded as the down projection uses it, y += h * W_down[j]
     for (int e = 0; e < cur.n; ++e) {
-      const float ae = __int_as_float(__shfl_sync(0xffffffffu, cur.a, e & 31));
+      const float ae = E::from_raw(__shfl_sync(0xffffffffu, cur.a, e & 31));
       uint32_t a;
       if (!(ok = acquire(a))) break;
       // eight independent accumulator chains
@@ -701,13 +710,14 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
     }
     if (!ok) break;
     if (cur.flags & kLast) {
+      const int ck = cur.flags >> 3;  // the job's sequence number
       // ---- job done: the warps add their partial rows into the team's row
       // buffer one after the other (warp order), each waiting only for its
       // predecessor; the last one stores the sum.  Warp 0 queues the job
       // after next before it hands the buffer on.
       uint64_t* wait_bar = w == 0 ? tfree : chain + (w - 1);
-      const uint32_t wait_par = w == 0 ? ((cur.k - 1) & 1) : (cur.k & 1);
-      if ((w > 0 || cur.k > 0) && !(ok = wait_or_abort(wait_bar, wait_par, abort_flag, p.diag))) break;
+      const uint32_t wait_par = w == 0 ? ((ck - 1) & 1) : (ck & 1);
+      if ((w > 0 || ck > 0) && !(ok = wait_or_abort(wait_bar, wait_par, abort_flag, p.diag))) break;
 #pragma unroll
       for (int k = 0; k < NV; ++k) {
         const int pc = lane + 32 * k;
@@ -735,7 +745,7 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
         }
       }
       if (w < kTeam - 1) {
-        if (leader && lane == 0) publish_job((cur.k + 2) & 3);
+        if (leader && lane == 0) publish_job((ck + 2) & 3);
         __syncwarp();
         if (lane == 0) mbar_arrive(chain + w);
         if (leader && lane == 0) prefetch_job();
@@ -743,7 +753,7 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
       if (w == kTeam - 1) {
         __syncwarp();
         if (lane == 0) mbar_arrive(tfree);  // the buffer has been read
-        const Job jb = jobq[cur.k & 3];
+        const Job jb = jobq[ck & 3];
         char* yrow = static_cast<char*>(p.y) + static_cast<int64_t>(jb.t) * rb;
         if (jb.nu <= 1) {
 #pragma unroll

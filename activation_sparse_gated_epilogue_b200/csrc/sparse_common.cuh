@@ -62,6 +62,11 @@ struct Elem<true> {
   __device__ __forceinline__ static float load_val(const void* p, int64_t i) {
     return __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(p)[i]) << 16);
   }
+  // the stored bits of value i, and the value they encode
+  __device__ __forceinline__ static uint32_t load_raw(const void* p, int64_t i) {
+    return static_cast<const uint16_t*>(p)[i];
+  }
+  __device__ __forceinline__ static float from_raw(uint32_t r) { return __uint_as_float(r << 16); }
   __device__ __forceinline__ static uint4 pack(const float (&o)[8]) {
     uint32_t w[4];
 #pragma unroll
@@ -101,6 +106,10 @@ struct Elem<false> {
   __device__ __forceinline__ static float load_val(const void* p, int64_t i) {
     return static_cast<const float*>(p)[i];
   }
+  __device__ __forceinline__ static uint32_t load_raw(const void* p, int64_t i) {
+    return static_cast<const uint32_t*>(p)[i];
+  }
+  __device__ __forceinline__ static float from_raw(uint32_t r) { return __uint_as_float(r); }
   __device__ __forceinline__ static uint4 pack(const float (&o)[4]) {
     return make_uint4(__float_as_uint(o[0]), __float_as_uint(o[1]), __float_as_uint(o[2]),
                       __float_as_uint(o[3]));
