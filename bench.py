@@ -47,7 +47,7 @@ HYB_INFER_K = 64
 # a kernel whose source changed since gets null.
 TRAFFIC = {
     "2eebdb20775a495c": 80.1e6,   # gate GEMM + TwELL, profiles/gate_gemm_twell_ffn_1b_bf16.md
-    "6033b28ca36d3085": 341.5e6,  # fused up/down main kernel, profiles/fused_up_down_ffn_1b_bf16.md
+    "a6110f8ae25a3be5": 365.8e6,  # fused up/down main kernel, profiles/fused_up_down_ffn_1b_bf16.md
 }
 
 
