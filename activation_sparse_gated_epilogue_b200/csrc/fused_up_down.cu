@@ -829,7 +829,7 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
 // ---------------------------------------------------------- small batches
 //
 // With few tokens (decode-sized batches) the persistent kernel's per-warp row
-// streams are short and its latency chain (five launches, the job queue, a
+// streams are short and its latency chain (three launches, the job queue, a
 // ring a few rows deep) dominates.  The small-batch path splits every token
 // into units of E entries (E = 8, doubled until the split tokens' partial
 // outputs fit the pool), gives each unit one CTA of kSmWarps warps and each
