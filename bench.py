@@ -338,7 +338,7 @@ def run_own(args, rank, world, local_rank):
               "ms": round(mg, 4), "share": round(mg / (mg + mf), 3),
               "algorithmic": f"2*N*d*F = {flops_gate:.3e} flop per launch",
               "peak_note": "bf16_tflops (burst) of measured peaks: the step keeps SM clocks at max"}
-    k_fused = {"kernel": "twell_fused_up_down (3 planning kernels + persistent main kernel)", "bound": "alu", "achieved": round(fused_tf, 2),
+    k_fused = {"kernel": "twell_fused_up_down (planning kernels + main kernel)", "bound": "alu", "achieved": round(fused_tf, 2),
                "peak": round(FP32_SIMT_TFLOPS, 1), "unit": "TFLOP/s",
                "frac": round(fused_tf / FP32_SIMT_TFLOPS, 4), "traffic": tr_fused,
                "ms": round(mf, 4), "share": round(mf / (mg + mf), 3),
