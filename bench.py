@@ -57,6 +57,8 @@ def parse():
     p.add_argument("--steps", type=int, default=300)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--workload", default="ffn_1b_bf16")
+    p.add_argument("--tokens", type=int, default=0,
+                   help="override the workload's token count (e.g. 1..64 for decode-shaped batches)")
     p.add_argument("--impl", default="own", choices=["own", "reference"])
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--sweep", action="store_true",
@@ -168,13 +170,20 @@ def replica_tokens_per_s(n_tokens: int, world: int, steps: int, max_ms: float) -
     return n_tokens * world * steps / (max_ms / 1e3)
 
 
+def workload_config(args):
+    """The workload's configuration, with --tokens applied."""
+    from activation_sparse_gated_epilogue_b200 import synth
+    cfg = synth.CONFIGS[args.workload]
+    return cfg.with_(n_tokens=args.tokens) if args.tokens > 0 else cfg
+
+
 def run_own(args, rank, world, local_rank):
     import activation_sparse_gated_epilogue_b200 as sge
     from activation_sparse_gated_epilogue_b200 import synth
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    cfg = synth.CONFIGS[args.workload]
+    cfg = workload_config(args)
     inp = synth.make_inputs(cfg)
     n, d, f, tile, cap = cfg.n_tokens, cfg.d_model, cfg.d_ff, cfg.tile, cfg.cap
     x, wg, wu, wd = (getattr(inp, k).to(dev) for k in ("x", "wg_t", "wu_t", "wd"))
@@ -680,7 +689,7 @@ def run_reference(args):
     """The oracle as the reference arm: each step is a bounded token sample."""
     import oracle
     from activation_sparse_gated_epilogue_b200 import synth
-    cfg = synth.CONFIGS[args.workload]
+    cfg = workload_config(args)
     inp = synth.make_inputs(cfg)
     xf, wgf, wuf, wdf = (inp.as_f64(k) for k in ("x", "wg_t", "wu_t", "wd"))
     oracle.build()
@@ -744,8 +753,7 @@ def main():
         return
     out = run_own(args, rank, world, local_rank)
     if rank == 0 and out is not None:
-        from activation_sparse_gated_epilogue_b200 import synth
-        out["cpu_baseline"] = None if args.no_cpu else cpu_baseline(synth.CONFIGS[args.workload])
+        out["cpu_baseline"] = None if args.no_cpu else cpu_baseline(workload_config(args))
         print(json.dumps(out), flush=True)
     if world > 1:
         torch.distributed.barrier()

@@ -312,8 +312,10 @@ def test_full_density_equals_dense(cuda_device):
 
 # --------------------------------------------------------------- end to end
 
-def _e2e_check(inp, dev, tile, cap, tol, rows=None):
+def _e2e_check(inp, dev, tile, cap, tol, rows=None, interleave=False):
     x, wg, wu, wd = _dev(inp, dev)
+    if interleave:                 # the bench's weight layout
+        _, wu, wd = sge.interleave_up_down(wu, wd)
     diag = sge.new_diag(dev)
     y, tw = sge.twell_ffn_forward(x, wg, wu, wd, tile, cap, diag=diag)
     torch.cuda.synchronize()
@@ -351,15 +353,18 @@ def test_e2e_0p5b_bf16(cuda_device):
     print(f"0.5B bf16: max-abs-rel {err:.2e}, {flips} flips")
 
 
+@pytest.mark.parametrize("interleave", [True, False])
 @pytest.mark.parametrize("name", ["ffn_1b_bf16", "ffn_2b_bf16"])
-def test_e2e_full_size_sampled_rows(cuda_device, name):
-    """Full-size workload in the bench's launch configuration; the oracle
-    checks a sample of rows (first, last, and a strided set)."""
+def test_e2e_full_size_sampled_rows(cuda_device, name, interleave):
+    """Full-size workload in the bench's launch configuration (interleaved
+    weights; separate ones too); the oracle checks a sample of rows (first,
+    last, and a strided set)."""
     cfg = synth.CONFIGS[name]
     inp = synth.make_inputs(cfg)
     n = cfg.n_tokens
     rows = np.unique(np.concatenate([[0, 1, n - 1], np.arange(5, n, n // 24)]))
-    err, flips, _ = _e2e_check(inp, cuda_device, cfg.tile, cfg.cap, BF16_TOL, rows=rows)
+    err, flips, _ = _e2e_check(inp, cuda_device, cfg.tile, cfg.cap, BF16_TOL, rows=rows,
+                               interleave=interleave)
     print(f"{name}: max-abs-rel {err:.2e} on {len(rows)} rows, {flips} flips")
 
 
