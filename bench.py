@@ -68,6 +68,8 @@ def parse():
                         "and the hybrid path that recomputes overflowing rows: one JSON line per C")
     p.add_argument("--profile", action="store_true",
                    help="run only warmup + steps of the sparse step (for ncu captures); no JSON")
+    p.add_argument("--profile-hybrid", action="store_true",
+                   help="with --profile: the hybrid inference step (gate, hybrid_pack, hybrid_ffn_fwd) instead")
     return p.parse_args()
 
 
@@ -226,8 +228,22 @@ def run_own(args, rank, world, local_rank):
     fused = lambda: sge.twell_fused_up_down(x, tw, wu_i, wd_i, y=y, workspace=ws)
     dense = lambda: sge.dense_ffn_fwd(x, wg, wu, wd_t, h=h, y=y_dense)
 
+    def hybrid_setup():
+        hk, hs = HYB_INFER_K, max(128, (n // 4 + 127) // 128 * 128)
+        hy = sge.Hybrid.empty(n, f, hk, hs, dev)
+        hws = sge.hybrid_fwd_workspace(d, f, hs, dev)
+        y_h = torch.empty_like(x)
+        hdiag = sge.new_diag(dev)
+        hpack = lambda: sge.hybrid_pack(tw, hk, hs, out=hy, diag=hdiag)
+        hfwd = lambda: sge.hybrid_ffn_fwd(x, hy, wu, wd, wd_t=wd_t, y=y_h, workspace=hws)
+        return hk, hs, hy, y_h, hdiag, hpack, hfwd
+
     if args.profile:
-        timed([gate, fused], args.steps, args.warmup)
+        if args.profile_hybrid:
+            _, _, _, _, _, hpack, hfwd = hybrid_setup()
+            timed([gate, hpack, hfwd], args.steps, args.warmup)
+        else:
+            timed([gate, fused], args.steps, args.warmup)
         return None
 
     # ---- the sparse forward: timed region
@@ -298,13 +314,7 @@ def run_own(args, rank, world, local_rank):
     # dense spill GEMMs on tensor cores, the others through the ELL kernel
     hyb = None
     if x.dtype == torch.bfloat16:
-        hk, hs = HYB_INFER_K, max(128, (n // 4 + 127) // 128 * 128)
-        hy = sge.Hybrid.empty(n, f, hk, hs, dev)
-        hws = sge.hybrid_fwd_workspace(d, f, hs, dev)
-        y_h = torch.empty_like(x)
-        hdiag = sge.new_diag(dev)
-        hpack = lambda: sge.hybrid_pack(tw, hk, hs, out=hy, diag=hdiag)
-        hfwd = lambda: sge.hybrid_ffn_fwd(x, hy, wu, wd, wd_t=wd_t, y=y_h, workspace=hws)
+        hk, hs, hy, y_h, hdiag, hpack, hfwd = hybrid_setup()
         hsteps = min(args.steps, 100)
         timed([gate, hpack, hfwd], 0, 3)
         barrier()
