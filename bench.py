@@ -703,8 +703,9 @@ def run_reference(args):
     inp = synth.make_inputs(cfg)
     xf, wgf, wuf, wdf = (inp.as_f64(k) for k in ("x", "wg_t", "wu_t", "wd"))
     oracle.build()
+    kind = oracle.VAL_F32 if cfg.dtype == "f32" else oracle.VAL_BF16
     t0 = time.perf_counter()
-    oracle.sparse_ffn(xf[:4], wgf, wuf, wdf, cfg.tile, cfg.cap, oracle.VAL_BF16)
+    oracle.sparse_ffn(xf[:4], wgf, wuf, wdf, cfg.tile, cfg.cap, kind)
     per_tok = (time.perf_counter() - t0) / 4
     budget = 150.0 / max(1, args.steps + args.warmup)
     k = int(max(1, min(cfg.n_tokens, budget / max(per_tok, 1e-6))))
@@ -712,7 +713,7 @@ def run_reference(args):
     for s in range(args.warmup + args.steps):
         off = (s * k) % max(1, cfg.n_tokens - k)
         t0 = time.perf_counter()
-        oracle.sparse_ffn(xf[off:off + k], wgf, wuf, wdf, cfg.tile, cfg.cap, oracle.VAL_BF16)
+        oracle.sparse_ffn(xf[off:off + k], wgf, wuf, wdf, cfg.tile, cfg.cap, kind)
         if s >= args.warmup:
             times.append(time.perf_counter() - t0)
     total = sum(times)

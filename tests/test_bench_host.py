@@ -1,0 +1,39 @@
+"""Host-side pieces of bench.py that need no GPU: the reference arm (the
+oracle timed on the host cores) keeps the bench's JSON contract, and the
+token-count override reaches the workload configuration."""
+import argparse
+import json
+
+import bench
+
+
+def _args(**kw):
+    base = dict(gpus=1, steps=1, warmup=0, workload="decode_1b_bf16", impl="reference", tokens=2,
+                no_cpu=False, sweep=False, cap_sweep=False, profile=False, profile_hybrid=False)
+    base.update(kw)
+    return argparse.Namespace(**base)
+
+
+def test_tokens_override():
+    assert bench.workload_config(_args(tokens=7)).n_tokens == 7
+    assert bench.workload_config(_args(tokens=0)).n_tokens == 64
+    assert bench.workload_config(_args(workload="ffn_1b_bf16", tokens=0)).n_tokens == 8192
+
+
+def test_reference_arm_json_contract():
+    out = bench.run_reference(_args())
+    json.dumps(out)
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "dtype", "config", "cpu_baseline", "e2e"):
+        assert key in out, key
+    assert out["impl"] == "reference" and out["metric"] == bench.METRIC
+    assert out["value"] > 0 and out["unit"] == "tokens/s" and out["steps"] == 1
+    assert out["config"]["workload"].startswith("decode_1b_bf16: N=2 ")
+    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["cores"] >= 1
+    assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["e2e"]["d2h_bytes_per_step"] == 0
+    assert out["e2e"]["value"] == out["value"]
+
+
+def test_reference_arm_fp32_workload():
+    out = bench.run_reference(_args(workload="tiny_fp32", tokens=4))
+    assert out["value"] > 0 and out["config"]["workload"].startswith("tiny_fp32: N=4 ")
