@@ -185,9 +185,12 @@ def run_own(args, rank, world, local_rank):
     import activation_sparse_gated_epilogue_b200 as sge
     from activation_sparse_gated_epilogue_b200 import synth
 
+    cfg = workload_config(args)
+    if cfg.dtype != "bf16":
+        raise SystemExit(f"bench.py measures the bf16 workloads; {cfg.name} is a parity case "
+                         "(tests/test_gpu_forward.py)")
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    cfg = workload_config(args)
     inp = synth.make_inputs(cfg)
     n, d, f, tile, cap = cfg.n_tokens, cfg.d_model, cfg.d_ff, cfg.tile, cfg.cap
     x, wg, wu, wd = (getattr(inp, k).to(dev) for k in ("x", "wg_t", "wu_t", "wd"))

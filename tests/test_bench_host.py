@@ -37,3 +37,9 @@ def test_reference_arm_json_contract():
 def test_reference_arm_fp32_workload():
     out = bench.run_reference(_args(workload="tiny_fp32", tokens=4))
     assert out["value"] > 0 and out["config"]["workload"].startswith("tiny_fp32: N=4 ")
+
+
+def test_own_arm_refuses_fp32_workloads_before_touching_a_gpu():
+    import pytest
+    with pytest.raises(SystemExit, match="parity case"):
+        bench.run_own(_args(workload="tiny_fp32", impl="own", tokens=0), 0, 1, 0)
