@@ -93,6 +93,8 @@ def test_gate_pack_gaussian_sign_flips(cuda_device, name, cap):
     (129, 1024, 512, 128, 128),
     (77, 520, 768, 32, 6),        # truncated tiles
     (64, 2560, 1024, 128, 128),   # the 2B d_model
+    (200, 4096, 1024, 128, 128),  # the longest rows (8 KB in bf16): 16 pieces per lane
+    (200, 2048, 1024, 128, 128),  # 8 KB rows in fp32
 ])
 def test_fused_up_down_matches_oracle(cuda_device, dtype, tol, n, d, f, tile, cap):
     """Both sides get the same TwELL (the oracle's pack of its fp64 G)."""
