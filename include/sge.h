@@ -18,9 +18,10 @@
  * writing the hidden activation h to memory (section 02, last paragraph).
  *
  * Conventions for every entry point:
- *  - All tensor pointers are DEVICE pointers, row-major and contiguous, owned
- *    by the caller; the library never allocates or frees device memory and
- *    keeps no pointer after the call returns.
+ *  - All tensor pointers are DEVICE pointers, row-major and contiguous (the
+ *    fused call's two weight matrices take a row stride, ldw), owned by the
+ *    caller; the library never allocates or frees device memory and keeps no
+ *    pointer after the call returns.
  *  - Every pointer must be 16-byte aligned; d_model must be a multiple of 8.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
  *    are asynchronous on that stream; outputs are overwritten (beta = 0).
