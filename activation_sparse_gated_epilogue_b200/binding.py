@@ -68,7 +68,6 @@ def library() -> ctypes.CDLL:
             "sge_interleave_up_down": (I, [P, P, P, I64, I64, I, P]),
             "twell_fused_up_down_noalloc_max_tokens": (I64, []),
             "dense_ffn_fwd": (I, [P, P, P, P, P, P, I64, I64, I64, P, P]),
-            "sge_l2_gather_probe": (I, [P, I64, I, P, I64, P, P, P]),
             "hybrid_pack": (I, [P, P, P, I, I, ctypes.POINTER(_SgeHybrid), P, P]),
             "hybrid_ffn_fwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I]),
             "hybrid_ffn_fwd": (I, [P, ctypes.POINTER(_SgeHybrid), P, P, P, P, P, I64, P,
@@ -266,20 +265,6 @@ def dense_ffn_fwd(x: torch.Tensor, wg_t: torch.Tensor, wu_t: torch.Tensor, wd_t:
     return y
 
 
-def l2_gather_probe(table: torch.Tensor, ids: torch.Tensor, sink: torch.Tensor,
-                    diag: Optional[torch.Tensor] = None, stream=None) -> None:
-    """Stream rows ids of table (2-D, contiguous) into shared memory on every
-    SM, the way the fused up/down kernel streams its weight rows (a
-    measurement helper; time it with CUDA events)."""
-    if table.dim() != 2 or not table.is_contiguous():
-        raise ValueError("table must be a contiguous 2-D tensor")
-    if ids.dtype != torch.int32 or not ids.is_contiguous():
-        raise ValueError("ids must be contiguous int32")
-    row_bytes = table.shape[1] * table.element_size()
-    _call("sge_l2_gather_probe", _ptr(table), table.shape[0], row_bytes, _ptr(ids), ids.numel(),
-          _ptr(sink), _ptr(diag), _stream(table.device, stream))
-
-
 @dataclass
 class Hybrid:
     """Device buffers of the hybrid format (see `sge_hybrid` in include/sge.h)."""
@@ -337,21 +322,24 @@ def hybrid_fwd_workspace(d_model: int, d_ff: int, s_max: int, device) -> torch.T
 
 
 def hybrid_ffn_fwd(x: torch.Tensor, hy: Hybrid, wu_t: torch.Tensor, wd: torch.Tensor,
-                   wd_t: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                   wd_t: Optional[torch.Tensor], y: Optional[torch.Tensor] = None,
                    workspace: Optional[torch.Tensor] = None, stream=None,
                    wg_t: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """y from the hybrid form; fills hy.ell_u and hy.spill_u.  With wg_t the
-    spill rows' activations are recomputed from the gate (and written to
-    hy.spill_a), so rows that reached the spill through an overflowing
-    TwELL tile come out exact."""
+    """y from the hybrid form; fills hy.ell_u and hy.spill_u.  ``wd_t`` is
+    W_down transposed, [d][F] (a weight layout the caller builds once; None
+    only when hy.s_max == 0).  With wg_t the spill rows' activations are
+    recomputed from the gate (and written to hy.spill_a), so rows that
+    reached the spill through an overflowing TwELL tile come out exact."""
     _check(x, "x", torch.bfloat16)
     n, d = x.shape
     f = hy.d_ff
     _check(wu_t, "wu_t", torch.bfloat16, (f, d))
     _check(wd, "wd", torch.bfloat16, (f, d))
     if wd_t is None:
-        wd_t = wd.t().contiguous()
-    _check(wd_t, "wd_t", torch.bfloat16, (d, f))
+        if hy.s_max > 0:
+            raise ValueError("wd_t (W_down transposed, [d][F]) is required when s_max > 0")
+    else:
+        _check(wd_t, "wd_t", torch.bfloat16, (d, f))
     if wg_t is not None:
         _check(wg_t, "wg_t", torch.bfloat16, (f, d))
     if y is None:

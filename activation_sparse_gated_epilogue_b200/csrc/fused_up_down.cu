@@ -50,6 +50,8 @@
 // Every wait is bounded: a wait that runs out of time sets SGE_FLAG_TIMEOUT in
 // diag and stops the CTA, after each warp has waited (again bounded) for its
 // own copies in flight.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "sge_host.h"
@@ -1373,23 +1375,49 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
+// Per device: the context the address was looked up in, and the address.  A
+// device reset or a new primary context maps the array afresh, so the
+// address is looked up again whenever the current context differs.
+CUcontext g_scratch_ctx[kMaxDevices] = {nullptr};
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
 
-// Device address of g_fused_scratch on the current device (looked up once).
+CUresult current_context(CUcontext* ctx) {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  });
+  if (!fn) return CUDA_ERROR_NOT_FOUND;
+  return fn(ctx);
+}
+
+// Device address of g_fused_scratch in the current device's current context
+// (looked up once per context).
 int scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "twell_fused_up_down_noalloc: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices)
     return fail(SGE_ERR_UNSUPPORTED, "twell_fused_up_down_noalloc: device %d beyond %d", dev, kMaxDevices);
+  // Before the runtime has set up this thread no context is current; the
+  // symbol lookup then makes the device's primary context current.
+  CUcontext ctx = nullptr;
+  if (current_context(&ctx) != CUDA_SUCCESS) ctx = nullptr;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
+  if (!ctx || !g_scratch_ptr[dev] || g_scratch_ctx[dev] != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_fused_scratch);
     if (e != cudaSuccess || !p)
       return fail(SGE_ERR_CUDA, "twell_fused_up_down_noalloc: cudaGetSymbolAddress: %s",
                   cudaGetErrorString(e));
+    if (current_context(&ctx) != CUDA_SUCCESS || !ctx)
+      return fail(SGE_ERR_CUDA, "twell_fused_up_down_noalloc: no current CUDA context");
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return SGE_OK;
@@ -1413,7 +1441,9 @@ extern "C" int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, 
                 kName, (long long)n_tokens, (long long)kNoAllocMaxTokens);
   int rc = check_args(kName, n_tokens, d_model, d_ff, ldw, tile, cap);
   if (rc) return rc;
-  if (n_tokens == 0) return SGE_OK;
+  void* scratch = nullptr;
+  // a call without tokens only sets up the array's address (start-up)
+  if (n_tokens == 0) return scratch_address(&scratch);
   if (!x || !count || !idx || !val || !wu_t || !wd || !y)
     return fail(SGE_ERR_ARG, "%s: null pointer", kName);
   if (!aligned16(x) || !aligned16(wu_t) || !aligned16(wd) || !aligned16(y) || !aligned16(val))
@@ -1422,7 +1452,6 @@ extern "C" int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, 
   if (slots > kNoAllocPoolSlots) slots = kNoAllocPoolSlots;
   if (WsLayout(n_tokens, d_model, slots).total > kNoAllocScratchBytes)
     return fail(SGE_ERR_UNSUPPORTED, "%s: built-in scratch too small for this shape", kName);
-  void* scratch = nullptr;
   rc = scratch_address(&scratch);
   if (rc) return rc;
   // The array keeps the previous call's contents; the planning kernels reset

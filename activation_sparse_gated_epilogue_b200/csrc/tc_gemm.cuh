@@ -15,7 +15,10 @@
 // by two B matrices at once into two accumulators (gate and up projections
 // of the dense gated FFN share the A tile).
 //
-// No cluster launch and no TMA multicast: every CTA loads its own tiles.
+// No TMA multicast loads anywhere: every CTA loads its own tiles.  The
+// single-CTA engine runs without clusters; the CTA-pair engine below runs in
+// 2-CTA clusters (cta_group::2), each CTA loading its half of the operands
+// into its own shared memory.
 // Every wait is bounded (sge::mbar_wait); a timeout sets SGE_FLAG_TIMEOUT in
 // diag, raises a CTA-wide abort flag, and the CTA drains its in-flight TMA
 // loads and MMAs (bounded) before freeing TMEM and returning.

@@ -42,15 +42,10 @@ FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # stored entries run on the tensor-core spill GEMMs)
 HYB_INFER_K = 64
 
-# DRAM bytes (read + write) per launch from the committed ncu captures
-# (profiles/*.md), keyed by the source hash of the kernel they were taken on;
-# a kernel whose source changed since gets null.
-TRAFFIC = {
-    "2eebdb20775a495c": 80.1e6,   # gate GEMM + TwELL, profiles/gate_gemm_twell_ffn_1b_bf16.md
-    # fused up/down main kernel, profiles/fused_up_down_ffn_1b_bf16.md (the source
-    # changed since the capture only in one comment)
-    "2725061022e5278b": 365.8e6,
-}
+# DRAM bytes (read + write) per launch from ncu captures of the kernels,
+# keyed by the hash of the source they were taken on; a kernel whose source
+# changed since its capture gets null.
+TRAFFIC = {}
 
 
 def parse():
@@ -268,24 +263,6 @@ def run_own(args, rank, world, local_rank):
     nnz = int(tw.count.to(torch.int64).sum().item())
     density = nnz / (n * f)
 
-    # ---- the L2-to-SM row gather ceiling the fused kernel's rows stream
-    # against, measured now with the same copy mechanism (random whole rows of
-    # a 64 MB table, every row read back): see sge_l2_gather_probe
-    probe_table = torch.empty((64 * 1024 * 1024) // (2 * d), d, dtype=torch.bfloat16, device=dev)
-    probe_ids = torch.randint(0, probe_table.shape[0], (1 << 19,), dtype=torch.int32, device=dev)
-    probe_sink = torch.zeros(1, dtype=torch.int32, device=dev)
-    probe_diag = sge.new_diag(dev)
-    for _ in range(3):
-        sge.l2_gather_probe(probe_table, probe_ids, probe_sink, diag=probe_diag)
-    pe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    pe[0].record(stream)
-    for _ in range(5):
-        sge.l2_gather_probe(probe_table, probe_ids, probe_sink, diag=probe_diag)
-    pe[1].record(stream)
-    torch.cuda.synchronize(dev)
-    probe_tbs = 5 * probe_ids.numel() * 2 * d / (pe[0].elapsed_time(pe[1]) / 1e3) / 1e12
-    del probe_table, probe_ids
-
     # ---- dense baselines on the same inputs (own tcgen05 and cuBLAS)
     evd = timed([dense], min(args.steps, 100), 3)
     ms_dense = statistics.mean(e[0].elapsed_time(e[1]) for e in evd)
@@ -369,13 +346,8 @@ def run_own(args, rank, world, local_rank):
                "algorithmic": f"4*nnz*d = {flops_fused:.3e} flop per launch (nnz={nnz})",
                "hbm_gbs_unique": round(bytes_fused / (mf / 1e3) / 1e9, 1),
                "peak_note": "fp32 FMA peak of the CUDA cores, 148 SMs x 128 lanes x 2 x 1.965 GHz",
-               # what the kernel is actually bound by: its weight rows
-               # (4*nnz*d bytes) streamed from L2, against the row-gather rate
-               # measured in this run by sge_l2_gather_probe
-               "l2_row_gather": {"achieved_tbs": round(4.0 * nnz * d / (mf / 1e3) / 1e12, 2),
-                                 "probe_tbs": round(probe_tbs, 2),
-                                 "frac": round(4.0 * nnz * d / (mf / 1e3) / 1e12 / probe_tbs, 4),
-                                 "bytes": int(4 * nnz * d)}}
+               # its weight rows (4*nnz*d bytes) streamed from L2 into the SMs
+               "l2_row_bytes_tbs": round(4.0 * nnz * d / (mf / 1e3) / 1e12, 2)}
     k_gate["traffic_unit"] = k_fused["traffic_unit"] = "bytes per launch (ncu dram read + write)"
     dominant = k_gate if mg >= mf else k_fused
     rest = k_fused if dominant is k_gate else k_gate

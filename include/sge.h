@@ -171,9 +171,14 @@ int twell_fused_up_down(const void* x, const uint8_t* count, const uint8_t* idx,
  * tokens (65536; about 6.6 MB, held on every GPU that loads the library
  * until the process exits).  Larger N is rejected with SGE_ERR_UNSUPPORTED.
  *
- * The first call on a device looks up the array's device address on that
- * device (cudaGetSymbolAddress); make that first call before any stream
- * capture.  Every call shares the one array, so calls that may overlap on
+ * The first call in a device's context looks up the array's device address
+ * there (cudaGetSymbolAddress) and, under CUDA's lazy module loading (the
+ * default), that lookup loads the library's device code, which commits
+ * device memory for the array.  A caller that may not allocate once it is
+ * serving therefore makes one call during start-up, before any stream
+ * capture: a call with n_tokens = 0 does only this set-up (its pointers may
+ * be NULL).  After a device reset, or in a new context, the next call looks
+ * the address up again.  Every call shares the one array, so calls that may overlap on
  * the GPU (different streams, or different host threads on the same device)
  * race and must be serialised by the caller.  Results agree with those of
  * twell_fused_up_down up to fp32 rounding order: the array's smaller pool for
@@ -216,23 +221,6 @@ int sge_interleave_up_down(const void* wu_t, const void* wd, void* w_ud, int64_t
 int dense_ffn_fwd(const void* x, const void* wg_t, const void* wu_t, const void* wd_t, void* h,
                   void* y, int64_t n_tokens, int64_t d_model, int64_t d_ff, int32_t* diag,
                   void* stream);
-
-/*
- * sge_l2_gather_probe -- measurement helper, not part of the FFN: streams the
- * rows ids[0 .. n_ids) of `table` (table_rows rows of row_bytes bytes,
- * row-major, 16-byte aligned) from memory into shared memory the way the
- * fused up/down kernel streams its W_up and W_down rows (bulk copies of whole
- * rows through per-warp rings, every row read back), on every SM.  With a
- * table that fits L2 and random ids, bytes / time is the L2-to-SM row
- * gather rate that bounds twell_fused_up_down.  Asynchronous on `stream`;
- * the caller times it with events.  ids outside [0, table_rows) are clamped.
- *   sink  device uint32[1] the kernel may write (keeps the reads live)
- *   diag  nullable int32[4]; SGE_FLAG_TIMEOUT if a wait gave up
- * Errors: SGE_ERR_ARG for bad sizes, a null or misaligned pointer;
- * SGE_ERR_UNSUPPORTED for rows too long for the rings (> about 100 KB).
- */
-int sge_l2_gather_probe(const void* table, int64_t table_rows, int row_bytes, const int32_t* ids,
-                        int64_t n_ids, uint32_t* sink, int32_t* diag, void* stream);
 
 /*
  * Hybrid format for training ("Sparser, Faster, Lighter Transformer Language

@@ -388,3 +388,18 @@ def test_grid_inputs_are_exact_in_fp32():
     g32 = (inp.x.float() @ inp.wg_t.float().T).double().numpy()
     np.testing.assert_array_equal(g32, g64)
     np.testing.assert_array_equal(oracle.gate_preact(x, w), g64)
+
+
+def test_gate_bias_is_exactly_additive():
+    """The density sweep's harness reuses G0 = G(tau = 0): with x's last
+    feature 1.0 and the bias (-tau) in W_gate's last input row, which the
+    oracle adds last, G(tau) = fl(G0 - tau) holds bit for bit."""
+    cfg = synth.CONFIGS["ffn_2b_bf16"].with_(n_tokens=48, d_model=96, d_ff=256)
+    for rho in (0.0025, 0.05):
+        inp = synth.make_inputs(cfg.with_(rho=rho))
+        x, wg = inp.as_f64("x"), inp.as_f64("wg_t")
+        assert np.all(x[:, -1] == 1.0) and np.all(wg[:, -1] == -inp.tau)
+        wg0 = wg.copy()
+        wg0[:, -1] = 0.0
+        np.testing.assert_array_equal(oracle.gate_preact(x, wg),
+                                      oracle.gate_preact(x, wg0) - inp.tau)

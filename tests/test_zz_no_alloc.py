@@ -35,18 +35,33 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def test_noalloc_matches_workspace_entry_point(cuda_device):
+def _upload_twell(tw: "oracle.TwELL", dev):
+    return sge.TwELL(torch.from_numpy(tw.count).to(dev), torch.from_numpy(tw.idx).to(dev),
+                     torch.from_numpy(tw.val).to(torch.bfloat16).to(dev), tw.tile, tw.cap)
+
+
+def test_noalloc_matches_oracle_and_workspace_entry_point(cuda_device):
+    """Both sides get the oracle's TwELL of the same inputs (a few heavy
+    tokens, so heavy-token units and light tokens both run): two calls in a
+    row of the allocation-free entry point match the oracle's fused up/down
+    and the workspace entry point within the bf16 bar."""
     lib, fn = _noalloc_fn()
     cfg = synth.CONFIGS["ffn_0p5b_bf16"]
     inp = synth.make_inputs(cfg, n_tokens=2048)
-    x, wg, wu, wd = (getattr(inp, k).to(cuda_device) for k in ("x", "wg_t", "wu_t", "wd"))
-    x[:6, :-1] *= 8.0              # a few heavy tokens: both halves of the kernel run
-    tw = sge.twell_gate_pack(x, wg, cfg.tile, cfg.cap)
-    y_ref = sge.twell_fused_up_down(x, tw, wu, wd)
+    inp.x[:6, :-1] *= 8.0          # exact in bf16 (a power of two)
+    xf, wgf, wuf, wdf = (inp.as_f64(k) for k in ("x", "wg_t", "wu_t", "wd"))
+    tw_ora = oracle.twell_pack(oracle.gate_preact(xf, wgf), cfg.tile, cfg.cap, oracle.VAL_BF16)
+    assert tw_ora.count[:6].sum() > 4 * tw_ora.count[6:].sum(1).max()   # the heavy tokens
+    want = oracle.fused_up_down(xf, tw_ora, wuf, wdf)
+    x, wu, wd = (getattr(inp, k).to(cuda_device) for k in ("x", "wu_t", "wd"))
+    tw = _upload_twell(tw_ora, cuda_device)
+    y_ws = sge.twell_fused_up_down(x, tw, wu, wd)
     n, d = x.shape
-    f = wg.shape[0]
+    f = wu.shape[0]
     stream = ctypes.c_void_p(torch.cuda.current_stream(cuda_device).cuda_stream)
-    want = y_ref.double().cpu().numpy()
+    torch.cuda.synchronize()
+    got_ws = y_ws.double().cpu().numpy()
+    assert oracle.max_abs_rel(got_ws, want) <= BF16_TOL
     for call in range(2):           # the second call reuses the array's old contents
         y = torch.full_like(x, float("nan"))
         rc = fn(_ptr(x), _ptr(tw.count), _ptr(tw.idx), _ptr(tw.val), _ptr(wu), _ptr(wd), d, _ptr(y),
@@ -56,6 +71,16 @@ def test_noalloc_matches_workspace_entry_point(cuda_device):
         got = y.double().cpu().numpy()
         assert np.isfinite(got).all()
         assert oracle.max_abs_rel(got, want) <= BF16_TOL, call
+        assert oracle.max_abs_rel(got, got_ws) <= BF16_TOL, call
+
+
+def test_noalloc_zero_tokens_sets_up_only(cuda_device):
+    """A call without tokens performs only the start-up lookup of the
+    array's address; its pointers may be NULL."""
+    lib, fn = _noalloc_fn()
+    torch.cuda.synchronize()
+    rc = fn(None, None, None, None, None, None, 64, None, 0, 64, 256, sge.SGE_BF16, 128, 128, None, None)
+    assert rc == 0, lib.sge_last_error()
 
 
 def test_noalloc_rejects_more_tokens_than_its_scratch_holds(cuda_device):
