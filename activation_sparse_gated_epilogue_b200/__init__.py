@@ -10,12 +10,13 @@ from .binding import (  # noqa: F401
     SGE_BF16, SGE_F32, TwELL, LibraryError, library, library_path,
     twell_gate_pack, twell_fused_up_down, twell_ffn_forward, dense_ffn_fwd, new_diag,
     fused_workspace, Hybrid, hybrid_pack, hybrid_ffn_fwd, hybrid_fwd_workspace,
-    hybrid_ffn_bwd, hybrid_bwd_workspace, interleave_up_down,
+    hybrid_ffn_bwd, hybrid_bwd_workspace, interleave_up_down, twell_hybrid_up_down, routed_workspace,
 )
 
 __all__ = [
     "SGE_BF16", "SGE_F32", "TwELL", "LibraryError", "library", "library_path",
     "twell_gate_pack", "twell_fused_up_down", "twell_ffn_forward", "dense_ffn_fwd", "new_diag",
     "fused_workspace", "Hybrid", "hybrid_pack", "hybrid_ffn_fwd", "hybrid_fwd_workspace",
-    "hybrid_ffn_bwd", "hybrid_bwd_workspace", "interleave_up_down",
+    "hybrid_ffn_bwd", "hybrid_bwd_workspace", "interleave_up_down", "twell_hybrid_up_down",
+    "routed_workspace",
 ]

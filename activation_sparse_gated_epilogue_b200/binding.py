@@ -66,6 +66,9 @@ def library() -> ctypes.CDLL:
             "twell_fused_up_down_noalloc": (I, [P, P, P, P, P, P, I64, P, I64, I64, I64, I, I, I,
                                                 P, P]),
             "sge_interleave_up_down": (I, [P, P, P, I64, I64, I, P]),
+            "twell_hybrid_up_down_workspace_bytes": (ctypes.c_size_t, [I64, I64, I64, I]),
+            "twell_hybrid_up_down": (I, [P, P, P, P, P, P, I64, P, P, I64, I64, I64, I, I, I, I, P,
+                                         ctypes.c_size_t, P, P]),
             "twell_fused_up_down_noalloc_max_tokens": (I64, []),
             "dense_ffn_fwd": (I, [P, P, P, P, P, P, I64, I64, I64, P, P]),
             "hybrid_pack": (I, [P, P, P, I, I, ctypes.POINTER(_SgeHybrid), P, P]),
@@ -230,6 +233,50 @@ def twell_fused_up_down(x: torch.Tensor, tw: TwELL, wu_t: torch.Tensor, wd: torc
         _check(diag, "diag", torch.int32, (4,))
     _call("twell_fused_up_down", _ptr(x), _ptr(tw.count), _ptr(tw.idx), _ptr(tw.val),
           _ptr(wu_t), _ptr(wd), ldw, _ptr(y), n, d, f, _dtype_code(x), tw.tile, tw.cap,
+          _ptr(workspace), workspace.numel(), _ptr(diag), _stream(x.device, stream))
+    return y
+
+
+def routed_workspace(n_tokens: int, d_model: int, d_ff: int, s_max: int, device) -> torch.Tensor:
+    """Scratch for twell_hybrid_up_down (the caching allocator's blocks are
+    512-byte aligned; 256 are needed)."""
+    nbytes = library().twell_hybrid_up_down_workspace_bytes(n_tokens, d_model, d_ff, s_max)
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def twell_hybrid_up_down(x: torch.Tensor, tw: TwELL, wu_t: torch.Tensor, wd: torch.Tensor,
+                         wd_t: Optional[torch.Tensor], ell_cap: int, s_max: int,
+                         y: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                         diag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """y from TwELL with tokens of more than ell_cap stored entries (the first
+    s_max of them) on the tensor-core spill GEMMs and the others through the
+    per-entry fused kernel.  bf16.  ``wd_t`` is W_down transposed, [d][F]
+    (None only when s_max == 0); wu_t and wd may be the row-strided halves of
+    interleave_up_down's matrix."""
+    _check(x, "x", torch.bfloat16)
+    n, d = x.shape
+    f = wu_t.shape[0]
+    ldw = _check_rows(wu_t, "wu_t", x.dtype, (f, d))
+    if _check_rows(wd, "wd", x.dtype, (f, d)) != ldw:
+        raise ValueError("wu_t and wd must have the same row stride")
+    if wd_t is None:
+        if s_max > 0:
+            raise ValueError("wd_t (W_down transposed, [d][F]) is required when s_max > 0")
+    else:
+        _check(wd_t, "wd_t", torch.bfloat16, (d, f))
+    _check(tw.count, "count", torch.uint8, (n, f // tw.tile))
+    _check(tw.idx, "idx", torch.uint8, (n, f // tw.tile, tw.cap))
+    _check(tw.val, "val", x.dtype, (n, f // tw.tile, tw.cap))
+    if y is None:
+        y = torch.empty_like(x)
+    _check(y, "y", x.dtype, (n, d))
+    if workspace is None:
+        workspace = routed_workspace(n, d, f, s_max, x.device)
+    _check(workspace, "workspace", torch.uint8)
+    if diag is not None:
+        _check(diag, "diag", torch.int32, (4,))
+    _call("twell_hybrid_up_down", _ptr(x), _ptr(tw.count), _ptr(tw.idx), _ptr(tw.val), _ptr(wu_t),
+          _ptr(wd), ldw, _ptr(wd_t), _ptr(y), n, d, f, tw.tile, tw.cap, ell_cap, s_max,
           _ptr(workspace), workspace.numel(), _ptr(diag), _stream(x.device, stream))
     return y
 

@@ -65,6 +65,40 @@ int set_smem_limit(const void* kernel, int bytes) {
   return SGE_OK;
 }
 
+int prefer_max_shared(const void* kernel) {
+  struct Entry {
+    int dev;
+    const void* kernel;
+  };
+  static Entry table[64];
+  static int used = 0;
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (table[i].dev == dev && table[i].kernel == kernel) return SGE_OK;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                       cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "cudaFuncSetAttribute(carveout): %s", cudaGetErrorString(e));
+  if (used < 64) table[used++] = Entry{dev, kernel};
+  return SGE_OK;
+}
+
+CUresult current_context(CUcontext* ctx) {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  });
+  if (!fn) return CUDA_ERROR_NOT_FOUND;
+  return fn(ctx);
+}
+
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;

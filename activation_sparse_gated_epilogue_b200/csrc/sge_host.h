@@ -24,8 +24,15 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Multiprocessor count of the current device (cached per device).
 int sm_count();
 
-// Sets the dynamic shared memory limit of a kernel once per process.
+// Sets the dynamic shared memory limit of a kernel once per device.
 int set_smem_limit(const void* kernel, int bytes);
+
+// Asks for the largest shared-memory carveout for a kernel, once per device.
+int prefer_max_shared(const void* kernel);
+
+// The calling thread's current CUDA context (nullptr if none), via the
+// driver entry point; CUDA_SUCCESS or the driver's error.
+CUresult current_context(CUcontext* ctx);
 
 // 2-D bf16 tensor map over a row-major [rows][cols] matrix with row pitch
 // `pitch_elems`, box [box_rows][64] (64 bf16 = one 128-byte swizzle row),

@@ -84,6 +84,36 @@ __device__ __forceinline__ int epi_k_limit(const E& e, int k) {
   return epi_k_limit_impl(e, k, 0);
 }
 
+// Split-K (CTA-pair engine): an epilogue may ask for its K range to be cut
+// into Epi::splits() parts, each an output tile of its own whose partial
+// product the epilogue combines (Epi::run_split); default 1.
+template <class E>
+__device__ __forceinline__ auto epi_splits_impl(const E& e, int) -> decltype(e.splits()) {
+  return e.splits();
+}
+template <class E>
+__device__ __forceinline__ int epi_splits_impl(const E&, long) {
+  return 1;
+}
+template <class E>
+__device__ __forceinline__ int epi_splits(const E& e) {
+  return epi_splits_impl(e, 0);
+}
+
+// The epilogue call of one output tile: run_split (given the split and the
+// number of splits) for epilogues that have it, run otherwise.
+template <int BN, class E>
+__device__ __forceinline__ auto epi_run_impl(const E& e, uint32_t taddr, int64_t row, int n_blk, int split,
+                                             int nsplit, int lane, int)
+    -> decltype(e.template run_split<BN>(taddr, row, n_blk, split, nsplit, lane)) {
+  return e.template run_split<BN>(taddr, row, n_blk, split, nsplit, lane);
+}
+template <int BN, class E>
+__device__ __forceinline__ void epi_run_impl(const E& e, uint32_t taddr, int64_t row, int n_blk, int, int,
+                                             int lane, long) {
+  e.template run<BN>(taddr, row, n_blk, lane);
+}
+
 __device__ __forceinline__ TileCoord tile_coord(int tile, int m_blocks) {
   return TileCoord{tile % m_blocks, tile / m_blocks};
 }
@@ -312,7 +342,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int m_blocks = (epi_m_limit(epi, M) + Shape::BM - 1) / Shape::BM;
   const int n_blocks = (N + BN - 1) / BN;
   const int k_blocks = (epi_k_limit(epi, K) + kBK - 1) / kBK;
-  const int num_tiles = k_blocks > 0 ? m_blocks * n_blocks : 0;
+  // split-K: K-blocks per split, and the number of non-empty splits
+  const int want_splits = max(1, min(epi_splits(epi), k_blocks));
+  const int kb_per = k_blocks > 0 ? (k_blocks + want_splits - 1) / want_splits : 0;
+  const int nsplit = kb_per > 0 ? (k_blocks + kb_per - 1) / kb_per : 1;
+  const int num_tiles = k_blocks > 0 ? m_blocks * n_blocks * nsplit : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -343,10 +377,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t ph = 0;
       uint32_t armed = 0, armed_par = 0;
       for (int tile = pair; tile < num_tiles && !*abort_flag; tile += n_pairs) {
-        const TileCoord tc = tile_coord(tile, m_blocks);
+        const int split = tile % nsplit;
+        const TileCoord tc = tile_coord(tile / nsplit, m_blocks);
         const int a_row = tc.m_blk * Shape::BM + static_cast<int>(rank) * kBM;
         const int b_row = tc.n_blk * BN + static_cast<int>(rank) * (BN / 2);
-        for (int kb = 0; kb < k_blocks; ++kb) {
+        const int kb_end = min(k_blocks, (split + 1) * kb_per);
+        for (int kb = split * kb_per; kb < kb_end; ++kb) {
           if (!wait_or_abort(&empty[s], ph ^ 1, abort_flag, diag)) break;
           uint8_t* sa = smem + s * Shape::STAGE_BYTES;
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * Shape::STAGE_BYTES);
@@ -382,7 +418,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * Shape::ACC_COLS;
         bool ok = true;
-        for (int kb = 0; kb < k_blocks; ++kb) {
+        const int split = tile % nsplit;
+        const int kb0 = split * kb_per, kb_end = min(k_blocks, kb0 + kb_per);
+        for (int kb = kb0; kb < kb_end; ++kb) {
           if (!wait_or_abort(&full[s], ph, abort_flag, diag)) {
             ok = false;
             break;
@@ -395,7 +433,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int b = 0; b < NB; ++b) {
               const uint64_t bdesc = umma_desc_sw128(sa + Shape::A_BYTES + b * Shape::B_BYTES + k * 32);
-              umma2_bf16(d_tmem + b * BN, adesc, bdesc, idesc, (kb | k) != 0);
+              umma2_bf16(d_tmem + b * BN, adesc, bdesc, idesc, (kb != kb0 || k != 0) ? 1u : 0u);
             }
           }
           umma2_commit_mc(&empty[s], 0x3);
@@ -422,10 +460,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const bool ok = wait_or_abort(&tmem_full[acc], (it >> 1) & 1, abort_flag, diag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const TileCoord tc = tile_coord(tile, m_blocks);
+      const TileCoord tc = tile_coord(tile / nsplit, m_blocks);
       const uint32_t taddr = tmem_base + acc * Shape::ACC_COLS + (static_cast<uint32_t>(quarter * 32) << 16);
       const int64_t row = static_cast<int64_t>(tc.m_blk) * Shape::BM + rank * kBM + quarter * 32 + lane;
-      epi.template run<BN>(taddr, row, tc.n_blk, lane);
+      epi_run_impl<BN>(epi, taddr, row, tc.n_blk, tile % nsplit, nsplit, lane, 0);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tmem_empty0 + acc * 8);

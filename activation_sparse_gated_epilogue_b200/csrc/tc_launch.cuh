@@ -47,14 +47,15 @@ int max_resident_pairs() {
   return n;
 }
 
+// `splits`: the K splits the epilogue asks for (Epi::splits), for the grid size.
 template <class Shape, class Epi>
 int launch_tc_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1,
                         int64_t m, int64_t n, int64_t k, const Epi& epi, int32_t* diag,
-                        cudaStream_t st, const char* what) {
+                        cudaStream_t st, const char* what, int splits = 1) {
   auto kern = tc_gemm_pair_kernel<Shape, Epi>;
   int rc = set_smem_limit(reinterpret_cast<const void*>(kern), Shape::SMEM_BYTES);
   if (rc) return rc;
-  const int64_t tiles = ((m + Shape::BM - 1) / Shape::BM) * ((n + Shape::BN - 1) / Shape::BN);
+  const int64_t tiles = ((m + Shape::BM - 1) / Shape::BM) * ((n + Shape::BN - 1) / Shape::BN) * splits;
   const int64_t resident = max_resident_pairs<Shape, Epi>();
   const int pairs = static_cast<int>(tiles < resident ? tiles : resident);
   cudaLaunchConfig_t cfg = {};

@@ -2,19 +2,23 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-One step = one pass of the whole sparse inference path over one batch:
-gate GEMM with the TwELL epilogue (twell_gate_pack) followed by the fused
-up/down kernel (twell_fused_up_down), on the 1B-shaped bf16 workload
-(N=8192 tokens, d=2048, F=8192, T=C=128, mean gate density 1%, per-token
-scale LogNormal(0, 0.7)) unless --workload names another.  Inputs are seeded
-synthetic data resident in HBM; L2 is flushed (a 256 MB write) between timed
-steps and the flush is outside the per-step CUDA events.
+One step = one pass of the whole sparse inference path over one batch: the
+gate GEMM with the TwELL epilogue (twell_gate_pack), then the up and down
+projections from TwELL (twell_hybrid_up_down: tokens with at most K = 32
+stored entries through a CUDA-core kernel beside the heavier ones, which run
+through two tcgen05 spill GEMMs), on the 1B-shaped bf16
+workload (N=8192 tokens, d=2048, F=8192, T=C=128, mean gate density 1%,
+per-token scale LogNormal(0, 0.7)) unless --workload names another.  Inputs
+are seeded synthetic data resident in HBM; L2 is flushed (a 256 MB write)
+between timed steps and the flush is outside the per-step CUDA events.
 
 Prints one JSON line (rank 0).  `value` is tokens/s over all ranks (weak
 scaling: every rank runs its own batch, no collective on the data path).
-Also reported: the library's dense bf16 FFN and a cuBLAS (torch.matmul)
-dense FFN on the same inputs, the roofline of each kernel, an end-to-end
-number through host buffers, and the fp64 CPU oracle on a bounded sample.
+Also reported: the same forward with every entry through the per-entry
+kernel (twell_fused_up_down), the hybrid format's pack-and-forward path, the
+library's dense bf16 FFN and a cuBLAS (torch.matmul) dense FFN on the same
+inputs, the roofline of each kernel, an end-to-end number through host
+buffers, and the fp64 CPU oracle on a bounded sample.
 """
 from __future__ import annotations
 
@@ -41,6 +45,10 @@ FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # ELL capacity of the hybrid format when it serves inference (tokens with more
 # stored entries run on the tensor-core spill GEMMs)
 HYB_INFER_K = 64
+# K of the routed step: tokens with more stored entries take the spill GEMMs
+# (measured at the 1B shape: K = 16 / 32 / 64 give 0.186 / 0.185 / 0.197 ms
+# for the call)
+ROUTED_K = 32
 
 # DRAM bytes (read + write) per launch from ncu captures of the kernels,
 # keyed by the hash of the source they were taken on; a kernel whose source
@@ -63,10 +71,14 @@ def parse():
     p.add_argument("--cap-sweep", action="store_true",
                    help="TwELL capacity C in {T/4, T/2, T}: footprint, overflow, truncation error, "
                         "and the hybrid path that recomputes overflowing rows: one JSON line per C")
+    p.add_argument("--ell-cap", type=int, default=ROUTED_K,
+                   help="K of the routed step: tokens with more stored entries run on the spill GEMMs")
     p.add_argument("--profile", action="store_true",
-                   help="run only warmup + steps of the sparse step (for ncu captures); no JSON")
-    p.add_argument("--profile-hybrid", action="store_true",
-                   help="with --profile: the hybrid inference step (gate, hybrid_pack, hybrid_ffn_fwd) instead")
+                   help="run only warmup + steps of one path (for ncu captures); no JSON")
+    p.add_argument("--profile-path", default="routed", choices=["routed", "fused", "hybrid"],
+                   help="with --profile: the routed step (default), the TwELL step (gate + "
+                        "twell_fused_up_down) or the hybrid format's path (gate, hybrid_pack, "
+                        "hybrid_ffn_fwd)")
     return p.parse_args()
 
 
@@ -176,6 +188,24 @@ def workload_config(args):
     return cfg.with_(n_tokens=args.tokens) if args.tokens > 0 else cfg
 
 
+def spill_rows_for(n: int) -> int:
+    """S_max of the hybrid format's path: a quarter of the batch, rounded up
+    to whole 256-row spill tiles."""
+    return max(256, (n // 4 + 255) // 256 * 256)
+
+
+def routed_split(count: torch.Tensor, cap: int, k: int, s_max: int):
+    """(spill rows, stored entries of the light and past-S_max tokens, all
+    stored entries) of a routed call on a TwELL with per-tile counts
+    `count`: tokens with more than k stored entries are heavy and the first
+    s_max of them (ascending token order) go to the spill."""
+    stored = torch.clamp(count.to(torch.int64), max=cap).sum(1)
+    heavy = torch.nonzero(stored > k).flatten()[:s_max]
+    total = int(stored.sum().item())
+    spilled = int(stored[heavy].sum().item())
+    return int(heavy.numel()), total - spilled, total
+
+
 def run_own(args, rank, world, local_rank):
     import activation_sparse_gated_epilogue_b200 as sge
     from activation_sparse_gated_epilogue_b200 import synth
@@ -188,16 +218,23 @@ def run_own(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     inp = synth.make_inputs(cfg)
     n, d, f, tile, cap = cfg.n_tokens, cfg.d_model, cfg.d_ff, cfg.tile, cfg.cap
+    # S_max = N: every heavy token can take the spill (the workspace holds
+    # the spill operands for N rows; the GEMMs run only the rows there are)
+    k_route, s_max = args.ell_cap, n
     x, wg, wu, wd = (getattr(inp, k).to(dev) for k in ("x", "wg_t", "wu_t", "wd"))
+    # weight layouts built once: W_up^T and W_down interleaved row by row (the
+    # per-entry kernel's rows, the up GEMM's B operand with row stride 2d) and
+    # W_down^T (the down GEMM's K-major B operand)
     wd_t = wd.t().contiguous()
-    # the fused kernel's weights: W_up^T and W_down interleaved row by row
     _w_ud, wu_i, wd_i = sge.interleave_up_down(wu, wd)
     tw = sge.TwELL.empty(n, f, tile, cap, x.dtype, dev)
     y = torch.empty_like(x)
+    y_fused = torch.empty_like(x)
     h = torch.empty((n, f), dtype=x.dtype, device=dev)
     y_dense = torch.empty_like(x)
     diag = sge.new_diag(dev)
     ws = sge.fused_workspace(n, d, dev)
+    ws_r = sge.routed_workspace(n, d, f, s_max, dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -225,43 +262,54 @@ def run_own(args, rank, world, local_rank):
         return reduce_max_over_ranks(v, dev)
 
     gate = lambda: sge.twell_gate_pack(x, wg, tile, cap, out=tw, diag=diag)
-    fused = lambda: sge.twell_fused_up_down(x, tw, wu_i, wd_i, y=y, workspace=ws)
+    routed = lambda: sge.twell_hybrid_up_down(x, tw, wu_i, wd_i, wd_t, k_route, s_max, y=y,
+                                              workspace=ws_r, diag=diag)
+    fused = lambda: sge.twell_fused_up_down(x, tw, wu_i, wd_i, y=y_fused, workspace=ws)
     dense = lambda: sge.dense_ffn_fwd(x, wg, wu, wd_t, h=h, y=y_dense)
 
     def hybrid_setup():
-        hk, hs = HYB_INFER_K, max(128, (n // 4 + 127) // 128 * 128)
+        hk, hs = HYB_INFER_K, spill_rows_for(n)
         hy = sge.Hybrid.empty(n, f, hk, hs, dev)
         hws = sge.hybrid_fwd_workspace(d, f, hs, dev)
         y_h = torch.empty_like(x)
         hdiag = sge.new_diag(dev)
         hpack = lambda: sge.hybrid_pack(tw, hk, hs, out=hy, diag=hdiag)
-        hfwd = lambda: sge.hybrid_ffn_fwd(x, hy, wu, wd, wd_t=wd_t, y=y_h, workspace=hws)
+        hfwd = lambda: sge.hybrid_ffn_fwd(x, hy, wu, wd, wd_t, y=y_h, workspace=hws)
         return hk, hs, hy, y_h, hdiag, hpack, hfwd
 
     if args.profile:
-        if args.profile_hybrid:
+        if args.profile_path == "hybrid":
             _, _, _, _, _, hpack, hfwd = hybrid_setup()
             timed([gate, hpack, hfwd], args.steps, args.warmup)
-        else:
+        elif args.profile_path == "fused":
             timed([gate, fused], args.steps, args.warmup)
+        else:
+            timed([gate, routed], args.steps, args.warmup)
         return None
 
     # ---- the sparse forward: timed region
-    timed([gate, fused], 0, args.warmup)
+    timed([gate, routed], 0, args.warmup)
     barrier()
     with ClockSampler(local_rank) as clk:
         barrier()
-        evs = timed([gate, fused], args.steps, 0)
+        evs = timed([gate, routed], args.steps, 0)
         barrier()
     clocks = clk.summary()
     t_gate = [e[0].elapsed_time(e[1]) for e in evs]
-    t_fused = [e[1].elapsed_time(e[2]) for e in evs]
-    total_ms = reduce_max(sum(a + b for a, b in zip(t_gate, t_fused)))
+    t_routed = [e[1].elapsed_time(e[2]) for e in evs]
+    total_ms = reduce_max(sum(a + b for a, b in zip(t_gate, t_routed)))
     ms_step = total_ms / args.steps
     value = replica_tokens_per_s(n, world, args.steps, total_ms)
-
-    nnz = int(tw.count.to(torch.int64).sum().item())
+    diag_host = diag.tolist()
+    n_spill, nnz_light, nnz = routed_split(tw.count, cap, k_route, s_max)
     density = nnz / (n * f)
+
+    # ---- the same forward through the per-entry kernel alone (TwELL step)
+    evf = timed([gate, fused], min(args.steps, 100), 3)
+    ms_fused_step = statistics.mean(e[0].elapsed_time(e[2]) for e in evf)
+    ms_fused = statistics.mean(e[1].elapsed_time(e[2]) for e in evf)
+    routed_vs_fused = float(((y.float() - y_fused.float()).abs().max()
+                             / y_fused.float().abs().max().clamp_min(1e-30)).item())
 
     # ---- dense baselines on the same inputs (own tcgen05 and cuBLAS)
     evd = timed([dense], min(args.steps, 100), 3)
@@ -281,7 +329,8 @@ def run_own(args, rank, world, local_rank):
     def e2e():
         x_dev2.copy_(x_host, non_blocking=True)
         sge.twell_gate_pack(x_dev2, wg, tile, cap, out=tw, diag=diag)
-        sge.twell_fused_up_down(x_dev2, tw, wu_i, wd_i, y=y, workspace=ws)
+        sge.twell_hybrid_up_down(x_dev2, tw, wu_i, wd_i, wd_t, k_route, s_max, y=y, workspace=ws_r,
+                                 diag=diag)
         y_host.copy_(y, non_blocking=True)
     e2e_steps = min(args.steps, 50)
     barrier()
@@ -289,69 +338,66 @@ def run_own(args, rank, world, local_rank):
     barrier()
     e2e_ms = reduce_max(sum(e[0].elapsed_time(e[1]) for e in eve))
     e2e_value = replica_tokens_per_s(n, world, e2e_steps, e2e_ms)
-    diag_host = diag.tolist()
 
-    # ---- the hybrid format used for inference (a further row of the method,
-    # not the step above): rows with more than K stored entries go through the
-    # dense spill GEMMs on tensor cores, the others through the ELL kernel
-    hyb = None
-    if x.dtype == torch.bfloat16:
-        hk, hs, hy, y_h, hdiag, hpack, hfwd = hybrid_setup()
-        hsteps = min(args.steps, 100)
-        timed([gate, hpack, hfwd], 0, 3)
-        barrier()
-        evh = timed([gate, hpack, hfwd], hsteps, 0)
-        barrier()
-        h_ms = reduce_max(sum(e[0].elapsed_time(e[3]) for e in evh)) / hsteps
-        dropped = int(hdiag[2].item())
-        err = float(((y_h.float() - y.float()).abs().max() / y.float().abs().max()).item())
-        hyb = {"value": round(replica_tokens_per_s(n, world, 1, h_ms), 1), "unit": "tokens/s", "ms_per_step": round(h_ms, 4),
-               "ell_cap_K": hk, "s_max": hs, "spill_rows": int(hy.n_spill.item()), "dropped_rows": dropped,
-               "ms_parts": {"gate": round(statistics.mean(e[0].elapsed_time(e[1]) for e in evh), 4),
-                            "hybrid_pack": round(statistics.mean(e[1].elapsed_time(e[2]) for e in evh), 4),
-                            "hybrid_ffn_fwd": round(statistics.mean(e[2].elapsed_time(e[3]) for e in evh), 4)},
-               "max_abs_rel_vs_fused": round(err, 6),
-               "note": "gate GEMM + TwELL, hybrid_pack, hybrid_ffn_fwd (spill rows' h goes through HBM)"}
+    # ---- the hybrid format's own path (pack into ELL + spill, then forward)
+    hk, hs, hy, y_h, hdiag, hpack, hfwd = hybrid_setup()
+    hsteps = min(args.steps, 100)
+    timed([gate, hpack, hfwd], 0, 3)
+    barrier()
+    evh = timed([gate, hpack, hfwd], hsteps, 0)
+    barrier()
+    h_ms = reduce_max(sum(e[0].elapsed_time(e[3]) for e in evh)) / hsteps
+    hyb = {"value": round(replica_tokens_per_s(n, world, 1, h_ms), 1), "unit": "tokens/s",
+           "ms_per_step": round(h_ms, 4), "ell_cap_K": hk, "s_max": hs,
+           "spill_rows": int(hy.n_spill.item()), "dropped_rows": int(hdiag[2].item()),
+           "ms_parts": {"gate": round(statistics.mean(e[0].elapsed_time(e[1]) for e in evh), 4),
+                        "hybrid_pack": round(statistics.mean(e[1].elapsed_time(e[2]) for e in evh), 4),
+                        "hybrid_ffn_fwd": round(statistics.mean(e[2].elapsed_time(e[3]) for e in evh), 4)},
+           "speedup_vs_own_dense": round(ms_dense / h_ms, 3),
+           "note": "gate GEMM + TwELL, hybrid_pack (ELL + dense spill rows), hybrid_ffn_fwd (saves u)"}
 
     if rank != 0:
         return None
 
     pk = peaks()
-    mg = statistics.mean(t_gate)
-    mf = statistics.mean(t_fused)
-    flops_gate = 2.0 * n * d * f
     bf16_peak = pk["bf16_tflops"]
+    mg = statistics.mean(t_gate)
+    mr = statistics.mean(t_routed)
+    flops_gate = 2.0 * n * d * f
     gate_tf = flops_gate / (mg / 1e3) / 1e12
-    flops_fused = 4.0 * nnz * d
-    fused_tf = flops_fused / (mf / 1e3) / 1e12
-    # unique HBM bytes of the fused kernel: x, the weight rows it touches
-    # (at most all of W_up and W_down), TwELL entries and counts, y
-    bytes_fused = (2 * n * d + 2 * 2 * f * d + 3 * nnz + n * (f // tile) + 2 * n * d)
+    # the routed call's algorithmic work: the spill rows' two GEMMs over all F
+    # hidden units on tensor cores, the other tokens' entries on CUDA cores
+    flops_spill = 4.0 * n_spill * d * f
+    flops_light = 4.0 * nnz_light * d
+    routed_roof_ms = (flops_spill / (bf16_peak * 1e12) + flops_light / (FP32_SIMT_TFLOPS * 1e12)) * 1e3
+    gate_roof_ms = flops_gate / (bf16_peak * 1e12) * 1e3
     gate_src = src_hash("gate_pack.cu", "tc_gemm.cuh", "sge_common.cuh")
-    fused_src = src_hash("fused_up_down.cu", "sparse_common.cuh", "sge_common.cuh")
-    tr_gate = TRAFFIC.get(gate_src)
-    tr_fused = TRAFFIC.get(fused_src)
-    tr_gate = None if tr_gate is None else int(tr_gate)
-    tr_fused = None if tr_fused is None else int(tr_fused)
+    routed_src = src_hash("routed.cu", "fused_kernels.cuh", "spill_gemm.cuh", "tc_gemm.cuh",
+                          "sparse_common.cuh", "sge_common.cuh")
+    tr_gate, tr_routed = TRAFFIC.get(gate_src), TRAFFIC.get(routed_src)
     k_gate = {"kernel": "twell_gate_pack (tcgen05 GEMM + TwELL epilogue)", "bound": "tensor",
               "achieved": round(gate_tf, 1), "peak": bf16_peak, "unit": "TFLOP/s",
-              "frac": round(gate_tf / bf16_peak, 4), "traffic": tr_gate,
-              "ms": round(mg, 4), "share": round(mg / (mg + mf), 3),
+              "frac": round(gate_tf / bf16_peak, 4),
+              "traffic": None if tr_gate is None else int(tr_gate),
+              "ms": round(mg, 4), "share": round(mg / (mg + mr), 3),
               "algorithmic": f"2*N*d*F = {flops_gate:.3e} flop per launch",
               "peak_note": "bf16_tflops (burst) of measured peaks: the step keeps SM clocks at max"}
-    k_fused = {"kernel": "twell_fused_up_down (planning kernels + main kernel)", "bound": "alu", "achieved": round(fused_tf, 2),
-               "peak": round(FP32_SIMT_TFLOPS, 1), "unit": "TFLOP/s",
-               "frac": round(fused_tf / FP32_SIMT_TFLOPS, 4), "traffic": tr_fused,
-               "ms": round(mf, 4), "share": round(mf / (mg + mf), 3),
-               "algorithmic": f"4*nnz*d = {flops_fused:.3e} flop per launch (nnz={nnz})",
-               "hbm_gbs_unique": round(bytes_fused / (mf / 1e3) / 1e9, 1),
-               "peak_note": "fp32 FMA peak of the CUDA cores, 148 SMs x 128 lanes x 2 x 1.965 GHz",
-               # its weight rows (4*nnz*d bytes) streamed from L2 into the SMs
-               "l2_row_bytes_tbs": round(4.0 * nnz * d / (mf / 1e3) / 1e12, 2)}
-    k_gate["traffic_unit"] = k_fused["traffic_unit"] = "bytes per launch (ncu dram read + write)"
-    dominant = k_gate if mg >= mf else k_fused
-    rest = k_fused if dominant is k_gate else k_gate
-    roofline_time_ms = flops_gate / (bf16_peak * 1e12) * 1e3 + flops_fused / (FP32_SIMT_TFLOPS * 1e12) * 1e3
+    k_routed = {"kernel": "twell_hybrid_up_down (plan 2 + spill prep + 2 tcgen05 spill GEMMs + "
+                          "per-entry kernel)", "bound": "tensor",
+                "achieved": round((flops_spill + flops_light) / (mr / 1e3) / 1e12, 1),
+                "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(routed_roof_ms / mr, 4),
+                "traffic": None if tr_routed is None else int(tr_routed),
+                "ms": round(mr, 4), "share": round(mr / (mg + mr), 3),
+                "algorithmic": f"4*S*d*F = {flops_spill:.3e} flop on tensor cores (S={n_spill} spill "
+                               f"rows) + 4*nnz_light*d = {flops_light:.3e} flop on CUDA cores "
+                               f"(nnz_light={nnz_light}): {routed_roof_ms:.4f} ms at the peaks",
+                "frac_note": "algorithmic time at the peaks / measured time"}
+    k_gate["traffic_unit"] = k_routed["traffic_unit"] = "bytes per launch (ncu dram read + write)"
+    dominant = k_gate if mg >= mr else k_routed
+    rest = k_routed if dominant is k_gate else k_gate
+    step_roof_ms = gate_roof_ms + routed_roof_ms
+    # the TwELL step's roofline (gate on tensor cores, 4*nnz*d on CUDA cores)
+    twell_roof_ms = gate_roof_ms + 4.0 * nnz * d / (FP32_SIMT_TFLOPS * 1e12) * 1e3
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -359,22 +405,38 @@ def run_own(args, rank, world, local_rank):
         "data": "synthetic (seeded; tokens x d_model x d_ff shaped like a 1B FFN)",
         "config": {"workload": f"{cfg.name}: N={n} d={d} F={f} T={tile} C={cap} "
                                f"target density {cfg.rho} sigma={cfg.sigma}",
-                   "realised_density": round(density, 5), "nnz": nnz,
+                   "step": f"twell_gate_pack + twell_hybrid_up_down (K={k_route}, S_max={s_max})",
+                   "realised_density": round(density, 5), "nnz": nnz, "spill_rows": n_spill,
+                   "nnz_per_entry_path": nnz_light,
                    "l2": "flushed between steps (256 MB write outside the step events)",
-                   "weights": "fused kernel reads W_up^T and W_down interleaved row by row ([F][2d], built once)",
+                   "weights": "W_up^T and W_down interleaved row by row ([F][2d]) and W_down^T "
+                              "([d][F]), both built once",
                    "parallelism": f"replicas x{world} (token batches independent)"},
         "roofline": {k: dominant[k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")},
         "kernels": [dominant, rest],
-        "step_roofline_ms": round(roofline_time_ms, 4),
-        "step_roofline_frac": round(roofline_time_ms / ms_step, 4),
+        "step_roofline_ms": round(step_roof_ms, 4),
+        "step_roofline_frac": round(step_roof_ms / ms_step, 4),
+        "twell_roofline_ms": round(twell_roof_ms, 4),
+        "twell_roofline_frac": round(twell_roof_ms / ms_step, 4),
+        "roofline_note": "step roofline: gate flops and spill flops at the bf16 peak, the "
+                         "per-entry tokens' 4*nnz*d at the fp32 FMA peak; twell roofline: gate "
+                         "flops at the bf16 peak and all 4*nnz*d at the fp32 FMA peak",
         "dense": {"own_tcgen05_ms": round(ms_dense, 4), "cublas_ms": round(ms_cublas, 4),
                   "speedup_vs_own_dense": round(ms_dense / ms_step, 3),
                   "speedup_vs_cublas_dense": round(ms_cublas / ms_step, 3)},
+        "twell_fused_step": {"ms_per_step": round(ms_fused_step, 4), "fused_ms": round(ms_fused, 4),
+                             "value": round(n / (ms_fused_step / 1e3), 1), "unit": "tokens/s",
+                             "speedup_vs_own_dense": round(ms_dense / ms_fused_step, 3),
+                             "max_abs_rel_routed_vs_fused": round(routed_vs_fused, 6),
+                             "note": "gate + twell_fused_up_down: every entry through the "
+                                     "per-entry kernel"},
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
                 "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
-        "gpu_launches": 4 * args.steps,
-        "launches_note": "per step: gate GEMM + TwELL epilogue; fused up/down = count, jobs, main kernel",
+        "gpu_launches": (2 if n <= 64 else 7) * args.steps,
+        "launches_note": "per step: gate GEMM + TwELL epilogue; twell_hybrid_up_down = count, jobs, "
+                         "spill prep, up GEMM, down GEMM, per-entry kernel (2 launches in all for "
+                         "batches of at most 64 tokens)",
         "hybrid_inference": hyb,
         "clocks": clocks,
         "diag": diag_host,
@@ -428,6 +490,9 @@ def run_sweep(args, local_rank):
         torch.cuda.synchronize(dev)
         return [[e[i].elapsed_time(e[i + 1]) for i in range(len(fns))] for e in evs]
 
+    s_max_r = n
+    ws_r = sge.routed_workspace(n, d, f, s_max_r, dev)
+    y_r = torch.empty_like(x)
     h = torch.empty((n, f), dtype=x.dtype, device=dev)
     y_dense = torch.empty_like(x)
     dense_ms = statistics.mean(t[0] for t in timed([lambda: sge.dense_ffn_fwd(x, wg, wu, wd_t, h=h, y=y_dense)],
@@ -439,6 +504,11 @@ def run_sweep(args, local_rank):
         wg[:, d - 1] = -tau                      # rounded to the weight dtype
         gate = lambda: sge.twell_gate_pack(x, wg, tile, cap, out=tw)
         fused = lambda: sge.twell_fused_up_down(x, tw, wu_i, wd_i, y=y, workspace=ws)
+        routed = lambda: sge.twell_hybrid_up_down(x, tw, wu_i, wd_i, wd_t, args.ell_cap, s_max_r,
+                                                  y=y_r, workspace=ws_r)
+        tr = timed([gate, routed], steps, 3)
+        routed_ms = statistics.mean(a + b for a, b in tr)
+        n_spill_r, nnz_light_r, _ = routed_split(tw.count, cap, args.ell_cap, s_max_r)
         t = timed([gate, fused], steps, 3)
         mg = statistics.mean(a for a, _ in t)
         mf = statistics.mean(b for _, b in t)
@@ -466,6 +536,13 @@ def run_sweep(args, local_rank):
             "dense_own_ms": round(dense_ms, 4), "speedup_vs_own_dense": round(dense_ms / step, 3),
             "hybrid_inference_ms": round(hms, 4), "hybrid_speedup_vs_own_dense": round(dense_ms / hms, 3),
             "hybrid_K": hk, "hybrid_spill_rows": int((per_tok > hk).sum().item()),
+            "routed_ms": round(routed_ms, 4), "routed_tokens_per_s": round(n / (routed_ms / 1e3), 1),
+            "routed_speedup_vs_own_dense": round(dense_ms / routed_ms, 3),
+            "routed_K": args.ell_cap, "routed_S_max": s_max_r, "routed_spill_rows": n_spill_r,
+            "routed_nnz_per_entry_path": nnz_light_r,
+            "routed_step_roofline_frac": round((flops_gate + 4.0 * n_spill_r * d * f) / (pk["bf16_tflops"] * 1e12) * 1e3
+                                               / routed_ms + 4.0 * nnz_light_r * d / (FP32_SIMT_TFLOPS * 1e12) * 1e3
+                                               / routed_ms, 4),
         })
     return out
 
@@ -618,11 +695,51 @@ def run_train(args, local_rank):
     ms = statistics.mean(t_sparse)
     ms_dense = statistics.mean(t_dense)
     n_spill = int(hy.n_spill.item())
-    kept = min(n_spill, cfg.s_max)
     nnz = int(hy.row_nnz.to(torch.int64).sum().item())
-    # activations saved between forward and backward (bytes)
-    hybrid_saved = (n * cfg.ell_cap * (2 + 2 + 2) + 4 * n * 3 + kept * f * 2 * 2)
-    dense_saved = n * f * 2 * 2          # G and U in bf16 (h recomputed)
+
+    # ---- activation memory, read from the caching allocator: what the
+    # forward leaves allocated for the backward (plus y), and the peak over
+    # forward + backward, both above what was allocated before the step
+    # (weights, x, dy); buffers and workspaces are allocated inside.
+    def measure(fwd, bwd):
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev)
+        saved = fwd()
+        torch.cuda.synchronize(dev)
+        held = torch.cuda.memory_allocated(dev) - base
+        out = bwd(saved)
+        torch.cuda.synchronize(dev)
+        peak = torch.cuda.max_memory_allocated(dev) - base
+        del saved, out
+        return held, peak
+
+    def hybrid_fwd():
+        tw_ = sge.twell_gate_pack(x, wg, cfg.tile, cfg.cap)     # transient
+        hy_ = sge.hybrid_pack(tw_, cfg.ell_cap, cfg.s_max)      # saved for the backward
+        ws_ = sge.hybrid_fwd_workspace(d, f, cfg.s_max, dev)
+        y_ = sge.hybrid_ffn_fwd(x, hy_, wu, wd, wd_t, workspace=ws_)
+        del tw_, ws_
+        return hy_, y_
+
+    def hybrid_bwd(saved):
+        hy_, _ = saved
+        ws_ = sge.hybrid_bwd_workspace(n, d, f, cfg.ell_cap, cfg.s_max, dev)
+        return sge.hybrid_ffn_bwd(x, dy, hy_, wg, wu, wd, workspace=ws_)
+
+    def dense_fwd():
+        return (torch.relu(xr @ wgr.t()) * (xr @ wur.t())) @ wdr
+
+    def dense_bwd(y_):
+        y_.backward(dy)
+        g = (xr.grad, wgr.grad, wur.grad, wdr.grad)
+        xr.grad = wgr.grad = wur.grad = wdr.grad = None
+        return g
+
+    del tw, hy, y, fws, bws
+    h_held, h_peak = measure(hybrid_fwd, hybrid_bwd)
+    d_held, d_peak = measure(dense_fwd, dense_bwd)
     return {
         "metric": "hybrid FFN training step tokens/s (1B shape, bf16)", "value": round(n / (ms / 1e3), 1),
         "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
@@ -633,8 +750,16 @@ def run_train(args, local_rank):
                    "nnz": nnz, "spill_rows": n_spill, "l2": "flushed between steps"},
         "dense_autograd_cublas_ms": round(ms_dense, 4),
         "speedup_vs_dense": round(ms_dense / ms, 3),
-        "saved_activation_bytes": {"hybrid": hybrid_saved, "dense": dense_saved,
-                                   "ratio": round(hybrid_saved / dense_saved, 4)},
+        "activation_memory_bytes": {
+            "hybrid_held_after_forward": int(h_held), "dense_held_after_forward": int(d_held),
+            "held_ratio": round(h_held / d_held, 4),
+            "hybrid_peak_forward_backward": int(h_peak), "dense_peak_forward_backward": int(d_peak),
+            "peak_ratio": round(h_peak / d_peak, 4),
+            "how": "torch.cuda.memory_allocated / max_memory_allocated around one forward and one "
+                   "backward, above the weights and inputs; held = activations saved for the "
+                   "backward plus y (hybrid: ELL rows, routing and the S_max-row spill buffers; "
+                   "dense autograd: relu(G), U and h); the peaks include workspaces, the "
+                   "hybrid's transient TwELL (C = T) and its fp32 weight gradients (dense: bf16)"},
         "gpu_launches_per_step": 24,
         "launches_note": "gate 1, pack 2, forward 4 (ELL, gather, 2 GEMMs), backward 17 (ELL, 4 bucket kernels, dW, gather, 6 transposes, 3 GEMMs)",
         "clocks": clk.summary(), "diag": diag.tolist(),

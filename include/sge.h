@@ -193,6 +193,69 @@ int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, const uint8
                                 int dtype, int tile, int cap, int32_t* diag, void* stream);
 
 /*
+ * twell_hybrid_up_down -- the up and down projections from TwELL with the
+ * heavy tokens routed to tensor cores (inference).  ("Sparser, Faster,
+ * Lighter Transformer Language Models", pwwt.cn summary, section 03 and
+ * figure "routing of the hybrid-format sparse operator": tokens with few
+ * active gates take the sparse path, the rare highly active tokens a dense
+ * backup path on tensor cores; kongchang.com page, "core idea": a fast path
+ * with a dense fallback.)  Computes the same y as twell_fused_up_down:
+ *   y[t] = sum over stored entries (j, a) of row t of bf16(a u) wd[j],
+ *   u = x[t] . wu_t[j], fp32 accumulation, y in bf16,
+ * up to the order of the fp32 sums (which differs from
+ * twell_fused_up_down's, so the last bits of y may differ).
+ *
+ * Routing: a token with more than K = ell_cap stored entries (the sum of
+ * min(count, C) over its tiles) is heavy; heavy tokens are ranked in
+ * ascending token order and the first S_max = s_max of them run as two
+ * tcgen05 GEMMs over all F hidden units (U = X_s W_up with an epilogue
+ * forming h = bf16(a u), zero where the TwELL stores no entry; then
+ * Y_s = H_s W_down scattered into y).  The light tokens run on CUDA cores
+ * at the same time, on a stream the library keeps per device (forked from
+ * and joined back into `stream` within the call); heavy tokens past S_max
+ * run through the per-entry kernel of twell_fused_up_down afterwards; no
+ * token is dropped.  Batches of at most 64 tokens,
+ * and s_max = 0, run the per-entry path for every token (a spill GEMM would
+ * stream all of W_up and W_down for a few rows).  No ELL repack and nothing
+ * saved for a backward pass (hybrid_pack / hybrid_ffn_fwd do that).
+ *
+ *   x [N][d], y [N][d]   bf16
+ *   count/idx/val        the TwELL of twell_gate_pack (bf16 values), tile T,
+ *                        capacity C
+ *   wu_t, wd, ldw        as for twell_fused_up_down (the interleaved layout
+ *                        of sge_interleave_up_down is the fastest); the
+ *                        spill GEMM reads wu_t with row stride ldw
+ *   wd_t [d][F]          bf16  W_down transposed (row i = column i of
+ *                        W_down), the K-major operand of the down GEMM; a
+ *                        weight layout built once; may be NULL if s_max = 0
+ *   ell_cap              K, 0 <= K <= 512
+ *   s_max                spill capacity in tokens, >= 0
+ *   workspace            >= twell_hybrid_up_down_workspace_bytes(N, d, F,
+ *                        s_max) bytes, 256-byte aligned, caller-owned, not
+ *                        shared by calls that may run concurrently (the
+ *                        per-entry kernel's lists and pool, the spill list,
+ *                        and the spill operands X_s [S_max][d], A_s and H_s
+ *                        [S_max][F] in bf16)
+ *   diag                 nullable; [SGE_DIAG_SPILL_ROWS] gains the number of
+ *                        heavy tokens (those past S_max included),
+ *                        [SGE_DIAG_FLAGS] SGE_FLAG_TIMEOUT if a wait gave up
+ * Deterministic: repeated calls give the same bits.  Rows with a tile whose
+ * count exceeds C use their stored entries only, as in twell_fused_up_down.
+ * Errors: as twell_fused_up_down; SGE_ERR_ARG for negative K or S_max,
+ * F % 8 != 0, a short or misaligned workspace, a missing wd_t;
+ * SGE_ERR_UNSUPPORTED for K > 512; SGE_ERR_CUDA if the library's stream or
+ * events cannot be created.
+ */
+size_t twell_hybrid_up_down_workspace_bytes(int64_t n_tokens, int64_t d_model, int64_t d_ff,
+                                            int s_max);
+
+int twell_hybrid_up_down(const void* x, const uint8_t* count, const uint8_t* idx, const void* val,
+                         const void* wu_t, const void* wd, int64_t ldw, const void* wd_t, void* y,
+                         int64_t n_tokens, int64_t d_model, int64_t d_ff, int tile, int cap,
+                         int ell_cap, int s_max, void* workspace, size_t workspace_bytes,
+                         int32_t* diag, void* stream);
+
+/*
  * sge_interleave_up_down -- builds the interleaved weight layout that
  * twell_fused_up_down streams fastest: w_ud [F][2d], row j = wu_t[j] (d
  * elements) then wd[j] (d elements).  A layout step for loading weights, done

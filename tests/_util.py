@@ -127,3 +127,30 @@ def check_1b_all_rows(y_gpu: np.ndarray, tw_gpu=None):
     err = oracle.max_abs_rel(y_gpu, y_ora)
     assert err <= BF16_TOL, err
     return err, flips
+
+
+def heavy_and_strided_rows(inp, n_heavy=128, stride=4):
+    """The n_heavy tokens with the largest per-token scale (the most active
+    gates) and every stride-th token."""
+    n = inp.x.shape[0]
+    heavy = np.argsort(-inp.scale)[:n_heavy]
+    return np.unique(np.concatenate([heavy, np.arange(0, n, stride), [n - 1]]))
+
+
+_SWEEP_CACHE = {}
+
+
+def sweep_gate0(inp, rows):
+    """Oracle gate pre-activations of the checked rows with the bias column
+    of W_gate set to zero, shared by the sweep's densities: the inputs differ
+    only in that column (x's last feature is 1.0), and the oracle sums the
+    bias term last, so G(tau) = fl(G0 - tau) bit for bit (pinned on the CPU
+    by tests/test_oracle_pins.py)."""
+    key = tuple(rows[:4]) + (len(rows),)
+    if key not in _SWEEP_CACHE:
+        _SWEEP_CACHE.clear()
+        xf = inp.as_f64("x")[rows]
+        wg0 = inp.as_f64("wg_t").copy()
+        wg0[:, -1] = 0.0
+        _SWEEP_CACHE[key] = (oracle.gate_preact(xf, wg0), np.abs(xf) @ np.abs(wg0).T)
+    return _SWEEP_CACHE[key]

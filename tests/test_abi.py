@@ -121,3 +121,35 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(4, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         sge.twell_gate_pack(x, torch.zeros(128, 64, dtype=torch.bfloat16), 128, 128)
+
+
+def _routed(lib, **kw):
+    p = ctypes.c_void_p(4096)
+    a = dict(x=p, count=p, idx=p, val=p, wu=p, wd=p, ldw=64, wd_t=p, y=p, n=1000, d=64, f=256,
+             tile=128, cap=128, k=16, s_max=64, ws=p, ws_bytes=1 << 40, diag=None, stream=None)
+    a.update(kw)
+    return lib.twell_hybrid_up_down(a["x"], a["count"], a["idx"], a["val"], a["wu"], a["wd"],
+                                    a["ldw"], a["wd_t"], a["y"], a["n"], a["d"], a["f"], a["tile"],
+                                    a["cap"], a["k"], a["s_max"], a["ws"], a["ws_bytes"], a["diag"],
+                                    a["stream"])
+
+
+def test_routed_rejects_bad_arguments(lib):
+    assert _routed(lib, n=0, x=None, ws=None) == 0          # empty input: no-op
+    assert _routed(lib, k=-1) == 1
+    assert b"capacity" in lib.sge_last_error()
+    assert _routed(lib, s_max=-3) == 1
+    assert _routed(lib, k=513) == 2                          # K beyond the light kernel's 512
+    assert _routed(lib, wd_t=None) == 1                      # the spill needs W_down^T
+    assert b"null" in lib.sge_last_error()
+    assert _routed(lib, f=260, tile=20, cap=20) == 1         # F % 8
+    assert _routed(lib, d=60, ldw=64) == 1                   # d % 8
+    need = lib.twell_hybrid_up_down_workspace_bytes(1000, 64, 256, 64)
+    assert _routed(lib, ws_bytes=need - 1) == 1
+    assert b"workspace" in lib.sge_last_error()
+    assert _routed(lib, ws=ctypes.c_void_p(4096 + 128), ws_bytes=need) == 1
+    assert b"aligned" in lib.sge_last_error()
+    # the spill operands grow the workspace with S_max
+    small = lib.twell_hybrid_up_down_workspace_bytes(1000, 64, 256, 0)
+    assert need >= small + 64 * (64 + 2 * 256) * 2
+    assert lib.twell_hybrid_up_down_workspace_bytes(1000, 64, 256, -1) == 0

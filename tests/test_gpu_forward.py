@@ -8,7 +8,8 @@ import activation_sparse_gated_epilogue_b200 as sge
 import oracle
 from activation_sparse_gated_epilogue_b200 import synth
 from tests._util import (BF16_TOL, F32_TOL, FLIP_EPS, assert_twell_equal, check_1b_all_rows,
-                         compare_twell_inexact, oracle_1b, to_f64)
+                         compare_twell_inexact, heavy_and_strided_rows, oracle_1b,
+                         sweep_gate0, to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -381,33 +382,6 @@ def test_e2e_1b_all_rows(cuda_device, interleave):
     print(f"1B: max-abs-rel {err:.2e} on all {cfg.n_tokens} rows, {flips} flips")
 
 
-def heavy_and_strided_rows(inp, n_heavy=128, stride=4):
-    """The n_heavy tokens with the largest per-token scale (the most active
-    gates) and every stride-th token."""
-    n = inp.x.shape[0]
-    heavy = np.argsort(-inp.scale)[:n_heavy]
-    return np.unique(np.concatenate([heavy, np.arange(0, n, stride), [n - 1]]))
-
-
-_SWEEP_CACHE = {}
-
-
-def _sweep_gate0(inp, rows):
-    """Oracle gate pre-activations of the checked rows with the bias column
-    of W_gate set to zero, shared by the sweep's densities: the inputs differ
-    only in that column (x's last feature is 1.0), and the oracle sums the
-    bias term last, so G(tau) = fl(G0 - tau) bit for bit (pinned on the CPU
-    by tests/test_oracle_pins.py)."""
-    key = tuple(rows[:4]) + (len(rows),)
-    if key not in _SWEEP_CACHE:
-        _SWEEP_CACHE.clear()
-        xf = inp.as_f64("x")[rows]
-        wg0 = inp.as_f64("wg_t").copy()
-        wg0[:, -1] = 0.0
-        _SWEEP_CACHE[key] = (oracle.gate_preact(xf, wg0), np.abs(xf) @ np.abs(wg0).T)
-    return _SWEEP_CACHE[key]
-
-
 @pytest.mark.parametrize("rho", [0.0025, 0.005, 0.01, 0.02, 0.05])
 def test_e2e_2b_density_sweep(cuda_device, rho):
     """The 2B workload at each density of the sweep (the heavy tail grows
@@ -422,7 +396,7 @@ def test_e2e_2b_density_sweep(cuda_device, rho):
     _, wu, wd = sge.interleave_up_down(wu, wd)
     y, tw = sge.twell_ffn_forward(x, wg, wu, wd, cfg.tile, cfg.cap)
     torch.cuda.synchronize()
-    g0, abs0 = _sweep_gate0(inp, rows)
+    g0, abs0 = sweep_gate0(inp, rows)
     g = g0 - inp.tau
     tw_ora = oracle.twell_pack(g, cfg.tile, cfg.cap, oracle.VAL_BF16)
     y_ora = oracle.fused_up_down(inp.as_f64("x")[rows], tw_ora, inp.as_f64("wu_t"),
