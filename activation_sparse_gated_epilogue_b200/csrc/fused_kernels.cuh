@@ -113,7 +113,8 @@ constexpr size_t kHdrBytes = 256;
 struct RouteArgs {
   int k;
   int s_max;
-  int light_apart;   // no job lists: tokens not on the spill go to another kernel
+  int light_apart;   // job lists for the light-token kernel: every token not on the
+                     // spill, unsplit, in size classes
   int2* blk_heavy;   // per count block: heavy tokens, their stored entries
   int* spill_rows;   // [s_max]
   int32_t* diag;     // nullable: gains the number of heavy tokens
@@ -357,9 +358,11 @@ static __global__ void __launch_bounds__(256) ud_jobs_kernel(int* __restrict__ n
       ntok[t] = -1;
       n = -1;
     }
-    if (route.light_apart) n = -1;  // every remaining token goes to the light-token kernel
   }
-  const bool split = n > U;
+  // routed calls list every token left off the spill, unsplit, in four size
+  // classes (more than 32, 8, 2 entries, the rest) for the light-token kernel
+  const bool routed_lists = route.k >= 0 && route.light_apart;
+  const bool split = !routed_lists && n > U;
   // split tokens: ceil(n / U) units each
   const int k = split ? (n + U - 1) / U : 0;
   int incl = k;
@@ -377,7 +380,7 @@ static __global__ void __launch_bounds__(256) ud_jobs_kernel(int* __restrict__ n
   }
   ubase = __shfl_sync(0xffffffffu, ubase, 0);
   sbase = __shfl_sync(0xffffffffu, sbase, 0);
-  bool light = n > 0 && n <= U;
+  bool light = n > 0 && (routed_lists || n <= U);
   if (split) {
     const int first = ubase + incl - k;
     const int sid = sbase + __popc(ms & lt);
@@ -400,7 +403,7 @@ static __global__ void __launch_bounds__(256) ud_jobs_kernel(int* __restrict__ n
       done[sid] = 0;
     }
   }
-  const int cls = light ? light_class(n, U) : -1;
+  const int cls = light ? light_class(n, routed_lists ? 64 : U) : -1;
 #pragma unroll
   for (int c = 0; c < kLightClasses; ++c) {
     const unsigned ml = __ballot_sync(0xffffffffu, cls == c);

@@ -197,7 +197,7 @@ constexpr int64_t kSmallGateRows = 256;
 template <int T>
 static int launch_bf16(const void* x, const void* wg_t, int64_t n, int64_t d, int64_t f, int cap,
                        uint8_t* count, uint8_t* idx, void* val, int32_t* diag, cudaStream_t st) {
-  using Shape = TcPairShape<256, 1>;
+  using Shape = TcPairShape<256, 1, 2>;
   CUtensorMap ma, mb;
   int rc = make_tmap_bf16(&ma, x, n, d, d, kBM);
   if (rc) return rc;

@@ -24,7 +24,7 @@
 // kernel; results do not depend on scheduling.  Per row the arithmetic is
 // that of the dense FFN restricted to the stored entries: fp32 accumulation,
 // h rounded to bf16 before the down projection, as in twell_fused_up_down.
-#include <mutex>
+#include <algorithm>
 
 #include "fused_kernels.cuh"
 #include "spill_gemm.cuh"
@@ -32,45 +32,12 @@
 
 namespace sge {
 
-// Exclusive prefix over the first nt (<= 256) capped tile counts of token t,
-// into pre[0 .. nt] (pre[nt] = the token's stored entries), by the `nthr`
-// threads of a group (thread index gt; 128 or 256 threads, which share the
-// named barrier `bar`; wsum holds nthr / 32 ints).  The caller synchronises
-// the group before pre[] is read.
-__device__ __forceinline__ void tile_prefix(const uint8_t* __restrict__ count, int64_t t, int nt, int cap,
-                                            int gt, int nthr, int bar, int* pre, int* wsum) {
-  const int lane = gt & 31, gw = gt >> 5, nw = nthr >> 5;
-  // each thread owns tiles 2 gt and 2 gt + 1 (nt <= 256 = 2 x 128)
-  int c0 = 0, c1 = 0;
-  const int b0 = 2 * gt;
-  if (b0 < nt) c0 = min(static_cast<int>(__ldg(count + t * nt + b0)), cap);
-  if (b0 + 1 < nt) c1 = min(static_cast<int>(__ldg(count + t * nt + b0 + 1)), cap);
-  int incl = c0 + c1;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) wsum[gw] = incl;
-  named_sync(bar, nthr);
-  int base = 0;
-  for (int w = 0; w < gw; ++w) base += wsum[w];
-  const int ex = base + incl - c0 - c1;
-  if (b0 < nt) pre[b0] = ex;
-  if (b0 + 1 < nt) pre[b0 + 1] = ex + c0;
-  if (gt == nthr - 1) {
-    int tot = 0;
-    for (int w = 0; w < nw; ++w) tot += wsum[w];
-    pre[nt] = tot;
-  }
-}
-
 // X_s and A_s rows of the kept spill tokens, a CTA per row (grid-stride over
-// the spill ranks): the x row is copied, the dense row of a is zeroed, then
-// every stored entry is written by its own thread (its tile found by a
-// binary search over the row's tile prefix).
-constexpr int kPrepThreads = 256;
-constexpr int kPrepCtas = 2048;  // about two rows per CTA for the largest spills
+// the spill ranks; CTAs small enough that every row is in flight at once):
+// the x row is copied and the dense row of a zeroed while the tile counts
+// load, then every stored entry is written by its own thread, which finds its
+// tile by a binary search over the row's tile prefix in shared memory.
+constexpr int kPrepThreads = 128;
 
 __global__ void __launch_bounds__(kPrepThreads) spill_prep_kernel(const uint16_t* __restrict__ x,
                                                                   const uint8_t* __restrict__ count,
@@ -84,19 +51,38 @@ __global__ void __launch_bounds__(kPrepThreads) spill_prep_kernel(const uint16_t
                                                                   uint16_t* __restrict__ as) {
   __shared__ int pre[257];
   __shared__ int wsum[kPrepThreads / 32];
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kept = min(*n_heavy, s_max);
   for (int r = blockIdx.x; r < kept; r += gridDim.x) {
     const int64_t t = spill_rows[r];
+    // each thread owns tiles 2 tid and 2 tid + 1 (nt <= 256)
+    const int b0 = 2 * tid;
+    const int c0 = b0 < nt ? min(static_cast<int>(__ldg(count + t * nt + b0)), cap) : 0;
+    const int c1 = b0 + 1 < nt ? min(static_cast<int>(__ldg(count + t * nt + b0 + 1)), cap) : 0;
     const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
     uint4* dst = reinterpret_cast<uint4*>(xs + static_cast<int64_t>(r) * d);
     for (int v = tid; v < d / 8; v += kPrepThreads) dst[v] = __ldg(src + v);
     uint16_t* arow = as + static_cast<int64_t>(r) * f;
     for (int v = tid; v < f / 8; v += kPrepThreads) reinterpret_cast<uint4*>(arow)[v] = make_uint4(0, 0, 0, 0);
-    tile_prefix(count, t, nt, cap, tid, kPrepThreads, 0, pre, wsum);
+    int incl = c0 + c1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int base = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kPrepThreads / 32; ++w) {
+      base += w < warp ? wsum[w] : 0;
+      total += wsum[w];
+    }
+    const int ex = base + incl - c0 - c1;
+    if (b0 < nt) pre[b0] = ex;
+    if (b0 + 1 < nt) pre[b0 + 1] = ex + c0;
     __syncthreads();  // the prefix is complete and the zeros have landed
-    const int n = pre[nt];
-    for (int e = tid; e < n; e += kPrepThreads) {
+    for (int e = tid; e < total; e += kPrepThreads) {
       int b = 0;  // the last tile whose prefix is <= e
       for (int step = 128; step > 0; step >>= 1)
         if (b + step < nt && pre[b + step] <= e) b += step;
@@ -105,28 +91,33 @@ __global__ void __launch_bounds__(kPrepThreads) spill_prep_kernel(const uint16_t
       const int j = b * tile + min(static_cast<int>(__ldg(idx + at)), tile - 1);
       arow[j] = __ldg(val + at);
     }
-    __syncthreads();  // pre[] is rewritten for the next row
+    __syncthreads();  // pre[] and wsum[] are rewritten for the next row
   }
 }
 
 // ------------------------------------------------------ light tokens
 //
-// Every token not on the spill, straight from TwELL.  A group of four
-// warps takes one token at a time (tokens in a static stride over the batch,
-// so no queue); it resolves the token's entries from the tile counts (up to
-// kLightMaxK at a time), then runs them in batches of kLightBatch: the W_up
-// and W_down rows of a batch are loaded together (one memory round trip per
-// batch), u is summed over the group's warps in warp order, h = bf16(a u),
-// and h W_down[j] is accumulated into the fp32 y row held in registers.  The
-// group also stores y = 0 for the tokens of its stride without stored
-// entries.  Light tokens have at most K <= kLightMaxK entries; heavy tokens
-// past S_max (only when the caller's S_max is too small) take as many rounds
-// of kLightMaxK entries as they need.  Few registers and little shared
-// memory per CTA, one CTA per SM: it runs beside the spill GEMMs' CTAs.
-constexpr int kLightBatch = 4;
-constexpr int kLightMaxK = 512;  // the largest K of a routed call
+// Every token not on the spill, straight from TwELL, one warp per token: the
+// warps pull tokens from the planning kernel's size-class lists (largest
+// class first) through a global cursor.  A warp keeps x[t] (bf16) and the
+// fp32 y[t] in registers and streams the token's entries through its own
+// ring of S (2 to 4) shared-memory slots filled by cp.async.bulk: a slot
+// holds an entry's W_up row in its first half and its W_down row in the
+// second (one 8 KB copy when the caller interleaves the two matrices row by
+// row with rows of a multiple of 512 bytes, two copies otherwise).  Per
+// entry: u = x . W_up[:, j] (exact bf16 products, fp32 sums, reduced over the
+// lanes), h = bf16(a u), y += h W_down[j].  Entries are resolved from the
+// tile counts 32 at a time, one round ahead of the copies.  The warps first
+// store y = 0 for the tokens without stored entries, each an equal share of
+// the batch.  Light tokens have at most K entries; heavy tokens past S_max
+// (when the caller's S_max is too small) take the same path, entry by
+// entry.  Every wait is bounded: a wait that runs out sets SGE_FLAG_TIMEOUT
+// and stops the CTA after its copies in flight have landed.
+constexpr int kRingMaxWarps = 8;
+constexpr int kRingMaxSlots = 4;
+constexpr int kRingSmem = 220 * 1024;  // slots of all warps
 
-struct LightParams {
+struct RingParams {
   const uint16_t* x;
   const uint8_t* count;
   const uint8_t* idx;
@@ -136,113 +127,202 @@ struct LightParams {
   int64_t w_ld;
   uint16_t* y;
   const int* ntok;
+  const int* hdr;       // job counts per class (kHLight), cursor (kHCursor)
+  int* cursor;
+  const int2* lights;   // [kLightClasses][n_rows]: (token, entries)
+  int32_t* diag;
   int64_t n_rows;
-  int d, nt, tile, cap, k;
+  int nt, tile, cap;
+  int row_bytes;   // d * 2
+  int slot_bytes;  // two halves of NV * 512 bytes
+  int slots;       // S, slots per warp
+  int w_one;       // one copy brings both rows of an entry
 };
 
-// Registers per thread: with G groups of 128 threads the CTA stays within
-// the 64 K registers an SM has minus the ~15 K of a spill GEMM CTA.
-template <int G>
-struct LightRegs {
-  static constexpr int kMax = G >= 3 ? 128 : 192;
-};
-
-template <int NV, int G>
-__global__ void __launch_bounds__(G * 128) __maxnreg__(LightRegs<G>::kMax)
-    light_fwd_kernel(const LightParams p) {
+template <int NV, int NTR>
+__global__ void __launch_bounds__(kRingMaxWarps * 32, 1) light_ring_kernel(const RingParams p) {
   using E = Elem<true>;
-  constexpr int VEC = E::VEC;
-  __shared__ int s_pre[G][257];
-  __shared__ int s_wsum[G][4];
-  __shared__ int s_j[G][kLightMaxK];
-  __shared__ float s_a[G][kLightMaxK];
-  __shared__ float s_part[G][4][kLightBatch];
-  __shared__ uint16_t s_h[G][kLightBatch];
-  const int g = threadIdx.x >> 7, gt = threadIdx.x & 127, lane = gt & 31, gw = gt >> 5;
-  const int nvec = p.d / VEC;
-  const int64_t groups = static_cast<int64_t>(gridDim.x) * G;
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * G + g; t < p.n_rows; t += groups) {
-    const int n = p.ntok[t];
-    uint4* yrow = reinterpret_cast<uint4*>(p.y + t * p.d);
-    if (n == 0) {
-      for (int v = gt; v < nvec; v += 128) yrow[v] = make_uint4(0, 0, 0, 0);
-      continue;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5, S = p.slots;
+  const int half = p.slot_bytes / 2;
+  uint8_t* ring = smem + warp * S * p.slot_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + warps * S * p.slot_bytes);
+  uint64_t* full = bars + warp * S;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + warps * S);
+  const int pieces = p.row_bytes / 16;
+
+  // slot bytes past a row stay zero for the whole kernel (loads need no test)
+  if (p.row_bytes < half)
+    for (int q = 0; q < 2 * S; ++q)
+      for (int o = p.row_bytes + lane * 16; o < half; o += 32 * 16)
+        *reinterpret_cast<uint4*>(ring + q * half + o) = make_uint4(0, 0, 0, 0);
+  if (lane == 0)
+    for (int q = 0; q < S; ++q) mbar_init(full + q, 1);
+  if (threadIdx.x == 0) *abort_flag = 0;
+  fence_mbar_init();
+  __syncthreads();
+
+  // y = 0 for the tokens without stored entries, an equal share per warp
+  {
+    const int64_t gw = static_cast<int64_t>(blockIdx.x) * warps + warp;
+    const int64_t ngw = static_cast<int64_t>(gridDim.x) * warps;
+    const int64_t per = (p.n_rows + ngw - 1) / ngw;
+    const int64_t t0 = gw * per, t1 = min(p.n_rows, t0 + per);
+    for (int64_t tb = t0; tb < t1; tb += 32) {
+      unsigned m = __ballot_sync(0xffffffffu, tb + lane < t1 && p.ntok[tb + lane] == 0);
+      while (m) {
+        const int i = __ffs(m) - 1;
+        m &= m - 1;
+        uint4* row = reinterpret_cast<uint4*>(p.y + (tb + i) * (p.row_bytes / 2));
+        for (int pc = lane; pc < pieces; pc += 32) row[pc] = make_uint4(0, 0, 0, 0);
+      }
     }
-    if (n < 0) continue;  // spill token
-    uint4 xv[NV];
-    const uint4* xrow = reinterpret_cast<const uint4*>(p.x + t * p.d);
+  }
+  int n_light[kLightClasses];
 #pragma unroll
-    for (int k = 0; k < NV; ++k) {
-      const int v = gt + k * 128;
-      xv[k] = v < nvec ? __ldg(xrow + v) : make_uint4(0, 0, 0, 0);
+  for (int c = 0; c < kLightClasses; ++c) n_light[c] = p.hdr[kHLight + c];
+
+  uint32_t parity = 0;  // bit q: phase parity of slot q's next completion
+  bool ok = true;
+  int issued_total = 0, consumed_total = 0;  // copies issued / consumed by this warp
+  while (ok) {
+    // ---- next token (largest class first)
+    int k = 0;
+    if (lane == 0) k = atomicAdd(p.cursor, 1);
+    k = __shfl_sync(0xffffffffu, k, 0);
+    int t = -1, n = 0;
+#pragma unroll
+    for (int c = 0; c < kLightClasses; ++c) {
+      if (t < 0 && k < n_light[c]) {
+        const int2 j = p.lights[c * p.n_rows + k];
+        t = j.x;
+        n = j.y;
+      }
+      k -= n_light[c];
     }
-    tile_prefix(p.count, t, p.nt, p.cap, gt, 128, 1 + g, s_pre[g], s_wsum[g]);
-    float acc[NV][VEC];
+    if (t < 0) break;
+    // ---- x row and the tile prefix of the token's counts
+    uint4 xr[NV];
+    const uint4* xrow = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(t) * (p.row_bytes / 2));
 #pragma unroll
-    for (int k = 0; k < NV; ++k)
+    for (int q = 0; q < NV; ++q) {
+      const int pc = lane + 32 * q;
+      xr[q] = pc < pieces ? __ldg(xrow + pc) : make_uint4(0, 0, 0, 0);
+    }
+    int pre[NTR];
+    {
+      const uint8_t* cnt = p.count + static_cast<int64_t>(t) * p.nt;
+      int c[NTR];
 #pragma unroll
-      for (int q = 0; q < VEC; ++q) acc[k][q] = 0.0f;
-    for (int c0 = 0; c0 < n; c0 += kLightMaxK) {
-    const int cn = min(kLightMaxK, n - c0);  // entries of this round
-    named_sync(1 + g, 128);  // the prefix (first round) or the last round's batches are done
-    for (int e = gt; e < cn; e += 128) {
-      const int eg = c0 + e;
+      for (int r = 0; r < NTR; ++r) {
+        const int b = lane + 32 * r;
+        c[r] = b < p.nt ? min(static_cast<int>(__ldg(cnt + b)), p.cap) : 0;
+      }
+      int carry = 0;
+#pragma unroll
+      for (int r = 0; r < NTR; ++r) {
+        int incl = c[r];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        pre[r] = carry + incl - c[r];
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+      }
+    }
+    // entry e of round e / 32 lives in lane e % 32: its column and raw value
+    auto resolve = [&](int round, int& jcol, uint32_t& araw) {
+      const int e = round * 32 + lane;
+      jcol = 0;
+      araw = 0;
       int b = 0;
-      for (int step = 128; step > 0; step >>= 1)
-        if (b + step < p.nt && s_pre[g][b + step] <= eg) b += step;
-      const int64_t at = (t * p.nt + b) * p.cap + (eg - s_pre[g][b]);
-      s_j[g][e] = b * p.tile + min(static_cast<int>(__ldg(p.idx + at)), p.tile - 1);
-      s_a[g][e] = E::from_raw(__ldg(p.val + at));
-    }
-    named_sync(1 + g, 128);
-    for (int e0 = 0; e0 < cn; e0 += kLightBatch) {
-      uint4 wu[kLightBatch][NV], wdv[kLightBatch][NV];
 #pragma unroll
-      for (int u = 0; u < kLightBatch; ++u) {
-        const int e = e0 + u;
-        const int j = e < cn ? s_j[g][e] : 0;
-        const uint4* ur = reinterpret_cast<const uint4*>(p.wu + static_cast<int64_t>(j) * p.w_ld);
-        const uint4* dr = reinterpret_cast<const uint4*>(p.wd + static_cast<int64_t>(j) * p.w_ld);
+      for (int step = 16 * NTR; step > 0; step >>= 1) {
+        const int cand = b + step;
+        const int v = prefix_at<NTR>(pre, cand < p.nt ? cand : 0);
+        if (cand < p.nt && v <= e) b = cand;
+      }
+      const int s = e - prefix_at<NTR>(pre, b);
+      if (e < n) {
+        const int64_t at = (static_cast<int64_t>(t) * p.nt + b) * p.cap + s;
+        jcol = b * p.tile + min(static_cast<int>(__ldg(p.idx + at)), p.tile - 1);
+        araw = __ldg(p.val + at);
+      }
+    };
+    int cur_j, nxt_j;
+    uint32_t cur_a, nxt_a;
+    resolve(0, cur_j, cur_a);
+    resolve(1, nxt_j, nxt_a);
+    // ---- the ring: entry e goes to slot (first + e) % S
+    const int first = issued_total % S;
+    float acc[NV][8];
 #pragma unroll
-        for (int k = 0; k < NV; ++k) {
-          const int v = gt + k * 128;
-          const bool in = e < cn && v < nvec;
-          wu[u][k] = in ? __ldg(ur + v) : make_uint4(0, 0, 0, 0);
-          wdv[u][k] = in ? __ldg(dr + v) : make_uint4(0, 0, 0, 0);
+    for (int q = 0; q < NV; ++q)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[q][i] = 0.0f;
+    // copies of the first min(n, slots) entries
+    int round_base = 0;  // first entry of the round held in cur_*
+    int next_issue = 0;
+    auto issue_next = [&]() {
+      const int e = next_issue;
+      const int jc = __shfl_sync(0xffffffffu, e - round_base < 32 ? cur_j : nxt_j, e & 31);
+      if (lane == 0) {
+        const int q = (first + e) % S;
+        uint8_t* dst = ring + q * p.slot_bytes;
+        fence_proxy_async_smem();  // the slot's earlier reads come before the copy
+        mbar_arrive_expect_tx(full + q, 2 * static_cast<uint32_t>(p.row_bytes));
+        if (p.w_one) {
+          bulk_load(dst, p.wu + static_cast<int64_t>(jc) * p.w_ld, 2 * p.row_bytes, full + q);
+        } else {
+          bulk_load(dst, p.wu + static_cast<int64_t>(jc) * p.w_ld, p.row_bytes, full + q);
+          bulk_load(dst + half, p.wd + static_cast<int64_t>(jc) * p.w_ld, p.row_bytes, full + q);
         }
       }
-      float part[kLightBatch];
+      ++next_issue;
+      ++issued_total;
+    };
+    while (next_issue < n && next_issue < S) issue_next();
+    for (int e = 0; e < n; ++e) {
+      const int q = (first + e) % S;
+      const float a = E::from_raw(__shfl_sync(0xffffffffu, cur_a, e & 31));
+      if (!(ok = ud_wait_or_abort(full + q, (parity >> q) & 1u, abort_flag, p.diag))) break;
+      parity ^= 1u << q;
+      ++consumed_total;
+      const uint32_t sa = smem_u32(ring + q * p.slot_bytes);
+      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int u = 0; u < kLightBatch; ++u) {
-        float s = 0.0f;
+      for (int k2 = 0; k2 < NV; ++k2)
+        E::dot2(xr[k2], lds128(sa + (lane + 32 * k2) * 16), s8[2 * (k2 & 3)], s8[2 * (k2 & 3) + 1]);
+      float u = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
 #pragma unroll
-        for (int k = 0; k < NV; ++k) s = E::dot(xv[k], wu[u][k], s);
-        part[u] = s;
+      for (int o = 16; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
+      const uint16_t h = E::h_of(a * u);
+#pragma unroll
+      for (int k2 = 0; k2 < NV; ++k2) E::axpy(h, lds128(sa + half + (lane + 32 * k2) * 16), acc[k2]);
+      __syncwarp();  // every lane has read the slot
+      if ((e & 31) == 31) {  // the next round becomes current; resolve the one after
+        cur_j = nxt_j;
+        cur_a = nxt_a;
+        round_base += 32;
+        resolve((e >> 5) + 2, nxt_j, nxt_a);
       }
-      const float tot = warp_reduce_multi<kLightBatch>(part, lane);
-      if ((lane & (32 / kLightBatch - 1)) == 0) s_part[g][gw][multi_entry<kLightBatch>(lane)] = tot;
-      named_sync(1 + g, 128);
-      if (gt < kLightBatch) {
-        const int e = e0 + gt;
-        // u summed over the group's warps in warp order
-        const float u = ((s_part[g][0][gt] + s_part[g][1][gt]) + s_part[g][2][gt]) + s_part[g][3][gt];
-        s_h[g][gt] = e < cn ? E::h_of(s_a[g][e] * u) : 0;
-      }
-      named_sync(1 + g, 128);
-#pragma unroll
-      for (int u = 0; u < kLightBatch; ++u) {
-        const uint16_t hb = s_h[g][u];
-#pragma unroll
-        for (int k = 0; k < NV; ++k) E::axpy(hb, wdv[u][k], acc[k]);
-      }
+      if (next_issue < n) issue_next();
     }
-    }
+    if (!ok) break;
+    uint4* yrow = reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(t) * (p.row_bytes / 2));
 #pragma unroll
-    for (int k = 0; k < NV; ++k) {
-      const int v = gt + k * 128;
-      if (v < nvec) yrow[v] = E::pack(acc[k]);
+    for (int q = 0; q < NV; ++q) {
+      const int pc = lane + 32 * q;
+      if (pc < pieces) yrow[pc] = E::pack(acc[q]);
     }
-    named_sync(1 + g, 128);  // s_pre / s_j / s_h are rewritten for the next token
+  }
+  // copies still in flight (only after a give-up) land before the CTA exits
+  for (int i = consumed_total; i < issued_total; ++i) {
+    const int q = i % S;
+    mbar_wait(full + q, (parity >> q) & 1u, p.diag);
+    parity ^= 1u << q;
   }
 }
 
@@ -269,64 +349,45 @@ struct RoutedLayout {
   }
 };
 
-template <int NV, int G>
-static int launch_light(const LightParams& p, cudaStream_t st) {
-  // kernels beside the spill GEMMs ask for the largest shared-memory
-  // carveout: an SM configured for a small one cannot take a GEMM CTA (about
-  // 197 KB) until it has drained
-  const int rc = prefer_max_shared(reinterpret_cast<const void*>(light_fwd_kernel<NV, G>));
+template <int NV, int NTR>
+static int launch_ring(const RingParams& p, int warps, int smem, cudaStream_t st) {
+  auto kern = light_ring_kernel<NV, NTR>;
+  const int rc = set_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (rc) return rc;
-  light_fwd_kernel<NV, G><<<sm_count(), G * 128, 0, st>>>(p);
+  kern<<<sm_count(), warps * 32, smem, st>>>(p);
   return check_launch("twell_hybrid_up_down (light tokens)");
 }
 
-static int launch_light_nv(const LightParams& p, cudaStream_t st) {
-  const int nvec = p.d / 8;
-  if (nvec <= 128) return launch_light<1, 3>(p, st);
-  if (nvec <= 256) return launch_light<2, 3>(p, st);
-  if (nvec <= 384) return launch_light<3, 2>(p, st);
-  return launch_light<4, 2>(p, st);
+template <int NV>
+static int ring_ntr(const RingParams& p, int warps, int smem, cudaStream_t st) {
+  if (p.nt <= 32) return launch_ring<NV, 1>(p, warps, smem, st);
+  if (p.nt <= 64) return launch_ring<NV, 2>(p, warps, smem, st);
+  if (p.nt <= 128) return launch_ring<NV, 4>(p, warps, smem, st);
+  return launch_ring<NV, 8>(p, warps, smem, st);
 }
 
-// The light-token kernel runs on a stream of the library's own, beside the
-// spill work on the caller's stream: the caller's stream forks into it after
-// planning and joins it before the call's last kernel.  One such stream and
-// its two events per device and context, created on first use; the mutex
-// keeps the record / wait sequences of concurrent calls apart.
-namespace {
-constexpr int kMaxDevices = 64;
-struct SideStream {
-  CUcontext ctx = nullptr;
-  cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
-};
-SideStream g_side[kMaxDevices];
-std::mutex g_side_mutex;
-
-int side_stream(SideStream** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "twell_hybrid_up_down: %s", cudaGetErrorString(e));
-  if (dev < 0 || dev >= kMaxDevices)
-    return fail(SGE_ERR_UNSUPPORTED, "twell_hybrid_up_down: device %d beyond %d", dev, kMaxDevices);
-  CUcontext ctx = nullptr;
-  if (current_context(&ctx) != CUDA_SUCCESS || !ctx)
-    return fail(SGE_ERR_CUDA, "twell_hybrid_up_down: no current CUDA context");
-  SideStream& sd = g_side[dev];
-  if (sd.ctx != ctx) {  // first use, or a new context (the old handles died with the old one)
-    sd = SideStream{};
-    if ((e = cudaStreamCreateWithFlags(&sd.s, cudaStreamNonBlocking)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming)) != cudaSuccess ||
-        (e = cudaEventCreateWithFlags(&sd.join, cudaEventDisableTiming)) != cudaSuccess) {
-      sd = SideStream{};
-      return fail(SGE_ERR_CUDA, "twell_hybrid_up_down: side stream: %s", cudaGetErrorString(e));
-    }
-    sd.ctx = ctx;
+// The light-token kernel: slots of two halves of nv * 512 bytes, as many
+// warps (at most kRingMaxWarps) and slots (2 to kRingMaxSlots, 3 preferred)
+// as the shared memory holds.
+static int run_ring(RingParams p, int nv, cudaStream_t st) {
+  p.slot_bytes = 2 * nv * 512;
+  int warps = kRingMaxWarps, slots = 3;
+  while (warps * slots * p.slot_bytes > kRingSmem) {
+    if (slots > 2) --slots;
+    else --warps;
   }
-  *out = &sd;
-  return SGE_OK;
+  if (warps < 1) return fail(SGE_ERR_UNSUPPORTED, "twell_hybrid_up_down: rows of %d bytes", p.row_bytes);
+  p.slots = slots;
+  p.w_one = p.w_one && 2 * p.row_bytes == p.slot_bytes;
+  const int smem = warps * slots * p.slot_bytes + warps * slots * 8 + 16;
+  switch (nv) {
+    case 2: return ring_ntr<2>(p, warps, smem, st);
+    case 4: return ring_ntr<4>(p, warps, smem, st);
+    case 8: return ring_ntr<8>(p, warps, smem, st);
+    case 12: return ring_ntr<12>(p, warps, smem, st);
+    default: return ring_ntr<16>(p, warps, smem, st);
+  }
 }
-}  // namespace
 
 }  // namespace sge
 
@@ -351,8 +412,6 @@ extern "C" int twell_hybrid_up_down(const void* x, const uint8_t* count, const u
   if (ell_cap < 0 || s_max < 0)
     return fail(SGE_ERR_ARG, "%s: negative ELL capacity K (%d) or spill capacity S_max (%d)", kName,
                 ell_cap, s_max);
-  if (ell_cap > kLightMaxK)
-    return fail(SGE_ERR_UNSUPPORTED, "%s: ELL capacity K = %d beyond %d", kName, ell_cap, kLightMaxK);
   if (d_ff % 8) return fail(SGE_ERR_ARG, "%s: d_ff %% 8 != 0", kName);
   if (n_tokens == 0) return SGE_OK;
   if (!x || !count || !idx || !val || !wu_t || !wd || !y || !workspace || (s_max > 0 && !wd_t))
@@ -376,9 +435,6 @@ extern "C" int twell_hybrid_up_down(const void* x, const uint8_t* count, const u
     if ((rc = fused_launch_plan(c, no_route(), st))) return rc;
     return fused_launch_main(c, st);
   }
-  SideStream* side = nullptr;
-  if ((rc = side_stream(&side))) return rc;
-  if ((rc = prefer_max_shared(reinterpret_cast<const void*>(spill_prep_kernel)))) return rc;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int* spill_rows = reinterpret_cast<int*>(ws + L.rows);
   int* n_heavy = c.prm.hdr + kHHeavy;
@@ -388,45 +444,35 @@ extern "C" int twell_hybrid_up_down(const void* x, const uint8_t* count, const u
   const RouteArgs route{ell_cap, s_max, 1, reinterpret_cast<int2*>(ws + L.heavy), spill_rows, diag};
   if ((rc = fused_launch_plan(c, route, st))) return rc;
 
+  // the light tokens, then the spill
   const int f = static_cast<int>(d_ff), d = static_cast<int>(d_model);
-  LightParams lp{static_cast<const uint16_t*>(x), count, idx, static_cast<const uint16_t*>(val),
-                 static_cast<const char*>(wu_t), static_cast<const char*>(wd), ldw * 2,
-                 static_cast<uint16_t*>(y), c.prm.ntok, n_tokens, d, f / tile, tile, cap, ell_cap};
-  std::lock_guard<std::mutex> lock(g_side_mutex);
-  cudaError_t e = cudaEventRecord(side->fork, st);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
-  if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "%s: fork: %s", kName, cudaGetErrorString(e));
-  rc = launch_light_nv(lp, side->s);
-  e = cudaEventRecord(side->join, side->s);  // recorded even after a failed launch
-  if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "%s: join: %s", kName, cudaGetErrorString(e));
-
-  // the spill on the caller's stream, beside the light tokens
-  if (!rc) {
-    const int prep_grid = s_max < kPrepCtas ? s_max : kPrepCtas;
+  RingParams rp{static_cast<const uint16_t*>(x), count, idx, static_cast<const uint16_t*>(val),
+                static_cast<const char*>(wu_t), static_cast<const char*>(wd), ldw * 2,
+                static_cast<uint16_t*>(y), c.prm.ntok, c.prm.hdr, c.prm.hdr + kHCursor, c.prm.lights,
+                diag, n_tokens, f / tile, tile, cap, d * 2, 0, 0, 0};
+  // one copy per entry when each wd row directly follows its wu_t row
+  // (run_ring also needs a row to fill half a slot exactly)
+  rp.w_one = static_cast<const char*>(wd) == static_cast<const char*>(wu_t) + 2 * d_model &&
+             ldw == 2 * d_model;
+  if ((rc = run_ring(rp, c.nv, st))) return rc;
+  {
+    const int prep_grid = static_cast<int>(std::min<int64_t>(s_max, 16 * static_cast<int64_t>(sm_count())));
     spill_prep_kernel<<<prep_grid, kPrepThreads, 0, st>>>(
         static_cast<const uint16_t*>(x), count, idx, static_cast<const uint16_t*>(val), spill_rows,
         n_heavy, s_max, d, f, f / tile, tile, cap, xs, as);
-    rc = check_launch("twell_hybrid_up_down (spill prep)");
+    if ((rc = check_launch("twell_hybrid_up_down (spill prep)"))) return rc;
   }
-  using S = TcPairShape<kSpillBN, 1>;
+  using S = TcPairShape<kSpillBN, 1, 2>;
   CUtensorMap ma, mb, mh, md;
-  if (!rc) rc = make_tmap_bf16(&ma, xs, s_max, d_model, d_model, kBM);
-  if (!rc) rc = make_tmap_bf16(&mb, wu_t, d_ff, d_model, ldw, S::BN / 2);
-  if (!rc) {
-    EpiSpillUp e1{as, nullptr, hs, n_heavy, s_max, f};
-    rc = launch_tc_gemm_pair<S>(ma, mb, mb, s_max, d_ff, d_model, e1, diag, st,
-                                "twell_hybrid_up_down (spill up)");
-  }
-  if (!rc) rc = make_tmap_bf16(&mh, hs, s_max, d_ff, d_ff, kBM);
-  if (!rc) rc = make_tmap_bf16(&md, wd_t, d_model, d_ff, d_ff, S::BN / 2);
-  if (!rc) {
-    EpiScatterRows e2{static_cast<uint16_t*>(y), spill_rows, n_heavy, s_max, d};
-    rc = launch_tc_gemm_pair<S>(mh, md, md, s_max, d_model, d_ff, e2, diag, st,
+  if ((rc = make_tmap_bf16(&ma, xs, s_max, d_model, d_model, kBM))) return rc;
+  if ((rc = make_tmap_bf16(&mb, wu_t, d_ff, d_model, ldw, S::BN / 2))) return rc;
+  EpiSpillUp e1{as, nullptr, hs, n_heavy, s_max, f};
+  if ((rc = launch_tc_gemm_pair<S>(ma, mb, mb, s_max, d_ff, d_model, e1, diag, st,
+                                   "twell_hybrid_up_down (spill up)")))
+    return rc;
+  if ((rc = make_tmap_bf16(&mh, hs, s_max, d_ff, d_ff, kBM))) return rc;
+  if ((rc = make_tmap_bf16(&md, wd_t, d_model, d_ff, d_ff, S::BN / 2))) return rc;
+  EpiScatterRows e2{static_cast<uint16_t*>(y), spill_rows, n_heavy, s_max, d};
+  return launch_tc_gemm_pair<S>(mh, md, md, s_max, d_model, d_ff, e2, diag, st,
                                 "twell_hybrid_up_down (spill down)");
-  }
-  // join: the caller's stream continues once the light tokens are done too
-  e = cudaStreamWaitEvent(st, side->join, 0);
-  if (rc) return rc;
-  if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "%s: join: %s", kName, cudaGetErrorString(e));
-  return SGE_OK;
 }

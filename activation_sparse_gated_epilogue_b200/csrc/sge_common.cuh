@@ -195,12 +195,6 @@ SGE_DEV uint16_t f32_to_bf16_bits(float v) {
   return *reinterpret_cast<uint16_t*>(&b);
 }
 
-// Barrier `id` (0..15) among `nthreads` threads of the CTA (a multiple of 32;
-// id 0 with the whole CTA is __syncthreads).
-SGE_DEV void named_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 SGE_DEV bool elect_one_sync() {
   uint32_t pred = 0;
   asm volatile(

@@ -2,14 +2,15 @@
 // (both operands K-major bf16, fp32 accumulation in tensor memory), with a
 // pluggable epilogue that reads the accumulator tile straight out of TMEM.
 //
-// One CTA per SM (192 threads, 6 warps), looping over output tiles:
+// One CTA per SM (6 or 10 warps), looping over output tiles:
 //   warp 0      TMA producer: A and B tiles (128-byte swizzle) into a ring of
 //               STAGES shared-memory stages, completion on `full` mbarriers.
 //   warp 1      TMEM allocator and MMA issuer: one elected thread issues
 //               tcgen05.mma (M = 128, N = BN, K = 16 per instruction) and
 //               releases each stage with tcgen05.commit -> `empty`.
-//   warps 2..5  epilogue: tcgen05.ld of the tile (thread i of warp w holds
-//               accumulator row 32*(w%4) + i), then the Epilogue functor.
+//   warps 2..    epilogue: tcgen05.ld of the tile (thread i of warp w holds
+//               accumulator row 32*(w%4) + i), then the Epilogue functor;
+//               4 warps, or 8 with the tile's columns in two halves.
 // The accumulator is double-buffered in TMEM so the epilogue of one tile
 // overlaps the main loop of the next.  With NB = 2 the engine multiplies A
 // by two B matrices at once into two accumulators (gate and up projections
@@ -30,12 +31,17 @@ namespace sge {
 
 constexpr int kBM = 128;  // UMMA M: rows of A per tile = TMEM lanes
 constexpr int kBK = 64;   // K per stage: one 128-byte swizzle row of bf16
-constexpr int kGemmThreads = 192;
 
-template <int BN_, int NB_>
+// Epilogue warps: 4 x HALVES.  With HALVES = 2 two warps share each TMEM
+// lane quarter and each takes half the tile's columns (the epilogue is then
+// called with BN / 2 columns); two-accumulator tiles (NB = 2) keep HALVES = 1.
+template <int BN_, int NB_, int HALVES_ = 1>
 struct TcShape {
   static constexpr int BN = BN_;
   static constexpr int NB = NB_;
+  static constexpr int HALVES = HALVES_;
+  static constexpr int THREADS = 64 + 128 * HALVES;
+  static_assert(HALVES == 1 || (HALVES == 2 && NB == 1), "column halves need one accumulator");
   static constexpr int A_BYTES = kBM * kBK * 2;
   static constexpr int B_BYTES = BN * kBK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + NB * B_BYTES;
@@ -137,7 +143,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
 }
 
 template <class Shape, class Epilogue>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(Shape::THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                    const __grid_constant__ CUtensorMap map_b0,
                    const __grid_constant__ CUtensorMap map_b1, int M, int N, int K,
@@ -168,7 +174,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tmem_full[a], 1);
-      mbar_init(&tmem_empty[a], 4);
+      mbar_init(&tmem_empty[a], 4 * Shape::HALVES);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -263,6 +269,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // --------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int half = (warp - 2) >> 2;  // column half (HALVES = 2)
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = it & 1;
@@ -270,9 +277,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const TileCoord tc = tile_coord(tile, m_blocks);
-      const uint32_t taddr = tmem_base + acc * Shape::ACC_COLS + (static_cast<uint32_t>(quarter * 32) << 16);
+      const uint32_t taddr = tmem_base + acc * Shape::ACC_COLS + half * (BN / Shape::HALVES) +
+                             (static_cast<uint32_t>(quarter * 32) << 16);
       const int64_t row = static_cast<int64_t>(tc.m_blk) * kBM + quarter * 32 + lane;
-      epi.template run<BN>(taddr, row, tc.n_blk, lane);
+      epi.template run<BN / Shape::HALVES>(taddr, row, tc.n_blk * Shape::HALVES + half, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tmem_empty[acc]);
@@ -298,10 +306,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // epilogue drains its own TMEM and releases the accumulator on the leader's
 // `tmem_empty` barrier (count 8: four warps in each CTA).  Per SM this moves
 // half the B bytes of the single-CTA engine for the same work.
-template <int BN_, int NB_>
+template <int BN_, int NB_, int HALVES_ = 1>
 struct TcPairShape {
   static constexpr int BN = BN_;  // N of one MMA (both CTAs together)
   static constexpr int NB = NB_;
+  static constexpr int HALVES = HALVES_;
+  static constexpr int THREADS = 64 + 128 * HALVES;
+  static_assert(HALVES == 1 || (HALVES == 2 && NB == 1), "column halves need one accumulator");
   static constexpr int BM = 2 * kBM;
   static constexpr int A_BYTES = kBM * kBK * 2;
   static constexpr int B_BYTES = (BN / 2) * kBK * 2;  // this CTA's half
@@ -316,7 +327,7 @@ struct TcPairShape {
 };
 
 template <class Shape, class Epilogue>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(Shape::THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
                         const __grid_constant__ CUtensorMap map_b0,
                         const __grid_constant__ CUtensorMap map_b1, int M, int N, int K,
@@ -355,7 +366,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tmem_full[a], 1);
-      mbar_init(&tmem_empty[a], 8);
+      mbar_init(&tmem_empty[a], 8 * Shape::HALVES);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -453,6 +464,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // --------------------------------------------------------- epilogue
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;  // column half (HALVES = 2)
     const uint32_t leader_tmem_empty0 = mapa_shared(smem_u32(&tmem_empty[0]), 0);
     int it = 0;
     for (int tile = pair; tile < num_tiles; tile += n_pairs, ++it) {
@@ -461,9 +473,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const TileCoord tc = tile_coord(tile / nsplit, m_blocks);
-      const uint32_t taddr = tmem_base + acc * Shape::ACC_COLS + (static_cast<uint32_t>(quarter * 32) << 16);
+      const uint32_t taddr = tmem_base + acc * Shape::ACC_COLS + half * (BN / Shape::HALVES) +
+                             (static_cast<uint32_t>(quarter * 32) << 16);
       const int64_t row = static_cast<int64_t>(tc.m_blk) * Shape::BM + rank * kBM + quarter * 32 + lane;
-      epi_run_impl<BN>(epi, taddr, row, tc.n_blk, tile % nsplit, nsplit, lane, 0);
+      epi_run_impl<BN / Shape::HALVES>(epi, taddr, row, tc.n_blk * Shape::HALVES + half, tile % nsplit,
+                                       nsplit, lane, 0);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tmem_empty0 + acc * 8);

@@ -15,7 +15,7 @@ int launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensor
   if (rc) return rc;
   const int64_t tiles = ((m + kBM - 1) / kBM) * ((n + Shape::BN - 1) / Shape::BN);
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  kern<<<grid, kGemmThreads, Shape::SMEM_BYTES, st>>>(ma, mb0, mb1, static_cast<int>(m),
+  kern<<<grid, Shape::THREADS, Shape::SMEM_BYTES, st>>>(ma, mb0, mb1, static_cast<int>(m),
                                                       static_cast<int>(n), static_cast<int>(k), epi,
                                                       diag);
   return check_launch(what);
@@ -29,7 +29,7 @@ int max_resident_pairs() {
   auto kern = tc_gemm_pair_kernel<Shape, Epi>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * (sm_count() / 2));
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(Shape::THREADS);
   cfg.dynamicSmemBytes = Shape::SMEM_BYTES;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -60,7 +60,7 @@ int launch_tc_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb0, const CUt
   const int pairs = static_cast<int>(tiles < resident ? tiles : resident);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(Shape::THREADS);
   cfg.dynamicSmemBytes = Shape::SMEM_BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];

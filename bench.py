@@ -4,7 +4,7 @@
 
 One step = one pass of the whole sparse inference path over one batch: the
 gate GEMM with the TwELL epilogue (twell_gate_pack), then the up and down
-projections from TwELL (twell_hybrid_up_down: tokens with at most K = 32
+projections from TwELL (twell_hybrid_up_down: tokens with at most K = 16
 stored entries through a CUDA-core kernel beside the heavier ones, which run
 through two tcgen05 spill GEMMs), on the 1B-shaped bf16
 workload (N=8192 tokens, d=2048, F=8192, T=C=128, mean gate density 1%,
@@ -46,9 +46,8 @@ FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # stored entries run on the tensor-core spill GEMMs)
 HYB_INFER_K = 64
 # K of the routed step: tokens with more stored entries take the spill GEMMs
-# (measured at the 1B shape: K = 16 / 32 / 64 give 0.186 / 0.185 / 0.197 ms
-# for the call)
-ROUTED_K = 32
+# (measured at the 1B shape: K = 16 / 32 gives 0.178 / 0.188 ms for the call)
+ROUTED_K = 16
 
 # DRAM bytes (read + write) per launch from ncu captures of the kernels,
 # keyed by the hash of the source they were taken on; a kernel whose source

@@ -210,11 +210,11 @@ int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, const uint8
  * ascending token order and the first S_max = s_max of them run as two
  * tcgen05 GEMMs over all F hidden units (U = X_s W_up with an epilogue
  * forming h = bf16(a u), zero where the TwELL stores no entry; then
- * Y_s = H_s W_down scattered into y).  The light tokens run on CUDA cores
- * at the same time, on a stream the library keeps per device (forked from
- * and joined back into `stream` within the call); heavy tokens past S_max
- * run through the per-entry kernel of twell_fused_up_down afterwards; no
- * token is dropped.  Batches of at most 64 tokens,
+ * Y_s = H_s W_down scattered into y).  Every other token (light, or heavy
+ * past S_max) runs on CUDA cores first, one warp per token streaming its
+ * entries' W_up and W_down rows through shared memory; no token is dropped
+ * (heavy tokens past S_max are slow on that path: size S_max for the heavy
+ * tokens expected).  Batches of at most 64 tokens,
  * and s_max = 0, run the per-entry path for every token (a spill GEMM would
  * stream all of W_up and W_down for a few rows).  No ELL repack and nothing
  * saved for a backward pass (hybrid_pack / hybrid_ffn_fwd do that).
@@ -228,7 +228,7 @@ int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, const uint8
  *   wd_t [d][F]          bf16  W_down transposed (row i = column i of
  *                        W_down), the K-major operand of the down GEMM; a
  *                        weight layout built once; may be NULL if s_max = 0
- *   ell_cap              K, 0 <= K <= 512
+ *   ell_cap              K >= 0
  *   s_max                spill capacity in tokens, >= 0
  *   workspace            >= twell_hybrid_up_down_workspace_bytes(N, d, F,
  *                        s_max) bytes, 256-byte aligned, caller-owned, not
@@ -242,9 +242,7 @@ int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, const uint8
  * Deterministic: repeated calls give the same bits.  Rows with a tile whose
  * count exceeds C use their stored entries only, as in twell_fused_up_down.
  * Errors: as twell_fused_up_down; SGE_ERR_ARG for negative K or S_max,
- * F % 8 != 0, a short or misaligned workspace, a missing wd_t;
- * SGE_ERR_UNSUPPORTED for K > 512; SGE_ERR_CUDA if the library's stream or
- * events cannot be created.
+ * F % 8 != 0, a short or misaligned workspace, a missing wd_t.
  */
 size_t twell_hybrid_up_down_workspace_bytes(int64_t n_tokens, int64_t d_model, int64_t d_ff,
                                             int s_max);

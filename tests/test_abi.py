@@ -139,7 +139,6 @@ def test_routed_rejects_bad_arguments(lib):
     assert _routed(lib, k=-1) == 1
     assert b"capacity" in lib.sge_last_error()
     assert _routed(lib, s_max=-3) == 1
-    assert _routed(lib, k=513) == 2                          # K beyond the light kernel's 512
     assert _routed(lib, wd_t=None) == 1                      # the spill needs W_down^T
     assert b"null" in lib.sge_last_error()
     assert _routed(lib, f=260, tile=20, cap=20) == 1         # F % 8
