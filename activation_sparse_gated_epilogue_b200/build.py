@@ -18,6 +18,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsge.so")
+# the test-only self-test library (failure handling of the GEMM engines)
+SELFTEST_SRC = os.path.join(CSRC, "selftest", "selftest.cu")
+SELFTEST_LIB = os.path.join(HERE, "libsge_selftest.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -46,8 +49,8 @@ def _stale(target, inputs):
     return any(os.path.getmtime(p) > t for p in inputs)
 
 
-def _compile(src, verbose):
-    obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+def _compile(src, verbose, obj=None):
+    obj = obj or os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
     cmd = [NVCC, *FLAGS, "-c", src, "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
@@ -76,10 +79,28 @@ def build(force: bool = False, verbose: bool = False) -> str:
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
         os.replace(tmp, LIB)
+    _build_selftest(force, verbose)
     if verbose:
         for log in logs:
             sys.stderr.write(log)
     return LIB
+
+
+def _build_selftest(force: bool, verbose: bool) -> str:
+    """libsge_selftest.so: the self-test kernels plus the host helpers."""
+    obj = os.path.join(BUILD, "selftest.o")
+    host = os.path.join(BUILD, "host.o")
+    if force or _stale(obj, [SELFTEST_SRC, *_deps()]):
+        _compile(SELFTEST_SRC, verbose, obj)
+    if force or _stale(SELFTEST_LIB, [obj, host]):
+        tmp = SELFTEST_LIB + f".tmp{os.getpid()}"
+        cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static",
+               "-Xcompiler", "-fPIC", obj, host, "-o", tmp]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+        os.replace(tmp, SELFTEST_LIB)
+    return SELFTEST_LIB
 
 
 if __name__ == "__main__":

@@ -33,11 +33,12 @@
 namespace sge {
 
 // X_s and A_s rows of the kept spill tokens, a CTA per row (grid-stride over
-// the spill ranks; CTAs small enough that every row is in flight at once):
-// the x row is copied and the dense row of a zeroed while the tile counts
-// load, then every stored entry is written by its own thread, which finds its
-// tile by a binary search over the row's tile prefix in shared memory.
-constexpr int kPrepThreads = 128;
+// the spill ranks): the x row is copied while the tile counts load; the dense
+// row of a is assembled in shared memory (zeroed, then every stored entry
+// written by its own thread, which finds its tile by a binary search over the
+// row's tile prefix) and stored with whole 16-byte vectors, so global memory
+// sees each row written once, in full lines.
+constexpr int kPrepThreads = 256;
 
 __global__ void __launch_bounds__(kPrepThreads) spill_prep_kernel(const uint16_t* __restrict__ x,
                                                                   const uint8_t* __restrict__ count,
@@ -49,22 +50,20 @@ __global__ void __launch_bounds__(kPrepThreads) spill_prep_kernel(const uint16_t
                                                                   int tile, int cap,
                                                                   uint16_t* __restrict__ xs,
                                                                   uint16_t* __restrict__ as) {
-  __shared__ int pre[257];
-  __shared__ int wsum[kPrepThreads / 32];
+  extern __shared__ __align__(16) uint8_t prep_smem[];
+  uint16_t* row = reinterpret_cast<uint16_t*>(prep_smem);              // f bf16
+  int* pre = reinterpret_cast<int*>(prep_smem + ((2 * f + 15) & ~15));  // nt + 1
+  int* wsum = pre + 260;                                                // warps
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kept = min(*n_heavy, s_max);
   for (int r = blockIdx.x; r < kept; r += gridDim.x) {
     const int64_t t = spill_rows[r];
-    // each thread owns tiles 2 tid and 2 tid + 1 (nt <= 256)
-    const int b0 = 2 * tid;
-    const int c0 = b0 < nt ? min(static_cast<int>(__ldg(count + t * nt + b0)), cap) : 0;
-    const int c1 = b0 + 1 < nt ? min(static_cast<int>(__ldg(count + t * nt + b0 + 1)), cap) : 0;
+    const int c = tid < nt ? min(static_cast<int>(__ldg(count + t * nt + tid)), cap) : 0;
     const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
     uint4* dst = reinterpret_cast<uint4*>(xs + static_cast<int64_t>(r) * d);
     for (int v = tid; v < d / 8; v += kPrepThreads) dst[v] = __ldg(src + v);
-    uint16_t* arow = as + static_cast<int64_t>(r) * f;
-    for (int v = tid; v < f / 8; v += kPrepThreads) reinterpret_cast<uint4*>(arow)[v] = make_uint4(0, 0, 0, 0);
-    int incl = c0 + c1;
+    for (int v = tid; v < f / 8; v += kPrepThreads) reinterpret_cast<uint4*>(row)[v] = make_uint4(0, 0, 0, 0);
+    int incl = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -78,22 +77,25 @@ __global__ void __launch_bounds__(kPrepThreads) spill_prep_kernel(const uint16_t
       base += w < warp ? wsum[w] : 0;
       total += wsum[w];
     }
-    const int ex = base + incl - c0 - c1;
-    if (b0 < nt) pre[b0] = ex;
-    if (b0 + 1 < nt) pre[b0 + 1] = ex + c0;
-    __syncthreads();  // the prefix is complete and the zeros have landed
+    if (tid < nt) pre[tid] = base + incl - c;
+    __syncthreads();  // the prefix is complete, the row is zero
     for (int e = tid; e < total; e += kPrepThreads) {
       int b = 0;  // the last tile whose prefix is <= e
       for (int step = 128; step > 0; step >>= 1)
         if (b + step < nt && pre[b + step] <= e) b += step;
       const int64_t at = (t * nt + b) * cap + (e - pre[b]);
       // a stored index is < T; kept inside its tile even if it is not
-      const int j = b * tile + min(static_cast<int>(__ldg(idx + at)), tile - 1);
-      arow[j] = __ldg(val + at);
+      row[b * tile + min(static_cast<int>(__ldg(idx + at)), tile - 1)] = __ldg(val + at);
     }
-    __syncthreads();  // pre[] and wsum[] are rewritten for the next row
+    __syncthreads();  // the row is assembled
+    uint4* arow = reinterpret_cast<uint4*>(as + static_cast<int64_t>(r) * f);
+    for (int v = tid; v < f / 8; v += kPrepThreads) arow[v] = reinterpret_cast<const uint4*>(row)[v];
+    __syncthreads();  // row[], pre[] and wsum[] are rewritten for the next row
   }
 }
+
+// Shared memory of the prep kernel for F hidden units.
+inline int prep_smem_bytes(int64_t f) { return static_cast<int>(((2 * f + 15) & ~15) + 4 * (260 + 8)); }
 
 // ------------------------------------------------------ light tokens
 //
@@ -456,8 +458,10 @@ extern "C" int twell_hybrid_up_down(const void* x, const uint8_t* count, const u
              ldw == 2 * d_model;
   if ((rc = run_ring(rp, c.nv, st))) return rc;
   {
-    const int prep_grid = static_cast<int>(std::min<int64_t>(s_max, 16 * static_cast<int64_t>(sm_count())));
-    spill_prep_kernel<<<prep_grid, kPrepThreads, 0, st>>>(
+    const int smem = prep_smem_bytes(d_ff);
+    if ((rc = set_smem_limit(reinterpret_cast<const void*>(spill_prep_kernel), smem))) return rc;
+    const int prep_grid = static_cast<int>(std::min<int64_t>(s_max, 8 * static_cast<int64_t>(sm_count())));
+    spill_prep_kernel<<<prep_grid, kPrepThreads, smem, st>>>(
         static_cast<const uint16_t*>(x), count, idx, static_cast<const uint16_t*>(val), spill_rows,
         n_heavy, s_max, d, f, f / tile, tile, cap, xs, as);
     if ((rc = check_launch("twell_hybrid_up_down (spill prep)"))) return rc;

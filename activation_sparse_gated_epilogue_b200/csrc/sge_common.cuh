@@ -21,7 +21,12 @@ namespace sge {
 // Deadline of one bounded wait, in nanoseconds of %globaltimer.  Every
 // legitimate wait in this library is microseconds; four seconds means the
 // pipeline is broken, and the kernel gives up instead of hanging the GPU.
-constexpr uint64_t kWaitNs = 4000000000ull;
+// (The test-only self-test library builds the same kernels with a short
+// deadline, to make a wait run out on purpose.)
+#ifndef SGE_WAIT_NS
+#define SGE_WAIT_NS 4000000000ull
+#endif
+constexpr uint64_t kWaitNs = SGE_WAIT_NS;
 // Tries of an mbarrier wait between two reads of %globaltimer (a power of two).
 constexpr uint32_t kWaitSpins = 1024;
 

@@ -44,20 +44,34 @@ struct EpiSpillUp {
 
   template <int BN>
   __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {
+    constexpr int CH = BN / 32;
     const int kept = min(*n_spill, s_max);
-#pragma unroll 1
-    for (int ch = 0; ch < BN / 32; ++ch) {
+    const bool live = row < kept;
+    // the row's activations for the whole tile, all loads in flight at once
+    // (one thread per row: each load is a separate line, so issuing them
+    // chunk by chunk would cost a memory round trip per chunk)
+    uint4 av[CH][4];
+#pragma unroll
+    for (int ch = 0; ch < CH; ++ch)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int col = n_blk * BN + ch * 32 + q * 8;
+        av[ch][q] = live && col + 8 <= n_cols
+                        ? *reinterpret_cast<const uint4*>(spill_a + row * n_cols + col)
+                        : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+    for (int ch = 0; ch < CH; ++ch) {
       uint32_t r[32];
       tmem_ld32(taddr + ch * 32, r);
       tmem_ld_wait();
       const int col0 = n_blk * BN + ch * 32;
-      if (row >= kept) continue;
+      if (!live) continue;
       const int64_t off = row * n_cols + col0;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         if (col0 + q * 8 + 8 > n_cols) break;
-        const uint4 av = *reinterpret_cast<const uint4*>(spill_a + off + q * 8);
-        const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+        const uint32_t aw[4] = {av[ch][q].x, av[ch][q].y, av[ch][q].z, av[ch][q].w};
         uint32_t uw[4], hw[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {

@@ -14,8 +14,11 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "sge.h")
 
 
-def declared_functions():
-    text = open(HEADER).read()
+SELFTEST_HEADER = os.path.join(ROOT, "include", "sge_selftest.h")
+
+
+def declared_functions(header=HEADER):
+    text = open(header).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
     return sorted(set(n for n in names if n not in ("defined",)))
@@ -40,6 +43,36 @@ def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert name in exported, name
         assert getattr(lib, name) is not None
+
+
+def test_every_header_is_covered():
+    """include/ holds the product library's header and the self-test
+    library's; the tests below check both."""
+    headers = sorted(os.listdir(os.path.join(ROOT, "include")))
+    assert headers == ["sge.h", "sge_selftest.h"], headers
+
+
+def test_selftest_library_exports_its_declared_symbols(lib):
+    path = sge_build.SELFTEST_LIB
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    names = declared_functions(SELFTEST_HEADER)
+    assert names == ["sge_selftest_wait_timeout"]
+    st = ctypes.CDLL(path)
+    for name in names:
+        assert name in exported, name
+        assert getattr(st, name) is not None
+
+
+def test_selftest_rejects_bad_arguments(lib):
+    st = ctypes.CDLL(sge_build.SELFTEST_LIB)
+    P = ctypes.c_void_p
+    st.sge_selftest_wait_timeout.argtypes = [ctypes.c_int, P, P, ctypes.c_int64, ctypes.c_int64,
+                                             ctypes.c_int64, P, P, P]
+    p = P(4096)
+    assert st.sge_selftest_wait_timeout(0, None, p, 256, 256, 256, p, p, None) == 1
+    assert st.sge_selftest_wait_timeout(1, p, p, 256, 256, 32, p, p, None) == 1    # k < 64
 
 
 def test_version_and_error_string(lib):
