@@ -76,8 +76,9 @@ def library() -> ctypes.CDLL:
             "hybrid_ffn_fwd": (I, [P, ctypes.POINTER(_SgeHybrid), P, P, P, P, P, I64, P,
                                    ctypes.c_size_t, P]),
             "hybrid_ffn_bwd_workspace_bytes": (ctypes.c_size_t, [I64, I64, I64, I, I]),
-            "hybrid_ffn_bwd": (I, [P, P, ctypes.POINTER(_SgeHybrid), P, P, P, P, P, P, P, I64, P,
+            "hybrid_ffn_bwd": (I, [P, P, ctypes.POINTER(_SgeHybrid), P, P, P, P, P, P, P, P, I64, P,
                                    ctypes.c_size_t, P]),
+            "sge_transpose_up_gate": (I, [P, P, P, I64, I64, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(lib, name)
@@ -407,22 +408,39 @@ def hybrid_bwd_workspace(n_tokens: int, d_model: int, d_ff: int, ell_cap: int, s
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
+def transpose_up_gate(wu_t: torch.Tensor, wg_t: torch.Tensor, stream=None) -> torch.Tensor:
+    """w_ug [d][2F] = [W_up | W_gate], hybrid_ffn_bwd's dX operand; a
+    weight-loading step, done once per weight update."""
+    _check(wu_t, "wu_t", torch.bfloat16)
+    f, d = wu_t.shape
+    _check(wg_t, "wg_t", torch.bfloat16, (f, d))
+    w_ug = torch.empty((d, 2 * f), dtype=torch.bfloat16, device=wu_t.device)
+    _call("sge_transpose_up_gate", _ptr(wu_t), _ptr(wg_t), _ptr(w_ug), f, d, _stream(wu_t.device, stream))
+    return w_ug
+
+
 def hybrid_ffn_bwd(x: torch.Tensor, dy: torch.Tensor, hy: Hybrid, wg_t: torch.Tensor,
                    wu_t: torch.Tensor, wd: torch.Tensor, workspace: Optional[torch.Tensor] = None,
-                   stream=None):
-    """Returns (dx bf16 [N][d], dwg_t, dwu_t, dwd fp32 [F][d])."""
+                   stream=None, w_ug: Optional[torch.Tensor] = None, out=None):
+    """Returns (dx bf16 [N][d], dwg_t, dwu_t, dwd fp32 [F][d]).  ``w_ug`` is
+    transpose_up_gate's [W_up | W_gate] (None: built in the workspace per
+    call); ``out`` optionally gives the four output tensors."""
     _check(x, "x", torch.bfloat16)
     n, d = x.shape
     f = hy.d_ff
     _check(dy, "dy", torch.bfloat16, (n, d))
     for name, w in (("wg_t", wg_t), ("wu_t", wu_t), ("wd", wd)):
         _check(w, name, torch.bfloat16, (f, d))
-    dx = torch.empty_like(x)
-    grads = [torch.empty((f, d), dtype=torch.float32, device=x.device) for _ in range(3)]
+    if w_ug is not None:
+        _check(w_ug, "w_ug", torch.bfloat16, (d, 2 * f))
+    if out is None:
+        out = (torch.empty_like(x),) + tuple(torch.empty((f, d), dtype=torch.float32, device=x.device)
+                                              for _ in range(3))
+    dx, dwg, dwu, dwd = out
     if workspace is None:
         workspace = hybrid_bwd_workspace(n, d, f, hy.ell_cap, hy.s_max, x.device)
     cs = hy.c_struct()
     _call("hybrid_ffn_bwd", _ptr(x), _ptr(dy), ctypes.byref(cs), _ptr(wg_t), _ptr(wu_t), _ptr(wd),
-          _ptr(dx), _ptr(grads[0]), _ptr(grads[1]), _ptr(grads[2]), d, _ptr(workspace),
+          _ptr(w_ug), _ptr(dx), _ptr(dwg), _ptr(dwu), _ptr(dwd), d, _ptr(workspace),
           workspace.numel(), _stream(x.device, stream))
-    return (dx, *grads)
+    return dx, dwg, dwu, dwd

@@ -11,17 +11,17 @@
 //   dW_down[j] += a_j u_j dy   dW_up[:, j] += du_j x   dW_gate[:, j] += dg_j x
 //
 // ELL rows: one CTA per token computes dh (dot products with rows of
-// W_down), du, dg (kept in fp32 for the weight gradients) and dx.  Weight
-// gradients of the ELL entries are summed per hidden unit over its tokens in
-// ascending token order: entries are bucketed by column (counting sort) and
-// each column's bucket is ordered by token, so the result is deterministic.
-// Spill rows: dense tcgen05 GEMMs on the gathered rows,
-//   dH = dY_s W_down^T (epilogue: dU = dH a, dG = dH u [a > 0], H = a u),
-//   dX_s = [dU | dG] [W_up ; W_gate]^T (scattered to dx),
-//   dW_down += H^T dY_s,  [dW_up ; dW_gate] += [dU | dG]^T X_s,
-// with the small operands transposed in the workspace so that every GEMM
-// reads K-major tiles.
+// W_down), du, dg (kept in fp32 for the weight gradients) and dx.  Spill
+// rows: dH = dY_s W_down^T on tcgen05 (gathered rows; epilogue: dU = dH a,
+// dG = dH u [a > 0], both bf16), then dX_s = [dU | dG] [W_up ; W_gate]^T on
+// tcgen05, scattered to dx.  Weight gradients: every stored entry, of ELL and
+// of spill rows alike (a spill row's entries are its active columns, a > 0),
+// is bucketed by hidden unit (counting sort) and each unit's bucket ordered
+// by token; one CTA per unit then sums its entries in ascending token order
+// and writes the unit's three fp32 gradient rows once.  The result is
+// deterministic.
 #include "sparse_common.cuh"
+#include "spill_gemm.cuh"
 #include "tc_launch.cuh"
 
 namespace sge {
@@ -52,17 +52,13 @@ struct BwdWs {
   int* col_count;    // [F]
   int* col_start;    // [F + 1]
   int* col_cursor;   // [F]
-  int2* csc;         // [N * K] (token, slot), bucketed by column
-  int2* csc_sorted;  // [N * K] same, ascending token within a column
+  int2* csc;         // [N * K + S_max * F] (token, slot), bucketed by column; a spill
+                     // row's entry has slot -(spill rank + 1)
+  int2* csc_sorted;  // same, ascending token within a column
   uint16_t* dys;     // [Sp][d]   gathered dy of the kept spill rows
-  uint16_t* xs;      // [Sp][d]   gathered x
   uint16_t* acat;    // [Sp][2F]  dU | dG
-  uint16_t* hs;      // [Sp][F]   H = a u
-  uint16_t* acat_t;  // [2F][Sp]
-  uint16_t* hs_t;    // [F][Sp]
-  uint16_t* dys_t;   // [d][Sp]
-  uint16_t* xs_t;    // [d][Sp]
-  uint16_t* bcat;    // [d][2F]   W_up | W_gate (row i = row i of W_up, W_gate)
+  uint16_t* bcat;    // [d][2F]   W_up | W_gate (row i = row i of W_up, W_gate), when the
+                     //           caller passes none
   size_t bytes;
 };
 
@@ -79,22 +75,17 @@ static BwdWs carve(void* base, int64_t n, int64_t d, int64_t f, int k, int s_max
     return q;
   };
   const size_t nk = static_cast<size_t>(n) * static_cast<size_t>(k > 0 ? k : 1);
+  const size_t ne = nk + static_cast<size_t>(s_max) * static_cast<size_t>(f);
   w.du = reinterpret_cast<float*>(take(nk * 4));
   w.dg = reinterpret_cast<float*>(take(nk * 4));
   w.col_count = reinterpret_cast<int*>(take(f * 4));
   w.col_start = reinterpret_cast<int*>(take((f + 1) * 4));
   w.col_cursor = reinterpret_cast<int*>(take(f * 4));
-  w.csc = reinterpret_cast<int2*>(take(nk * 8));
-  w.csc_sorted = reinterpret_cast<int2*>(take(nk * 8));
+  w.csc = reinterpret_cast<int2*>(take(ne * 8));
+  w.csc_sorted = reinterpret_cast<int2*>(take(ne * 8));
   if (s_max > 0) {
     w.dys = reinterpret_cast<uint16_t*>(take(sp * d * 2));
-    w.xs = reinterpret_cast<uint16_t*>(take(sp * d * 2));
     w.acat = reinterpret_cast<uint16_t*>(take(sp * 2 * f * 2));
-    w.hs = reinterpret_cast<uint16_t*>(take(sp * f * 2));
-    w.acat_t = reinterpret_cast<uint16_t*>(take(2 * f * sp * 2));
-    w.hs_t = reinterpret_cast<uint16_t*>(take(f * sp * 2));
-    w.dys_t = reinterpret_cast<uint16_t*>(take(d * sp * 2));
-    w.xs_t = reinterpret_cast<uint16_t*>(take(d * sp * 2));
     w.bcat = reinterpret_cast<uint16_t*>(take(d * 2 * f * 2));
   }
   w.bytes = off;
@@ -268,6 +259,41 @@ __global__ void __launch_bounds__(256) csc_scatter_kernel(BwdHybrid hv, int* col
   }
 }
 
+// Entries of the kept spill rows (their active columns, a > 0): counted per
+// column, then scattered with slot -(spill rank + 1).  Grid: (F / 2048
+// chunks) x (S_max ranks); eight columns per thread.
+__global__ void __launch_bounds__(256) csc_count_spill_kernel(BwdHybrid hv, int* col_count) {
+  const int r = blockIdx.y;
+  if (r >= min(*hv.n_spill, hv.s_max)) return;
+  const int j0 = (blockIdx.x * 256 + threadIdx.x) * 8;
+  if (j0 >= hv.f) return;
+  const uint4 av = *reinterpret_cast<const uint4*>(hv.spill_a + static_cast<int64_t>(r) * hv.f + j0);
+  const uint32_t w[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (__uint_as_float(w[i] << 16) > 0.0f) atomicAdd(&col_count[j0 + 2 * i], 1);
+    if (__uint_as_float(w[i] & 0xFFFF0000u) > 0.0f) atomicAdd(&col_count[j0 + 2 * i + 1], 1);
+  }
+}
+
+__global__ void __launch_bounds__(256) csc_scatter_spill_kernel(BwdHybrid hv, int* col_cursor, int2* csc) {
+  const int r = blockIdx.y;
+  if (r >= min(*hv.n_spill, hv.s_max)) return;
+  const int j0 = (blockIdx.x * 256 + threadIdx.x) * 8;
+  if (j0 >= hv.f) return;
+  const int t = hv.spill_rows[r];
+  const uint4 av = *reinterpret_cast<const uint4*>(hv.spill_a + static_cast<int64_t>(r) * hv.f + j0);
+  const uint32_t w[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      if (__uint_as_float(h ? (w[i] & 0xFFFF0000u) : (w[i] << 16)) > 0.0f) {
+        const int pos = atomicAdd(&col_cursor[j0 + 2 * i + h], 1);
+        csc[pos] = make_int2(t, -(r + 1));
+      }
+}
+
 // Per column (one warp): order the bucket by token.  Tokens are unique in a
 // column, so an entry's position is the number of smaller tokens.
 __global__ void __launch_bounds__(256) csc_sort_kernel(const int* col_start, int f, const int2* csc,
@@ -284,8 +310,9 @@ __global__ void __launch_bounds__(256) csc_sort_kernel(const int* col_start, int
   }
 }
 
-// Per column j (one CTA): weight-gradient rows from the ELL entries, summed
-// in ascending token order, written (overwriting) in fp32.
+// Per column j (one CTA): weight-gradient rows from the column's entries (ELL
+// and spill rows), summed in ascending token order, written (overwriting) in
+// fp32.
 struct DwParams {
   const uint16_t* x;
   const uint16_t* dy;
@@ -311,10 +338,21 @@ __global__ void __launch_bounds__(kBwdThreads) dw_ell_kernel(DwParams p) {
   const int s0 = p.ws.col_start[j], s1 = p.ws.col_start[j + 1];
   for (int i = s0; i < s1; ++i) {
     const int2 te = p.ws.csc_sorted[i];
-    const int64_t rk = static_cast<int64_t>(te.x) * p.hv.k + te.y;
-    const float a = __uint_as_float(static_cast<uint32_t>(p.hv.ell_a[rk]) << 16);
-    const float u = __uint_as_float(static_cast<uint32_t>(p.hv.ell_u[rk]) << 16);
-    const float h = a * u, du = p.ws.du[rk], dg = p.ws.dg[rk];
+    float a, u, du, dg;
+    if (te.y >= 0) {  // an ELL entry: slot te.y of row te.x
+      const int64_t rk = static_cast<int64_t>(te.x) * p.hv.k + te.y;
+      a = __uint_as_float(static_cast<uint32_t>(p.hv.ell_a[rk]) << 16);
+      u = __uint_as_float(static_cast<uint32_t>(p.hv.ell_u[rk]) << 16);
+      du = p.ws.du[rk];
+      dg = p.ws.dg[rk];
+    } else {  // an active column of spill rank -te.y - 1
+      const int64_t r = -te.y - 1;
+      a = __uint_as_float(static_cast<uint32_t>(p.hv.spill_a[r * p.hv.f + j]) << 16);
+      u = __uint_as_float(static_cast<uint32_t>(p.hv.spill_u[r * p.hv.f + j]) << 16);
+      du = __uint_as_float(static_cast<uint32_t>(p.ws.acat[r * 2 * p.hv.f + j]) << 16);
+      dg = __uint_as_float(static_cast<uint32_t>(p.ws.acat[r * 2 * p.hv.f + p.hv.f + j]) << 16);
+    }
+    const float h = a * u;
     const uint4* dyr = reinterpret_cast<const uint4*>(p.dy + static_cast<int64_t>(te.x) * p.d);
     const uint4* xr = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(te.x) * p.d);
 #pragma unroll
@@ -354,31 +392,6 @@ __global__ void __launch_bounds__(kBwdThreads) dw_ell_kernel(DwParams p) {
 }
 
 // -------------------------------------------------------- spill rows
-
-__global__ void __launch_bounds__(256) gather2_kernel(const uint16_t* __restrict__ a,
-                                                      const uint16_t* __restrict__ b,
-                                                      const int32_t* __restrict__ rows,
-                                                      const int32_t* __restrict__ n_rows_dev,
-                                                      int cap_rows, int d, uint16_t* da, uint16_t* db) {
-  const int r = blockIdx.x;
-  const int kept = min(*n_rows_dev, cap_rows);
-  const int nvec = d / 8;
-  uint4* oa = reinterpret_cast<uint4*>(da + static_cast<int64_t>(r) * d);
-  uint4* ob = reinterpret_cast<uint4*>(db + static_cast<int64_t>(r) * d);
-  if (r < kept) {
-    const uint4* ia = reinterpret_cast<const uint4*>(a + static_cast<int64_t>(rows[r]) * d);
-    const uint4* ib = reinterpret_cast<const uint4*>(b + static_cast<int64_t>(rows[r]) * d);
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-      oa[v] = __ldg(ia + v);
-      ob[v] = __ldg(ib + v);
-    }
-  } else {
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-      oa[v] = make_uint4(0, 0, 0, 0);
-      ob[v] = make_uint4(0, 0, 0, 0);
-    }
-  }
-}
 
 // dst[c][col_off + r] = src[r][c] for r < rows, c < cols (bf16, 32x32 tiles).
 __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restrict__ src, int rows,
@@ -424,13 +437,11 @@ __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restri
 }
 
 // Epilogue of dH = dY_s W_down^T: dU = dH a, dG = dH u [a > 0] -> acat
-// (dU in columns [0, F), dG in [F, 2F)), H = a u -> hs; zero rows past the
-// kept spill rows so that they add nothing in the later GEMMs.
+// (dU in columns [0, F), dG in [F, 2F)); zero rows past the kept spill rows.
 struct EpiBwdSpill {
   const uint16_t* spill_a;
   const uint16_t* spill_u;
   uint16_t* acat;
-  uint16_t* hs;
   const int32_t* n_spill;
   int s_max;
   int f;
@@ -458,14 +469,14 @@ struct EpiBwdSpill {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         if (col0 + q * 8 + 8 > f) break;
-        uint32_t du[4] = {0, 0, 0, 0}, dg[4] = {0, 0, 0, 0}, hw[4] = {0, 0, 0, 0};
+        uint32_t du[4] = {0, 0, 0, 0}, dg[4] = {0, 0, 0, 0};
         if (row < kept) {
           const uint4 av = *reinterpret_cast<const uint4*>(spill_a + off + q * 8);
           const uint4 uv = *reinterpret_cast<const uint4*>(spill_u + off + q * 8);
           const uint32_t aw[4] = {av.x, av.y, av.z, av.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            float o[2][3];
+            float o[2][2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const float dh = __uint_as_float(r[q * 8 + 2 * i + h]);
@@ -473,82 +484,14 @@ struct EpiBwdSpill {
               const float u = __uint_as_float(h ? (uw[i] & 0xFFFF0000u) : (uw[i] << 16));
               o[h][0] = dh * a;
               o[h][1] = a > 0.0f ? dh * u : 0.0f;
-              o[h][2] = a * u;
             }
             du[i] = static_cast<uint32_t>(f32_to_bf16_bits(o[0][0])) | (static_cast<uint32_t>(f32_to_bf16_bits(o[1][0])) << 16);
             dg[i] = static_cast<uint32_t>(f32_to_bf16_bits(o[0][1])) | (static_cast<uint32_t>(f32_to_bf16_bits(o[1][1])) << 16);
-            hw[i] = static_cast<uint32_t>(f32_to_bf16_bits(o[0][2])) | (static_cast<uint32_t>(f32_to_bf16_bits(o[1][2])) << 16);
           }
         }
         *reinterpret_cast<uint4*>(acat + offc + q * 8) = make_uint4(du[0], du[1], du[2], du[3]);
         *reinterpret_cast<uint4*>(acat + offc + f + q * 8) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
-        *reinterpret_cast<uint4*>(hs + off + q * 8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
       }
-    }
-  }
-};
-
-// Epilogue: out[row] += D (fp32).  Rows [0, split) go to out0, rows
-// [split, 2 split) to out1 (row - split).
-struct EpiAddF32 {
-  float* out0;
-  float* out1;
-  int64_t split;
-  int n_cols;
-  const int32_t* k_count;  // nullable: K is the kept spill rows, rounded up to 64
-  int k_cap;
-
-  __device__ __forceinline__ int k_limit(int k) const {
-    if (!k_count) return k;
-    const int c = min(*k_count, k_cap);
-    return min(k, (c + 63) / 64 * 64);
-  }
-
-  template <int BN>
-  __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {
-    // the warp's 32 rows pass through shared memory so that each row is
-    // added with contiguous 128-byte accesses (a thread per row would add 16
-    // bytes at a time to 32 different rows)
-    __shared__ __align__(16) float stage[4][32][36];
-    float(*buf)[36] = stage[(threadIdx.x >> 5) & 3];
-    const int64_t row0 = row - lane;
-    const int rr = lane >> 3, c4 = (lane & 7) * 4;
-#pragma unroll 1
-    for (int ch = 0; ch < BN / 32; ++ch) {
-      uint32_t r[32];
-      tmem_ld32(taddr + ch * 32, r);
-      tmem_ld_wait();
-      const int col0 = n_blk * BN + ch * 32;
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        *reinterpret_cast<float4*>(&buf[lane][4 * q]) =
-            make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                        __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
-      __syncwarp();
-      if (col0 + c4 + 4 <= n_cols) {
-        // all 8 rows' loads in flight before any add
-        float4* o[8];
-        float4 v[8];
-#pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int64_t g = row0 + rr + 4 * it;
-          float* out = g < split ? out0 + g * n_cols
-                                 : (out1 && g < 2 * split ? out1 + (g - split) * n_cols : nullptr);
-          o[it] = out ? reinterpret_cast<float4*>(out + col0 + c4) : nullptr;
-          v[it] = o[it] ? *o[it] : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          if (!o[it]) continue;
-          const float4 add = *reinterpret_cast<const float4*>(&buf[rr + 4 * it][c4]);
-          v[it].x += add.x;
-          v[it].y += add.y;
-          v[it].z += add.z;
-          v[it].w += add.w;
-          *o[it] = v[it];
-        }
-      }
-      __syncwarp();
     }
   }
 };
@@ -621,9 +564,32 @@ extern "C" size_t hybrid_ffn_bwd_workspace_bytes(int64_t n_tokens, int64_t d_mod
   return carve(nullptr, n_tokens, d_model, d_ff, ell_cap, s_max).bytes;
 }
 
+// [W_up | W_gate] as the dX GEMM's K-major B operand: w_ug[i][j] =
+// W_up[i][j] = wu_t[j][i], w_ug[i][F + j] = W_gate[i][j] = wg_t[j][i].
+static int build_up_gate(const void* wu_t, const void* wg_t, uint16_t* w_ug, int64_t f, int64_t d,
+                         cudaStream_t st) {
+  int rc = launch_transpose(static_cast<const uint16_t*>(wu_t), static_cast<int>(f), static_cast<int>(d), d,
+                            w_ug, 2 * f, 0, st);
+  if (rc) return rc;
+  return launch_transpose(static_cast<const uint16_t*>(wg_t), static_cast<int>(f), static_cast<int>(d), d,
+                          w_ug, 2 * f, static_cast<int>(f), st);
+}
+
+extern "C" int sge_transpose_up_gate(const void* wu_t, const void* wg_t, void* w_ug, int64_t d_ff,
+                                     int64_t d_model, void* stream) {
+  clear_error();
+  if (d_ff < 8 || d_ff % 8 || d_model < 8 || d_model % 8 || d_ff > (1 << 30) || d_model > (1 << 30))
+    return fail(SGE_ERR_ARG, "sge_transpose_up_gate: d_ff and d_model must be multiples of 8");
+  if (!wu_t || !wg_t || !w_ug) return fail(SGE_ERR_ARG, "sge_transpose_up_gate: null pointer");
+  if (!aligned16(wu_t) || !aligned16(wg_t) || !aligned16(w_ug))
+    return fail(SGE_ERR_ARG, "sge_transpose_up_gate: pointer not 16-byte aligned");
+  return build_up_gate(wu_t, wg_t, static_cast<uint16_t*>(w_ug), d_ff, d_model,
+                       static_cast<cudaStream_t>(stream));
+}
+
 extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* hy,
-                              const void* wg_t, const void* wu_t, const void* wd, void* dx,
-                              float* dwg_t, float* dwu_t, float* dwd, int64_t d_model,
+                              const void* wg_t, const void* wu_t, const void* wd, const void* w_ug,
+                              void* dx, float* dwg_t, float* dwu_t, float* dwd, int64_t d_model,
                               void* workspace, size_t workspace_bytes, void* stream) {
   clear_error();
   if (!hy) return fail(SGE_ERR_ARG, "hybrid_ffn_bwd: null hybrid descriptor");
@@ -639,13 +605,19 @@ extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* h
   if (!x || !dy || !wg_t || !wu_t || !wd || !dx || !dwg_t || !dwu_t || !dwd)
     return fail(SGE_ERR_ARG, "hybrid_ffn_bwd: null pointer");
   if (!aligned16(x) || !aligned16(dy) || !aligned16(wg_t) || !aligned16(wu_t) || !aligned16(wd) ||
-      !aligned16(dx) || !aligned16(dwg_t) || !aligned16(dwu_t) || !aligned16(dwd))
+      !aligned16(dx) || !aligned16(dwg_t) || !aligned16(dwu_t) || !aligned16(dwd) || (w_ug && !aligned16(w_ug)))
     return fail(SGE_ERR_ARG, "hybrid_ffn_bwd: pointer not 16-byte aligned");
   const BwdWs need = carve(nullptr, n, d, f, k, s_max);
   if (!workspace || workspace_bytes < need.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return fail(SGE_ERR_ARG, "hybrid_ffn_bwd: workspace of %zu bytes, %zu needed (256-byte aligned)",
                 workspace_bytes, need.bytes);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n == 0) {
+    cudaMemsetAsync(dwg_t, 0, sizeof(float) * f * d, st);
+    cudaMemsetAsync(dwu_t, 0, sizeof(float) * f * d, st);
+    cudaMemsetAsync(dwd, 0, sizeof(float) * f * d, st);
+    return check_launch("hybrid_ffn_bwd (zero gradients)");
+  }
   const BwdWs ws = carve(workspace, n, d, f, k, s_max);
   BwdHybrid hv{n, static_cast<int>(f), k, s_max, hy->row_nnz, hy->spill_slot, hy->spill_rows,
                hy->n_spill, hy->ell_idx, static_cast<const uint16_t*>(hy->ell_a),
@@ -653,92 +625,61 @@ extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* h
                static_cast<const uint16_t*>(hy->spill_u)};
   const auto* xb = static_cast<const uint16_t*>(x);
   const auto* dyb = static_cast<const uint16_t*>(dy);
-  int rc;
-  if (n > 0) {
-    // ---- ELL rows: dh, du, dg, dx
-    EllBwdParams p{xb, dyb, static_cast<const uint16_t*>(wg_t), static_cast<const uint16_t*>(wu_t),
-                   static_cast<const uint16_t*>(wd), static_cast<uint16_t*>(dx), hv, ws,
-                   static_cast<int>(d)};
-    DwParams q{xb, dyb, hv, ws, dwg_t, dwu_t, dwd, static_cast<int>(d)};
-    const int64_t nvec = d / 8;
-    if (nvec <= kBwdThreads) rc = launch_ell_bwd<1>(p, n, st);
-    else if (nvec <= 2 * kBwdThreads) rc = launch_ell_bwd<2>(p, n, st);
-    else if (nvec <= 3 * kBwdThreads) rc = launch_ell_bwd<3>(p, n, st);
-    else rc = launch_ell_bwd<4>(p, n, st);
-    if (rc) return rc;
-    // ---- column buckets of the ELL entries, ordered by token
-    cudaError_t e = cudaMemsetAsync(ws.col_count, 0, sizeof(int) * f, st);
-    if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "hybrid_ffn_bwd: %s", cudaGetErrorString(e));
-    const unsigned rb = static_cast<unsigned>((n + 7) / 8);
-    csc_count_kernel<<<rb, 256, 0, st>>>(hv, ws.col_count);
-    csc_scan_kernel<<<1, 1024, 0, st>>>(ws.col_count, static_cast<int>(f), ws.col_start, ws.col_cursor);
-    csc_scatter_kernel<<<rb, 256, 0, st>>>(hv, ws.col_cursor, ws.csc);
-    csc_sort_kernel<<<static_cast<unsigned>((f + 7) / 8), 256, 0, st>>>(ws.col_start, static_cast<int>(f),
-                                                                       ws.csc, ws.csc_sorted);
-    if ((rc = check_launch("hybrid_ffn_bwd (column buckets)"))) return rc;
-    // ---- weight gradients of the ELL entries (overwrite)
-    if (nvec <= kBwdThreads) rc = launch_dw<1>(q, static_cast<int>(f), st);
-    else if (nvec <= 2 * kBwdThreads) rc = launch_dw<2>(q, static_cast<int>(f), st);
-    else if (nvec <= 3 * kBwdThreads) rc = launch_dw<3>(q, static_cast<int>(f), st);
-    else rc = launch_dw<4>(q, static_cast<int>(f), st);
-    if (rc) return rc;
-  } else {
-    cudaMemsetAsync(dwg_t, 0, sizeof(float) * f * d, st);
-    cudaMemsetAsync(dwu_t, 0, sizeof(float) * f * d, st);
-    cudaMemsetAsync(dwd, 0, sizeof(float) * f * d, st);
-    return SGE_OK;
-  }
-  if (s_max == 0) return SGE_OK;
-
-  // ---- spill rows on tensor cores
+  const int64_t nvec = d / 8;
   const int sp = (s_max + 63) / 64 * 64;
-  gather2_kernel<<<sp, 256, 0, st>>>(dyb, xb, hy->spill_rows, hy->n_spill, s_max, static_cast<int>(d),
-                                      ws.dys, ws.xs);
-  if ((rc = check_launch("hybrid_ffn_bwd (gather)"))) return rc;
-  using S = TcPairShape<256, 1>;
-  CUtensorMap m1a, m1b;
-  if ((rc = make_tmap_bf16(&m1a, ws.dys, sp, d, d, kBM))) return rc;
-  // tile widths for few spill rows: N = F in 128-wide tiles (dH), N = d in
-  // 64-wide tiles (dX), so that the GEMMs with one or two row tiles still
-  // spread over the SMs
-  using Sh = TcPairShape<128, 1>;
-  using Sx = TcPairShape<64, 1>;
-  if ((rc = make_tmap_bf16(&m1b, wd, f, d, d, Sh::BN / 2))) return rc;
-  EpiBwdSpill e1{hv.spill_a, hv.spill_u, ws.acat, ws.hs, hy->n_spill, s_max, static_cast<int>(f), sp};
-  if ((rc = launch_tc_gemm_pair<Sh>(m1a, m1b, m1b, sp, f, d, e1, nullptr, st, "hybrid_ffn_bwd (dH)")))
-    return rc;
-  // operands of the remaining GEMMs, K-major
-  // (spill-row operands: only as many rows as the weight-gradient GEMMs read)
-  if ((rc = launch_transpose(ws.acat, sp, static_cast<int>(2 * f), 2 * f, ws.acat_t, sp, 0, st, hy->n_spill, s_max)))
-    return rc;
-  if ((rc = launch_transpose(ws.hs, sp, static_cast<int>(f), f, ws.hs_t, sp, 0, st, hy->n_spill, s_max))) return rc;
-  if ((rc = launch_transpose(ws.dys, sp, static_cast<int>(d), d, ws.dys_t, sp, 0, st, hy->n_spill, s_max))) return rc;
-  if ((rc = launch_transpose(ws.xs, sp, static_cast<int>(d), d, ws.xs_t, sp, 0, st, hy->n_spill, s_max))) return rc;
-  if ((rc = launch_transpose(static_cast<const uint16_t*>(wu_t), static_cast<int>(f), static_cast<int>(d), d,
-                             ws.bcat, 2 * f, 0, st)))
-    return rc;
-  if ((rc = launch_transpose(static_cast<const uint16_t*>(wg_t), static_cast<int>(f), static_cast<int>(d), d,
-                             ws.bcat, 2 * f, static_cast<int>(f), st)))
-    return rc;
-  // dX_s = [dU | dG] [W_up ; W_gate]^T  -> dx rows
+  int rc;
+  // ---- ELL rows: dh, du, dg, dx
+  EllBwdParams p{xb, dyb, static_cast<const uint16_t*>(wg_t), static_cast<const uint16_t*>(wu_t),
+                 static_cast<const uint16_t*>(wd), static_cast<uint16_t*>(dx), hv, ws, static_cast<int>(d)};
+  if (nvec <= kBwdThreads) rc = launch_ell_bwd<1>(p, n, st);
+  else if (nvec <= 2 * kBwdThreads) rc = launch_ell_bwd<2>(p, n, st);
+  else if (nvec <= 3 * kBwdThreads) rc = launch_ell_bwd<3>(p, n, st);
+  else rc = launch_ell_bwd<4>(p, n, st);
+  if (rc) return rc;
+  // ---- spill rows: dH = dY_s W_down^T on tensor cores, epilogue dU | dG
+  using Sh = TcPairShape<128, 1>;  // N = F in 128-wide tiles: few spill row tiles still spread
+  using Sx = TcPairShape<64, 1>;   // N = d in 64-wide tiles, for the same reason
+  if (s_max > 0) {
+    gather_rows_kernel<<<sp, 256, 0, st>>>(dyb, hy->spill_rows, hy->n_spill, s_max, static_cast<int>(d),
+                                           ws.dys);
+    if ((rc = check_launch("hybrid_ffn_bwd (gather)"))) return rc;
+    CUtensorMap m1a, m1b;
+    if ((rc = make_tmap_bf16(&m1a, ws.dys, sp, d, d, kBM))) return rc;
+    if ((rc = make_tmap_bf16(&m1b, wd, f, d, d, Sh::BN / 2))) return rc;
+    EpiBwdSpill e1{hv.spill_a, hv.spill_u, ws.acat, hy->n_spill, s_max, static_cast<int>(f), sp};
+    if ((rc = launch_tc_gemm_pair<Sh>(m1a, m1b, m1b, sp, f, d, e1, nullptr, st, "hybrid_ffn_bwd (dH)")))
+      return rc;
+  }
+  // ---- every stored entry (ELL and spill rows) bucketed by hidden unit,
+  // ordered by token
+  cudaError_t e = cudaMemsetAsync(ws.col_count, 0, sizeof(int) * f, st);
+  if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "hybrid_ffn_bwd: %s", cudaGetErrorString(e));
+  const unsigned rb = static_cast<unsigned>((n + 7) / 8);
+  const dim3 sgrid(static_cast<unsigned>((f + 2047) / 2048), static_cast<unsigned>(s_max > 0 ? s_max : 1));
+  csc_count_kernel<<<rb, 256, 0, st>>>(hv, ws.col_count);
+  if (s_max > 0) csc_count_spill_kernel<<<sgrid, 256, 0, st>>>(hv, ws.col_count);
+  csc_scan_kernel<<<1, 1024, 0, st>>>(ws.col_count, static_cast<int>(f), ws.col_start, ws.col_cursor);
+  csc_scatter_kernel<<<rb, 256, 0, st>>>(hv, ws.col_cursor, ws.csc);
+  if (s_max > 0) csc_scatter_spill_kernel<<<sgrid, 256, 0, st>>>(hv, ws.col_cursor, ws.csc);
+  csc_sort_kernel<<<static_cast<unsigned>((f + 7) / 8), 256, 0, st>>>(ws.col_start, static_cast<int>(f),
+                                                                     ws.csc, ws.csc_sorted);
+  if ((rc = check_launch("hybrid_ffn_bwd (column buckets)"))) return rc;
+  // ---- weight gradients, each row written once
+  DwParams q{xb, dyb, hv, ws, dwg_t, dwu_t, dwd, static_cast<int>(d)};
+  if (nvec <= kBwdThreads) rc = launch_dw<1>(q, static_cast<int>(f), st);
+  else if (nvec <= 2 * kBwdThreads) rc = launch_dw<2>(q, static_cast<int>(f), st);
+  else if (nvec <= 3 * kBwdThreads) rc = launch_dw<3>(q, static_cast<int>(f), st);
+  else rc = launch_dw<4>(q, static_cast<int>(f), st);
+  if (rc || s_max == 0) return rc;
+  // ---- dX_s = [dU | dG] [W_up ; W_gate]^T -> dx rows of the spill tokens
+  const uint16_t* bcat = static_cast<const uint16_t*>(w_ug);
+  if (!bcat) {
+    if ((rc = build_up_gate(wu_t, wg_t, ws.bcat, f, d, st))) return rc;
+    bcat = ws.bcat;
+  }
   CUtensorMap m2a, m2b;
   if ((rc = make_tmap_bf16(&m2a, ws.acat, sp, 2 * f, 2 * f, kBM))) return rc;
-  if ((rc = make_tmap_bf16(&m2b, ws.bcat, d, 2 * f, 2 * f, Sx::BN / 2))) return rc;
+  if ((rc = make_tmap_bf16(&m2b, bcat, d, 2 * f, 2 * f, Sx::BN / 2))) return rc;
   EpiScatterRowsBwd e2{static_cast<uint16_t*>(dx), hy->spill_rows, hy->n_spill, s_max, static_cast<int>(d)};
-  if ((rc = launch_tc_gemm_pair<Sx>(m2a, m2b, m2b, sp, d, 2 * f, e2, nullptr, st, "hybrid_ffn_bwd (dX)")))
-    return rc;
-  // dW_down += H^T dY_s
-  CUtensorMap m3a, m3b;
-  if ((rc = make_tmap_bf16(&m3a, ws.hs_t, f, sp, sp, kBM))) return rc;
-  if ((rc = make_tmap_bf16(&m3b, ws.dys_t, d, sp, sp, S::BN / 2))) return rc;
-  EpiAddF32 e3{dwd, nullptr, f, static_cast<int>(d), hy->n_spill, s_max};
-  if ((rc = launch_tc_gemm_pair<S>(m3a, m3b, m3b, f, d, sp, e3, nullptr, st, "hybrid_ffn_bwd (dW_down)")))
-    return rc;
-  // [dW_up ; dW_gate] += [dU | dG]^T X_s
-  CUtensorMap m4a, m4b;
-  if ((rc = make_tmap_bf16(&m4a, ws.acat_t, 2 * f, sp, sp, kBM))) return rc;
-  if ((rc = make_tmap_bf16(&m4b, ws.xs_t, d, sp, sp, S::BN / 2))) return rc;
-  EpiAddF32 e4{dwu_t, dwg_t, f, static_cast<int>(d), hy->n_spill, s_max};
-  return launch_tc_gemm_pair<S>(m4a, m4b, m4b, 2 * f, d, sp, e4, nullptr, st,
-                                "hybrid_ffn_bwd (dW_up, dW_gate)");
+  return launch_tc_gemm_pair<Sx>(m2a, m2b, m2b, sp, d, 2 * f, e2, nullptr, st, "hybrid_ffn_bwd (dX)");
 }

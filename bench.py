@@ -658,11 +658,17 @@ def run_train(args, local_rank):
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    # weight layouts built once per weight update: W_down^T (the forward's
+    # spill down GEMM) and [W_up | W_gate] (the backward's dX GEMM)
+    w_ug = sge.transpose_up_gate(wu, wg)
+    grads = (torch.empty_like(x),) + tuple(torch.empty((f, d), dtype=torch.float32, device=dev)
+                                           for _ in range(3))
+
     def step():
         sge.twell_gate_pack(x, wg, cfg.tile, cfg.cap, out=tw)
         sge.hybrid_pack(tw, cfg.ell_cap, cfg.s_max, out=hy, diag=diag)
         sge.hybrid_ffn_fwd(x, hy, wu, wd, wd_t=wd_t, y=y, workspace=fws)
-        return sge.hybrid_ffn_bwd(x, dy, hy, wg, wu, wd, workspace=bws)
+        return sge.hybrid_ffn_bwd(x, dy, hy, wg, wu, wd, workspace=bws, w_ug=w_ug, out=grads)
 
     xr = x.detach().clone().requires_grad_(True)
     wgr, wur, wdr = (w.detach().clone().requires_grad_(True) for w in (wg, wu, wd))
@@ -725,7 +731,7 @@ def run_train(args, local_rank):
     def hybrid_bwd(saved):
         hy_, _ = saved
         ws_ = sge.hybrid_bwd_workspace(n, d, f, cfg.ell_cap, cfg.s_max, dev)
-        return sge.hybrid_ffn_bwd(x, dy, hy_, wg, wu, wd, workspace=ws_)
+        return sge.hybrid_ffn_bwd(x, dy, hy_, wg, wu, wd, workspace=ws_, w_ug=w_ug)
 
     def dense_fwd():
         return (torch.relu(xr @ wgr.t()) * (xr @ wur.t())) @ wdr
@@ -736,7 +742,7 @@ def run_train(args, local_rank):
         xr.grad = wgr.grad = wur.grad = wdr.grad = None
         return g
 
-    del tw, hy, y, fws, bws
+    del tw, hy, y, fws, bws, grads
     h_held, h_peak = measure(hybrid_fwd, hybrid_bwd)
     d_held, d_peak = measure(dense_fwd, dense_bwd)
     return {
@@ -759,8 +765,9 @@ def run_train(args, local_rank):
                    "backward plus y (hybrid: ELL rows, routing and the S_max-row spill buffers; "
                    "dense autograd: relu(G), U and h); the peaks include workspaces, the "
                    "hybrid's transient TwELL (C = T) and its fp32 weight gradients (dense: bf16)"},
-        "gpu_launches_per_step": 24,
-        "launches_note": "gate 1, pack 2, forward 4 (ELL, gather, 2 GEMMs), backward 17 (ELL, 4 bucket kernels, dW, gather, 6 transposes, 3 GEMMs)",
+        "gpu_launches_per_step": 21,
+        "launches_note": "gate 1, pack 3 (counts, route, fill), forward 4 (ELL, gather, 2 GEMMs), backward 13 "
+                         "(ELL, gather, dH GEMM, bucket memset, 2 counts, scan, 2 scatters, sort, dW, dX GEMM)",
         "clocks": clk.summary(), "diag": diag.tolist(),
     }
 

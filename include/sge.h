@@ -377,10 +377,14 @@ int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* wu_t, const 
  *   dx = sum_j du W_up[:, j] + dg W_gate[:, j],
  *   dW_down[j] = sum_t a u dy_t, dW_up[:, j] = sum_t du x_t,
  *   dW_gate[:, j] = sum_t dg x_t.
- * ELL rows run on CUDA cores (weight gradients summed per hidden unit in
- * ascending token order); spill rows run as tcgen05 GEMMs whose results are
- * added to the same fp32 rows.  Deterministic.
+ * ELL rows run on CUDA cores; spill rows' dh and dx run as tcgen05 GEMMs.
+ * The weight gradients sum every stored entry (ELL entries and the spill
+ * rows' active columns) per hidden unit in ascending token order, one fp32
+ * row written once per unit.  Deterministic.
  *   x, dy, dx [N][d] bf16; wg_t, wu_t, wd [F][d] bf16;
+ *   w_ug [d][2F] bf16 or NULL: [W_up | W_gate] (row i = W_up[i, :] then
+ *   W_gate[i, :]), the dX GEMM's operand, built once per weight update by
+ *   sge_transpose_up_gate; NULL builds it in the workspace on every call;
  *   dwg_t, dwu_t [F][d] fp32 (neuron-major like the weights), dwd [F][d] fp32,
  *   all overwritten; dropped rows get dx = 0 and add nothing.
  *   workspace >= hybrid_ffn_bwd_workspace_bytes(N, d, F, K, S_max) bytes,
@@ -390,9 +394,20 @@ size_t hybrid_ffn_bwd_workspace_bytes(int64_t n_tokens, int64_t d_model, int64_t
                                       int s_max);
 
 int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* hy, const void* wg_t,
-                   const void* wu_t, const void* wd, void* dx, float* dwg_t, float* dwu_t,
-                   float* dwd, int64_t d_model, void* workspace, size_t workspace_bytes,
+                   const void* wu_t, const void* wd, const void* w_ug, void* dx, float* dwg_t,
+                   float* dwu_t, float* dwd, int64_t d_model, void* workspace, size_t workspace_bytes,
                    void* stream);
+
+/*
+ * sge_transpose_up_gate -- builds w_ug [d][2F] = [W_up | W_gate] (row i:
+ * W_up[i, :] = column i of wu_t, then W_gate[i, :]) for hybrid_ffn_bwd, a
+ * layout step for loading (or updating) the weights, not part of a step.
+ *   wu_t, wg_t [F][d] bf16; w_ug [d][2F] bf16, caller-allocated.
+ * Errors: SGE_ERR_ARG for null or misaligned pointers, F or d not a multiple
+ * of 8.  Stream-ordered.
+ */
+int sge_transpose_up_gate(const void* wu_t, const void* wg_t, void* w_ug, int64_t d_ff,
+                          int64_t d_model, void* stream);
 
 #ifdef __cplusplus
 }

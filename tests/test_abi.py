@@ -185,3 +185,12 @@ def test_routed_rejects_bad_arguments(lib):
     small = lib.twell_hybrid_up_down_workspace_bytes(1000, 64, 256, 0)
     assert need >= small + 64 * (64 + 2 * 256) * 2
     assert lib.twell_hybrid_up_down_workspace_bytes(1000, 64, 256, -1) == 0
+
+
+def test_transpose_up_gate_rejects_bad_arguments(lib):
+    p = ctypes.c_void_p(4096)
+    assert lib.sge_transpose_up_gate(p, p, p, 100, 64, None) == 1     # F % 8
+    assert lib.sge_transpose_up_gate(p, None, p, 128, 64, None) == 1
+    assert b"null" in lib.sge_last_error()
+    assert lib.sge_transpose_up_gate(ctypes.c_void_p(4100), p, p, 128, 64, None) == 1
+    assert b"aligned" in lib.sge_last_error()

@@ -226,7 +226,10 @@ def test_hybrid_train_workload_full_gradients(cuda_device):
     hy = sge.hybrid_pack(tw, cfg.ell_cap, cfg.s_max, diag=diag)
     y = sge.hybrid_ffn_fwd(x, hy, wu, wd, wd.t().contiguous())
     got = sge.hybrid_ffn_bwd(x, dy, hy, wg, wu, wd)
+    # the dX operand built once (a weight-loading step) gives the same bits
+    got2 = sge.hybrid_ffn_bwd(x, dy, hy, wg, wu, wd, w_ug=sge.transpose_up_gate(wu, wg))
     torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(got, got2))
     n_spill = int(hy.n_spill.item())
     assert 0 < n_spill <= cfg.s_max and int(diag[2]) == 0, n_spill
     o = _train_oracle(inp)
