@@ -324,9 +324,16 @@ struct DwParams {
   int d;
 };
 
+constexpr int kDwStage = 256;  // entries of a column whose metadata is staged at once
+
 template <int NV>
 __global__ void __launch_bounds__(kBwdThreads) dw_ell_kernel(DwParams p) {
   constexpr int VEC = 8;
+  // the entries' tokens and (h, du, dg), loaded for a whole round of the
+  // column's bucket by all threads at once; the rows of x and dy then
+  // stream two entries at a time
+  __shared__ int s_t[kDwStage];
+  __shared__ float s_h[kDwStage], s_du[kDwStage], s_dg[kDwStage];
   const int j = blockIdx.x;
   const int tid = threadIdx.x;
   const int nvec = p.d / VEC;
@@ -336,41 +343,68 @@ __global__ void __launch_bounds__(kBwdThreads) dw_ell_kernel(DwParams p) {
 #pragma unroll
     for (int q = 0; q < VEC; ++q) ad[k][q] = au[k][q] = ag[k][q] = 0.0f;
   const int s0 = p.ws.col_start[j], s1 = p.ws.col_start[j + 1];
-  for (int i = s0; i < s1; ++i) {
-    const int2 te = p.ws.csc_sorted[i];
-    float a, u, du, dg;
-    if (te.y >= 0) {  // an ELL entry: slot te.y of row te.x
-      const int64_t rk = static_cast<int64_t>(te.x) * p.hv.k + te.y;
-      a = __uint_as_float(static_cast<uint32_t>(p.hv.ell_a[rk]) << 16);
-      u = __uint_as_float(static_cast<uint32_t>(p.hv.ell_u[rk]) << 16);
-      du = p.ws.du[rk];
-      dg = p.ws.dg[rk];
-    } else {  // an active column of spill rank -te.y - 1
-      const int64_t r = -te.y - 1;
-      a = __uint_as_float(static_cast<uint32_t>(p.hv.spill_a[r * p.hv.f + j]) << 16);
-      u = __uint_as_float(static_cast<uint32_t>(p.hv.spill_u[r * p.hv.f + j]) << 16);
-      du = __uint_as_float(static_cast<uint32_t>(p.ws.acat[r * 2 * p.hv.f + j]) << 16);
-      dg = __uint_as_float(static_cast<uint32_t>(p.ws.acat[r * 2 * p.hv.f + p.hv.f + j]) << 16);
+  for (int r0 = s0; r0 < s1; r0 += kDwStage) {
+    const int rn = min(kDwStage, s1 - r0);
+    __syncthreads();  // the previous round's metadata has been used
+    for (int i = tid; i < rn; i += kBwdThreads) {
+      const int2 te = p.ws.csc_sorted[r0 + i];
+      float a, u, du, dg;
+      if (te.y >= 0) {  // an ELL entry: slot te.y of row te.x
+        const int64_t rk = static_cast<int64_t>(te.x) * p.hv.k + te.y;
+        a = __uint_as_float(static_cast<uint32_t>(p.hv.ell_a[rk]) << 16);
+        u = __uint_as_float(static_cast<uint32_t>(p.hv.ell_u[rk]) << 16);
+        du = p.ws.du[rk];
+        dg = p.ws.dg[rk];
+      } else {  // an active column of spill rank -te.y - 1
+        const int64_t r = -te.y - 1;
+        a = __uint_as_float(static_cast<uint32_t>(p.hv.spill_a[r * p.hv.f + j]) << 16);
+        u = __uint_as_float(static_cast<uint32_t>(p.hv.spill_u[r * p.hv.f + j]) << 16);
+        du = __uint_as_float(static_cast<uint32_t>(p.ws.acat[r * 2 * p.hv.f + j]) << 16);
+        dg = __uint_as_float(static_cast<uint32_t>(p.ws.acat[r * 2 * p.hv.f + p.hv.f + j]) << 16);
+      }
+      s_t[i] = te.x;
+      s_h[i] = a * u;
+      s_du[i] = du;
+      s_dg[i] = dg;
     }
-    const float h = a * u;
-    const uint4* dyr = reinterpret_cast<const uint4*>(p.dy + static_cast<int64_t>(te.x) * p.d);
-    const uint4* xr = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(te.x) * p.d);
+    __syncthreads();
+    for (int i = 0; i < rn; i += 2) {
+      const bool two = i + 1 < rn;
+      const uint4* dyr0 = reinterpret_cast<const uint4*>(p.dy + static_cast<int64_t>(s_t[i]) * p.d);
+      const uint4* xr0 = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(s_t[i]) * p.d);
+      const uint4* dyr1 = reinterpret_cast<const uint4*>(p.dy + static_cast<int64_t>(s_t[two ? i + 1 : i]) * p.d);
+      const uint4* xr1 = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(s_t[two ? i + 1 : i]) * p.d);
+      uint4 y0[NV], x0[NV], y1[NV], x1[NV];
 #pragma unroll
-    for (int k = 0; k < NV; ++k) {
-      const int v = tid + k * kBwdThreads;
-      if (v >= nvec) continue;
-      const uint4 yv = __ldg(dyr + v), xv = __ldg(xr + v);
-      const uint32_t ys[4] = {yv.x, yv.y, yv.z, yv.w}, xs[4] = {xv.x, xv.y, xv.z, xv.w};
+      for (int k = 0; k < NV; ++k) {
+        const int v = tid + k * kBwdThreads;
+        const bool in = v < nvec;
+        y0[k] = in ? __ldg(dyr0 + v) : make_uint4(0, 0, 0, 0);
+        x0[k] = in ? __ldg(xr0 + v) : make_uint4(0, 0, 0, 0);
+        y1[k] = in && two ? __ldg(dyr1 + v) : make_uint4(0, 0, 0, 0);
+        x1[k] = in && two ? __ldg(xr1 + v) : make_uint4(0, 0, 0, 0);
+      }
+      // entry i, then entry i + 1: the sums keep ascending token order
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float y0 = __uint_as_float(ys[q] << 16), y1 = __uint_as_float(ys[q] & 0xFFFF0000u);
-        const float x0 = __uint_as_float(xs[q] << 16), x1 = __uint_as_float(xs[q] & 0xFFFF0000u);
-        ad[k][2 * q] = fmaf(h, y0, ad[k][2 * q]);
-        ad[k][2 * q + 1] = fmaf(h, y1, ad[k][2 * q + 1]);
-        au[k][2 * q] = fmaf(du, x0, au[k][2 * q]);
-        au[k][2 * q + 1] = fmaf(du, x1, au[k][2 * q + 1]);
-        ag[k][2 * q] = fmaf(dg, x0, ag[k][2 * q]);
-        ag[k][2 * q + 1] = fmaf(dg, x1, ag[k][2 * q + 1]);
+      for (int e = 0; e < 2; ++e) {
+        if (e == 1 && !two) break;
+        const float h = s_h[i + e], du = s_du[i + e], dg = s_dg[i + e];
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+          const uint4 yv = e ? y1[k] : y0[k], xv = e ? x1[k] : x0[k];
+          const uint32_t ys[4] = {yv.x, yv.y, yv.z, yv.w}, xs[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float ya = __uint_as_float(ys[q] << 16), yb = __uint_as_float(ys[q] & 0xFFFF0000u);
+            const float xa = __uint_as_float(xs[q] << 16), xb = __uint_as_float(xs[q] & 0xFFFF0000u);
+            ad[k][2 * q] = fmaf(h, ya, ad[k][2 * q]);
+            ad[k][2 * q + 1] = fmaf(h, yb, ad[k][2 * q + 1]);
+            au[k][2 * q] = fmaf(du, xa, au[k][2 * q]);
+            au[k][2 * q + 1] = fmaf(du, xb, au[k][2 * q + 1]);
+            ag[k][2 * q] = fmaf(dg, xa, ag[k][2 * q]);
+            ag[k][2 * q + 1] = fmaf(dg, xb, ag[k][2 * q + 1]);
+          }
+        }
       }
     }
   }
