@@ -414,6 +414,34 @@ static __global__ void __launch_bounds__(256) ud_jobs_kernel(int* __restrict__ n
   }
 }
 
+// v += the VEC floats at src + u * stride for u = 0 .. nu - 1, in unit order
+// (the fp32 partial rows of a split token's units); the loads of eight units
+// are issued together, then added in order.
+template <int VEC>
+__device__ __forceinline__ void sum_partials(const float* src, int64_t stride, int nu, float (&v)[VEC]) {
+  constexpr int B = 8;
+  for (int u0 = 0; u0 < nu; u0 += B) {
+    float4 f[B][VEC / 4];
+#pragma unroll
+    for (int b = 0; b < B; ++b)
+#pragma unroll
+      for (int q = 0; q < VEC / 4; ++q)
+        f[b][q] = u0 + b < nu ? __ldcg(reinterpret_cast<const float4*>(src + (u0 + b) * stride) + q)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      if (u0 + b >= nu) break;
+#pragma unroll
+      for (int q = 0; q < VEC / 4; ++q) {
+        v[4 * q] += f[b][q].x;
+        v[4 * q + 1] += f[b][q].y;
+        v[4 * q + 2] += f[b][q].z;
+        v[4 * q + 3] += f[b][q].w;
+      }
+    }
+  }
+}
+
 // -------------------------------------------------------------- main kernel
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -880,18 +908,7 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
                 float v[VEC];
 #pragma unroll
                 for (int q = 0; q < VEC; ++q) v[q] = 0.0f;
-                for (int u = 0; u < jb.nu; ++u) {
-                  const float4* src =
-                      reinterpret_cast<const float4*>(p.pool + static_cast<int64_t>(jb.base + u) * p.d + pc * VEC);
-#pragma unroll
-                  for (int q = 0; q < VEC / 4; ++q) {
-                    const float4 f = __ldcg(src + q);
-                    v[4 * q] += f.x;
-                    v[4 * q + 1] += f.y;
-                    v[4 * q + 2] += f.z;
-                    v[4 * q + 3] += f.w;
-                  }
-                }
+                sum_partials<VEC>(p.pool + static_cast<int64_t>(jb.base) * p.d + pc * VEC, p.d, jb.nu, v);
                 reinterpret_cast<uint4*>(yrow)[pc] = E::pack(v);
               }
             }
@@ -1201,15 +1218,7 @@ __global__ void __launch_bounds__(kSmWarps * 32, 1) us_main_kernel(const UsParam
           float v[VEC];
 #pragma unroll
           for (int q = 0; q < VEC; ++q) v[q] = 0.0f;
-          for (int w = 0; w < nu; ++w)
-#pragma unroll
-            for (int q = 0; q < VEC / 4; ++q) {
-              const float4 f = __ldcg(reinterpret_cast<const float4*>(base + static_cast<int64_t>(w) * p.d + pc * VEC) + q);
-              v[4 * q] += f.x;
-              v[4 * q + 1] += f.y;
-              v[4 * q + 2] += f.z;
-              v[4 * q + 3] += f.w;
-            }
+          sum_partials<VEC>(base + pc * VEC, p.d, nu, v);
           reinterpret_cast<uint4*>(yrow)[pc] = E::pack(v);
         }
       }
