@@ -908,7 +908,18 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
                 float v[VEC];
 #pragma unroll
                 for (int q = 0; q < VEC; ++q) v[q] = 0.0f;
-                sum_partials<VEC>(p.pool + static_cast<int64_t>(jb.base) * p.d + pc * VEC, p.d, jb.nu, v);
+                for (int u = 0; u < jb.nu; ++u) {
+                  const float4* src =
+                      reinterpret_cast<const float4*>(p.pool + static_cast<int64_t>(jb.base + u) * p.d + pc * VEC);
+#pragma unroll
+                  for (int q = 0; q < VEC / 4; ++q) {
+                    const float4 f = __ldcg(src + q);
+                    v[4 * q] += f.x;
+                    v[4 * q + 1] += f.y;
+                    v[4 * q + 2] += f.z;
+                    v[4 * q + 3] += f.w;
+                  }
+                }
                 reinterpret_cast<uint4*>(yrow)[pc] = E::pack(v);
               }
             }
