@@ -339,7 +339,9 @@ extern "C" int hybrid_pack(const uint8_t* count, const uint8_t* idx, const void*
 
 extern "C" size_t hybrid_ffn_fwd_workspace_bytes(int64_t d_model, int64_t d_ff, int s_max) {
   if (d_model < 0 || d_ff < 0 || s_max < 0) return 0;
-  return static_cast<size_t>(s_max) * static_cast<size_t>(d_model + d_ff) * 2 + 256;
+  if (s_max == 0) return 256;
+  // X_s and H_s in bf16, then the split-K partial products and counters
+  return align256(static_cast<size_t>(s_max) * static_cast<size_t>(d_model + d_ff) * 2) + kSplitPartBytes + 256;
 }
 
 template <int NV>
@@ -385,7 +387,7 @@ extern "C" int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* w
   gather_rows_kernel<<<hy->s_max, 256, 0, st>>>(static_cast<const uint16_t*>(x), hy->spill_rows,
                                                  hy->n_spill, hy->s_max, static_cast<int>(d_model), xs);
   if ((rc = check_launch("hybrid_ffn_fwd (gather)"))) return rc;
-  using S = TcPairShape<256, 1>;
+  using S = TcPairShape<256, 1, 2>;
   CUtensorMap ma, mb, mh, md;
   if ((rc = make_tmap_bf16(&ma, xs, hy->s_max, d_model, d_model, kBM))) return rc;
   if (wg_t) {
@@ -409,8 +411,15 @@ extern "C" int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* w
   }
   if ((rc = make_tmap_bf16(&mh, hs, hy->s_max, hy->d_ff, hy->d_ff, kBM))) return rc;
   if ((rc = make_tmap_bf16(&md, wd_t, d_model, hy->d_ff, hy->d_ff, S::BN / 2))) return rc;
+  char* split_base = reinterpret_cast<char*>(workspace) +
+                     align256(static_cast<size_t>(hy->s_max) * static_cast<size_t>(d_model + hy->d_ff) * 2);
+  float* part = reinterpret_cast<float*>(split_base);
+  const int tiles_n = static_cast<int>((d_model + S::BN - 1) / S::BN);
   EpiScatterRows e2{static_cast<uint16_t*>(y), hy->spill_rows, hy->n_spill, hy->s_max,
-                    static_cast<int>(d_model)};
-  return launch_tc_gemm_pair<S>(mh, md, md, hy->s_max, d_model, hy->d_ff, e2, nullptr, st,
-                                "hybrid_ffn_fwd (spill down)");
+                    static_cast<int>(d_model), part, tiles_n, S::BN};
+  if ((rc = launch_tc_gemm_pair<S>(mh, md, md, hy->s_max, d_model, hy->d_ff, e2, nullptr, st,
+                                   "hybrid_ffn_fwd (spill down)", kSplitMax)))
+    return rc;
+  return launch_split_scatter(part, hy->spill_rows, hy->n_spill, hy->s_max, static_cast<int>(d_model),
+                              tiles_n * S::BN, static_cast<uint16_t*>(y), st, "hybrid_ffn_fwd (split sum)");
 }

@@ -59,10 +59,10 @@ struct BwdWs {
   uint16_t* acat;    // [Sp][2F]  dU | dG
   uint16_t* bcat;    // [d][2F]   W_up | W_gate (row i = row i of W_up, W_gate), when the
                      //           caller passes none
+  float* part;       // split-K partial products of the dX GEMM
   size_t bytes;
 };
 
-static size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 
 static BwdWs carve(void* base, int64_t n, int64_t d, int64_t f, int k, int s_max) {
   BwdWs w{};
@@ -87,6 +87,7 @@ static BwdWs carve(void* base, int64_t n, int64_t d, int64_t f, int k, int s_max
     w.dys = reinterpret_cast<uint16_t*>(take(sp * d * 2));
     w.acat = reinterpret_cast<uint16_t*>(take(sp * 2 * f * 2));
     w.bcat = reinterpret_cast<uint16_t*>(take(d * 2 * f * 2));
+    w.part = reinterpret_cast<float*>(take(kSplitPartBytes));
   }
   w.bytes = off;
   return w;
@@ -530,43 +531,6 @@ struct EpiBwdSpill {
   }
 };
 
-// Epilogue: row r of D goes to dst[rows[r]] (bf16) for the kept rows.
-struct EpiScatterRowsBwd {
-  uint16_t* dst;
-  const int32_t* rows;
-  const int32_t* n_spill;
-  int s_max;
-  int n_cols;
-
-  // only the kept spill rows are computed
-  __device__ __forceinline__ int m_limit(int m) const { return min(m, min(*n_spill, s_max)); }
-
-  template <int BN>
-  __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {
-    const int kept = min(*n_spill, s_max);
-    const int64_t t = row < kept ? rows[row] : -1;
-#pragma unroll 1
-    for (int ch = 0; ch < BN / 32; ++ch) {
-      uint32_t r[32];
-      tmem_ld32(taddr + ch * 32, r);
-      tmem_ld_wait();
-      const int col0 = n_blk * BN + ch * 32;
-      if (t < 0) continue;
-      uint16_t* o = dst + t * n_cols + col0;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (col0 + q * 8 + 8 > n_cols) break;
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          w[i] = static_cast<uint32_t>(f32_to_bf16_bits(__uint_as_float(r[q * 8 + 2 * i]))) |
-                 (static_cast<uint32_t>(f32_to_bf16_bits(__uint_as_float(r[q * 8 + 2 * i + 1]))) << 16);
-        *reinterpret_cast<uint4*>(o + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    }
-  }
-};
-
 static int launch_transpose(const uint16_t* src, int rows, int cols, int64_t src_pitch,
                             uint16_t* dst, int64_t dst_pitch, int col_off, cudaStream_t st,
                             const int32_t* rows_dev = nullptr, int rows_cap = 0) {
@@ -672,7 +636,7 @@ extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* h
   if (rc) return rc;
   // ---- spill rows: dH = dY_s W_down^T on tensor cores, epilogue dU | dG
   using Sh = TcPairShape<128, 1>;  // N = F in 128-wide tiles: few spill row tiles still spread
-  using Sx = TcPairShape<64, 1>;   // N = d in 64-wide tiles, for the same reason
+  using Sx = TcPairShape<256, 1, 2>;  // N = d: few tiles, K = 2F split over the CTA pairs
   if (s_max > 0) {
     gather_rows_kernel<<<sp, 256, 0, st>>>(dyb, hy->spill_rows, hy->n_spill, s_max, static_cast<int>(d),
                                            ws.dys);
@@ -714,6 +678,12 @@ extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* h
   CUtensorMap m2a, m2b;
   if ((rc = make_tmap_bf16(&m2a, ws.acat, sp, 2 * f, 2 * f, kBM))) return rc;
   if ((rc = make_tmap_bf16(&m2b, bcat, d, 2 * f, 2 * f, Sx::BN / 2))) return rc;
-  EpiScatterRowsBwd e2{static_cast<uint16_t*>(dx), hy->spill_rows, hy->n_spill, s_max, static_cast<int>(d)};
-  return launch_tc_gemm_pair<Sx>(m2a, m2b, m2b, sp, d, 2 * f, e2, nullptr, st, "hybrid_ffn_bwd (dX)");
+  const int tiles_n = static_cast<int>((d + Sx::BN - 1) / Sx::BN);
+  EpiScatterRows e2{static_cast<uint16_t*>(dx), hy->spill_rows, hy->n_spill, s_max, static_cast<int>(d),
+                    ws.part, tiles_n, Sx::BN};
+  if ((rc = launch_tc_gemm_pair<Sx>(m2a, m2b, m2b, sp, d, 2 * f, e2, nullptr, st, "hybrid_ffn_bwd (dX)",
+                                    kSplitMax)))
+    return rc;
+  return launch_split_scatter(ws.part, hy->spill_rows, hy->n_spill, s_max, static_cast<int>(d),
+                              tiles_n * Sx::BN, static_cast<uint16_t*>(dx), st, "hybrid_ffn_bwd (split sum)");
 }

@@ -11,10 +11,13 @@
 //
 //   plan    stored entries per token; tokens with more than K stored entries
 //           are heavy and ranked in ascending token order; the first S_max
-//           go to the spill list (fused_kernels.cuh's planning kernels)
-//   light   on a stream of the library's own, at the same time as the spill:
-//           every other token through CUDA cores (light_fwd_kernel below),
-//           y = 0 for tokens without stored entries
+//           go to the spill list, every other non-empty token to a size
+//           class of the light lists (fused_kernels.cuh's planning kernels)
+//   light   the light tokens (and heavy ones past S_max) through CUDA
+//           cores, one warp per token, its entries' W_up and W_down rows
+//           streamed through a ring of shared-memory slots filled by bulk
+//           copies (light_ring_kernel below); y = 0 for tokens without
+//           stored entries
 //   prep    per spill row: its x row into X_s, its stored activations
 //           scattered into a dense row of A_s (zeros elsewhere)
 //   GEMM 1  U = X_s W_up on tcgen05 (CTA pairs), epilogue H_s = bf16(A_s (.) U)
@@ -335,7 +338,7 @@ constexpr int kSpillBN = 256;
 
 struct RoutedLayout {
   WsLayout fused;
-  size_t heavy, rows, xs, as, hs, total;
+  size_t heavy, rows, xs, as, hs, part, total;
   RoutedLayout(int64_t n, int64_t d, int64_t f, int64_t s_max, int64_t pool_slots)
       : fused(n, d, pool_slots) {
     auto up = [](size_t v, size_t a) { return (v + a - 1) / a * a; };
@@ -347,6 +350,7 @@ struct RoutedLayout {
     xs = o;        o = up(o + 2 * sm * static_cast<size_t>(d), 1024);
     as = o;        o = up(o + 2 * sm * static_cast<size_t>(f), 1024);
     hs = o;        o = up(o + 2 * sm * static_cast<size_t>(f), 1024);
+    part = o;      o = up(o + (sm > 0 ? kSplitPartBytes : 0), 1024);
     total = o;
   }
 };
@@ -443,6 +447,7 @@ extern "C" int twell_hybrid_up_down(const void* x, const uint8_t* count, const u
   uint16_t* xs = reinterpret_cast<uint16_t*>(ws + L.xs);
   uint16_t* as = reinterpret_cast<uint16_t*>(ws + L.as);
   uint16_t* hs = reinterpret_cast<uint16_t*>(ws + L.hs);
+  float* part = reinterpret_cast<float*>(ws + L.part);
   const RouteArgs route{ell_cap, s_max, 1, reinterpret_cast<int2*>(ws + L.heavy), spill_rows, diag};
   if ((rc = fused_launch_plan(c, route, st))) return rc;
 
@@ -476,7 +481,11 @@ extern "C" int twell_hybrid_up_down(const void* x, const uint8_t* count, const u
     return rc;
   if ((rc = make_tmap_bf16(&mh, hs, s_max, d_ff, d_ff, kBM))) return rc;
   if ((rc = make_tmap_bf16(&md, wd_t, d_model, d_ff, d_ff, S::BN / 2))) return rc;
-  EpiScatterRows e2{static_cast<uint16_t*>(y), spill_rows, n_heavy, s_max, d};
-  return launch_tc_gemm_pair<S>(mh, md, md, s_max, d_model, d_ff, e2, diag, st,
-                                "twell_hybrid_up_down (spill down)");
+  const int tiles_n = (d + S::BN - 1) / S::BN;
+  EpiScatterRows e2{static_cast<uint16_t*>(y), spill_rows, n_heavy, s_max, d, part, tiles_n, S::BN};
+  if ((rc = launch_tc_gemm_pair<S>(mh, md, md, s_max, d_model, d_ff, e2, diag, st,
+                                   "twell_hybrid_up_down (spill down)", kSplitMax)))
+    return rc;
+  return launch_split_scatter(part, spill_rows, n_heavy, s_max, d, tiles_n * S::BN, static_cast<uint16_t*>(y),
+                              st, "twell_hybrid_up_down (split sum)");
 }

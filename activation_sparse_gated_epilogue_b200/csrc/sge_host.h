@@ -21,6 +21,8 @@ int check_launch(const char* what);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+inline size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
 // Multiprocessor count of the current device (cached per device).
 int sm_count();
 

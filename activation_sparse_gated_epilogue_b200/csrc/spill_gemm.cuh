@@ -7,6 +7,7 @@
 // the dense backup path on tensor cores).
 #pragma once
 
+#include "sge_host.h"
 #include "tc_gemm.cuh"
 
 namespace sge {
@@ -142,40 +143,156 @@ struct EpiSpillGateUp {
 };
 
 // Epilogue of Y_s = H_s W_down: row r of the tile goes to y[spill_rows[r]].
+// Split-K of the scatter GEMMs.  With few spill rows the output has fewer
+// tiles than there are CTA pairs (130 spill rows and d = 2048: 8 tiles of
+// 256 x 256 for 74 pairs), so the GEMM would stream the weights through a
+// few SMs only.  The epilogue then asks for K to be cut into up to
+// kSplitMax parts, so that tiles x parts fill the pairs; each part stores
+// its fp32 product, and split_scatter_kernel adds the parts in part order
+// and writes the bf16 rows: results do not depend on timing.
+constexpr int kSplitMax = 16;
+// capacity of the partial-product area in 256 x 256 fp32 tiles (at least
+// the number of CTA pairs that can be resident)
+constexpr int kSplitTiles = 80;
+constexpr size_t kSplitPartBytes = static_cast<size_t>(kSplitTiles) * 256 * 256 * 4 + 256;
+
+// Y_s = H_s W (W's rows K-major): row r of the product goes to y[rows[r]]
+// (bf16) for the kept spill rows r < min(*n_spill, s_max).  With `part`
+// (kSplitPartBytes) K may be split: the parts go to part[split][row][col]
+// (rows padded to the launch's 256-row tiles, columns to its n_tiles_n
+// tiles), the number of parts to the word after them, and
+// split_scatter_kernel finishes the rows; with part == nullptr every tile
+// takes all of K.
 struct EpiScatterRows {
   uint16_t* y;
   const int32_t* rows;
   const int32_t* n_spill;
   int s_max;
   int n_cols;
+  float* part = nullptr;
+  int n_tiles_n = 1;  // output column tiles of the launch (N / Shape::BN rounded up)
+  int tile_n = 256;   // Shape::BN
 
   // only the kept spill rows are computed
   __device__ __forceinline__ int m_limit(int m) const { return min(m, min(*n_spill, s_max)); }
 
+  __device__ __forceinline__ int splits() const {
+    if (part == nullptr) return 1;
+    const int units = ((min(*n_spill, s_max) + 255) / 256) * n_tiles_n;
+    if (units == 0) return 1;
+    const int pairs = min(static_cast<int>(cluster_count_x()), kSplitTiles);
+    return max(1, min(kSplitMax, pairs / units));
+  }
+
   template <int BN>
-  __device__ __forceinline__ void run(uint32_t taddr, int64_t row, int n_blk, int lane) const {
+  __device__ __forceinline__ void run_split(uint32_t taddr, int64_t row, int n_blk, int split, int nsplit,
+                                            int lane) const {
     const int kept = min(*n_spill, s_max);
+    if (part != nullptr && row == 0 && n_blk == 0 && split == 0)
+      reinterpret_cast<int*>(part)[kSplitTiles * 256 * 256] = nsplit;  // for split_scatter_kernel
     const int64_t t = row < kept ? rows[row] : -1;
+    if (nsplit == 1) {
+      uint16_t* o = t >= 0 ? y + t * n_cols : nullptr;
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        uint32_t r[32];
+        tmem_ld32(taddr + ch * 32, r);
+        tmem_ld_wait();
+        const int col0 = n_blk * BN + ch * 32;
+        if (t < 0) continue;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (col0 + q * 8 + 8 > n_cols) break;
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            w[i] = static_cast<uint32_t>(f32_to_bf16_bits(__uint_as_float(r[q * 8 + 2 * i]))) |
+                   (static_cast<uint32_t>(f32_to_bf16_bits(__uint_as_float(r[q * 8 + 2 * i + 1]))) << 16);
+          *reinterpret_cast<uint4*>(o + col0 + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      return;
+    }
+    // part[split][row][col], rows padded to the launch's row tiles
+    const int64_t ncp = static_cast<int64_t>(n_tiles_n) * tile_n;
+    const int64_t rows_pad = static_cast<int64_t>((kept + 255) / 256) * 256;
+    float* dst = part + (split * rows_pad + row) * ncp + n_blk * BN;
 #pragma unroll 1
     for (int ch = 0; ch < BN / 32; ++ch) {
       uint32_t r[32];
       tmem_ld32(taddr + ch * 32, r);
       tmem_ld_wait();
-      const int col0 = n_blk * BN + ch * 32;
       if (t < 0) continue;
-      uint16_t* o = y + t * n_cols + col0;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (col0 + q * 8 + 8 > n_cols) break;
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          w[i] = static_cast<uint32_t>(f32_to_bf16_bits(__uint_as_float(r[q * 8 + 2 * i]))) |
-                 (static_cast<uint32_t>(f32_to_bf16_bits(__uint_as_float(r[q * 8 + 2 * i + 1]))) << 16);
-        *reinterpret_cast<uint4*>(o + q * 8) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
+      for (int q = 0; q < 8; ++q)
+        __stcg(reinterpret_cast<float4*>(dst + ch * 32) + q,
+               make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                           __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3])));
     }
   }
 };
+
+// Finishes a split scatter GEMM: y[rows[r]][c] = bf16(sum over parts, in
+// part order, of part[s][r][c]) for the kept rows; nothing when the GEMM
+// did not split (it wrote y itself).  A thread per 8 columns of a row, the
+// loads of four parts in flight at once.
+static __global__ void __launch_bounds__(256) split_scatter_kernel(const float* __restrict__ part,
+                                                                   const int32_t* __restrict__ rows,
+                                                                   const int32_t* __restrict__ n_spill,
+                                                                   int s_max, int n_cols, int ncp,
+                                                                   uint16_t* __restrict__ y) {
+  const int nsplit = reinterpret_cast<const int*>(part)[kSplitTiles * 256 * 256];
+  const int kept = min(*n_spill, s_max);
+  if (nsplit <= 1 || kept <= 0) return;
+  const int64_t rows_pad = static_cast<int64_t>((kept + 255) / 256) * 256;
+  const int per_row = n_cols / 8;
+  const int64_t total = static_cast<int64_t>(kept) * per_row;
+  for (int64_t i = blockIdx.x * 256ll + threadIdx.x; i < total; i += static_cast<int64_t>(gridDim.x) * 256) {
+    const int r = static_cast<int>(i / per_row);
+    const int c = static_cast<int>(i % per_row) * 8;
+    const float* src = part + static_cast<int64_t>(r) * ncp + c;
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = 0.0f;
+    for (int s0 = 0; s0 < nsplit; s0 += 4) {
+      float4 f[4][2];
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          f[b][h] = s0 + b < nsplit
+                        ? __ldcg(reinterpret_cast<const float4*>(src + (s0 + b) * rows_pad * ncp) + h)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        if (s0 + b >= nsplit) break;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          v[4 * h] += f[b][h].x;
+          v[4 * h + 1] += f[b][h].y;
+          v[4 * h + 2] += f[b][h].z;
+          v[4 * h + 3] += f[b][h].w;
+        }
+      }
+    }
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      w[k] = static_cast<uint32_t>(f32_to_bf16_bits(v[2 * k])) |
+             (static_cast<uint32_t>(f32_to_bf16_bits(v[2 * k + 1])) << 16);
+    *reinterpret_cast<uint4*>(y + static_cast<int64_t>(rows[r]) * n_cols + c) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// Launches split_scatter_kernel after a scatter GEMM launched with `part`
+// (ncp = the GEMM's n_tiles_n * tile_n).
+static inline int launch_split_scatter(const float* part, const int32_t* rows, const int32_t* n_spill,
+                                       int s_max, int n_cols, int ncp, uint16_t* y, cudaStream_t st,
+                                       const char* what) {
+  const int64_t work = (static_cast<int64_t>(s_max) * (n_cols / 8) + 255) / 256;
+  const int grid = static_cast<int>(work < 4 * sm_count() ? (work > 0 ? work : 1) : 4 * sm_count());
+  split_scatter_kernel<<<grid, 256, 0, st>>>(part, rows, n_spill, s_max, n_cols, ncp, y);
+  return check_launch(what);
+}
 
 }  // namespace sge

@@ -234,8 +234,10 @@ int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, const uint8
  *                        s_max) bytes, 256-byte aligned, caller-owned, not
  *                        shared by calls that may run concurrently (the
  *                        per-entry kernel's lists and pool, the spill list,
- *                        and the spill operands X_s [S_max][d], A_s and H_s
- *                        [S_max][F] in bf16)
+ *                        the spill operands X_s [S_max][d], A_s and H_s
+ *                        [S_max][F] in bf16, and 21 MB for the down GEMM's
+ *                        split-K parts, used when the heavy tokens make
+ *                        fewer output tiles than there are CTA pairs)
  *   diag                 nullable; [SGE_DIAG_SPILL_ROWS] gains the number of
  *                        heavy tokens (those past S_max included),
  *                        [SGE_DIAG_FLAGS] SGE_FLAG_TIMEOUT if a wait gave up
@@ -349,6 +351,9 @@ int hybrid_pack(const uint8_t* count, const uint8_t* idx, const void* val, int t
  *             (fp32 accumulation; u_e saved to ell_u in bf16)
  *   spill rows: U = X_s W_up (all F columns, tcgen05), saved to spill_u;
  *             H = bf16(A (.) U); Y_s = H W_down (tcgen05), scattered to y.
+ *             When the spill rows make fewer output tiles of Y_s than
+ *             there are CTA pairs, its K (= F) is split over the pairs and
+ *             the fp32 parts are added in a fixed order (deterministic).
  *             With wg_t given, A is first recomputed from the gate,
  *             A = bf16(ReLU(X_s W_gate)) (one tcgen05 GEMM with two B
  *             operands, W_gate and W_up) and written to spill_a: the rows
@@ -360,7 +365,8 @@ int hybrid_pack(const uint8_t* count, const uint8_t* idx, const void* val, int t
  *   x [N][d], y [N][d], wu_t [F][d], wd [F][d], wd_t [d][F] (W_down
  *   transposed, the K-major operand of the spill GEMM; may be NULL when
  *   S_max == 0), wg_t [F][d] or NULL; workspace >=
- *   hybrid_ffn_fwd_workspace_bytes(d, F, S_max).
+ *   hybrid_ffn_fwd_workspace_bytes(d, F, S_max), 16-byte aligned: X_s and
+ *   H_s [S_max][d + F] bf16, then (S_max > 0) 21 MB of split-K parts.
  */
 size_t hybrid_ffn_fwd_workspace_bytes(int64_t d_model, int64_t d_ff, int s_max);
 
@@ -377,7 +383,9 @@ int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* wu_t, const 
  *   dx = sum_j du W_up[:, j] + dg W_gate[:, j],
  *   dW_down[j] = sum_t a u dy_t, dW_up[:, j] = sum_t du x_t,
  *   dW_gate[:, j] = sum_t dg x_t.
- * ELL rows run on CUDA cores; spill rows' dh and dx run as tcgen05 GEMMs.
+ * ELL rows run on CUDA cores; spill rows' dh and dx run as tcgen05 GEMMs
+ * (the dx GEMM's K = 2F split over the CTA pairs when its output has fewer
+ * tiles than there are pairs; parts added in a fixed order).
  * The weight gradients sum every stored entry (ELL entries and the spill
  * rows' active columns) per hidden unit in ascending token order, one fp32
  * row written once per unit.  Deterministic.
