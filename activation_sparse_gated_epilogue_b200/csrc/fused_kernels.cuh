@@ -200,6 +200,8 @@ static __global__ void __launch_bounds__(256) ud_count_kernel(const uint8_t* __r
                                                        RouteArgs route) {
   __shared__ long long wsum[8];
   __shared__ int2 wheavy[8];
+  grid_dep_launch();
+  grid_dep_wait();  // the counts come from the gate GEMM (no-op for a plain launch)
   const int64_t t = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   if (blockIdx.x == 0 && threadIdx.x < 16) {
     const int w = threadIdx.x;
@@ -298,6 +300,8 @@ static __global__ void __launch_bounds__(256) ud_jobs_kernel(int* __restrict__ n
                                                       int* hdr, int2* __restrict__ lights,
                                                       Job* __restrict__ units, int* __restrict__ done,
                                                       int64_t pool_slots, RouteArgs route) {
+  grid_dep_launch();
+  grid_dep_wait();
   __shared__ long long hsum[3][8];
   __shared__ int wrank[8];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1422,15 +1426,14 @@ static int fused_prepare(FusedCall& c, const char* name, const void* x, const ui
 // lists.
 static int fused_launch_plan(const FusedCall& c, const RouteArgs& route, cudaStream_t st) {
   const UdParams& prm = c.prm;
-  ud_count_kernel<<<static_cast<unsigned>(c.nblk), 256, 0, st>>>(
-      prm.count, prm.n_rows, prm.nt, prm.cap, const_cast<int*>(prm.ntok), c.blk, prm.hdr, route);
-  int rc = check_launch("fused up/down (count)");
+  int rc = launch_pdl(ud_count_kernel, dim3(static_cast<unsigned>(c.nblk)), dim3(256), 0, st,
+                      "fused up/down (count)", prm.count, prm.n_rows, prm.nt, prm.cap,
+                      const_cast<int*>(prm.ntok), c.blk, prm.hdr, route);
   if (rc) return rc;
-  ud_jobs_kernel<<<static_cast<unsigned>(c.nblk), 256, 0, st>>>(
-      const_cast<int*>(prm.ntok), prm.n_rows, c.blk, c.nblk, static_cast<int64_t>(c.grid) * prm.teams,
-      prm.hdr, const_cast<int2*>(prm.lights), const_cast<Job*>(prm.units), prm.done, c.pool_slots,
-      route);
-  return check_launch("fused up/down (jobs)");
+  return launch_pdl(ud_jobs_kernel, dim3(static_cast<unsigned>(c.nblk)), dim3(256), 0, st,
+                    "fused up/down (jobs)", const_cast<int*>(prm.ntok), prm.n_rows, c.blk, c.nblk,
+                    static_cast<int64_t>(c.grid) * prm.teams, prm.hdr, const_cast<int2*>(prm.lights),
+                    const_cast<Job*>(prm.units), prm.done, c.pool_slots, route);
 }
 
 static int fused_launch_main(const FusedCall& c, cudaStream_t st) {

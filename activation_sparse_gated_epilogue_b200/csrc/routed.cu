@@ -54,6 +54,8 @@ __global__ void __launch_bounds__(kPrepThreads) spill_prep_kernel(const uint16_t
                                                                   uint16_t* __restrict__ xs,
                                                                   uint16_t* __restrict__ as) {
   extern __shared__ __align__(16) uint8_t prep_smem[];
+  grid_dep_launch();
+  grid_dep_wait();
   uint16_t* row = reinterpret_cast<uint16_t*>(prep_smem);              // f bf16
   int* pre = reinterpret_cast<int*>(prep_smem + ((2 * f + 15) & ~15));  // nt + 1
   int* wsum = pre + 260;                                                // warps
@@ -146,6 +148,8 @@ struct RingParams {
 
 template <int NV, int NTR>
 __global__ void __launch_bounds__(kRingMaxWarps * 32, 1) light_ring_kernel(const RingParams p) {
+  grid_dep_launch();
+  grid_dep_wait();  // lists and counts come from the planning kernels
   using E = Elem<true>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -360,8 +364,7 @@ static int launch_ring(const RingParams& p, int warps, int smem, cudaStream_t st
   auto kern = light_ring_kernel<NV, NTR>;
   const int rc = set_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (rc) return rc;
-  kern<<<sm_count(), warps * 32, smem, st>>>(p);
-  return check_launch("twell_hybrid_up_down (light tokens)");
+  return launch_pdl(kern, dim3(sm_count()), dim3(warps * 32), smem, st, "twell_hybrid_up_down (light tokens)", p);
 }
 
 template <int NV>
@@ -466,10 +469,11 @@ extern "C" int twell_hybrid_up_down(const void* x, const uint8_t* count, const u
     const int smem = prep_smem_bytes(d_ff);
     if ((rc = set_smem_limit(reinterpret_cast<const void*>(spill_prep_kernel), smem))) return rc;
     const int prep_grid = static_cast<int>(std::min<int64_t>(s_max, 8 * static_cast<int64_t>(sm_count())));
-    spill_prep_kernel<<<prep_grid, kPrepThreads, smem, st>>>(
-        static_cast<const uint16_t*>(x), count, idx, static_cast<const uint16_t*>(val), spill_rows,
-        n_heavy, s_max, d, f, f / tile, tile, cap, xs, as);
-    if ((rc = check_launch("twell_hybrid_up_down (spill prep)"))) return rc;
+    if ((rc = launch_pdl(spill_prep_kernel, dim3(prep_grid), dim3(kPrepThreads), smem, st,
+                         "twell_hybrid_up_down (spill prep)", static_cast<const uint16_t*>(x), count, idx,
+                         static_cast<const uint16_t*>(val), spill_rows, n_heavy, s_max, d, f, f / tile,
+                         tile, cap, xs, as)))
+      return rc;
   }
   using S = TcPairShape<kSpillBN, 1, 2>;
   CUtensorMap ma, mb, mh, md;

@@ -200,6 +200,15 @@ SGE_DEV uint16_t f32_to_bf16_bits(float v) {
   return *reinterpret_cast<uint16_t*>(&b);
 }
 
+// Programmatic dependent launch.  grid_dep_wait: block until the grid this
+// one depends on has completed and its memory operations are visible (a
+// no-op when the grid was launched without the attribute); every kernel
+// launched with it calls this before touching global memory another kernel
+// writes or reads.  grid_dep_launch: let the next grid of the stream start
+// launching (its CTAs then wait in their own grid_dep_wait).
+SGE_DEV void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+SGE_DEV void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 SGE_DEV bool elect_one_sync() {
   uint32_t pred = 0;
   asm volatile(

@@ -36,6 +36,27 @@ int prefer_max_shared(const void* kernel);
 // driver entry point; CUDA_SUCCESS or the driver's error.
 CUresult current_context(CUcontext* ctx);
 
+// Launch with programmatic stream serialization: the kernel may start
+// while its predecessor in the stream finishes and must call grid_dep_wait()
+// before touching global memory.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+               const char* what, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return check_launch(what);
+}
+
 // 2-D bf16 tensor map over a row-major [rows][cols] matrix with row pitch
 // `pitch_elems`, box [box_rows][64] (64 bf16 = one 128-byte swizzle row),
 // 128-byte swizzle, out-of-bounds elements read as zero.

@@ -241,6 +241,8 @@ static __global__ void __launch_bounds__(256) split_scatter_kernel(const float* 
                                                                    const int32_t* __restrict__ n_spill,
                                                                    int s_max, int n_cols, int ncp,
                                                                    uint16_t* __restrict__ y) {
+  grid_dep_launch();
+  grid_dep_wait();  // the parts come from the GEMM before
   const int nsplit = reinterpret_cast<const int*>(part)[kSplitTiles * 256 * 256];
   const int kept = min(*n_spill, s_max);
   if (nsplit <= 1 || kept <= 0) return;
@@ -291,8 +293,8 @@ static inline int launch_split_scatter(const float* part, const int32_t* rows, c
                                        const char* what) {
   const int64_t work = (static_cast<int64_t>(s_max) * (n_cols / 8) + 255) / 256;
   const int grid = static_cast<int>(work < 4 * sm_count() ? (work > 0 ? work : 1) : 4 * sm_count());
-  split_scatter_kernel<<<grid, 256, 0, st>>>(part, rows, n_spill, s_max, n_cols, ncp, y);
-  return check_launch(what);
+  return launch_pdl(split_scatter_kernel, dim3(grid), dim3(256), 0, st, what, part, rows, n_spill, s_max,
+                    n_cols, ncp, y);
 }
 
 }  // namespace sge

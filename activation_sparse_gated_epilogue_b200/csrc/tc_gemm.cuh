@@ -162,10 +162,6 @@ __global__ void __launch_bounds__(Shape::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m_blocks = (epi_m_limit(epi, M) + kBM - 1) / kBM;
-  const int n_blocks = (N + BN - 1) / BN;
-  const int k_blocks = (epi_k_limit(epi, K) + kBK - 1) / kBK;
-  const int num_tiles = k_blocks > 0 ? m_blocks * n_blocks : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -188,6 +184,12 @@ __global__ void __launch_bounds__(Shape::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  grid_dep_launch();
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  const int m_blocks = (epi_m_limit(epi, M) + kBM - 1) / kBM;
+  const int n_blocks = (N + BN - 1) / BN;
+  const int k_blocks = (epi_k_limit(epi, K) + kBK - 1) / kBK;
+  const int num_tiles = k_blocks > 0 ? m_blocks * n_blocks : 0;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
@@ -350,14 +352,6 @@ __global__ void __launch_bounds__(Shape::THREADS, 1)
   const bool leader = rank == 0;
   const int pair = static_cast<int>(cluster_id_x());
   const int n_pairs = static_cast<int>(cluster_count_x());
-  const int m_blocks = (epi_m_limit(epi, M) + Shape::BM - 1) / Shape::BM;
-  const int n_blocks = (N + BN - 1) / BN;
-  const int k_blocks = (epi_k_limit(epi, K) + kBK - 1) / kBK;
-  // split-K: K-blocks per split, and the number of non-empty splits
-  const int want_splits = max(1, min(epi_splits(epi), k_blocks));
-  const int kb_per = k_blocks > 0 ? (k_blocks + want_splits - 1) / want_splits : 0;
-  const int nsplit = kb_per > 0 ? (k_blocks + kb_per - 1) / kb_per : 1;
-  const int num_tiles = k_blocks > 0 ? m_blocks * n_blocks * nsplit : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -380,6 +374,18 @@ __global__ void __launch_bounds__(Shape::THREADS, 1)
   cluster_sync();  // both CTAs' barriers exist before any remote arrive / TMA
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // with programmatic dependent launch the set-up above overlaps the previous
+  // kernel; everything below may read what it wrote
+  grid_dep_launch();
+  grid_dep_wait();
+  const int m_blocks = (epi_m_limit(epi, M) + Shape::BM - 1) / Shape::BM;
+  const int n_blocks = (N + BN - 1) / BN;
+  const int k_blocks = (epi_k_limit(epi, K) + kBK - 1) / kBK;
+  // split-K: K-blocks per split, and the number of non-empty splits
+  const int want_splits = max(1, min(epi_splits(epi), k_blocks));
+  const int kb_per = k_blocks > 0 ? (k_blocks + want_splits - 1) / want_splits : 0;
+  const int nsplit = kb_per > 0 ? (k_blocks + kb_per - 1) / kb_per : 1;
+  const int num_tiles = k_blocks > 0 ? m_blocks * n_blocks * nsplit : 0;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer

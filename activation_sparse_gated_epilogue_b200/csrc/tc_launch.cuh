@@ -63,13 +63,17 @@ int launch_tc_gemm_pair(const CUtensorMap& ma, const CUtensorMap& mb0, const CUt
   cfg.blockDim = dim3(Shape::THREADS);
   cfg.dynamicSmemBytes = Shape::SMEM_BYTES;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  // programmatic dependent launch: the kernel's set-up (barriers, TMEM,
+  // descriptors) overlaps the end of the previous kernel in the stream
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb0, mb1, static_cast<int>(m),
                                      static_cast<int>(n), static_cast<int>(k), epi, diag);
   if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));

@@ -432,10 +432,11 @@ def run_own(args, rank, world, local_rank):
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
                 "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
-        "gpu_launches": (2 if n <= 64 else 7) * args.steps,
+        "gpu_launches": (3 if n <= 64 else 8) * args.steps,
         "launches_note": "per step: gate GEMM + TwELL epilogue; twell_hybrid_up_down = count, jobs, "
-                         "spill prep, up GEMM, down GEMM, per-entry kernel (2 launches in all for "
-                         "batches of at most 64 tokens)",
+                         "light-token kernel, spill prep, up GEMM, down GEMM, split sum (the last "
+                         "exits at once when the down GEMM did not split K); for batches of at most "
+                         "64 tokens: gate, plan and the small-batch kernel",
         "hybrid_inference": hyb,
         "clocks": clocks,
         "diag": diag_host,

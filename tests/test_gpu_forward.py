@@ -40,6 +40,9 @@ def _upload_twell(tw: oracle.TwELL, dtype, dev):
     (64, 512, 1024, 128, 12),
     (1, 136, 512, 128, 128),      # one token (batches of <= 256 rows: single-CTA tiles)
     (200, 264, 384, 64, 64),      # ragged rows inside one 128-row tile
+    (128, 200, 640, 128, 128),    # one full row tile
+    (100, 264, 384, 64, 64),
+    (33, 136, 256, 16, 16),
 ])
 def test_gate_pack_exact_on_grid_inputs(cuda_device, dtype, n, d, f, tile, cap):
     """Grid inputs make G exact in fp32, so counts, indices and values are
@@ -68,12 +71,15 @@ def test_gate_pack_identity_weights(cuda_device):
     assert_twell_equal(tw, ora)
 
 
-@pytest.mark.parametrize("name,cap", [("ffn_0p5b_bf16", 128), ("tiny_fp32", 64), ("tiny_fp32", 16)])
-def test_gate_pack_gaussian_sign_flips(cuda_device, name, cap):
+@pytest.mark.parametrize("name,cap,n", [("ffn_0p5b_bf16", 128, 512), ("tiny_fp32", 64, 512),
+                                        ("tiny_fp32", 16, 512), ("ffn_1b_bf16", 128, 100),
+                                        ("ffn_1b_bf16", 128, 200)])
+def test_gate_pack_gaussian_sign_flips(cuda_device, name, cap, n):
     """Realistic inputs: tiles disagree only where near-zero gates explain it
-    (|g| < 1e-3); values agree within one bf16 ulp / the fp32 tolerance."""
+    (|g| < 1e-3); values agree within the fp32 accumulation bound.  100 and
+    200 tokens take the single-CTA tiles of small batches."""
     cfg = synth.CONFIGS[name]
-    inp = synth.make_inputs(cfg, n_tokens=512)
+    inp = synth.make_inputs(cfg, n_tokens=n)
     x, wg, _, _ = _dev(inp, cuda_device)
     tw = sge.twell_gate_pack(x, wg, cfg.tile, cap)
     g = oracle.gate_preact(inp.as_f64("x"), inp.as_f64("wg_t"))
