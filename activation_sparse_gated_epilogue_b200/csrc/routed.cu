@@ -13,16 +13,20 @@
 //           are heavy and ranked in ascending token order; the first S_max
 //           go to the spill list, every other non-empty token to a size
 //           class of the light lists (fused_kernels.cuh's planning kernels)
+//   prep    per spill row: its x row into X_s, its stored activations
+//           scattered into a dense row of A_s (zeros elsewhere)
+//   GEMM 1  U = X_s W_up on tcgen05 (CTA pairs), epilogue H_s = bf16(A_s (.) U)
 //   light   the light tokens (and heavy ones past S_max) through CUDA
 //           cores, one warp per token, its entries' W_up and W_down rows
 //           streamed through a ring of shared-memory slots filled by bulk
 //           copies (light_ring_kernel below); y = 0 for tokens without
-//           stored entries
-//   prep    per spill row: its x row into X_s, its stored activations
-//           scattered into a dense row of A_s (zeros elsewhere)
-//   GEMM 1  U = X_s W_up on tcgen05 (CTA pairs), epilogue H_s = bf16(A_s (.) U)
+//           stored entries.  Its CTAs start while GEMM 1's last wave runs.
 //   GEMM 2  Y_s = H_s W_down on tcgen05, epilogue scatters row r to y[token r]
+//           (with split-K and a part-sum kernel when the spill rows make
+//           few output tiles)
 //
+// Consecutive launches use programmatic dependent launch: each kernel's
+// set-up overlaps the end of the previous one.
 // Every token's y is written exactly once, by GEMM 2 or by the light-token
 // kernel; results do not depend on scheduling.  Per row the arithmetic is
 // that of the dense FFN restricted to the stored entries: fp32 accumulation,
@@ -147,9 +151,7 @@ struct RingParams {
 };
 
 template <int NV, int NTR>
-__global__ void __launch_bounds__(kRingMaxWarps * 32, 1) light_ring_kernel(const RingParams p) {
-  grid_dep_launch();
-  grid_dep_wait();  // lists and counts come from the planning kernels
+__device__ __forceinline__ void light_ring_body(const RingParams& p) {
   using E = Elem<true>;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -359,6 +361,20 @@ struct RoutedLayout {
   }
 };
 
+// The light-token kernel runs after the spill up GEMM in the stream but does
+// not wait for it: it needs only the planning kernels' lists, complete once
+// the up GEMM has passed its own dependency wait (the GEMM engine lets its
+// successor launch only after that wait), and it touches nothing the GEMM
+// writes.  So its CTAs start on the SMs the GEMM's last wave of tiles leaves
+// idle.  It waits for the GEMM before exiting, so that the down GEMM, which
+// waits for this kernel, also finds H_s complete.
+template <int NV, int NTR>
+__global__ void __launch_bounds__(kRingMaxWarps * 32, 1) light_ring_kernel(const RingParams p) {
+  grid_dep_launch();
+  light_ring_body<NV, NTR>(p);
+  grid_dep_wait();
+}
+
 template <int NV, int NTR>
 static int launch_ring(const RingParams& p, int warps, int smem, cudaStream_t st) {
   auto kern = light_ring_kernel<NV, NTR>;
@@ -454,7 +470,7 @@ extern "C" int twell_hybrid_up_down(const void* x, const uint8_t* count, const u
   const RouteArgs route{ell_cap, s_max, 1, reinterpret_cast<int2*>(ws + L.heavy), spill_rows, diag};
   if ((rc = fused_launch_plan(c, route, st))) return rc;
 
-  // the light tokens, then the spill
+  // the spill prep, the up GEMM, the light tokens, the down GEMM
   const int f = static_cast<int>(d_ff), d = static_cast<int>(d_model);
   RingParams rp{static_cast<const uint16_t*>(x), count, idx, static_cast<const uint16_t*>(val),
                 static_cast<const char*>(wu_t), static_cast<const char*>(wd), ldw * 2,
@@ -464,7 +480,6 @@ extern "C" int twell_hybrid_up_down(const void* x, const uint8_t* count, const u
   // (run_ring also needs a row to fill half a slot exactly)
   rp.w_one = static_cast<const char*>(wd) == static_cast<const char*>(wu_t) + 2 * d_model &&
              ldw == 2 * d_model;
-  if ((rc = run_ring(rp, c.nv, st))) return rc;
   {
     const int smem = prep_smem_bytes(d_ff);
     if ((rc = set_smem_limit(reinterpret_cast<const void*>(spill_prep_kernel), smem))) return rc;
@@ -483,6 +498,8 @@ extern "C" int twell_hybrid_up_down(const void* x, const uint8_t* count, const u
   if ((rc = launch_tc_gemm_pair<S>(ma, mb, mb, s_max, d_ff, d_model, e1, diag, st,
                                    "twell_hybrid_up_down (spill up)")))
     return rc;
+  // the light tokens, overlapping the up GEMM's last wave (see light_ring_kernel)
+  if ((rc = run_ring(rp, c.nv, st))) return rc;
   if ((rc = make_tmap_bf16(&mh, hs, s_max, d_ff, d_ff, kBM))) return rc;
   if ((rc = make_tmap_bf16(&md, wd_t, d_model, d_ff, d_ff, S::BN / 2))) return rc;
   const int tiles_n = (d + S::BN - 1) / S::BN;

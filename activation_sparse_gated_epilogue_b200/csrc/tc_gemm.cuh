@@ -184,8 +184,8 @@ __global__ void __launch_bounds__(Shape::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  grid_dep_launch();
   grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   const int m_blocks = (epi_m_limit(epi, M) + kBM - 1) / kBM;
   const int n_blocks = (N + BN - 1) / BN;
   const int k_blocks = (epi_k_limit(epi, K) + kBK - 1) / kBK;
@@ -375,9 +375,11 @@ __global__ void __launch_bounds__(Shape::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   // with programmatic dependent launch the set-up above overlaps the previous
-  // kernel; everything below may read what it wrote
-  grid_dep_launch();
+  // kernel; everything below may read what it wrote.  The successor may
+  // launch only after this wait: a successor that skips its own wait can
+  // then rely on every kernel before this one having completed.
   grid_dep_wait();
+  grid_dep_launch();
   const int m_blocks = (epi_m_limit(epi, M) + Shape::BM - 1) / Shape::BM;
   const int n_blocks = (N + BN - 1) / BN;
   const int k_blocks = (epi_k_limit(epi, K) + kBK - 1) / kBK;
