@@ -502,6 +502,8 @@ constexpr int kHasX = 4;   //              the x row leads the chunk's stream
 // p.slots slots (see the file comment).
 template <bool BF16, int NTR, int NV>
 __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(const UdParams p) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   using E = Elem<BF16>;
   constexpr int VEC = E::VEC;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -1008,6 +1010,8 @@ static __global__ void __launch_bounds__(kSmallTokens) us_plan_kernel(const uint
                                                               int* __restrict__ ufirst,
                                                               int* __restrict__ pbase,
                                                               int* __restrict__ done) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   __shared__ int tmp[kSmallTokens / 32 + 1];
   const int t = threadIdx.x;
   int n = 0;
@@ -1081,6 +1085,8 @@ struct UsParams {
 // of a row per lane.
 template <bool BF16, int NTR, int NV>
 __global__ void __launch_bounds__(kSmWarps * 32, 1) us_main_kernel(const UsParams p) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   using E = Elem<BF16>;
   constexpr int VEC = E::VEC;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -1247,8 +1253,7 @@ static int launch_small(const UsParams& prm, int smem, int grid, cudaStream_t st
   auto kern = us_main_kernel<BF16, NTR, NV>;
   const int rc = set_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (rc) return rc;
-  kern<<<grid, kSmWarps * 32, smem, st>>>(prm);
-  return check_launch("twell_fused_up_down (small batch)");
+  return launch_pdl(kern, dim3(grid), dim3(kSmWarps * 32), smem, st, "twell_fused_up_down (small batch)", prm);
 }
 
 template <bool BF16, int NV>
@@ -1297,8 +1302,7 @@ static int launch_main(const UdParams& prm, int smem, int grid, cudaStream_t st)
   auto kern = ud_main_kernel<BF16, NTR, NV>;
   const int rc = set_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (rc) return rc;
-  kern<<<grid, prm.teams * kTeam * 32, smem, st>>>(prm);
-  return check_launch("twell_fused_up_down");
+  return launch_pdl(kern, dim3(grid), dim3(prm.teams * kTeam * 32), smem, st, "twell_fused_up_down", prm);
 }
 
 template <bool BF16, int NV>
@@ -1346,9 +1350,9 @@ static int run_small(const UdParams& prm, const WsLayout& L, uint8_t* ws, int64_
   up.cap = prm.cap;
   up.pieces = prm.row_bytes / 16;
   up.w_ld = prm.w_ld;
-  us_plan_kernel<<<1, kSmallTokens, 0, st>>>(prm.count, prm.n_rows, prm.nt, prm.cap, pool_slots, prm.hdr,
-                                             const_cast<int*>(prm.ntok), ufirst, pbase, prm.done);
-  const int rc = check_launch("twell_fused_up_down (small-batch plan)");
+  const int rc = launch_pdl(us_plan_kernel, dim3(1), dim3(kSmallTokens), 0, st,
+                            "twell_fused_up_down (small-batch plan)", prm.count, prm.n_rows, prm.nt, prm.cap,
+                            pool_slots, prm.hdr, const_cast<int*>(prm.ntok), ufirst, pbase, prm.done);
   if (rc) return rc;
   const int smem = (kSmWarps * prm.d * 4 + 4 * static_cast<int>(prm.n_rows + 1) + 15) & ~15;
   return bf16 ? small_nv<true>(up, nv, smem, sm_count(), st) : small_nv<false>(up, nv, smem, sm_count(), st);

@@ -46,6 +46,8 @@ struct HybridView {
 // it from the gate.
 __global__ void __launch_bounds__(256) hybrid_nnz_kernel(const uint8_t* __restrict__ count, int nt,
                                                          int cap, HybridView hv) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   const int64_t t = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   if (t >= hv.n) return;
   const uint8_t* c = count + t * nt;
@@ -75,6 +77,8 @@ __global__ void __launch_bounds__(256) hybrid_nnz_kernel(const uint8_t* __restri
 // One CTA: routing and the ascending ranks of the spill rows (block-wide
 // exclusive scan over contiguous row ranges of the per-row counts).
 __global__ void __launch_bounds__(kPackThreads) hybrid_route_kernel(HybridView hv, int32_t* diag) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   __shared__ int s_scan[kPackThreads];
   const int tid = threadIdx.x;
   const int64_t per = (hv.n + kPackThreads - 1) / kPackThreads;
@@ -117,6 +121,8 @@ __global__ void __launch_bounds__(256) hybrid_fill_kernel(const uint8_t* __restr
                                                           const uint8_t* __restrict__ idx,
                                                           const uint16_t* __restrict__ val,
                                                           int nt, int tile, int cap, HybridView hv) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= hv.n) return;
@@ -182,6 +188,8 @@ struct EllFwdParams {
 // rows are left to the spill GEMMs.
 template <int NV>
 __global__ void __launch_bounds__(kEllThreads) hybrid_ell_fwd_kernel(EllFwdParams p) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   using E = Elem<true>;
   constexpr int VEC = E::VEC;
   __shared__ int s_j[kEllMaxK];
@@ -326,15 +334,13 @@ extern "C" int hybrid_pack(const uint8_t* count, const uint8_t* idx, const void*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const HybridView hv = view_of(hy);
   const int nt = static_cast<int>(hy->d_ff / tile);
-  hybrid_nnz_kernel<<<static_cast<unsigned>((hy->n_tokens + 255) / 256), 256, 0, st>>>(count, nt, cap, hv);
-  rc = check_launch("hybrid_pack (count)");
-  if (rc) return rc;
-  hybrid_route_kernel<<<1, kPackThreads, 0, st>>>(hv, diag);
-  rc = check_launch("hybrid_pack (route)");
-  if (rc) return rc;
-  hybrid_fill_kernel<<<static_cast<unsigned>((hy->n_tokens + 7) / 8), 256, 0, st>>>(
-      count, idx, static_cast<const uint16_t*>(val), nt, tile, cap, hv);
-  return check_launch("hybrid_pack (fill)");
+  if ((rc = launch_pdl(hybrid_nnz_kernel, dim3(static_cast<unsigned>((hy->n_tokens + 255) / 256)), dim3(256), 0, st,
+                       "hybrid_pack (counts)", count, nt, cap, hv)))
+    return rc;
+  if ((rc = launch_pdl(hybrid_route_kernel, dim3(1), dim3(kPackThreads), 0, st, "hybrid_pack (route)", hv, diag)))
+    return rc;
+  return launch_pdl(hybrid_fill_kernel, dim3(static_cast<unsigned>((hy->n_tokens + 7) / 8)), dim3(256), 0, st,
+                    "hybrid_pack (fill)", count, idx, static_cast<const uint16_t*>(val), nt, tile, cap, hv);
 }
 
 extern "C" size_t hybrid_ffn_fwd_workspace_bytes(int64_t d_model, int64_t d_ff, int s_max) {
@@ -346,8 +352,8 @@ extern "C" size_t hybrid_ffn_fwd_workspace_bytes(int64_t d_model, int64_t d_ff, 
 
 template <int NV>
 static int launch_ell_fwd(const EllFwdParams& p, int64_t n, cudaStream_t st) {
-  hybrid_ell_fwd_kernel<NV><<<static_cast<unsigned>(n), kEllThreads, 0, st>>>(p);
-  return check_launch("hybrid_ffn_fwd (ELL rows)");
+  return launch_pdl(hybrid_ell_fwd_kernel<NV>, dim3(static_cast<unsigned>(n)), dim3(kEllThreads), 0, st,
+                    "hybrid_ffn_fwd (ELL rows)", p);
 }
 
 extern "C" int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* wu_t, const void* wd,
@@ -384,9 +390,10 @@ extern "C" int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* w
   // Y_s = H_s W_down scattered to y.
   uint16_t* xs = static_cast<uint16_t*>(workspace);
   uint16_t* hs = xs + static_cast<size_t>(hy->s_max) * d_model;
-  gather_rows_kernel<<<hy->s_max, 256, 0, st>>>(static_cast<const uint16_t*>(x), hy->spill_rows,
-                                                 hy->n_spill, hy->s_max, static_cast<int>(d_model), xs);
-  if ((rc = check_launch("hybrid_ffn_fwd (gather)"))) return rc;
+  if ((rc = launch_pdl(gather_rows_kernel, dim3(hy->s_max), dim3(256), 0, st, "hybrid_ffn_fwd (gather)",
+                       static_cast<const uint16_t*>(x), hy->spill_rows, hy->n_spill, hy->s_max,
+                       static_cast<int>(d_model), xs)))
+    return rc;
   using S = TcPairShape<256, 1, 2>;
   CUtensorMap ma, mb, mh, md;
   if ((rc = make_tmap_bf16(&ma, xs, hy->s_max, d_model, d_model, kBM))) return rc;

@@ -109,6 +109,8 @@ struct EllBwdParams {
 
 template <int NV>
 __global__ void __launch_bounds__(kBwdThreads) ell_bwd_kernel(EllBwdParams p) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   using E = Elem<true>;
   constexpr int VEC = E::VEC;
   __shared__ int s_j[kBwdMaxK];
@@ -214,6 +216,8 @@ __global__ void __launch_bounds__(kBwdThreads) ell_bwd_kernel(EllBwdParams p) {
 // ------------------------------------------------- column buckets (CSC)
 
 __global__ void __launch_bounds__(256) csc_count_kernel(BwdHybrid hv, int* col_count) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= hv.n) return;
@@ -225,6 +229,8 @@ __global__ void __launch_bounds__(256) csc_count_kernel(BwdHybrid hv, int* col_c
 // One CTA: exclusive scan of the column counts.
 __global__ void __launch_bounds__(1024) csc_scan_kernel(const int* col_count, int f, int* col_start,
                                                         int* col_cursor) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   __shared__ int s[1024];
   const int tid = threadIdx.x;
   const int per = (f + 1023) / 1024;
@@ -249,6 +255,8 @@ __global__ void __launch_bounds__(1024) csc_scan_kernel(const int* col_count, in
 }
 
 __global__ void __launch_bounds__(256) csc_scatter_kernel(BwdHybrid hv, int* col_cursor, int2* csc) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= hv.n) return;
@@ -264,6 +272,8 @@ __global__ void __launch_bounds__(256) csc_scatter_kernel(BwdHybrid hv, int* col
 // column, then scattered with slot -(spill rank + 1).  Grid: (F / 2048
 // chunks) x (S_max ranks); eight columns per thread.
 __global__ void __launch_bounds__(256) csc_count_spill_kernel(BwdHybrid hv, int* col_count) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   const int r = blockIdx.y;
   if (r >= min(*hv.n_spill, hv.s_max)) return;
   const int j0 = (blockIdx.x * 256 + threadIdx.x) * 8;
@@ -278,6 +288,8 @@ __global__ void __launch_bounds__(256) csc_count_spill_kernel(BwdHybrid hv, int*
 }
 
 __global__ void __launch_bounds__(256) csc_scatter_spill_kernel(BwdHybrid hv, int* col_cursor, int2* csc) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   const int r = blockIdx.y;
   if (r >= min(*hv.n_spill, hv.s_max)) return;
   const int j0 = (blockIdx.x * 256 + threadIdx.x) * 8;
@@ -299,6 +311,8 @@ __global__ void __launch_bounds__(256) csc_scatter_spill_kernel(BwdHybrid hv, in
 // column, so an entry's position is the number of smaller tokens.
 __global__ void __launch_bounds__(256) csc_sort_kernel(const int* col_start, int f, const int2* csc,
                                                        int2* sorted) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   const int c = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (c >= f) return;
@@ -329,6 +343,8 @@ constexpr int kDwStage = 256;  // entries of a column whose metadata is staged a
 
 template <int NV>
 __global__ void __launch_bounds__(kBwdThreads) dw_ell_kernel(DwParams p) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   constexpr int VEC = 8;
   // the entries' tokens and (h, du, dg), loaded for a whole round of the
   // column's bucket by all threads at once; the rows of x and dy then
@@ -433,6 +449,8 @@ __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restri
                                                         int cols, int64_t src_pitch, uint16_t* dst,
                                                         int64_t dst_pitch, int col_off,
                                                         const int32_t* rows_dev, int rows_cap) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   // 64 x 64 tiles moved with 16-byte loads and stores (rows, cols, pitches,
   // col_off and the row limit are multiples of 8); the shared tile's row
   // pitch of 66 elements keeps the column reads off one bank
@@ -535,21 +553,19 @@ static int launch_transpose(const uint16_t* src, int rows, int cols, int64_t src
                             uint16_t* dst, int64_t dst_pitch, int col_off, cudaStream_t st,
                             const int32_t* rows_dev = nullptr, int rows_cap = 0) {
   dim3 grid((cols + 63) / 64, (rows + 63) / 64);
-  transpose_kernel<<<grid, 256, 0, st>>>(src, rows, cols, src_pitch, dst, dst_pitch, col_off, rows_dev,
-                                         rows_cap);
-  return check_launch("hybrid_ffn_bwd (transpose)");
+  return launch_pdl(transpose_kernel, grid, dim3(256), 0, st, "hybrid_ffn_bwd (transpose)", src, rows, cols,
+                    src_pitch, dst, dst_pitch, col_off, rows_dev, rows_cap);
 }
 
 template <int NV>
 static int launch_ell_bwd(const EllBwdParams& p, int64_t n, cudaStream_t st) {
-  ell_bwd_kernel<NV><<<static_cast<unsigned>(n), kBwdThreads, 0, st>>>(p);
-  return check_launch("hybrid_ffn_bwd (ELL rows)");
+  return launch_pdl(ell_bwd_kernel<NV>, dim3(static_cast<unsigned>(n)), dim3(kBwdThreads), 0, st,
+                    "hybrid_ffn_bwd (ELL rows)", p);
 }
 
 template <int NV>
 static int launch_dw(const DwParams& q, int f, cudaStream_t st) {
-  dw_ell_kernel<NV><<<f, kBwdThreads, 0, st>>>(q);
-  return check_launch("hybrid_ffn_bwd (weight gradients)");
+  return launch_pdl(dw_ell_kernel<NV>, dim3(f), dim3(kBwdThreads), 0, st, "hybrid_ffn_bwd (weight gradients)", q);
 }
 
 }  // namespace sge
@@ -638,9 +654,9 @@ extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* h
   using Sh = TcPairShape<128, 1>;  // N = F in 128-wide tiles: few spill row tiles still spread
   using Sx = TcPairShape<256, 1, 2>;  // N = d: few tiles, K = 2F split over the CTA pairs
   if (s_max > 0) {
-    gather_rows_kernel<<<sp, 256, 0, st>>>(dyb, hy->spill_rows, hy->n_spill, s_max, static_cast<int>(d),
-                                           ws.dys);
-    if ((rc = check_launch("hybrid_ffn_bwd (gather)"))) return rc;
+    if ((rc = launch_pdl(gather_rows_kernel, dim3(sp), dim3(256), 0, st, "hybrid_ffn_bwd (gather)", dyb,
+                         hy->spill_rows, hy->n_spill, s_max, static_cast<int>(d), ws.dys)))
+      return rc;
     CUtensorMap m1a, m1b;
     if ((rc = make_tmap_bf16(&m1a, ws.dys, sp, d, d, kBM))) return rc;
     if ((rc = make_tmap_bf16(&m1b, wd, f, d, d, Sh::BN / 2))) return rc;
@@ -654,14 +670,20 @@ extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* h
   if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "hybrid_ffn_bwd: %s", cudaGetErrorString(e));
   const unsigned rb = static_cast<unsigned>((n + 7) / 8);
   const dim3 sgrid(static_cast<unsigned>((f + 2047) / 2048), static_cast<unsigned>(s_max > 0 ? s_max : 1));
-  csc_count_kernel<<<rb, 256, 0, st>>>(hv, ws.col_count);
-  if (s_max > 0) csc_count_spill_kernel<<<sgrid, 256, 0, st>>>(hv, ws.col_count);
-  csc_scan_kernel<<<1, 1024, 0, st>>>(ws.col_count, static_cast<int>(f), ws.col_start, ws.col_cursor);
-  csc_scatter_kernel<<<rb, 256, 0, st>>>(hv, ws.col_cursor, ws.csc);
-  if (s_max > 0) csc_scatter_spill_kernel<<<sgrid, 256, 0, st>>>(hv, ws.col_cursor, ws.csc);
-  csc_sort_kernel<<<static_cast<unsigned>((f + 7) / 8), 256, 0, st>>>(ws.col_start, static_cast<int>(f),
-                                                                     ws.csc, ws.csc_sorted);
-  if ((rc = check_launch("hybrid_ffn_bwd (column buckets)"))) return rc;
+  const char* what = "hybrid_ffn_bwd (column buckets)";
+  if ((rc = launch_pdl(csc_count_kernel, dim3(rb), dim3(256), 0, st, what, hv, ws.col_count))) return rc;
+  if (s_max > 0 && (rc = launch_pdl(csc_count_spill_kernel, sgrid, dim3(256), 0, st, what, hv, ws.col_count)))
+    return rc;
+  if ((rc = launch_pdl(csc_scan_kernel, dim3(1), dim3(1024), 0, st, what, ws.col_count, static_cast<int>(f),
+                       ws.col_start, ws.col_cursor)))
+    return rc;
+  if ((rc = launch_pdl(csc_scatter_kernel, dim3(rb), dim3(256), 0, st, what, hv, ws.col_cursor, ws.csc))) return rc;
+  if (s_max > 0 && (rc = launch_pdl(csc_scatter_spill_kernel, sgrid, dim3(256), 0, st, what, hv, ws.col_cursor,
+                                    ws.csc)))
+    return rc;
+  if ((rc = launch_pdl(csc_sort_kernel, dim3(static_cast<unsigned>((f + 7) / 8)), dim3(256), 0, st, what,
+                       ws.col_start, static_cast<int>(f), ws.csc, ws.csc_sorted)))
+    return rc;
   // ---- weight gradients, each row written once
   DwParams q{xb, dyb, hv, ws, dwg_t, dwu_t, dwd, static_cast<int>(d)};
   if (nvec <= kBwdThreads) rc = launch_dw<1>(q, static_cast<int>(f), st);

@@ -17,6 +17,8 @@ static __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t*
                                                           const int32_t* __restrict__ rows,
                                                           const int32_t* __restrict__ n_rows_dev,
                                                           int cap_rows, int d, uint16_t* dst) {
+  grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
+  grid_dep_launch();
   const int r = blockIdx.x;
   const int kept = min(*n_rows_dev, cap_rows);
   uint4* out = reinterpret_cast<uint4*>(dst + static_cast<int64_t>(r) * d);

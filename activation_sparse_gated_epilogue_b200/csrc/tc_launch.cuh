@@ -15,10 +15,8 @@ int launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensor
   if (rc) return rc;
   const int64_t tiles = ((m + kBM - 1) / kBM) * ((n + Shape::BN - 1) / Shape::BN);
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  kern<<<grid, Shape::THREADS, Shape::SMEM_BYTES, st>>>(ma, mb0, mb1, static_cast<int>(m),
-                                                      static_cast<int>(n), static_cast<int>(k), epi,
-                                                      diag);
-  return check_launch(what);
+  return launch_pdl(kern, dim3(grid), dim3(Shape::THREADS), Shape::SMEM_BYTES, st, what, ma, mb0, mb1,
+                    static_cast<int>(m), static_cast<int>(n), static_cast<int>(k), epi, diag);
 }
 
 // Number of CTA pairs that can be resident at once (cached per kernel).
