@@ -958,8 +958,9 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
 // With few tokens (decode-sized batches) the persistent kernel's per-warp row
 // streams are short and its latency chain (three launches, the job queue, a
 // ring a few rows deep) dominates.  The small-batch path splits every token
-// into units of E entries (E = 8, doubled until the split tokens' partial
-// outputs fit the pool), gives each unit one CTA of kSmWarps warps and each
+// into units of E entries (E = 8, doubled until there is at most one unit
+// per CTA and the split tokens' partial outputs fit the pool), gives each
+// unit one CTA of kSmWarps warps and each
 // warp one entry at a time: the warp loads x[t], the W_up row and the W_down
 // row with plain 16-byte loads issued together, so a unit costs one memory
 // round trip.  The warps' partial rows are summed in warp order in shared
@@ -1005,7 +1006,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* tmp, int* total)
 // counters.  One CTA of kSmallTokens threads, a thread per token.
 static __global__ void __launch_bounds__(kSmallTokens) us_plan_kernel(const uint8_t* __restrict__ count,
                                                               int64_t n_rows, int nt, int cap,
-                                                              int64_t pool_slots, int* hdr,
+                                                              int64_t pool_slots, int n_cta, int* hdr,
                                                               int* __restrict__ ntok,
                                                               int* __restrict__ ufirst,
                                                               int* __restrict__ pbase,
@@ -1033,13 +1034,18 @@ static __global__ void __launch_bounds__(kSmallTokens) us_plan_kernel(const uint
     ntok[t] = n;
     done[t] = 0;
   }
-  // the smallest E (kSmWarps times a power of two) whose split tokens fit the pool
+  // the smallest E (kSmWarps times a power of two) that gives at most one
+  // unit per CTA of the launch and whose split tokens fit the pool: each
+  // unit pays a fixed chain of dependent round trips and a cross-warp sum,
+  // so fewer, longer units are faster once every CTA has one (64 tokens of
+  // the 1B workload: E = 8 -> 32 took the kernel from 39.6 to 23.7 us)
   int E = kSmWarps;
   for (;;) {
     const int nu = t < n_rows ? max(1, (n + E - 1) / E) : 0;
-    int split = 0;
+    int split = 0, all = 0;
     block_exclusive_scan(nu > 1 ? nu : 0, tmp, &split);
-    if (split <= pool_slots || E >= (1 << 24)) break;
+    block_exclusive_scan(nu, tmp, &all);
+    if ((split <= pool_slots && all <= n_cta) || E >= (1 << 24)) break;
     E *= 2;
   }
   const int nu = t < n_rows ? max(1, (n + E - 1) / E) : 0;
@@ -1352,7 +1358,7 @@ static int run_small(const UdParams& prm, const WsLayout& L, uint8_t* ws, int64_
   up.w_ld = prm.w_ld;
   const int rc = launch_pdl(us_plan_kernel, dim3(1), dim3(kSmallTokens), 0, st,
                             "twell_fused_up_down (small-batch plan)", prm.count, prm.n_rows, prm.nt, prm.cap,
-                            pool_slots, prm.hdr, const_cast<int*>(prm.ntok), ufirst, pbase, prm.done);
+                            pool_slots, sm_count(), prm.hdr, const_cast<int*>(prm.ntok), ufirst, pbase, prm.done);
   if (rc) return rc;
   const int smem = (kSmWarps * prm.d * 4 + 4 * static_cast<int>(prm.n_rows + 1) + 15) & ~15;
   return bf16 ? small_nv<true>(up, nv, smem, sm_count(), st) : small_nv<false>(up, nv, smem, sm_count(), st);
