@@ -51,8 +51,13 @@ ROUTED_K = 16
 
 # DRAM bytes (read + write) per launch from ncu captures of the kernels,
 # keyed by the hash of the source they were taken on; a kernel whose source
-# changed since its capture gets null.
-TRAFFIC = {}
+# changed since its capture gets null.  Captured on the 1B workload with
+# --profile (one launch per kernel, L2 cold): the gate GEMM, and the routed
+# call as the sum of its seven launches.
+TRAFFIC = {
+    "012f82b18eff59bd": 79441664,    # twell_gate_pack
+    "67d7c91a0b780ff8": 227635968,   # twell_hybrid_up_down
+}
 
 
 def parse():
@@ -832,7 +837,9 @@ def run_reference(args):
             "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{cfg.name}: N={cfg.n_tokens} d={cfg.d_model} F={cfg.d_ff} "
-                                   f"T={cfg.tile} C={cfg.cap}",
+                                   f"T={cfg.tile} C={cfg.cap} target density {cfg.rho} sigma={cfg.sigma}",
+                       "step": "fp64 oracle on the host cores: gate GEMM, TwELL pack, up/down over "
+                               "the stored entries",
                        "sample_tokens_per_step": k},
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": host_cores(),
                              "kind": "oracle",
