@@ -11,7 +11,7 @@ from .binding import (  # noqa: F401
     twell_gate_pack, twell_fused_up_down, twell_ffn_forward, dense_ffn_fwd, new_diag,
     fused_workspace, Hybrid, hybrid_pack, hybrid_ffn_fwd, hybrid_fwd_workspace,
     hybrid_ffn_bwd, hybrid_bwd_workspace, interleave_up_down, twell_hybrid_up_down, routed_workspace,
-    transpose_up_gate,
+    transpose_up_gate, debug_flags,
 )
 
 __all__ = [
@@ -19,5 +19,5 @@ __all__ = [
     "twell_gate_pack", "twell_fused_up_down", "twell_ffn_forward", "dense_ffn_fwd", "new_diag",
     "fused_workspace", "Hybrid", "hybrid_pack", "hybrid_ffn_fwd", "hybrid_fwd_workspace",
     "hybrid_ffn_bwd", "hybrid_bwd_workspace", "interleave_up_down", "twell_hybrid_up_down",
-    "routed_workspace", "transpose_up_gate",
+    "routed_workspace", "transpose_up_gate", "debug_flags",
 ]

@@ -18,7 +18,9 @@ SGE_F32, SGE_BF16 = 0, 1
 _DTYPES = {torch.float32: SGE_F32, torch.bfloat16: SGE_BF16}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "libsge.so")
+# SGE_DEBUG=1 loads the debug build (index checks in every kernel, read with
+# debug_flags); it is built by ``python -m activation_sparse_gated_epilogue_b200.build --debug``
+_LIB_PATH = os.path.join(_HERE, "libsge_debug.so" if os.environ.get("SGE_DEBUG") == "1" else "libsge.so")
 _lib = None
 
 
@@ -58,6 +60,7 @@ def library() -> ctypes.CDLL:
         P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
         sigs = {
             "sge_version": (I, []),
+            "sge_debug_flags": (I, [I]),
             "sge_last_error": (ctypes.c_char_p, []),
             "twell_gate_pack": (I, [P, P, I64, I64, I64, I, I, I, P, P, P, P, P]),
             "twell_fused_up_down_workspace_bytes": (ctypes.c_size_t, [I64, I64]),
@@ -86,6 +89,15 @@ def library() -> ctypes.CDLL:
             fn.argtypes = args
         _lib = lib
     return _lib
+
+
+def debug_flags(clear: bool = True) -> int:
+    """OR of the SGE_FLAG_* bits the debug build's index checks raised since
+    the last clear (synchronises the device); -1 with the release build."""
+    r = library().sge_debug_flags(1 if clear else 0)
+    if r == -2:
+        raise LibraryError("sge_debug_flags", 3, library().sge_last_error().decode())
+    return r
 
 
 def _call(name: str, *args) -> None:

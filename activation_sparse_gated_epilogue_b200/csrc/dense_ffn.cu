@@ -83,6 +83,7 @@ using namespace sge;
 extern "C" int dense_ffn_fwd(const void* x, const void* wg_t, const void* wu_t, const void* wd_t,
                              void* h, void* y, int64_t n_tokens, int64_t d_model, int64_t d_ff,
                              int32_t* diag, void* stream) {
+  NvtxRange nvtx_range("dense_ffn_fwd");
   clear_error();
   if (n_tokens < 0 || d_model < 1 || d_ff < 1) return fail(SGE_ERR_ARG, "dense_ffn_fwd: bad sizes");
   if (d_model % 8 || d_ff % 8) return fail(SGE_ERR_ARG, "dense_ffn_fwd: d_model and d_ff must be multiples of 8");

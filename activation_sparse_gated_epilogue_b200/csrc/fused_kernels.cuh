@@ -53,6 +53,7 @@
 #pragma once
 
 #include "sge_host.h"
+#include "debug_checks.cuh"
 #include "sparse_common.cuh"
 
 namespace sge {
@@ -705,7 +706,7 @@ __global__ void __launch_bounds__(UdLaunch<NV>::kWarps * 32, 1) ud_main_kernel(c
     c.a = 0;
     if (lane < c.n) {
       const int64_t at = (static_cast<int64_t>(c.t) * p.nt + b) * p.cap + s;
-      c.ji = __ldg(p.idx + at);
+      c.ji = clamp_index(__ldg(p.idx + at), p.tile);
       c.a = E::load_raw(p.val, at);
     }
     ++rci;
@@ -1170,7 +1171,7 @@ __global__ void __launch_bounds__(kSmWarps * 32, 1) us_main_kernel(const UsParam
         float a = 0.0f;
         if (my < e_end) {
           const int64_t at = (static_cast<int64_t>(t) * p.nt + b) * p.cap + s;
-          j = min(b * p.tile + static_cast<int>(__ldg(p.idx + at)), p.nt * p.tile - 1);
+          j = b * p.tile + clamp_index(__ldg(p.idx + at), p.tile);
           a = E::load_val(p.val, at);
         }
         const int cnt = min(32, (e_end - e + kSmWarps - 1) / kSmWarps);

@@ -21,6 +21,7 @@ extern "C" int twell_fused_up_down(const void* x, const uint8_t* count, const ui
                                    void* y, int64_t n_tokens, int64_t d_model, int64_t d_ff,
                                    int dtype, int tile, int cap, void* workspace,
                                    size_t workspace_bytes, int32_t* diag, void* stream) {
+  NvtxRange nvtx_range("twell_fused_up_down");
   static const char* kName = "twell_fused_up_down";
   clear_error();
   int rc = check_args(kName, n_tokens, d_model, d_ff, ldw, tile, cap);
@@ -145,6 +146,7 @@ extern "C" int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, 
 
 extern "C" int sge_interleave_up_down(const void* wu_t, const void* wd, void* w_ud, int64_t d_ff,
                                       int64_t d_model, int dtype, void* stream) {
+  NvtxRange nvtx_range("sge_interleave_up_down");
   static const char* kName = "sge_interleave_up_down";
   clear_error();
   if (dtype != SGE_BF16 && dtype != SGE_F32) return fail(SGE_ERR_UNSUPPORTED, "%s: dtype %d", kName, dtype);

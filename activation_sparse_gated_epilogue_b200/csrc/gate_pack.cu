@@ -235,6 +235,7 @@ using namespace sge;
 extern "C" int twell_gate_pack(const void* x, const void* wg_t, int64_t n_tokens, int64_t d_model,
                                int64_t d_ff, int dtype, int tile, int cap, uint8_t* count,
                                uint8_t* idx, void* val, int32_t* diag, void* stream) {
+  NvtxRange nvtx_range("twell_gate_pack");
   clear_error();
   if (n_tokens < 0 || d_model < 1 || d_ff < 1)
     return fail(SGE_ERR_ARG, "twell_gate_pack: bad sizes N=%lld d=%lld F=%lld", (long long)n_tokens,

@@ -21,6 +21,14 @@ int fail(int code, const char* fmt, ...) {
 
 void clear_error() { g_err[0] = 0; }
 
+static DebugReader g_debug_readers[32];
+static int g_debug_reader_count = 0;
+
+bool register_debug_reader(DebugReader reader) {
+  if (g_debug_reader_count < 32) g_debug_readers[g_debug_reader_count++] = reader;
+  return true;
+}
+
 int check_launch(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SGE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
@@ -133,5 +141,23 @@ int make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t c
 }  // namespace sge
 
 extern "C" int sge_version(void) { return 100; }
+
+extern "C" int sge_debug_flags(int clear) {
+#ifdef SGE_DEBUG
+  int flags = 0;
+  for (int i = 0; i < sge::g_debug_reader_count; ++i) {
+    const int v = sge::g_debug_readers[i](clear != 0);
+    if (v < 0) {
+      sge::fail(SGE_ERR_CUDA, "sge_debug_flags: %s", cudaGetErrorString(cudaGetLastError()));
+      return -2;
+    }
+    flags |= v;
+  }
+  return flags;
+#else
+  (void)clear;
+  return -1;
+#endif
+}
 
 extern "C" const char* sge_last_error(void) { return sge::g_err; }

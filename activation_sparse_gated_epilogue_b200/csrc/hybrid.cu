@@ -15,6 +15,8 @@
 //                   backward pass); spill rows: gathered and run as tcgen05
 //                   GEMMs, U = X_s W_up (u saved, h = a (.) u), Y_s = H_s W_down,
 //                   the rows scattered back into y.
+#include "block_scan.cuh"
+#include "debug_checks.cuh"
 #include "sparse_common.cuh"
 #include "spill_gemm.cuh"
 #include "tc_launch.cuh"
@@ -75,38 +77,57 @@ __global__ void __launch_bounds__(256) hybrid_nnz_kernel(const uint8_t* __restri
 }
 
 // One CTA: routing and the ascending ranks of the spill rows (block-wide
-// exclusive scan over contiguous row ranges of the per-row counts).
+// exclusive scan over contiguous row ranges of the per-row counts; up to
+// kRouteRegs rows per thread have their counts loaded together).
+constexpr int kRouteRegs = 16;
 __global__ void __launch_bounds__(kPackThreads) hybrid_route_kernel(HybridView hv, int32_t* diag) {
   grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
   grid_dep_launch();
-  __shared__ int s_scan[kPackThreads];
+  __shared__ int wsum[33];
   const int tid = threadIdx.x;
   const int64_t per = (hv.n + kPackThreads - 1) / kPackThreads;
-  const int64_t r0 = tid * per, r1 = min(hv.n, r0 + per);
-  int local = 0;
-  for (int64_t t = r0; t < r1; ++t) local += hv.row_nnz[t] > hv.k;
-  s_scan[tid] = local;
-  __syncthreads();
-  for (int o = 1; o < kPackThreads; o <<= 1) {  // inclusive Hillis-Steele scan
-    const int v = tid >= o ? s_scan[tid - o] : 0;
-    __syncthreads();
-    s_scan[tid] += v;
-    __syncthreads();
-  }
-  int rank = s_scan[tid] - local;
-  for (int64_t t = r0; t < r1; ++t) {
-    int slot = -1;
-    if (hv.row_nnz[t] > hv.k) {
-      if (rank < hv.s_max) {
-        slot = rank;
-        hv.spill_rows[rank] = static_cast<int32_t>(t);
-      }
-      ++rank;
+  const int64_t r0 = min(hv.n, tid * per), r1 = min(hv.n, r0 + per);
+  int total = 0;
+  if (per <= kRouteRegs) {
+    // up to kRouteRegs rows per thread: their counts loaded together
+    bool heavy[kRouteRegs];
+    int local = 0;
+#pragma unroll
+    for (int i = 0; i < kRouteRegs; ++i) {
+      heavy[i] = r0 + i < r1 && hv.row_nnz[r0 + i] > hv.k;
+      local += heavy[i];
     }
-    hv.spill_slot[t] = slot;
+    int rank = block_scan_exclusive(local, wsum, &total);
+#pragma unroll
+    for (int i = 0; i < kRouteRegs; ++i) {
+      if (r0 + i >= r1) break;
+      int slot = -1;
+      if (heavy[i]) {
+        if (rank < hv.s_max) {
+          slot = rank;
+          hv.spill_rows[rank] = static_cast<int32_t>(r0 + i);
+        }
+        ++rank;
+      }
+      hv.spill_slot[r0 + i] = slot;
+    }
+  } else {
+    int local = 0;
+    for (int64_t t = r0; t < r1; ++t) local += hv.row_nnz[t] > hv.k;
+    int rank = block_scan_exclusive(local, wsum, &total);
+    for (int64_t t = r0; t < r1; ++t) {
+      int slot = -1;
+      if (hv.row_nnz[t] > hv.k) {
+        if (rank < hv.s_max) {
+          slot = rank;
+          hv.spill_rows[rank] = static_cast<int32_t>(t);
+        }
+        ++rank;
+      }
+      hv.spill_slot[t] = slot;
+    }
   }
   if (tid == kPackThreads - 1) {
-    const int total = s_scan[tid];
     *hv.n_spill = total;
     if (diag) {
       atomicAdd(reinterpret_cast<int*>(diag + SGE_DIAG_SPILL_ROWS), total);
@@ -149,7 +170,7 @@ __global__ void __launch_bounds__(256) hybrid_fill_kernel(const uint8_t* __restr
     const int off = base + incl - cb;
     const int64_t seg = t * nt + b;
     for (int s = 0; s < cb; ++s) {
-      const int j = b * tile + idx[seg * cap + s];
+      const int j = b * tile + clamp_index(idx[seg * cap + s], tile);
       const uint16_t a = val[seg * cap + s];
       if (ell) {
         hv.ell_idx[t * hv.k + off + s] = static_cast<uint16_t>(j);
@@ -217,7 +238,7 @@ __global__ void __launch_bounds__(kEllThreads) hybrid_ell_fwd_kernel(EllFwdParam
     for (int q = 0; q < VEC; ++q) acc[k][q] = 0.0f;
   }
   for (int e = tid; e < nnz; e += kEllThreads) {
-    s_j[e] = p.hv.ell_idx[t * p.hv.k + e];
+    s_j[e] = static_cast<int>(checked_index(p.hv.ell_idx[t * p.hv.k + e], p.hv.f));
     s_h[e] = __uint_as_float(static_cast<uint32_t>(p.hv.ell_a[t * p.hv.k + e]) << 16);
   }
   __syncthreads();
@@ -322,6 +343,7 @@ using namespace sge;
 
 extern "C" int hybrid_pack(const uint8_t* count, const uint8_t* idx, const void* val, int tile,
                            int cap, sge_hybrid* hy, int32_t* diag, void* stream) {
+  NvtxRange nvtx_range("hybrid_pack");
   clear_error();
   int rc = check_hybrid(hy, "hybrid_pack");
   if (rc) return rc;
@@ -359,6 +381,7 @@ static int launch_ell_fwd(const EllFwdParams& p, int64_t n, cudaStream_t st) {
 extern "C" int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* wu_t, const void* wd,
                               const void* wd_t, const void* wg_t, void* y, int64_t d_model,
                               void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("hybrid_ffn_fwd");
   clear_error();
   int rc = check_hybrid(hy, "hybrid_ffn_fwd");
   if (rc) return rc;

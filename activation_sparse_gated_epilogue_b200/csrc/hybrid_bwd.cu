@@ -20,6 +20,8 @@
 // by token; one CTA per unit then sums its entries in ascending token order
 // and writes the unit's three fp32 gradient rows once.  The result is
 // deterministic.
+#include "block_scan.cuh"
+#include "debug_checks.cuh"
 #include "sparse_common.cuh"
 #include "spill_gemm.cuh"
 #include "tc_launch.cuh"
@@ -139,7 +141,7 @@ __global__ void __launch_bounds__(kBwdThreads) ell_bwd_kernel(EllBwdParams p) {
   }
   const int64_t rk = t * p.hv.k;
   for (int e = tid; e < nnz; e += kBwdThreads) {
-    s_j[e] = p.hv.ell_idx[rk + e];
+    s_j[e] = static_cast<int>(checked_index(p.hv.ell_idx[rk + e], p.hv.f));
     s_c[0][e] = __uint_as_float(static_cast<uint32_t>(p.hv.ell_a[rk + e]) << 16);
     s_c[1][e] = __uint_as_float(static_cast<uint32_t>(p.hv.ell_u[rk + e]) << 16);
   }
@@ -223,35 +225,50 @@ __global__ void __launch_bounds__(256) csc_count_kernel(BwdHybrid hv, int* col_c
   if (t >= hv.n) return;
   const int nnz = hv.row_nnz[t];
   if (nnz > hv.k) return;
-  for (int e = lane; e < nnz; e += 32) atomicAdd(&col_count[hv.ell_idx[t * hv.k + e]], 1);
+  for (int e = lane; e < nnz; e += 32) atomicAdd(&col_count[checked_index(hv.ell_idx[t * hv.k + e], hv.f)], 1);
 }
 
 // One CTA: exclusive scan of the column counts.
+// Bucket starts: an exclusive scan of the column counts, 1024 threads with
+// `per` consecutive columns each.  Up to kScanRegs columns per thread are
+// loaded together into registers (one memory round trip), then scanned.
+constexpr int kScanRegs = 16;
+
 __global__ void __launch_bounds__(1024) csc_scan_kernel(const int* col_count, int f, int* col_start,
                                                         int* col_cursor) {
   grid_dep_wait();  // a no-op unless launched with programmatic dependent launch
   grid_dep_launch();
-  __shared__ int s[1024];
+  __shared__ int wsum[33];
   const int tid = threadIdx.x;
-  const int per = (f + 1023) / 1024;
-  const int c0 = tid * per, c1 = min(f, c0 + per);
-  int local = 0;
-  for (int c = c0; c < c1; ++c) local += col_count[c];
-  s[tid] = local;
-  __syncthreads();
-  for (int o = 1; o < 1024; o <<= 1) {
-    const int v = tid >= o ? s[tid - o] : 0;
-    __syncthreads();
-    s[tid] += v;
-    __syncthreads();
+  const int per = (f + 1023) / 1024;  // consecutive columns per thread
+  const int c0 = min(f, tid * per), c1 = min(f, c0 + per);
+  int total = 0;
+  if (per <= kScanRegs) {
+    int v[kScanRegs];
+#pragma unroll
+    for (int i = 0; i < kScanRegs; ++i) v[i] = c0 + i < c1 ? __ldg(col_count + c0 + i) : 0;
+    int local = 0;
+#pragma unroll
+    for (int i = 0; i < kScanRegs; ++i) local += v[i];
+    int run = block_scan_exclusive(local, wsum, &total);
+#pragma unroll
+    for (int i = 0; i < kScanRegs; ++i)
+      if (c0 + i < c1) {
+        col_start[c0 + i] = run;
+        col_cursor[c0 + i] = run;
+        run += v[i];
+      }
+  } else {
+    int local = 0;
+    for (int c = c0; c < c1; ++c) local += __ldg(col_count + c);
+    int run = block_scan_exclusive(local, wsum, &total);
+    for (int c = c0; c < c1; ++c) {
+      col_start[c] = run;
+      col_cursor[c] = run;
+      run += __ldg(col_count + c);
+    }
   }
-  int run = s[tid] - local;
-  for (int c = c0; c < c1; ++c) {
-    col_start[c] = run;
-    col_cursor[c] = run;
-    run += col_count[c];
-  }
-  if (tid == 1023) col_start[f] = s[1023];
+  if (tid == 1023) col_start[f] = total;
 }
 
 __global__ void __launch_bounds__(256) csc_scatter_kernel(BwdHybrid hv, int* col_cursor, int2* csc) {
@@ -263,7 +280,7 @@ __global__ void __launch_bounds__(256) csc_scatter_kernel(BwdHybrid hv, int* col
   const int nnz = hv.row_nnz[t];
   if (nnz > hv.k) return;
   for (int e = lane; e < nnz; e += 32) {
-    const int pos = atomicAdd(&col_cursor[hv.ell_idx[t * hv.k + e]], 1);
+    const int pos = atomicAdd(&col_cursor[checked_index(hv.ell_idx[t * hv.k + e], hv.f)], 1);
     csc[pos] = make_int2(static_cast<int>(t), e);
   }
 }
@@ -364,7 +381,10 @@ __global__ void __launch_bounds__(kBwdThreads) dw_ell_kernel(DwParams p) {
     const int rn = min(kDwStage, s1 - r0);
     __syncthreads();  // the previous round's metadata has been used
     for (int i = tid; i < rn; i += kBwdThreads) {
-      const int2 te = p.ws.csc_sorted[r0 + i];
+      int2 te = p.ws.csc_sorted[r0 + i];
+      te.x = static_cast<int>(checked_index(te.x, p.hv.n));
+      if (te.y >= 0) te.y = static_cast<int>(checked_index(te.y, p.hv.k));
+      else te.y = -1 - static_cast<int>(checked_index(-te.y - 1, p.hv.s_max));
       float a, u, du, dg;
       if (te.y >= 0) {  // an ELL entry: slot te.y of row te.x
         const int64_t rk = static_cast<int64_t>(te.x) * p.hv.k + te.y;
@@ -591,6 +611,7 @@ static int build_up_gate(const void* wu_t, const void* wg_t, uint16_t* w_ug, int
 
 extern "C" int sge_transpose_up_gate(const void* wu_t, const void* wg_t, void* w_ug, int64_t d_ff,
                                      int64_t d_model, void* stream) {
+  NvtxRange nvtx_range("sge_transpose_up_gate");
   clear_error();
   if (d_ff < 8 || d_ff % 8 || d_model < 8 || d_model % 8 || d_ff > (1 << 30) || d_model > (1 << 30))
     return fail(SGE_ERR_ARG, "sge_transpose_up_gate: d_ff and d_model must be multiples of 8");
@@ -605,6 +626,7 @@ extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* h
                               const void* wg_t, const void* wu_t, const void* wd, const void* w_ug,
                               void* dx, float* dwg_t, float* dwu_t, float* dwd, int64_t d_model,
                               void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("hybrid_ffn_bwd");
   clear_error();
   if (!hy) return fail(SGE_ERR_ARG, "hybrid_ffn_bwd: null hybrid descriptor");
   if (hy->dtype != SGE_BF16) return fail(SGE_ERR_UNSUPPORTED, "hybrid_ffn_bwd: bf16 only");

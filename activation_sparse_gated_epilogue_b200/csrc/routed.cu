@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kPrepThreads) spill_prep_kernel(const uint16_t
         if (b + step < nt && pre[b + step] <= e) b += step;
       const int64_t at = (t * nt + b) * cap + (e - pre[b]);
       // a stored index is < T; kept inside its tile even if it is not
-      row[b * tile + min(static_cast<int>(__ldg(idx + at)), tile - 1)] = __ldg(val + at);
+      row[b * tile + clamp_index(__ldg(idx + at), tile)] = __ldg(val + at);
     }
     __syncthreads();  // the row is assembled
     uint4* arow = reinterpret_cast<uint4*>(as + static_cast<int64_t>(r) * f);
@@ -207,7 +207,7 @@ __device__ __forceinline__ void light_ring_body(const RingParams& p) {
     for (int c = 0; c < kLightClasses; ++c) {
       if (t < 0 && k < n_light[c]) {
         const int2 j = p.lights[c * p.n_rows + k];
-        t = j.x;
+        t = static_cast<int>(checked_index(j.x, p.n_rows));
         n = j.y;
       }
       k -= n_light[c];
@@ -258,7 +258,7 @@ __device__ __forceinline__ void light_ring_body(const RingParams& p) {
       const int s = e - prefix_at<NTR>(pre, b);
       if (e < n) {
         const int64_t at = (static_cast<int64_t>(t) * p.nt + b) * p.cap + s;
-        jcol = b * p.tile + min(static_cast<int>(__ldg(p.idx + at)), p.tile - 1);
+        jcol = b * p.tile + clamp_index(__ldg(p.idx + at), p.tile);
         araw = __ldg(p.val + at);
       }
     };
@@ -430,6 +430,7 @@ extern "C" int twell_hybrid_up_down(const void* x, const uint8_t* count, const u
                                     int64_t d_ff, int tile, int cap, int ell_cap, int s_max,
                                     void* workspace, size_t workspace_bytes, int32_t* diag,
                                     void* stream) {
+  NvtxRange nvtx_range("twell_hybrid_up_down");
   static const char* kName = "twell_hybrid_up_down";
   clear_error();
   int rc = check_args(kName, n_tokens, d_model, d_ff, ldw, tile, cap);

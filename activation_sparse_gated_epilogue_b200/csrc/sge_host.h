@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include <string>
@@ -12,12 +13,26 @@
 
 namespace sge {
 
+// Debug builds: each translation unit registers the reader of its device
+// debug word (read, optionally cleared; -1 on a CUDA error) at load time.
+using DebugReader = int (*)(bool clear);
+bool register_debug_reader(DebugReader reader);
+
 // Records a message for sge_last_error() and returns `code`.
 int fail(int code, const char* fmt, ...);
 void clear_error();
 
 // SGE_OK, or SGE_ERR_CUDA with the message of the pending launch error.
 int check_launch(const char* what);
+
+// An NVTX range over a library call on the calling host thread (names the
+// call in profiler timelines; next to free when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

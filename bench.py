@@ -55,8 +55,8 @@ ROUTED_K = 16
 # --profile (one launch per kernel, L2 cold): the gate GEMM, and the routed
 # call as the sum of its seven launches.
 TRAFFIC = {
-    "012f82b18eff59bd": 79441664,    # twell_gate_pack
-    "67d7c91a0b780ff8": 227635968,   # twell_hybrid_up_down
+    "57e9b5ffe93f838e": 80238080,    # twell_gate_pack
+    "e717b2c31ab7b1fa": 227009792,   # twell_hybrid_up_down
 }
 
 

@@ -76,9 +76,24 @@ extern "C" {
 #define SGE_DIAG_DROPPED_ROWS 2
 #define SGE_DIAG_FLAGS 3
 #define SGE_FLAG_TIMEOUT 1
+#define SGE_FLAG_BOUNDS 2  /* debug builds: an index outside its range */
 
 /* Library version (major * 10000 + minor * 100 + patch). */
 int sge_version(void);
+
+/*
+ * sge_debug_flags -- the debug build's index checks.  libsge_debug.so is the
+ * same library compiled with SGE_DEBUG: every computed index a kernel uses
+ * to address memory that comes from data (stored TwELL columns, token and
+ * spill lists, ELL columns, weight-gradient buckets) is checked against its
+ * range; one outside it sets SGE_FLAG_BOUNDS in a device word and is
+ * replaced by an index inside the range, so the kernel finishes without
+ * touching memory it does not own (no trap).  Returns the OR of the flags
+ * raised since the last clear (synchronising the device), clearing them if
+ * `clear` is nonzero; -1 in the release build (no checks compiled); -2 on a
+ * CUDA error (message in sge_last_error).
+ */
+int sge_debug_flags(int clear);
 
 /* Message of the last failed call on this host thread ("" if none). */
 const char* sge_last_error(void);

@@ -65,6 +65,21 @@ def test_selftest_library_exports_its_declared_symbols(lib):
         assert getattr(st, name) is not None
 
 
+def test_debug_library_exports_the_same_symbols(lib):
+    """libsge_debug.so (the index-checking build) exports every symbol of
+    the header, like the release library; the release build's
+    sge_debug_flags answers -1 without touching the device."""
+    path = sge_build.build_debug()
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    for name in declared_functions():
+        assert name in exported, name
+    lib.sge_debug_flags.restype = ctypes.c_int
+    lib.sge_debug_flags.argtypes = [ctypes.c_int]
+    assert lib.sge_debug_flags(0) == -1
+
+
 def test_selftest_rejects_bad_arguments(lib):
     st = ctypes.CDLL(sge_build.SELFTEST_LIB)
     P = ctypes.c_void_p
