@@ -433,10 +433,22 @@ extern "C" int hybrid_ffn_fwd(const void* x, const sge_hybrid* hy, const void* w
       return rc;
   } else {
     if ((rc = make_tmap_bf16(&mb, wu_t, hy->d_ff, d_model, d_model, S::BN / 2))) return rc;
+    // few spill rows: K (= d) split over the CTA pairs, the parts finished by
+    // split_spill_up_kernel (which shares the down GEMM's part area)
+    float* part_up = reinterpret_cast<float*>(
+        reinterpret_cast<char*>(workspace) +
+        align256(static_cast<size_t>(hy->s_max) * static_cast<size_t>(d_model + hy->d_ff) * 2));
+    const int tiles_up = static_cast<int>((hy->d_ff + S::BN - 1) / S::BN);
     EpiSpillUp e1{static_cast<const uint16_t*>(hy->spill_a), static_cast<uint16_t*>(hy->spill_u), hs,
-                  hy->n_spill, hy->s_max, static_cast<int>(hy->d_ff)};
+                  hy->n_spill, hy->s_max, static_cast<int>(hy->d_ff), part_up, tiles_up, S::BN};
     if ((rc = launch_tc_gemm_pair<S>(ma, mb, mb, hy->s_max, hy->d_ff, d_model, e1, nullptr, st,
-                                     "hybrid_ffn_fwd (spill up)")))
+                                     "hybrid_ffn_fwd (spill up)", kSplitMax)))
+      return rc;
+    if ((rc = launch_pdl(split_spill_up_kernel, dim3(split_grid(hy->s_max, static_cast<int>(hy->d_ff))), dim3(256),
+                         0, st, "hybrid_ffn_fwd (spill up part sums)", static_cast<const float*>(part_up),
+                         static_cast<const uint16_t*>(hy->spill_a), static_cast<uint16_t*>(hy->spill_u), hs,
+                         static_cast<const int32_t*>(hy->n_spill), hy->s_max, static_cast<int>(hy->d_ff),
+                         tiles_up * S::BN)))
       return rc;
   }
   if ((rc = make_tmap_bf16(&mh, hs, hy->s_max, hy->d_ff, hy->d_ff, kBM))) return rc;

@@ -519,6 +519,25 @@ struct EpiBwdSpill {
   int s_max;
   int f;
   int64_t m_rows;  // rows of the padded spill buffers
+  float* part = nullptr;  // split-K parts (split_bwd_spill_kernel finishes them)
+  int n_tiles_n = 1;
+  int tile_n = 256;
+
+  __device__ __forceinline__ int splits() const {
+    return part == nullptr ? 1 : split_count(min(*n_spill, s_max), n_tiles_n);
+  }
+
+  template <int BN>
+  __device__ __forceinline__ void run_split(uint32_t taddr, int64_t row, int n_blk, int split, int nsplit,
+                                            int lane) const {
+    if (part != nullptr && row == 0 && n_blk == 0 && split == 0) *split_word(part) = nsplit;
+    if (nsplit == 1) {
+      run<BN>(taddr, row, n_blk, lane);
+      return;
+    }
+    store_part<BN>(part, min(*n_spill, s_max), static_cast<int64_t>(n_tiles_n) * tile_n, split, row, n_blk,
+                   taddr);
+  }
 
   // rows up to the kept spill rows rounded up to 64 (the K the later GEMMs
   // read): the zero rows past the kept ones matter only that far
@@ -568,6 +587,54 @@ struct EpiBwdSpill {
     }
   }
 };
+
+// Finishes a split dH = dY_s W_down: dh = the parts summed in part order,
+// dU = bf16(dh a), dG = bf16(dh u) where a > 0 (else 0), for the kept rows,
+// and zero rows up to the kept rows rounded up to 64 (the K the later GEMMs
+// read); nothing when the GEMM did not split.  A thread per 8 columns.
+static __global__ void __launch_bounds__(256) split_bwd_spill_kernel(const float* __restrict__ part,
+                                                                     const uint16_t* __restrict__ spill_a,
+                                                                     const uint16_t* __restrict__ spill_u,
+                                                                     uint16_t* __restrict__ acat,
+                                                                     const int32_t* __restrict__ n_spill,
+                                                                     int s_max, int f, int ncp) {
+  grid_dep_wait();  // the parts come from the GEMM before
+  grid_dep_launch();
+  const int nsplit = split_word_read(part);
+  const int kept = min(*n_spill, s_max);
+  if (nsplit <= 1 || kept <= 0) return;
+  const int64_t rows_pad = static_cast<int64_t>((kept + 255) / 256) * 256;
+  const int64_t rows = (kept + 63) / 64 * 64;
+  const int per_row = f / 8;
+  const int64_t total = rows * per_row;
+  for (int64_t i = blockIdx.x * 256ll + threadIdx.x; i < total; i += static_cast<int64_t>(gridDim.x) * 256) {
+    const int64_t r = i / per_row;
+    const int c = static_cast<int>(i % per_row) * 8;
+    uint32_t du[4] = {0, 0, 0, 0}, dg[4] = {0, 0, 0, 0};
+    if (r < kept) {
+      float dh[8];
+      sum_parts8(part, nsplit, rows_pad, ncp, r, c, dh);
+      const uint4 av = *reinterpret_cast<const uint4*>(spill_a + r * f + c);
+      const uint4 uv = *reinterpret_cast<const uint4*>(spill_u + r * f + c);
+      const uint32_t aw[4] = {av.x, av.y, av.z, av.w}, uw[4] = {uv.x, uv.y, uv.z, uv.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float o[2][2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float a = __uint_as_float(h ? (aw[k] & 0xFFFF0000u) : (aw[k] << 16));
+          const float u = __uint_as_float(h ? (uw[k] & 0xFFFF0000u) : (uw[k] << 16));
+          o[h][0] = dh[2 * k + h] * a;
+          o[h][1] = a > 0.0f ? dh[2 * k + h] * u : 0.0f;
+        }
+        du[k] = static_cast<uint32_t>(f32_to_bf16_bits(o[0][0])) | (static_cast<uint32_t>(f32_to_bf16_bits(o[1][0])) << 16);
+        dg[k] = static_cast<uint32_t>(f32_to_bf16_bits(o[0][1])) | (static_cast<uint32_t>(f32_to_bf16_bits(o[1][1])) << 16);
+      }
+    }
+    *reinterpret_cast<uint4*>(acat + r * 2 * f + c) = make_uint4(du[0], du[1], du[2], du[3]);
+    *reinterpret_cast<uint4*>(acat + r * 2 * f + f + c) = make_uint4(dg[0], dg[1], dg[2], dg[3]);
+  }
+}
 
 static int launch_transpose(const uint16_t* src, int rows, int cols, int64_t src_pitch,
                             uint16_t* dst, int64_t dst_pitch, int col_off, cudaStream_t st,
@@ -673,7 +740,7 @@ extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* h
   else rc = launch_ell_bwd<4>(p, n, st);
   if (rc) return rc;
   // ---- spill rows: dH = dY_s W_down^T on tensor cores, epilogue dU | dG
-  using Sh = TcPairShape<128, 1>;  // N = F in 128-wide tiles: few spill row tiles still spread
+  using Sh = TcPairShape<256, 1, 2>;  // N = F: with few spill rows K is split over the CTA pairs
   using Sx = TcPairShape<256, 1, 2>;  // N = d: few tiles, K = 2F split over the CTA pairs
   if (s_max > 0) {
     if ((rc = launch_pdl(gather_rows_kernel, dim3(sp), dim3(256), 0, st, "hybrid_ffn_bwd (gather)", dyb,
@@ -682,8 +749,18 @@ extern "C" int hybrid_ffn_bwd(const void* x, const void* dy, const sge_hybrid* h
     CUtensorMap m1a, m1b;
     if ((rc = make_tmap_bf16(&m1a, ws.dys, sp, d, d, kBM))) return rc;
     if ((rc = make_tmap_bf16(&m1b, wd, f, d, d, Sh::BN / 2))) return rc;
-    EpiBwdSpill e1{hv.spill_a, hv.spill_u, ws.acat, hy->n_spill, s_max, static_cast<int>(f), sp};
-    if ((rc = launch_tc_gemm_pair<Sh>(m1a, m1b, m1b, sp, f, d, e1, nullptr, st, "hybrid_ffn_bwd (dH)")))
+    // few spill rows: K (= d) split over the CTA pairs, the parts finished by
+    // split_bwd_spill_kernel (the part area is the dX GEMM's, used later)
+    const int tiles_h = static_cast<int>((f + Sh::BN - 1) / Sh::BN);
+    EpiBwdSpill e1{hv.spill_a, hv.spill_u, ws.acat, hy->n_spill, s_max, static_cast<int>(f), sp,
+                   ws.part, tiles_h, Sh::BN};
+    if ((rc = launch_tc_gemm_pair<Sh>(m1a, m1b, m1b, sp, f, d, e1, nullptr, st, "hybrid_ffn_bwd (dH)",
+                                      kSplitMax)))
+      return rc;
+    if ((rc = launch_pdl(split_bwd_spill_kernel, dim3(split_grid(sp, static_cast<int>(f))), dim3(256), 0, st,
+                         "hybrid_ffn_bwd (dH part sums)", static_cast<const float*>(ws.part), hv.spill_a,
+                         hv.spill_u, ws.acat, static_cast<const int32_t*>(hy->n_spill), s_max,
+                         static_cast<int>(f), tiles_h * Sh::BN)))
       return rc;
   }
   // ---- every stored entry (ELL and spill rows) bucketed by hidden unit,
