@@ -203,7 +203,8 @@ static int launch_bf16(const void* x, const void* wg_t, int64_t n, int64_t d, in
   if (rc) return rc;
   if (n <= kSmallGateRows) {
     using Small = TcShape<128, 1>;
-    rc = make_tmap_bf16(&mb, wg_t, f, d, d, Small::BN);
+    rc = make_tmap_bf16(&ma, x, n, d, d, a_box_rows(n));  // the engine loads a_box_rows(n) rows of A
+    if (!rc) rc = make_tmap_bf16(&mb, wg_t, f, d, d, Small::BN);
     if (rc) return rc;
     EpiTwell<T> epi{count, idx, static_cast<uint16_t*>(val), n, static_cast<int>(f), cap, diag};
     return launch_tc_gemm<Small>(ma, mb, mb, n, f, d, epi, diag, st,

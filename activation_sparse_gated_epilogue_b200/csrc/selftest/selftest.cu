@@ -49,7 +49,7 @@ extern "C" int sge_selftest_wait_timeout(int pair, const void* a, const void* b,
     return launch_tc_gemm_pair<S>(ma, mb, mb, m, n, k, epi, diag, st, "selftest (pair engine)");
   }
   using S = TcShape<128, 1>;
-  int rc = make_tmap_bf16(&ma, a, m, k, k, kBM);
+  int rc = make_tmap_bf16(&ma, a, m, k, k, a_box_rows(m));
   if (!rc) rc = make_tmap_bf16(&mb, b, n, k, k, S::BN / 2);
   if (rc) return rc;
   return launch_tc_gemm<S>(ma, mb, mb, m, n, k, epi, diag, st, "selftest (single-CTA engine)");

@@ -43,6 +43,8 @@ def _upload_twell(tw: oracle.TwELL, dtype, dev):
     (128, 200, 640, 128, 128),    # one full row tile
     (100, 264, 384, 64, 64),
     (33, 136, 256, 16, 16),
+    (9, 136, 512, 128, 128),      # A boxes of 16 and 32 rows for small batches
+    (20, 264, 384, 64, 64),
 ])
 def test_gate_pack_exact_on_grid_inputs(cuda_device, dtype, n, d, f, tile, cap):
     """Grid inputs make G exact in fp32, so counts, indices and values are
