@@ -4,9 +4,9 @@
 
 One step = one pass of the whole sparse inference path over one batch: the
 gate GEMM with the TwELL epilogue (twell_gate_pack), then the up and down
-projections from TwELL (twell_hybrid_up_down: tokens with at most K = 16
-stored entries through a CUDA-core kernel beside the heavier ones, which run
-through two tcgen05 spill GEMMs), on the 1B-shaped bf16
+projections from TwELL (twell_hybrid_up_down: tokens with at most K = F/512
+stored entries (16 at the 1B shape) through a CUDA-core kernel, the heavier
+ones through two tcgen05 spill GEMMs), on the 1B-shaped bf16
 workload (N=8192 tokens, d=2048, F=8192, T=C=128, mean gate density 1%,
 per-token scale LogNormal(0, 0.7)) unless --workload names another.  Inputs
 are seeded synthetic data resident in HBM; L2 is flushed (a 256 MB write)
@@ -45,9 +45,14 @@ FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # ELL capacity of the hybrid format when it serves inference (tokens with more
 # stored entries run on the tensor-core spill GEMMs)
 HYB_INFER_K = 64
-# K of the routed step: tokens with more stored entries take the spill GEMMs
-# (measured at the 1B shape: K = 16 / 32 gives 0.178 / 0.188 ms for the call)
-ROUTED_K = 16
+# K of the routed step: tokens with more stored entries take the spill GEMMs.
+# A spill row costs the two GEMMs' work over all F hidden units, an entry of
+# the light kernel one 8 KB weight-row copy, so the break-even grows with F:
+# K = F / 512 (measured, routed call alone: 1B (F = 8192) flat for K = 12..20
+# at 0.155-0.156 ms, 0.161-0.165 ms at K = 8 or 24..48; 2B at 1% (F = 10240)
+# 0.594-0.608 ms at K = 16, 0.526-0.533 at K = 20, 0.518-0.524 at K = 48).
+def routed_k(d_ff: int) -> int:
+    return max(8, d_ff // 512)
 
 # DRAM bytes (read + write) per launch from ncu captures of the kernels,
 # keyed by the hash of the source they were taken on; a kernel whose source
@@ -75,8 +80,9 @@ def parse():
     p.add_argument("--cap-sweep", action="store_true",
                    help="TwELL capacity C in {T/4, T/2, T}: footprint, overflow, truncation error, "
                         "and the hybrid path that recomputes overflowing rows: one JSON line per C")
-    p.add_argument("--ell-cap", type=int, default=ROUTED_K,
-                   help="K of the routed step: tokens with more stored entries run on the spill GEMMs")
+    p.add_argument("--ell-cap", type=int, default=0,
+                   help="K of the routed step: tokens with more stored entries run on the spill GEMMs "
+                        "(default: d_ff / 512)")
     p.add_argument("--profile", action="store_true",
                    help="run only warmup + steps of one path (for ncu captures); no JSON")
     p.add_argument("--profile-path", default="routed", choices=["routed", "fused", "hybrid"],
@@ -224,7 +230,7 @@ def run_own(args, rank, world, local_rank):
     n, d, f, tile, cap = cfg.n_tokens, cfg.d_model, cfg.d_ff, cfg.tile, cfg.cap
     # S_max = N: every heavy token can take the spill (the workspace holds
     # the spill operands for N rows; the GEMMs run only the rows there are)
-    k_route, s_max = args.ell_cap, n
+    k_route, s_max = args.ell_cap or routed_k(f), n
     x, wg, wu, wd = (getattr(inp, k).to(dev) for k in ("x", "wg_t", "wu_t", "wd"))
     # weight layouts built once: W_up^T and W_down interleaved row by row (the
     # per-entry kernel's rows, the up GEMM's B operand with row stride 2d) and
@@ -497,6 +503,7 @@ def run_sweep(args, local_rank):
 
     s_max_r = n
     ws_r = sge.routed_workspace(n, d, f, s_max_r, dev)
+    k_r = args.ell_cap or routed_k(f)
     y_r = torch.empty_like(x)
     h = torch.empty((n, f), dtype=x.dtype, device=dev)
     y_dense = torch.empty_like(x)
@@ -509,11 +516,11 @@ def run_sweep(args, local_rank):
         wg[:, d - 1] = -tau                      # rounded to the weight dtype
         gate = lambda: sge.twell_gate_pack(x, wg, tile, cap, out=tw)
         fused = lambda: sge.twell_fused_up_down(x, tw, wu_i, wd_i, y=y, workspace=ws)
-        routed = lambda: sge.twell_hybrid_up_down(x, tw, wu_i, wd_i, wd_t, args.ell_cap, s_max_r,
+        routed = lambda: sge.twell_hybrid_up_down(x, tw, wu_i, wd_i, wd_t, k_r, s_max_r,
                                                   y=y_r, workspace=ws_r)
         tr = timed([gate, routed], steps, 3)
         routed_ms = statistics.mean(a + b for a, b in tr)
-        n_spill_r, nnz_light_r, _ = routed_split(tw.count, cap, args.ell_cap, s_max_r)
+        n_spill_r, nnz_light_r, _ = routed_split(tw.count, cap, k_r, s_max_r)
         t = timed([gate, fused], steps, 3)
         mg = statistics.mean(a for a, _ in t)
         mf = statistics.mean(b for _, b in t)
@@ -543,7 +550,7 @@ def run_sweep(args, local_rank):
             "hybrid_K": hk, "hybrid_spill_rows": int((per_tok > hk).sum().item()),
             "routed_ms": round(routed_ms, 4), "routed_tokens_per_s": round(n / (routed_ms / 1e3), 1),
             "routed_speedup_vs_own_dense": round(dense_ms / routed_ms, 3),
-            "routed_K": args.ell_cap, "routed_S_max": s_max_r, "routed_spill_rows": n_spill_r,
+            "routed_K": k_r, "routed_S_max": s_max_r, "routed_spill_rows": n_spill_r,
             "routed_nnz_per_entry_path": nnz_light_r,
             "routed_step_roofline_frac": round((flops_gate + 4.0 * n_spill_r * d * f) / (pk["bf16_tflops"] * 1e12) * 1e3
                                                / routed_ms + 4.0 * nnz_light_r * d / (FP32_SIMT_TFLOPS * 1e12) * 1e3
