@@ -381,9 +381,11 @@ def run_own(args, rank, world, local_rank):
     flops_light = 4.0 * nnz_light * d
     routed_roof_ms = (flops_spill / (bf16_peak * 1e12) + flops_light / (FP32_SIMT_TFLOPS * 1e12)) * 1e3
     gate_roof_ms = flops_gate / (bf16_peak * 1e12) * 1e3
-    gate_src = src_hash("gate_pack.cu", "tc_gemm.cuh", "sge_common.cuh")
-    routed_src = src_hash("routed.cu", "fused_kernels.cuh", "spill_gemm.cuh", "tc_gemm.cuh",
-                          "sparse_common.cuh", "sge_common.cuh")
+    # each hash covers the kernel's source and every header it includes
+    gate_src = src_hash("gate_pack.cu", "tc_launch.cuh", "tc_gemm.cuh", "sge_common.cuh", "sge_host.h")
+    routed_src = src_hash("routed.cu", "fused_kernels.cuh", "spill_gemm.cuh", "tc_launch.cuh",
+                          "tc_gemm.cuh", "sparse_common.cuh", "debug_checks.cuh", "sge_common.cuh",
+                          "sge_host.h")
     tr_gate, tr_routed = TRAFFIC.get(gate_src), TRAFFIC.get(routed_src)
     k_gate = {"kernel": "twell_gate_pack (tcgen05 GEMM + TwELL epilogue)", "bound": "tensor",
               "achieved": round(gate_tf, 1), "peak": bf16_peak, "unit": "TFLOP/s",

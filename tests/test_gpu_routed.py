@@ -117,10 +117,12 @@ def test_routed_zero_and_full_density(cuda_device):
             assert oracle.max_abs_rel(to_f64(y), want) <= BF16_TOL
 
 
-@pytest.mark.parametrize("k", [32, 64, 128])
-def test_routed_1b_all_rows(cuda_device, k):
-    """The 1B workload as the bench runs it (gate GEMM + TwELL on the GPU,
-    interleaved weights, S_max = N/4): every row against the oracle."""
+@pytest.mark.parametrize("k,s_div", [(16, 1), (32, 4), (64, 4), (128, 4)])
+def test_routed_1b_all_rows(cuda_device, k, s_div):
+    """The 1B workload (gate GEMM + TwELL on the GPU, interleaved weights),
+    every row against the oracle.  K = F/512 = 16 with S_max = N is the
+    launch configuration bench.py times; the others move the light/heavy
+    boundary and cap the spill at N/4."""
     inp = oracle_1b()[0]
     cfg = inp.cfg
     dev = cuda_device
@@ -128,7 +130,7 @@ def test_routed_1b_all_rows(cuda_device, k):
     _, wu_i, wd_i = sge.interleave_up_down(wu, wd)
     tw = sge.twell_gate_pack(x, wg, cfg.tile, cfg.cap)
     diag = sge.new_diag(dev)
-    y = sge.twell_hybrid_up_down(x, tw, wu_i, wd_i, wd.t().contiguous(), k, cfg.n_tokens // 4,
+    y = sge.twell_hybrid_up_down(x, tw, wu_i, wd_i, wd.t().contiguous(), k, cfg.n_tokens // s_div,
                                  diag=diag)
     torch.cuda.synchronize()
     assert int(diag[3]) == 0
@@ -136,11 +138,16 @@ def test_routed_1b_all_rows(cuda_device, k):
     print(f"routed 1B K={k}: {int(diag[1])} spill rows, max-abs-rel {err:.2e}, {flips} flips")
 
 
-@pytest.mark.parametrize("rho", [0.0025, 0.05])
-def test_routed_2b_sweep_ends(cuda_device, rho):
-    """The 2B workload at the sweep's lightest and densest points (at 5%
-    most tokens are heavy and those past S_max = N/4 run per entry): the
-    128 heaviest tokens and every 4th token against the oracle."""
+@pytest.mark.parametrize("rho,k,s_div", [
+    (0.0025, 20, 1), (0.005, 20, 1), (0.01, 20, 1), (0.02, 20, 1), (0.05, 20, 1),
+    (0.0025, 64, 4), (0.05, 64, 4),
+])
+def test_routed_2b_sweep(cuda_device, rho, k, s_div):
+    """The 2B workload at every density of the sweep in bench.py's launch
+    configuration (K = F/512 = 20, S_max = N), and at the lightest and
+    densest points with K = 64, S_max = N/4 (at 5% most tokens are heavy and
+    those past S_max run per entry): the 128 heaviest tokens and every 4th
+    token against the oracle."""
     cfg = synth.CONFIGS["ffn_2b_bf16"].with_(rho=rho)
     inp = synth.make_inputs(cfg)
     rows = heavy_and_strided_rows(inp)
@@ -149,9 +156,10 @@ def test_routed_2b_sweep_ends(cuda_device, rho):
     _, wu_i, wd_i = sge.interleave_up_down(wu, wd)
     tw = sge.twell_gate_pack(x, wg, cfg.tile, cfg.cap)
     diag = sge.new_diag(dev)
-    y = sge.twell_hybrid_up_down(x, tw, wu_i, wd_i, wd.t().contiguous(), 64, cfg.n_tokens // 4,
+    y = sge.twell_hybrid_up_down(x, tw, wu_i, wd_i, wd.t().contiguous(), k, cfg.n_tokens // s_div,
                                  diag=diag)
     torch.cuda.synchronize()
+    assert int(diag[3]) == 0
     g0, abs0 = sweep_gate0(inp, rows)
     g = g0 - inp.tau
     tw_ora = oracle.twell_pack(g, cfg.tile, cfg.cap, oracle.VAL_BF16)
@@ -161,7 +169,35 @@ def test_routed_2b_sweep_ends(cuda_device, rho):
     assert not shifted.any()
     err = oracle.max_abs_rel(to_f64(y)[rows], y_ora)
     assert err <= BF16_TOL, err
-    print(f"routed 2B rho={rho}: {int(diag[1])} heavy tokens, max-abs-rel {err:.2e}, {flips} flips")
+    print(f"routed 2B rho={rho} K={k}: {int(diag[1])} heavy tokens, max-abs-rel {err:.2e}, {flips} flips")
+
+
+@pytest.mark.parametrize("n", [64, 32, 8, 1])
+def test_routed_decode_1b_all_rows(cuda_device, n):
+    """The decode-shaped workload (a small batch against the 1B weights) as
+    bench.py runs it: the gate GEMM on single-CTA tiles, then the routed call
+    with K = F/512 = 16, S_max = N, which takes the small-batch path; every
+    row against the oracle's whole forward."""
+    cfg = synth.CONFIGS["decode_1b_bf16"].with_(n_tokens=n)
+    inp = synth.make_inputs(cfg)
+    dev = cuda_device
+    x, wg, wu, wd = (getattr(inp, nm).to(dev) for nm in ("x", "wg_t", "wu_t", "wd"))
+    _, wu_i, wd_i = sge.interleave_up_down(wu, wd)
+    tw = sge.twell_gate_pack(x, wg, cfg.tile, cfg.cap)
+    diag = sge.new_diag(dev)
+    y = sge.twell_hybrid_up_down(x, tw, wu_i, wd_i, wd.t().contiguous(), cfg.d_ff // 512, n,
+                                 diag=diag)
+    torch.cuda.synchronize()
+    assert int(diag[3]) == 0
+    xf, wgf, wuf, wdf = (inp.as_f64(nm) for nm in ("x", "wg_t", "wu_t", "wd"))
+    y_ora, tw_ora, g = oracle.sparse_ffn(xf, wgf, wuf, wdf, cfg.tile, cfg.cap, oracle.VAL_BF16)
+    abs_sum = np.abs(xf) @ np.abs(wgf).T
+    _, shifted, flips, _ = compare_twell_inexact(tw, tw_ora, g, oracle.VAL_BF16, abs_sum,
+                                                 d_model=cfg.d_model)
+    assert not shifted.any()          # C = T: no truncated tile
+    err = oracle.max_abs_rel(to_f64(y), y_ora)
+    assert err <= BF16_TOL, err
+    print(f"routed decode N={n}: max-abs-rel {err:.2e}, {flips} flips")
 
 
 def test_routed_heavy_tokens_past_s_max(cuda_device):
