@@ -60,8 +60,8 @@ def routed_k(d_ff: int) -> int:
 # --profile (one launch per kernel, L2 cold): the gate GEMM, and the routed
 # call as the sum of its seven launches.
 TRAFFIC = {
-    "57e9b5ffe93f838e": 80238080,    # twell_gate_pack
-    "e717b2c31ab7b1fa": 227009792,   # twell_hybrid_up_down
+    "e0bf0d70a6a99597": 79755264,    # twell_gate_pack
+    "3f0db3f8024f022c": 227535616,   # twell_hybrid_up_down
 }
 
 
@@ -780,9 +780,11 @@ def run_train(args, local_rank):
                    "backward plus y (hybrid: ELL rows, routing and the S_max-row spill buffers; "
                    "dense autograd: relu(G), U and h); the peaks include workspaces, the "
                    "hybrid's transient TwELL (C = T) and its fp32 weight gradients (dense: bf16)"},
-        "gpu_launches_per_step": 21,
-        "launches_note": "gate 1, pack 3 (counts, route, fill), forward 4 (ELL, gather, 2 GEMMs), backward 13 "
-                         "(ELL, gather, dH GEMM, bucket memset, 2 counts, scan, 2 scatters, sort, dW, dX GEMM)",
+        "gpu_launches_per_step": 23,
+        "launches_note": "library kernels per step: gate 1, pack 3 (counts, route, fill), forward 6 (ELL, "
+                         "gather, up GEMM, its split-K sum, down GEMM, its split-K sum), backward 13 (ELL, "
+                         "gather, dH GEMM, its split-K sum, 2 counts, scan, 2 scatters, sort, dW, dX GEMM, "
+                         "its split-K sum); plus one cudaMemsetAsync of the bucket counts",
         "clocks": clk.summary(), "diag": diag.tolist(),
     }
 
