@@ -216,6 +216,23 @@ def routed_split(count: torch.Tensor, cap: int, k: int, s_max: int):
     return int(heavy.numel()), total - spilled, total
 
 
+def twell_bytes(count: torch.Tensor, cap: int, elt: int) -> dict:
+    """Sizes of a TwELL with per-tile counts `count` ([N][F/T] u8), u8
+    indices and `elt`-byte values: the allocated layout, the algorithmic
+    bytes (one count per (row, tile), one index and one value per stored
+    entry) and the bytes of the 32-byte DRAM sectors a reader of the stored
+    entries touches.  Each tile's index run starts on a C-byte boundary and
+    its value run on a C*elt-byte boundary, so for C a multiple of 32 a tile
+    with c stored entries touches ceil(c/32) + ceil(c*elt/32) sectors."""
+    n, nt = count.shape
+    c = torch.clamp(count.to(torch.int64), max=cap)
+    stored = int(c.sum().item())
+    sectors = int(((c + 31) // 32 + (c * elt + 31) // 32).sum().item())
+    return {"allocated": n * nt * (1 + (1 + elt) * cap), "algorithmic": n * nt + (1 + elt) * stored,
+            "sector_granular": n * nt + 32 * sectors if cap % 32 == 0 else None,
+            "unit": "bytes", "note": "counts read whole; sectors of the stored index and value runs"}
+
+
 def run_own(args, rank, world, local_rank):
     import activation_sparse_gated_epilogue_b200 as sge
     from activation_sparse_gated_epilogue_b200 import synth
@@ -420,6 +437,7 @@ def run_own(args, rank, world, local_rank):
                    "step": f"twell_gate_pack + twell_hybrid_up_down (K={k_route}, S_max={s_max})",
                    "realised_density": round(density, 5), "nnz": nnz, "spill_rows": n_spill,
                    "nnz_per_entry_path": nnz_light,
+                   "twell_bytes": twell_bytes(tw.count, cap, x.element_size()),
                    "l2": "flushed between steps (256 MB write outside the step events)",
                    "weights": "W_up^T and W_down interleaved row by row ([F][2d]) and W_down^T "
                               "([d][F]), both built once",

@@ -43,3 +43,19 @@ def test_own_arm_refuses_fp32_workloads_before_touching_a_gpu():
     import pytest
     with pytest.raises(SystemExit, match="parity case"):
         bench.run_own(_args(workload="tiny_fp32", impl="own", tokens=0), 0, 1, 0)
+
+
+def test_twell_bytes_counts_sectors_per_tile():
+    """Counts 0, 1, 32, 33 and 200 (> C = 128, so 128 stored) in bf16:
+    0 + 2 + 3 + 5 + 12 sectors of 32 B over the index and value runs."""
+    import torch
+    count = torch.tensor([[0, 1, 32, 33, 200]], dtype=torch.uint8)
+    got = bench.twell_bytes(count, 128, 2)
+    assert got["allocated"] == 5 * (1 + 3 * 128)
+    assert got["algorithmic"] == 5 + 3 * (0 + 1 + 32 + 33 + 128)
+    assert got["sector_granular"] == 5 + 32 * (0 + 2 + 3 + 5 + 12)
+    assert bench.twell_bytes(count, 48, 2)["sector_granular"] is None
+
+
+def test_routed_k_rule():
+    assert bench.routed_k(8192) == 16 and bench.routed_k(10240) == 20 and bench.routed_k(1024) == 8
