@@ -59,3 +59,15 @@ def test_twell_bytes_counts_sectors_per_tile():
 
 def test_routed_k_rule():
     assert bench.routed_k(8192) == 16 and bench.routed_k(10240) == 20 and bench.routed_k(1024) == 8
+
+
+def test_routed_split_counts_heavy_tokens_in_order():
+    """Stored entries per token 3, 40, 0, 17, 200 (capped at C = 128 per
+    tile) with K = 16, S_max = 2: tokens 1 and 3 take the spill, token 4
+    (heavy, past S_max) stays with the per-entry path."""
+    import torch
+    count = torch.tensor([[3, 0], [20, 20], [0, 0], [17, 0], [100, 100]], dtype=torch.uint8)
+    n_spill, nnz_light, nnz = bench.routed_split(count, 128, 16, 2)
+    assert (n_spill, nnz_light, nnz) == (2, 3 + 200, 3 + 40 + 17 + 200)
+    # C = 10 stores 3, 20, 0, 10, 20 entries: tokens 1 and 4 are heavy
+    assert bench.routed_split(count, 10, 16, 8) == (2, 3 + 10, 3 + 20 + 10 + 20)
