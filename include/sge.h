@@ -246,8 +246,8 @@ int twell_fused_up_down_noalloc(const void* x, const uint8_t* count, const uint8
  *   ell_cap              K >= 0.  A spill row costs the two GEMMs over all
  *                        F hidden units, a light entry one copy of its
  *                        weight rows, so the break-even grows with F: K =
- *                        F/512 measured within 2% of the best K at F = 8192 and
- *                        F = 10240
+ *                        F/512 measured within 2% of the best K at 1%
+ *                        density for F = 8192 and F = 10240
  *   s_max                spill capacity in tokens, >= 0
  *   workspace            >= twell_hybrid_up_down_workspace_bytes(N, d, F,
  *                        s_max) bytes, 256-byte aligned, caller-owned, not
