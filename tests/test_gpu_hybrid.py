@@ -169,6 +169,43 @@ def test_hybrid_bwd_is_deterministic(cuda_device):
         assert torch.equal(u, v)
 
 
+@pytest.mark.parametrize("tau", [1e3, -1e3])
+def test_hybrid_bwd_zero_and_full_density(cuda_device, tau):
+    """No active gate (tau = 1e3): every row is an empty ELL row, and y, dx
+    and all three weight gradients are exactly zero.  Every gate active
+    (tau = -1e3): every row holds F entries, so with K = 16 and S_max = N all
+    rows take the dense spill GEMMs and each hidden unit's gradient bucket
+    holds all N tokens (more than one round of staged entries); the results
+    match the oracle."""
+    n, d, f, k = 300, 256, 1024, 16
+    cfg = synth.CONFIGS["train_1b_hybrid"].with_(n_tokens=n, d_model=d, d_ff=f, spill_frac=None,
+                                                 rho=0.02, seed=4)
+    inp = synth.make_inputs(cfg, tau=tau)
+    x, wg, wu, wd, dy = (inp.as_f64(nm) for nm in ("x", "wg_t", "wu_t", "wd", "dy"))
+    tw = oracle.twell_pack(oracle.gate_preact(x, wg), 128, 128, oracle.VAL_BF16)
+    assert int(tw.count.astype(np.int64).sum()) == (0 if tau > 0 else n * f)
+    ora = oracle.hybrid_pack(tw, k, n)
+    y_ora = oracle.hybrid_fwd(x, ora, wu, wd)
+    want = oracle.hybrid_bwd(x, dy, ora, wg, wu, wd)
+
+    dev = cuda_device
+    xd, dyd = inp.x.to(dev), inp.dy.to(dev)
+    w_dev = [getattr(inp, nm).to(dev) for nm in ("wg_t", "wu_t", "wd")]
+    hy = sge.hybrid_pack(_upload_twell(tw, dev), k, n)
+    y = sge.hybrid_ffn_fwd(xd, hy, w_dev[1], w_dev[2], w_dev[2].t().contiguous())
+    got = sge.hybrid_ffn_bwd(xd, dyd, hy, *w_dev)
+    torch.cuda.synchronize()
+    assert int(hy.n_spill.item()) == (0 if tau > 0 else n)
+    if tau > 0:
+        for t in (y,) + tuple(got):
+            assert not torch.any(t != 0)
+        return
+    assert oracle.max_abs_rel(to_f64(y), y_ora) <= BF16_TOL
+    for name, a, b in zip(("dx", "dW_gate", "dW_up", "dW_down"), got, want):
+        err = oracle.max_abs_rel(to_f64(a), b)
+        assert err <= BF16_TOL, (name, err)
+
+
 def test_hybrid_inference_1b_all_rows(cuda_device):
     """The hybrid path as the bench runs it for inference on the 1B workload
     (K = 64, S_max = N/4: about 1,400 heavy rows on the tensor-core spill),
