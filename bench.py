@@ -80,9 +80,9 @@ def parse():
     p.add_argument("--cap-sweep", action="store_true",
                    help="TwELL capacity C in {T/4, T/2, T}: footprint, overflow, truncation error, "
                         "and the hybrid path that recomputes overflowing rows: one JSON line per C")
-    p.add_argument("--ell-cap", type=int, default=0,
+    p.add_argument("--ell-cap", type=int, default=None,
                    help="K of the routed step: tokens with more stored entries run on the spill GEMMs "
-                        "(default: d_ff / 512)")
+                        "(default: d_ff / 512; 0 spills every non-empty token)")
     p.add_argument("--profile", action="store_true",
                    help="run only warmup + steps of one path (for ncu captures); no JSON")
     p.add_argument("--profile-path", default="routed", choices=["routed", "fused", "hybrid"],
@@ -247,7 +247,7 @@ def run_own(args, rank, world, local_rank):
     n, d, f, tile, cap = cfg.n_tokens, cfg.d_model, cfg.d_ff, cfg.tile, cfg.cap
     # S_max = N: every heavy token can take the spill (the workspace holds
     # the spill operands for N rows; the GEMMs run only the rows there are)
-    k_route, s_max = args.ell_cap or routed_k(f), n
+    k_route, s_max = routed_k(f) if args.ell_cap is None else args.ell_cap, n
     x, wg, wu, wd = (getattr(inp, k).to(dev) for k in ("x", "wg_t", "wu_t", "wd"))
     # weight layouts built once: W_up^T and W_down interleaved row by row (the
     # per-entry kernel's rows, the up GEMM's B operand with row stride 2d) and
@@ -523,7 +523,7 @@ def run_sweep(args, local_rank):
 
     s_max_r = n
     ws_r = sge.routed_workspace(n, d, f, s_max_r, dev)
-    k_r = args.ell_cap or routed_k(f)
+    k_r = routed_k(f) if args.ell_cap is None else args.ell_cap
     y_r = torch.empty_like(x)
     h = torch.empty((n, f), dtype=x.dtype, device=dev)
     y_dense = torch.empty_like(x)
