@@ -262,8 +262,8 @@ def twell_hybrid_up_down(x: torch.Tensor, tw: TwELL, wu_t: torch.Tensor, wd: tor
                          y: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                          diag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """y from TwELL with tokens of more than ell_cap stored entries (the first
-    s_max of them) on the tensor-core spill GEMMs and the others through the
-    per-entry fused kernel.  bf16.  ``wd_t`` is W_down transposed, [d][F]
+    s_max of them) on the tensor-core spill GEMMs and the others per entry on
+    CUDA cores (batches of at most 64 tokens: every token per entry).  bf16.  ``wd_t`` is W_down transposed, [d][F]
     (None only when s_max == 0); wu_t and wd may be the row-strided halves of
     interleave_up_down's matrix."""
     _check(x, "x", torch.bfloat16)
